@@ -1,0 +1,460 @@
+"""Benchmark: FP4 quantized linear layer fwd+bwd on a Llama-3.1-8B MLP shape.
+
+One step = the whole hot path over one batch: six quantizations (X, W along K
+for Fprop; dY along N and W along N for Dgrad; dY and X along the tokens for
+Wgrad; NVFP4 tensor-amax passes included) and the three block-scaled FP4
+GEMMs, through the library's C ABI. The headline `value` is 6 M N K / step
+time (TFLOP/s) with inputs resident in HBM; `e2e` is the same metric through
+qfp4_linear_fwd/bwd with host buffers (pinned H2D of X, W, dY and D2H of Y,
+dX, dW inside the timed region). `quantize` reports the quantizer sweep
+workload's GB/s. Synthetic inputs from fp4_precision_b200.inputs.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 runs N independent replicas (one per GPU, launched by torchrun); the
+path has no exchange step, so there is no data-path collective.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "FP4 linear fwd+bwd TFLOPS (8B MLP shapes) & quantize GB/s, as % of roofline"
+WORKLOAD = "mlp_up"  # Llama-3.1-8B MLP up/gate: X [16384x4096], W [28672x4096], dY [16384x28672]
+RECIPE = "QUARTET2_NVFP4"
+NOMINAL_FP4_OVER_BF16 = 4.0  # dense FP4 9 PF / dense BF16 2.25 PF (nominal ratio)
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f), "measured"
+    except OSError:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from fp4_precision_b200 import inputs
+    from fp4_precision_b200 import qfp4 as Q
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    wl = inputs.workload(WORKLOAD, device=dev)
+    X, W, dY = wl["X"], wl["W"], wl["dY"]
+    M, K = X.shape
+    N = W.shape[0]
+    rec = Q.recipe(RECIPE)
+    seed = Q.make_seed(rot=0x0123_4567, sr=0x89AB_CDEF)
+    stream = torch.cuda.current_stream()
+    ws = torch.empty((Q.quantize_workspace_bytes(),), dtype=torch.uint8, device=dev)
+
+    # quantized operands of the step, allocated once
+    c = rec.fprop, rec.dgrad, rec.wgrad
+    ops = [(X, c[0].fmt, c[0].rnd_a, c[0].had, Q.ROW, Q.make_seed(seed.rot, seed.sr, 0, 0)),
+           (W, c[0].fmt, c[0].rnd_b, c[0].had, Q.ROW, Q.make_seed(seed.rot, seed.sr, 0, 1)),
+           (dY, c[1].fmt, c[1].rnd_a, c[1].had, Q.ROW, Q.make_seed(seed.rot, seed.sr, 1, 2)),
+           (W, c[1].fmt, c[1].rnd_b, c[1].had, Q.COL, Q.make_seed(seed.rot, seed.sr, 1, 3)),
+           (dY, c[2].fmt, c[2].rnd_a, c[2].had, Q.COL, Q.make_seed(seed.rot, seed.sr, 2, 4)),
+           (X, c[2].fmt, c[2].rnd_b, c[2].had, Q.COL, Q.make_seed(seed.rot, seed.sr, 2, 5))]
+    qs = []
+    for (t, fmt, rnd, had, axis, sd) in ops:
+        rows, k = (t.shape[0], t.shape[1]) if axis == Q.ROW else (t.shape[1], t.shape[0])
+        qs.append(Q.empty_qtensor(fmt, rows, k, dev))
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    dX = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+    dW = torch.empty((N, K), dtype=torch.float32, device=dev)
+    gemm_flops = [2.0 * M * N * K] * 3
+    quant_elems = [t.numel() for (t, *_rest) in ops]
+
+    def step(ev=None):
+        # ev: list of (start, end) event pairs per kernel group, or None
+        for i, (t, fmt, rnd, had, axis, sd) in enumerate(ops):
+            if ev is not None:
+                ev[i][0].record(stream)
+            Q.quantize(t, fmt, rnd, had, axis, sd, out=qs[i], workspace=ws, stream=stream)
+            if ev is not None:
+                ev[i][1].record(stream)
+            if i == 1:
+                if ev is not None:
+                    ev[6][0].record(stream)
+                Q.gemm(qs[0], qs[1], torch.bfloat16, out=Y, stream=stream)
+                if ev is not None:
+                    ev[6][1].record(stream)
+            if i == 3:
+                if ev is not None:
+                    ev[7][0].record(stream)
+                Q.gemm(qs[2], qs[3], torch.bfloat16, out=dX, stream=stream)
+                if ev is not None:
+                    ev[7][1].record(stream)
+        if ev is not None:
+            ev[8][0].record(stream)
+        Q.gemm(qs[4], qs[5], torch.float32, out=dW, stream=stream)
+        if ev is not None:
+            ev[8][1].record(stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        step()
+    Q.status()
+    barrier()
+
+    # timed region: K steps, events on the launching stream
+    evs = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)] for _ in range(9)]
+           for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    Q.launch_count(reset=True)
+    with ClockSampler(local_rank) as clk:
+        barrier()
+        t0.record(stream)
+        for s in range(args.steps):
+            step(evs[s])
+        t1.record(stream)
+        barrier()
+    launches = Q.launch_count(reset=True)
+    Q.status()
+    ms = t0.elapsed_time(t1)
+    if world > 1:
+        tt = torch.tensor([ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    ms_step = ms / args.steps
+    per = [[evs[s][j][0].elapsed_time(evs[s][j][1]) for s in range(args.steps)] for j in range(9)]
+    gemm_ms = [statistics.mean(per[6 + g]) for g in range(3)]
+    quant_ms = [statistics.mean(per[i]) for i in range(6)]
+    flops_step = 6.0 * M * N * K
+    value = world * flops_step / (ms_step * 1e-3) / 1e12
+
+    peaks, src = measured_peaks()
+    fp4_peak = peaks["bf16_tflops_sustained"] * NOMINAL_FP4_OVER_BF16
+    gemm_achieved = sum(gemm_flops) / (sum(gemm_ms) * 1e-3) / 1e12
+
+    # quantizer sweep workload (GB/s of algorithmic bytes), L2 flushed between launches
+    quant = quant_sweep(Q, inputs, dev, stream, peaks)
+
+    # linear API (device-resident) and end to end with host buffers
+    api_ms = linear_api_time(Q, X, W, dY, rec, seed, args, stream, dev)
+    e2e = None if args.no_e2e else e2e_time(Q, X, W, dY, rec, seed, args, stream, dev, world)
+
+    out = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "e2m1", "data": "synthetic",
+        "config": {"workload": "Llama-3.1-8B MLP up/gate linear fwd+bwd, X[16384x4096] W[28672x4096] "
+                               "dY[16384x28672], NVFP4 Quartet II recipe",
+                   "M": M, "N": N, "K": K, "recipe": RECIPE,
+                   "l2": "inputs larger than L2 (dY 940 MB, W 235 MB, X 134 MB); no flush between steps",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": {"bound": "tensor", "kernel": "gemm_bs_fp4 (tcgen05 kind::mxf4nvf4)",
+                     "achieved": round(gemm_achieved, 1),
+                     "peak": round(fp4_peak, 1), "unit": "TFLOP/s", "frac": round(gemm_achieved / fp4_peak, 4),
+                     "traffic": None,
+                     "peak_source": f"{src}: bf16_tflops_sustained {peaks['bf16_tflops_sustained']} x nominal FP4/BF16 "
+                                    f"ratio {NOMINAL_FP4_OVER_BF16}",
+                     "per_gemm_ms": {"fprop": round(gemm_ms[0], 4), "dgrad": round(gemm_ms[1], 4),
+                                     "wgrad": round(gemm_ms[2], 4)}},
+        "step_breakdown_ms": {"quantize": [round(v, 4) for v in quant_ms], "gemm": [round(v, 4) for v in gemm_ms]},
+        "quantize": quant,
+        "linear_api_ms_per_step": round(api_ms, 4),
+        "e2e": e2e,
+        "gpu_launches": launches,
+        "clocks": clk.summary(),
+    }
+    return out
+
+
+def quant_sweep(Q, inputs, dev, stream, peaks):
+    """The quantizer-sweep tensor [8192x4096]: GB/s of algorithmic bytes
+    (2 B read + 0.5 B codes + scale bytes per element; the NVFP4 amax pass
+    counted separately at 2 B/elem), L2 flushed before every launch."""
+    import torch
+    T = inputs.workload("sweep", device=dev)["T"]
+    R, C = T.shape
+    flush = torch.empty((256 << 20,), dtype=torch.uint8, device=dev)
+    ws = torch.empty((Q.quantize_workspace_bytes(),), dtype=torch.uint8, device=dev)
+    amax = Q.amax(T, Q.HAD_NONE, Q.ROW, workspace=ws, stream=stream)
+    res = {}
+    cases = [("nvfp4_rtn_none_row", Q.NVFP4, Q.RTN, Q.HAD_NONE, Q.ROW),
+             ("nvfp4_q2_rand16_row", Q.NVFP4, Q.QUARTET2, Q.HAD_RAND16, Q.ROW),
+             ("nvfp4_sr_rand16_row", Q.NVFP4, Q.SR, Q.HAD_RAND16, Q.ROW),
+             ("nvfp4_q2_rand16_col", Q.NVFP4, Q.QUARTET2, Q.HAD_RAND16, Q.COL),
+             ("mxfp4_rtn_det32_col", Q.MXFP4, Q.RTN, Q.HAD_DET32, Q.COL),
+             ("mxfp4_rtn_none_row", Q.MXFP4, Q.RTN, Q.HAD_NONE, Q.ROW)]
+    seed = Q.make_seed(5, 6)
+    for name, fmt, rnd, had, axis in cases:
+        rows, k = (R, C) if axis == Q.ROW else (C, R)
+        q = Q.empty_qtensor(fmt, rows, k, dev)
+        # a pre-computed amax isolates the one-pass quantizer kernel
+        am = Q.amax(T, had, axis, seed, workspace=ws, stream=stream) if fmt == Q.NVFP4 else None
+        times = []
+        for it in range(8):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            Q.quantize(T, fmt, rnd, had, axis, seed, amax_in=am, out=q, workspace=ws, stream=stream)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            if it >= 3:
+                times.append(e0.elapsed_time(e1))
+        ms = statistics.median(times)
+        byts = R * C * (2 + 0.5 + (1 / 16 if fmt == Q.NVFP4 else 1 / 32))
+        gbs = byts / (ms * 1e-3) / 1e9
+        res[name] = {"ms": round(ms, 4), "GB/s": round(gbs, 1), "frac_of_measured_hbm": round(gbs / peaks["hbm_gbs"], 3)}
+    # the amax pass alone
+    times = []
+    for it in range(8):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        Q.amax(T, Q.HAD_RAND16, Q.ROW, seed, out=amax, workspace=ws, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if it >= 3:
+            times.append(e0.elapsed_time(e1))
+    ms = statistics.median(times)
+    gbs = R * C * 2 / (ms * 1e-3) / 1e9
+    res["amax_rand16_row"] = {"ms": round(ms, 4), "GB/s": round(gbs, 1),
+                              "frac_of_measured_hbm": round(gbs / peaks["hbm_gbs"], 3)}
+    Q.status()
+    return {"workload": "quantizer sweep tensor [8192x4096] bf16, Student-t(3)*0.02*LogNormal(0,1) column gains",
+            "bytes_per_elem": "2 read + 0.5 codes + 1/16 (NVFP4) or 1/32 (MXFP4) scales; amax pass 2 read",
+            "l2": "256 MiB buffer written before every launch", "unit": "GB/s", "cases": res}
+
+
+def linear_api_time(Q, X, W, dY, rec, seed, args, stream, dev):
+    import torch
+    M, K = X.shape
+    N = W.shape[0]
+    wsf = torch.empty((Q.linear_workspace_bytes(False, M, N, K, rec),), dtype=torch.uint8, device=dev)
+    wsb = torch.empty((Q.linear_workspace_bytes(True, M, N, K, rec),), dtype=torch.uint8, device=dev)
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    dX = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+    dW = torch.empty((N, K), dtype=torch.float32, device=dev)
+    for _ in range(2):
+        Q.linear_fwd(X, W, rec, seed, Y=Y, workspace=wsf, stream=stream)
+        Q.linear_bwd(dY, X, W, rec, seed, dX=dX, dW=dW, workspace=wsb, stream=stream)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n = max(3, args.steps // 2)
+    e0.record(stream)
+    for _ in range(n):
+        Q.linear_fwd(X, W, rec, seed, Y=Y, workspace=wsf, stream=stream)
+        Q.linear_bwd(dY, X, W, rec, seed, dX=dX, dW=dW, workspace=wsb, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    Q.status()
+    return e0.elapsed_time(e1) / n
+
+
+def e2e_time(Q, X, W, dY, rec, seed, args, stream, dev, world):
+    """qfp4_linear_fwd/bwd with host buffers: pinned H2D of the step's inputs and
+    D2H of its outputs inside the timed region."""
+    import torch
+    M, K = X.shape
+    N = W.shape[0]
+    hX, hW, hdY = (t.cpu().pin_memory() for t in (X, W, dY))
+    hY = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+    hdX = torch.empty((M, K), dtype=torch.bfloat16).pin_memory()
+    hdW = torch.empty((N, K), dtype=torch.float32).pin_memory()
+    dXd, dWd, dYd = torch.empty_like(X), torch.empty_like(W), torch.empty_like(dY)
+    wsf = torch.empty((Q.linear_workspace_bytes(False, M, N, K, rec),), dtype=torch.uint8, device=dev)
+    wsb = torch.empty((Q.linear_workspace_bytes(True, M, N, K, rec),), dtype=torch.uint8, device=dev)
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    gX = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+    gW = torch.empty((N, K), dtype=torch.float32, device=dev)
+
+    def one():
+        dXd.copy_(hX, non_blocking=True)
+        dWd.copy_(hW, non_blocking=True)
+        dYd.copy_(hdY, non_blocking=True)
+        Q.linear_fwd(dXd, dWd, rec, seed, Y=Y, workspace=wsf, stream=stream)
+        Q.linear_bwd(dYd, dXd, dWd, rec, seed, dX=gX, dW=gW, workspace=wsb, stream=stream)
+        hY.copy_(Y, non_blocking=True)
+        hdX.copy_(gX, non_blocking=True)
+        hdW.copy_(gW, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    n = max(2, min(args.steps, 5))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    Q.status()
+    ms = e0.elapsed_time(e1) / n
+    if world > 1:
+        import torch.distributed as dist
+        tt = torch.tensor([ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    h2d = (M * K + N * K + M * N) * 2
+    d2h = M * N * 2 + M * K * 2 + N * K * 4
+    return {"value": round(world * 6.0 * M * N * K / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+            "ms_per_step": round(ms, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+# ---------------------------------------------------------------------------
+def oracle_sample(m_rows: int, n_rows: int, steps: int = 1):
+    """The CPU oracle on a bounded sample of the workload: the linear fwd+bwd of
+    the first m_rows tokens and n_rows output features (all six quantizations
+    and the three fp64 GEMMs of that sub-layer, full K). Returns (seconds per
+    sample step, flops of the sample, threads)."""
+    import oracle as O
+    from fp4_precision_b200 import inputs
+    wl = inputs.workload(WORKLOAD, device="cpu", M=m_rows)
+    X, W, dY = wl["X"], wl["W"][:n_rows].contiguous(), wl["dY"][:, :n_rows].contiguous()
+    M, K = X.shape
+    N = W.shape[0]
+    r = O.preset(RECIPE)
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        O.linear_fwd(X, W, r, 1, 2)
+        O.linear_bwd(dY, X, W, r, 1, 2)
+    dt = (time.perf_counter() - t0) / steps
+    return dt, 6.0 * M * N * K, os.cpu_count()
+
+
+def cpu_baseline_obj(m_rows=128, n_rows=8192):
+    dt, flops, cores = oracle_sample(m_rows, n_rows)
+    return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": f"linear fwd+bwd of the first {m_rows} tokens x {n_rows} output features (full K = 4096) of "
+                      f"the MLP up/gate workload: six quantizations (fp32 decisions) + three fp64 GEMMs; {dt:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    m_rows, n_rows = 64, 2048
+    times = []
+    for _ in range(args.warmup):
+        oracle_sample(m_rows, n_rows)
+    for _ in range(args.steps):
+        dt, flops, cores = oracle_sample(m_rows, n_rows)
+        times.append(dt)
+    ms = statistics.mean(times) * 1e3
+    value = flops / (ms * 1e-3) / 1e12
+    return {"metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms, 2), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": "Llama-3.1-8B MLP up/gate linear fwd+bwd, X[16384x4096] W[28672x4096] "
+                                   "dY[16384x28672], NVFP4 Quartet II recipe", "recipe": RECIPE,
+                       "sample_tokens": m_rows, "sample_out_features": n_rows},
+            "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
+                             "sample": f"linear fwd+bwd of {m_rows} tokens x {n_rows} output features (full K) "
+                                       f"per step"},
+            "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.gpus != world and world == 1 and args.gpus > 1:
+        print(json.dumps({"error": "launch with torchrun for --gpus > 1"}))
+        return 2
+    if args.impl == "reference":
+        out = run_reference(args, rank, world)
+        if out is not None:
+            print(json.dumps(out))
+        return 0
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    out = run_ours(args, rank, world, local_rank)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline_obj()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out))
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,548 @@
+// qfp4_api.cu - the extern "C" entry points of include/qfp4.h: argument
+// validation, TMA descriptor encoding, launch of the quantizer and GEMM
+// kernels, and the linear layer's composition of six quantizations and three
+// GEMMs (page "New AMD paper overturns conventional wisdom: FP4 training...",
+// section "Poiskovaya eksperimental'naya rabota": Fprop Y = X W^T, Dgrad
+// dX = dY W, Wgrad dW = dY^T X).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstring>
+#include <mutex>
+
+#include "../../include/qfp4.h"
+#include "qfp4_internal.h"
+
+namespace qfp4 {
+namespace {
+
+thread_local int t_last_cuda_error = 0;
+thread_local int64_t t_launches = 0;
+
+int cuda_fail(cudaError_t e) {
+    t_last_cuda_error = (int)e;
+    return QFP4_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+int block_of(int fmt) { return fmt == kNvfp4 ? 16 : 32; }
+int had_n(int had) {
+    return (had == QFP4_HAD_DET16 || had == QFP4_HAD_RAND16)   ? 16
+           : (had == QFP4_HAD_DET32 || had == QFP4_HAD_RAND32) ? 32
+                                                               : 0;
+}
+bool had_random(int had) { return had == QFP4_HAD_RAND16 || had == QFP4_HAD_RAND32; }
+
+// ---- device check (sm_100), cached per device --------------------------------
+int check_device(int* sm_count) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    static std::mutex mu;
+    static int cached_ok[64] = {0};  // 0 unknown, 1 sm_100, -1 other
+    static int cached_sms[64] = {0};
+    if (dev < 0 || dev >= 64) return QFP4_ERR_UNSUPPORTED_ARCH;
+    std::lock_guard<std::mutex> lock(mu);
+    if (cached_ok[dev] == 0) {
+        int major = 0, minor = 0, sms = 0;
+        if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess)
+            return cuda_fail(e);
+        if ((e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess)
+            return cuda_fail(e);
+        if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+            return cuda_fail(e);
+        cached_ok[dev] = (major == 10 && minor == 0) ? 1 : -1;
+        cached_sms[dev] = sms;
+    }
+    if (sm_count) *sm_count = cached_sms[dev];
+    return cached_ok[dev] == 1 ? QFP4_OK : QFP4_ERR_UNSUPPORTED_ARCH;
+}
+
+// ---- TMA descriptors (driver entry point fetched through the runtime) --------
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 5-D view of a bf16 R x C tensor for the column quantizer: dimensions
+// (column, r % 2, r / G, (r / 2) % 4, (r / 8) % (G / 8)), box (64, 2, 4, 4,
+// G / 8), 128-byte swizzle. The box lands in shared memory with x-row r at
+// 128-byte row s = r%2 + 2 (r/G % 4) + 8 ((r/2) % 4) + 32 ((r/8) % (G/8)).
+int make_col_tmap(CUtensorMap* tm, const void* x, int64_t R, int64_t C, int64_t ld, int G) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return cuda_fail(cudaErrorNotSupported);
+    const cuuint64_t dims[5] = {(cuuint64_t)C, 2, (cuuint64_t)(R / G), 4, (cuuint64_t)(G / 8)};
+    const cuuint64_t strides[4] = {(cuuint64_t)ld * 2, (cuuint64_t)G * ld * 2, (cuuint64_t)2 * ld * 2,
+                                   (cuuint64_t)8 * ld * 2};
+    const cuuint32_t box[5] = {64, 2, 4, 4, (cuuint32_t)(G / 8)};
+    const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(x), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
+    return QFP4_OK;
+}
+
+// 2-D view of packed FP4 codes [rows][k/2] as bytes, box (128 bytes, box_rows),
+// 128-byte swizzle: the K-major operand layout of the MMA.
+int make_codes_tmap(CUtensorMap* tm, const void* codes, int64_t rows, int64_t k, int box_rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return cuda_fail(cudaErrorNotSupported);
+    const cuuint64_t dims[2] = {(cuuint64_t)(k / 2), (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)(k / 2)};
+    const cuuint32_t box[2] = {128, (cuuint32_t)box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(codes), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
+    return QFP4_OK;
+}
+
+int write_one(float* dst, cudaStream_t s) {
+    static const float one = 1.0f;
+    cudaError_t e = cudaMemcpyAsync(dst, &one, sizeof(float), cudaMemcpyHostToDevice, s);
+    return e == cudaSuccess ? QFP4_OK : cuda_fail(e);
+}
+
+int amax_partial_count(int sms, int64_t tiles) {
+    int64_t n = 4 * (int64_t)sms;
+    if (n > tiles) n = tiles;
+    if (n > kMaxAmaxPartials) n = kMaxAmaxPartials;
+    return n < 1 ? 1 : (int)n;
+}
+
+// Philox4x32-10 word 0 of counter (0, 0, kTagSign | stream << 4, 0): the 32
+// random Hadamard sign bits of a call (the kernels receive them as an argument).
+uint32_t host_sign_bits(uint64_t seed, uint32_t stream) {
+    uint32_t c0 = 0, c1 = 0, c2 = (uint32_t)kTagSign | (stream << 4), c3 = 0;
+    uint32_t k0 = (uint32_t)seed, k1 = (uint32_t)(seed >> 32);
+    for (int r = 0; r < 10; ++r) {
+        if (r) {
+            k0 += 0x9E3779B9u;
+            k1 += 0xBB67AE85u;
+        }
+        const uint64_t p0 = (uint64_t)0xD2511F53u * c0;
+        const uint64_t p1 = (uint64_t)0xCD9E8D57u * c2;
+        const uint32_t n0 = (uint32_t)(p1 >> 32) ^ c1 ^ k0, n1 = (uint32_t)p1;
+        const uint32_t n2 = (uint32_t)(p0 >> 32) ^ c3 ^ k1, n3 = (uint32_t)p0;
+        c0 = n0; c1 = n1; c2 = n2; c3 = n3;
+    }
+    return c0;
+}
+
+struct Geometry {
+    int64_t rows, k;
+};
+
+int validate_input(const void* x, int64_t R, int64_t C, int64_t ld, int32_t had, int32_t axis, Geometry* g) {
+    if (R < 0 || C < 0 || R > 0x7fffffffLL || C > 0x7fffffffLL) return QFP4_ERR_INVALID_ARG;
+    if (axis != QFP4_AXIS_ROW && axis != QFP4_AXIS_COL) return QFP4_ERR_INVALID_ARG;
+    if (had < QFP4_HAD_NONE || had > QFP4_HAD_RAND32) return QFP4_ERR_INVALID_ARG;
+    if (ld < C) return QFP4_ERR_INVALID_ARG;
+    if (R > 0 && C > 0) {
+        if (x == nullptr) return QFP4_ERR_INVALID_ARG;
+        if (!aligned16(x) || (ld % 8) != 0) return QFP4_ERR_MISALIGNED;
+    }
+    g->rows = axis == QFP4_AXIS_ROW ? R : C;
+    g->k = axis == QFP4_AXIS_ROW ? C : R;
+    const int nh = had_n(had);
+    if (nh && g->k % nh != 0) return QFP4_ERR_INVALID_ARG;
+    return QFP4_OK;
+}
+
+// Amax pass into `partials` (their count returned in *n_partials).
+int run_amax(const void* x, int64_t R, int64_t C, int64_t ld, int32_t had, int32_t axis, uint32_t signs,
+             const Geometry& g, float* partials, int* n_partials, int sms, cudaStream_t s) {
+    QuantParams p{};
+    p.x = static_cast<const uint16_t*>(x);
+    p.R = R; p.C = C; p.ld = ld;
+    p.rows = g.rows; p.k = g.k;
+    p.signs = signs;
+    p.amax_out = partials;
+    const int nh = had_n(had);
+    CUtensorMap tm;
+    std::memset(&tm, 0, sizeof tm);
+    int64_t tiles;
+    if (axis == QFP4_AXIS_ROW) {
+        tiles = ((g.rows + 127) / 128) * ((g.k + 127) / 128);
+    } else {
+        const int G = col_group(16, nh);
+        int rc = make_col_tmap(&tm, x, R, C, ld, G);
+        if (rc) return rc;
+        tiles = ((g.rows + 127) / 128) * ((g.k + 4 * G - 1) / (4 * G));
+    }
+    *n_partials = amax_partial_count(sms, tiles);
+    cudaError_t e = launch_amax(p, axis, nh, &tm, *n_partials, s);
+    return e == cudaSuccess ? QFP4_OK : cuda_fail(e);
+}
+
+int quantize_impl(const void* x, int64_t R, int64_t C, int64_t ld, int32_t fmt, int32_t rounding, int32_t had,
+                  int32_t axis, const qfp4_seed* seed, const float* amax_in, qfp4_tensor* out, void* workspace,
+                  size_t workspace_bytes, cudaStream_t s) {
+    int sms = 0;
+    int rc = check_device(&sms);
+    if (rc) return rc;
+    if (fmt != QFP4_NVFP4 && fmt != QFP4_MXFP4) return QFP4_ERR_INVALID_ARG;
+    if (rounding < QFP4_RTN || rounding > QFP4_QUARTET2) return QFP4_ERR_INVALID_ARG;
+    if (out == nullptr || seed == nullptr) return QFP4_ERR_INVALID_ARG;
+    if (seed->rot_stream >= (1u << 28) || seed->sr_stream >= (1u << 28)) return QFP4_ERR_INVALID_ARG;
+    Geometry g;
+    if ((rc = validate_input(x, R, C, ld, had, axis, &g))) return rc;
+    const int NB = block_of(fmt);
+    if (g.k % NB != 0) return QFP4_ERR_INVALID_ARG;
+    if (out->tensor_scale == nullptr) return QFP4_ERR_INVALID_ARG;
+    const bool nonempty = g.rows > 0 && g.k > 0;
+    if (nonempty) {
+        if (out->codes == nullptr || out->scales == nullptr) return QFP4_ERR_INVALID_ARG;
+        if (!aligned16(out->codes) || !aligned16(out->scales)) return QFP4_ERR_MISALIGNED;
+    }
+    const bool need_ws = nonempty && fmt == QFP4_NVFP4 && amax_in == nullptr;
+    if (need_ws) {
+        if (workspace == nullptr || workspace_bytes < qfp4_quantize_workspace_bytes()) return QFP4_ERR_WORKSPACE;
+        if (!aligned16(workspace)) return QFP4_ERR_MISALIGNED;
+    }
+    out->rows = g.rows;
+    out->k = g.k;
+    out->fmt = fmt;
+    out->had = had;
+    out->rot_seed = had_random(had) ? seed->rot : 0;
+    out->rot_stream = had_random(had) ? seed->rot_stream : 0;
+    out->reserved = 0;
+    if (!nonempty) return write_one(out->tensor_scale, s);
+
+    const uint32_t signs = had_random(had) ? host_sign_bits(seed->rot, seed->rot_stream) : 0u;
+    const int nh = had_n(had);
+    QuantParams p{};
+    p.x = static_cast<const uint16_t*>(x);
+    p.R = R; p.C = C; p.ld = ld;
+    p.rows = g.rows; p.k = g.k;
+    p.codes = out->codes;
+    p.scales = out->scales;
+    p.tensor_scale = out->tensor_scale;
+    p.kb4 = (g.k / NB + 3) / 4 * 4;
+    p.signs = signs;
+    p.sr_seed = seed->sr;
+    p.sr_tag_elem = (uint32_t)kTagElement | (seed->sr_stream << 4);
+    p.sr_tag_scale = (uint32_t)kTagScale | (seed->sr_stream << 4);
+    p.amax_in = amax_in;
+    if (need_ws) {
+        int n = 0;
+        float* partials = static_cast<float*>(workspace);
+        if ((rc = run_amax(x, R, C, ld, had, axis, signs, g, partials, &n, sms, s))) return rc;
+        p.amax_partials = partials;
+        p.n_partials = n;
+    }
+    CUtensorMap tm;
+    std::memset(&tm, 0, sizeof tm);
+    if (axis == QFP4_AXIS_COL) {
+        if ((rc = make_col_tmap(&tm, x, R, C, ld, col_group(NB, nh)))) return rc;
+    }
+    cudaError_t e = launch_quant(p, fmt, rounding, nh, axis, &tm, s);
+    return e == cudaSuccess ? QFP4_OK : cuda_fail(e);
+}
+
+int gemm_impl(const qfp4_tensor* A, const qfp4_tensor* B, void* D, int64_t ldd, int32_t out_dtype, cudaStream_t s) {
+    int rc = check_device(nullptr);
+    if (rc) return rc;
+    if (A == nullptr || B == nullptr) return QFP4_ERR_INVALID_ARG;
+    if (out_dtype != QFP4_OUT_BF16 && out_dtype != QFP4_OUT_F32) return QFP4_ERR_INVALID_ARG;
+    if (A->fmt != B->fmt || (A->fmt != QFP4_NVFP4 && A->fmt != QFP4_MXFP4)) return QFP4_ERR_INVALID_ARG;
+    if (A->k != B->k || A->k < 0 || A->rows < 0 || B->rows < 0) return QFP4_ERR_INVALID_ARG;
+    if (A->had != B->had) return QFP4_ERR_INVALID_ARG;
+    if (had_random(A->had) && (A->rot_seed != B->rot_seed || A->rot_stream != B->rot_stream))
+        return QFP4_ERR_INVALID_ARG;
+    if (A->k % 64 != 0) return QFP4_ERR_INVALID_ARG;
+    if (A->rows > 0x7fffffffLL || B->rows > 0x7fffffffLL || A->k > 0x7fffffffLL) return QFP4_ERR_INVALID_ARG;
+    const int64_t M = A->rows, N = B->rows, K = A->k;
+    if (M == 0 || N == 0) return QFP4_OK;
+    const size_t esz = out_dtype == QFP4_OUT_F32 ? 4 : 2;
+    if (D == nullptr || ldd < N) return QFP4_ERR_INVALID_ARG;
+    if (!aligned16(D) || (ldd * (int64_t)esz) % 16 != 0) return QFP4_ERR_MISALIGNED;
+    if (K == 0) {
+        cudaError_t e = cudaMemset2DAsync(D, (size_t)ldd * esz, 0, (size_t)N * esz, (size_t)M, s);
+        return e == cudaSuccess ? QFP4_OK : cuda_fail(e);
+    }
+    if (!A->codes || !B->codes || !A->scales || !B->scales || !A->tensor_scale || !B->tensor_scale)
+        return QFP4_ERR_INVALID_ARG;
+    if (!aligned16(A->codes) || !aligned16(B->codes) || !aligned16(A->scales) || !aligned16(B->scales))
+        return QFP4_ERR_MISALIGNED;
+    CUtensorMap tA, tB;
+    if ((rc = make_codes_tmap(&tA, A->codes, M, K, kGemmBM))) return rc;
+    if ((rc = make_codes_tmap(&tB, B->codes, N, K, kGemmBN))) return rc;
+    GemmParams p{};
+    p.sfa = A->scales;
+    p.sfb = B->scales;
+    p.ga = A->tensor_scale;
+    p.gb = B->tensor_scale;
+    p.D = D;
+    p.ldd = ldd;
+    p.out_f32 = out_dtype == QFP4_OUT_F32;
+    p.M = (int)M; p.N = (int)N; p.K = (int)K;
+    const int NB = block_of(A->fmt);
+    p.atoms_k = (int)((K / NB + 3) / 4);
+    cudaError_t e = launch_gemm(p, A->fmt, &tA, &tB, s);
+    return e == cudaSuccess ? QFP4_OK : cuda_fail(e);
+}
+
+// ---- linear layer -------------------------------------------------------------
+size_t round_up(size_t v) { return (v + 255) / 256 * 256; }
+
+struct Carver {
+    uint8_t* base;
+    size_t off;
+    void* take(size_t bytes) {
+        void* p = base ? base + off : nullptr;
+        off += round_up(bytes);
+        return p;
+    }
+};
+
+// Carve one quantized operand (rows x k) out of the workspace.
+void carve_operand(Carver& c, qfp4_tensor* t, int fmt, int64_t rows, int64_t k) {
+    std::memset(t, 0, sizeof *t);
+    t->codes = static_cast<uint8_t*>(c.take(qfp4_codes_bytes(rows, k)));
+    t->scales = static_cast<uint8_t*>(c.take(qfp4_scales_bytes(fmt, rows, k)));
+    t->tensor_scale = static_cast<float*>(c.take(sizeof(float)));
+}
+
+bool valid_cfg(const qfp4_gemm_cfg& g) {
+    return (g.fmt == QFP4_NVFP4 || g.fmt == QFP4_MXFP4) && g.rnd_a >= QFP4_RTN && g.rnd_a <= QFP4_QUARTET2 &&
+           g.rnd_b >= QFP4_RTN && g.rnd_b <= QFP4_QUARTET2 && g.had >= QFP4_HAD_NONE && g.had <= QFP4_HAD_RAND32;
+}
+bool valid_dtype(int32_t d) { return d == QFP4_OUT_BF16 || d == QFP4_OUT_F32; }
+
+int linear_layout(int backward, int64_t M, int64_t N, int64_t K, const qfp4_recipe* r, uint8_t* ws, qfp4_tensor* t,
+                  float** partials, size_t* total) {
+    Carver c{ws, 0};
+    *partials = static_cast<float*>(c.take(qfp4_quantize_workspace_bytes()));
+    if (!backward) {
+        carve_operand(c, &t[0], r->fprop.fmt, M, K);  // X along K
+        carve_operand(c, &t[1], r->fprop.fmt, N, K);  // W along K
+    } else {
+        carve_operand(c, &t[0], r->dgrad.fmt, M, N);  // dY along N
+        carve_operand(c, &t[1], r->dgrad.fmt, K, N);  // W^T: W along N
+        carve_operand(c, &t[2], r->wgrad.fmt, N, M);  // dY^T: dY along M
+        carve_operand(c, &t[3], r->wgrad.fmt, K, M);  // X^T: X along M
+    }
+    *total = c.off;
+    return QFP4_OK;
+}
+
+int check_linear_args(int64_t M, int64_t N, int64_t K, const qfp4_recipe* r, const qfp4_seed* seed) {
+    if (r == nullptr || seed == nullptr) return QFP4_ERR_INVALID_ARG;
+    if (M <= 0 || N <= 0 || K <= 0 || (M % 128) || (N % 128) || (K % 128)) return QFP4_ERR_INVALID_ARG;
+    if (!valid_cfg(r->fprop) || !valid_cfg(r->dgrad) || !valid_cfg(r->wgrad)) return QFP4_ERR_INVALID_ARG;
+    if (!valid_dtype(r->y_dtype) || !valid_dtype(r->dx_dtype) || !valid_dtype(r->dw_dtype)) return QFP4_ERR_INVALID_ARG;
+    return QFP4_OK;
+}
+
+qfp4_seed op_seed(const qfp4_seed* s, uint32_t gemm, uint32_t operand) {
+    qfp4_seed o;
+    o.rot = s->rot;
+    o.sr = s->sr;
+    o.rot_stream = gemm;
+    o.sr_stream = operand;
+    return o;
+}
+
+}  // namespace
+
+void count_launch() { ++t_launches; }
+
+}  // namespace qfp4
+
+using namespace qfp4;
+
+extern "C" {
+
+const char* qfp4_strerror(int status) {
+    switch (status) {
+        case QFP4_OK: return "ok";
+        case QFP4_ERR_INVALID_ARG: return "invalid argument";
+        case QFP4_ERR_MISALIGNED: return "misaligned pointer or row stride";
+        case QFP4_ERR_UNSUPPORTED_ARCH: return "device is not sm_100 (B200)";
+        case QFP4_ERR_WORKSPACE: return "workspace missing or too small";
+        case QFP4_ERR_CUDA: return "CUDA error";
+        case QFP4_ERR_TIMEOUT: return "device-side bounded wait expired";
+        default: return "unknown status";
+    }
+}
+
+int qfp4_last_cuda_error(void) { return t_last_cuda_error; }
+
+int64_t qfp4_launch_count(int32_t reset) {
+    const int64_t n = t_launches;
+    if (reset) t_launches = 0;
+    return n;
+}
+
+size_t qfp4_codes_bytes(int64_t rows, int64_t k) { return (rows <= 0 || k <= 0) ? 0 : (size_t)(rows * k / 2); }
+
+size_t qfp4_scales_bytes(int32_t fmt, int64_t rows, int64_t k) {
+    if ((fmt != QFP4_NVFP4 && fmt != QFP4_MXFP4) || rows <= 0 || k <= 0) return 0;
+    const int64_t kb = (k + block_of(fmt) - 1) / block_of(fmt);
+    return (size_t)(((rows + 127) / 128) * ((kb + 3) / 4) * 512);
+}
+
+int64_t qfp4_scale_offset(int32_t fmt, int64_t rows, int64_t k, int64_t r, int64_t c) {
+    if ((fmt != QFP4_NVFP4 && fmt != QFP4_MXFP4) || rows <= 0 || k <= 0) return -1;
+    const int64_t kb = (k + block_of(fmt) - 1) / block_of(fmt);
+    const int64_t rows_p = (rows + 127) / 128 * 128, kb4 = (kb + 3) / 4 * 4;
+    if (r < 0 || c < 0 || r >= rows_p || c >= kb4) return -1;
+    return ((r / 128) * (kb4 / 4) + c / 4) * 512 + (r % 32) * 16 + ((r / 32) % 4) * 4 + (c % 4);
+}
+
+size_t qfp4_quantize_workspace_bytes(void) { return (size_t)kMaxAmaxPartials * sizeof(float); }
+
+int qfp4_amax(const void* x, int64_t R, int64_t C, int64_t ld, int32_t had, int32_t axis, const qfp4_seed* seed,
+              float* amax, void* workspace, size_t workspace_bytes, void* stream) {
+    int sms = 0;
+    int rc = check_device(&sms);
+    if (rc) return rc;
+    Geometry g;
+    if ((rc = validate_input(x, R, C, ld, had, axis, &g))) return rc;
+    if (amax == nullptr || (had_random(had) && seed == nullptr)) return QFP4_ERR_INVALID_ARG;
+    if (workspace == nullptr || workspace_bytes < qfp4_quantize_workspace_bytes()) return QFP4_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return QFP4_ERR_MISALIGNED;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (g.rows == 0 || g.k == 0) {
+        cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(float), s);
+        return e == cudaSuccess ? QFP4_OK : cuda_fail(e);
+    }
+    const uint32_t signs = had_random(had) ? host_sign_bits(seed->rot, seed->rot_stream) : 0u;
+    int n = 0;
+    float* partials = static_cast<float*>(workspace);
+    if ((rc = run_amax(x, R, C, ld, had, axis, signs, g, partials, &n, sms, s))) return rc;
+    cudaError_t e = launch_reduce_max(partials, n, amax, s);
+    return e == cudaSuccess ? QFP4_OK : cuda_fail(e);
+}
+
+int qfp4_quantize(const void* x, int64_t R, int64_t C, int64_t ld, int32_t fmt, int32_t rounding, int32_t had,
+                  int32_t axis, const qfp4_seed* seed, const float* amax_in, qfp4_tensor* out, void* workspace,
+                  size_t workspace_bytes, void* stream) {
+    return quantize_impl(x, R, C, ld, fmt, rounding, had, axis, seed, amax_in, out, workspace, workspace_bytes,
+                         static_cast<cudaStream_t>(stream));
+}
+
+int qfp4_gemm(const qfp4_tensor* A, const qfp4_tensor* B, void* D, int64_t ldd, int32_t out_dtype, void* stream) {
+    return gemm_impl(A, B, D, ldd, out_dtype, static_cast<cudaStream_t>(stream));
+}
+
+int qfp4_recipe_preset(int32_t preset, qfp4_recipe* out) {
+    if (out == nullptr) return QFP4_ERR_INVALID_ARG;
+    std::memset(out, 0, sizeof *out);
+    out->y_dtype = QFP4_OUT_BF16;
+    out->dx_dtype = QFP4_OUT_BF16;
+    out->dw_dtype = QFP4_OUT_F32;
+    switch (preset) {
+        case QFP4_PRESET_NVIDIA_NVFP4:  // 16x16 random Hadamard on Wgrad inputs, SR of the gradient
+            out->fprop = {QFP4_NVFP4, QFP4_RTN, QFP4_RTN, QFP4_HAD_NONE};
+            out->dgrad = {QFP4_NVFP4, QFP4_SR, QFP4_RTN, QFP4_HAD_NONE};
+            out->wgrad = {QFP4_NVFP4, QFP4_SR, QFP4_RTN, QFP4_HAD_RAND16};
+            return QFP4_OK;
+        case QFP4_PRESET_QUARTET2_NVFP4:  // RTN forward; random rotation + Quartet II scale SR backward
+            out->fprop = {QFP4_NVFP4, QFP4_RTN, QFP4_RTN, QFP4_HAD_DET16};
+            out->dgrad = {QFP4_NVFP4, QFP4_QUARTET2, QFP4_QUARTET2, QFP4_HAD_RAND16};
+            out->wgrad = {QFP4_NVFP4, QFP4_QUARTET2, QFP4_QUARTET2, QFP4_HAD_RAND16};
+            return QFP4_OK;
+        case QFP4_PRESET_AMD_MXFP4_H:  // MXFP4 everywhere, deterministic Hadamard on Wgrad
+            out->fprop = {QFP4_MXFP4, QFP4_RTN, QFP4_RTN, QFP4_HAD_NONE};
+            out->dgrad = {QFP4_MXFP4, QFP4_RTN, QFP4_RTN, QFP4_HAD_NONE};
+            out->wgrad = {QFP4_MXFP4, QFP4_RTN, QFP4_RTN, QFP4_HAD_DET32};
+            return QFP4_OK;
+        default: return QFP4_ERR_INVALID_ARG;
+    }
+}
+
+size_t qfp4_linear_workspace_bytes(int32_t backward, int64_t M, int64_t N, int64_t K, const qfp4_recipe* recipe) {
+    if (recipe == nullptr || M < 0 || N < 0 || K < 0) return 0;
+    qfp4_tensor t[4];
+    float* partials;
+    size_t total = 0;
+    linear_layout(backward, M, N, K, recipe, nullptr, t, &partials, &total);
+    return total;
+}
+
+int qfp4_linear_fwd(const void* X, const void* W, void* Y, int64_t M, int64_t N, int64_t K, const qfp4_recipe* recipe,
+                    const qfp4_seed* seed, void* workspace, size_t workspace_bytes, void* stream) {
+    int rc = check_linear_args(M, N, K, recipe, seed);
+    if (rc) return rc;
+    if (!X || !W || !Y) return QFP4_ERR_INVALID_ARG;
+    if (workspace == nullptr || workspace_bytes < qfp4_linear_workspace_bytes(0, M, N, K, recipe))
+        return QFP4_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return QFP4_ERR_MISALIGNED;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    qfp4_tensor t[4];
+    float* partials;
+    size_t total;
+    linear_layout(0, M, N, K, recipe, static_cast<uint8_t*>(workspace), t, &partials, &total);
+    const qfp4_gemm_cfg& c = recipe->fprop;
+    const size_t pws = qfp4_quantize_workspace_bytes();
+    qfp4_seed sx = op_seed(seed, 0, 0), sw = op_seed(seed, 0, 1);
+    if ((rc = quantize_impl(X, M, K, K, c.fmt, c.rnd_a, c.had, QFP4_AXIS_ROW, &sx, nullptr, &t[0], partials, pws, s)))
+        return rc;
+    if ((rc = quantize_impl(W, N, K, K, c.fmt, c.rnd_b, c.had, QFP4_AXIS_ROW, &sw, nullptr, &t[1], partials, pws, s)))
+        return rc;
+    return gemm_impl(&t[0], &t[1], Y, N, recipe->y_dtype, s);
+}
+
+int qfp4_linear_bwd(const void* dY, const void* X, const void* W, void* dX, void* dW, int64_t M, int64_t N, int64_t K,
+                    const qfp4_recipe* recipe, const qfp4_seed* seed, void* workspace, size_t workspace_bytes,
+                    void* stream) {
+    int rc = check_linear_args(M, N, K, recipe, seed);
+    if (rc) return rc;
+    if (!dY || !X || !W || !dX || !dW) return QFP4_ERR_INVALID_ARG;
+    if (workspace == nullptr || workspace_bytes < qfp4_linear_workspace_bytes(1, M, N, K, recipe))
+        return QFP4_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return QFP4_ERR_MISALIGNED;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    qfp4_tensor t[4];
+    float* partials;
+    size_t total;
+    linear_layout(1, M, N, K, recipe, static_cast<uint8_t*>(workspace), t, &partials, &total);
+    const size_t pws = qfp4_quantize_workspace_bytes();
+    const qfp4_gemm_cfg& d = recipe->dgrad;
+    const qfp4_gemm_cfg& w = recipe->wgrad;
+    // Dgrad dX[M,K] = dY[M,N] . W[N,K]: reduce over N.
+    qfp4_seed s0 = op_seed(seed, 1, 2), s1 = op_seed(seed, 1, 3);
+    if ((rc = quantize_impl(dY, M, N, N, d.fmt, d.rnd_a, d.had, QFP4_AXIS_ROW, &s0, nullptr, &t[0], partials, pws, s)))
+        return rc;
+    if ((rc = quantize_impl(W, N, K, K, d.fmt, d.rnd_b, d.had, QFP4_AXIS_COL, &s1, nullptr, &t[1], partials, pws, s)))
+        return rc;
+    if ((rc = gemm_impl(&t[0], &t[1], dX, K, recipe->dx_dtype, s))) return rc;
+    // Wgrad dW[N,K] = dY^T[N,M] . X[M,K]: reduce over M (tokens).
+    qfp4_seed s2 = op_seed(seed, 2, 4), s3 = op_seed(seed, 2, 5);
+    if ((rc = quantize_impl(dY, M, N, N, w.fmt, w.rnd_a, w.had, QFP4_AXIS_COL, &s2, nullptr, &t[2], partials, pws, s)))
+        return rc;
+    if ((rc = quantize_impl(X, M, K, K, w.fmt, w.rnd_b, w.had, QFP4_AXIS_COL, &s3, nullptr, &t[3], partials, pws, s)))
+        return rc;
+    return gemm_impl(&t[2], &t[3], dW, K, recipe->dw_dtype, s);
+}
+
+int qfp4_status(void* stream) {
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e);
+    uint32_t v = 0;
+    if ((e = cudaMemcpyFromSymbol(&v, g_dev_error, sizeof v)) != cudaSuccess) return cuda_fail(e);
+    if (v != 0) {
+        const uint32_t zero = 0;
+        if ((e = cudaMemcpyToSymbol(g_dev_error, &zero, sizeof zero)) != cudaSuccess) return cuda_fail(e);
+        return QFP4_ERR_TIMEOUT;
+    }
+    return QFP4_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,260 @@
+// qfp4_device.cuh - device helpers shared by the sm_100a kernels of this library:
+// Philox4x32-10, bf16 unpacking, FP4/FP8 conversions, the library's device
+// error word, and thin inline-PTX wrappers for mbarrier, TMA and tcgen05.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+namespace qfp4 {
+
+// ---------------------------------------------------------------------------
+// error word: set by a kernel whose bounded wait expired; read by qfp4_status()
+enum : uint32_t { DEV_ERR_NONE = 0, DEV_ERR_TIMEOUT = 1 };
+// (the library is one translation unit, see qfp4_lib.cu, so this is its only definition)
+__device__ uint32_t g_dev_error = 0;
+
+__device__ __forceinline__ void raise_device_error(uint32_t code) { atomicOr(&g_dev_error, code); }
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+
+// A bounded wait gives up after this many nanoseconds (kernels here run for
+// microseconds to milliseconds; a legitimate wait is far shorter).
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+// ---------------------------------------------------------------------------
+// Philox4x32-10 (Salmon, Moraes, Dror, Shaw, SC'11): key = 64-bit seed,
+// counter = (i/4 lo, i/4 hi, tag | stream << 4, 0).
+__device__ __forceinline__ uint4 philox4x32_10(uint4 ctr, uint32_t key_lo, uint32_t key_hi) {
+#pragma unroll
+    for (int round = 0; round < 10; ++round) {
+        if (round != 0) {
+            key_lo += 0x9E3779B9u;
+            key_hi += 0xBB67AE85u;
+        }
+        const uint32_t m0_lo = 0xD2511F53u * ctr.x;
+        const uint32_t m0_hi = __umulhi(0xD2511F53u, ctr.x);
+        const uint32_t m1_lo = 0xCD9E8D57u * ctr.z;
+        const uint32_t m1_hi = __umulhi(0xCD9E8D57u, ctr.z);
+        ctr = make_uint4(m1_hi ^ ctr.y ^ key_lo, m1_lo, m0_hi ^ ctr.w ^ key_hi, m0_lo);
+    }
+    return ctr;
+}
+
+// Four consecutive words of stream (tag, stream) starting at item 4*quad.
+__device__ __forceinline__ uint4 philox_quad(uint64_t seed, uint32_t tag_stream, uint64_t quad) {
+    return philox4x32_10(make_uint4((uint32_t)quad, (uint32_t)(quad >> 32), tag_stream, 0u), (uint32_t)seed,
+                         (uint32_t)(seed >> 32));
+}
+
+// Uniform in [0, 1) on the 2^-24 grid.
+__device__ __forceinline__ float uniform24(uint32_t w) { return __uint2float_rn(w >> 8) * 0x1p-24f; }
+
+// ---------------------------------------------------------------------------
+// bf16 pairs -> fp32 (exact)
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// ---------------------------------------------------------------------------
+// E2M1: two fp32 -> one byte, `lo` in the low nibble (round-to-nearest-even,
+// saturating to +-6). Four pairs -> one 32-bit word, element 0 lowest.
+__device__ __forceinline__ uint32_t e2m1x8_rn(const float* v) {
+    uint32_t out;
+    asm("{\n\t"
+        ".reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t"
+        "}"
+        : "=r"(out)
+        : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
+    // a zero magnitude keeps code 0 whatever the sign (no -0 codes)
+    const uint32_t mag = out & 0x77777777u;
+    const uint32_t nonzero = (mag + 0x77777777u) & 0x88888888u;
+    return mag | (out & nonzero);
+}
+
+// E2M1 magnitude grid step for |u| < 6: 0.5 below 2, 1 below 4, 2 above.
+__device__ __forceinline__ float e2m1_step(float a) { return a < 2.0f ? 0.5f : (a < 4.0f ? 1.0f : 2.0f); }
+
+// Stochastic rounding of u onto the E2M1 grid with uniform rho: the lower grid
+// neighbour lo, gap `step`, round up iff rho < (|u| - lo) / step; |u| >= 6 -> 6.
+// Returns the exactly representable rounded value (sign kept).
+__device__ __forceinline__ float e2m1_sr_value(float u, float rho) {
+    const float a = fabsf(u);
+    float m;
+    if (a >= 6.0f) {
+        m = 6.0f;
+    } else {
+        const float step = e2m1_step(a);
+        const float t = a / step;          // exact: power-of-two divisor
+        const float fl = floorf(t);
+        const float p = t - fl;            // exact: fraction of an exactly scaled value
+        m = (fl + (rho < p ? 1.0f : 0.0f)) * step;
+    }
+    return copysignf(m, u);
+}
+
+// E2M1 code value (signed) of a 4-bit code.
+__device__ __forceinline__ float e2m1_decode(uint32_t code) {
+    const uint32_t idx = code & 7u;
+    float m = (idx < 4u) ? 0.5f * (float)idx : (idx == 4u ? 2.0f : (idx == 5u ? 3.0f : (idx == 6u ? 4.0f : 6.0f)));
+    return (code & 8u) ? -m : m;
+}
+
+// ---------------------------------------------------------------------------
+// E4M3 (OCP FN): fp32 -> code, round-to-nearest-even, saturating at 448.
+__device__ __forceinline__ uint32_t e4m3_rn(float t) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(t));
+    return r & 0xFFu;
+}
+
+// E4M3 code -> fp32 (exact, through f16).
+__device__ __forceinline__ float e4m3_decode(uint32_t code) {
+    uint32_t h2;
+    const uint16_t c = (uint16_t)code;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(c));
+    return __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
+}
+
+// Stochastic rounding of t >= 0 onto the E4M3 grid (saturating at 448).
+__device__ __forceinline__ uint32_t e4m3_sr(float t, float rho) {
+    if (!(t < 448.0f)) return 0x7Eu;
+    uint32_t c = e4m3_rn(t);
+    if (e4m3_decode(c) > t) c -= 1u;  // c = largest code with value <= t
+    const float lo = e4m3_decode(c);
+    const float hi = e4m3_decode(c + 1u);
+    const float p = (t - lo) / (hi - lo);
+    return rho < p ? c + 1u : c;
+}
+
+// floor(log2(a)) of a positive finite fp32, exact (subnormals included).
+__device__ __forceinline__ int floor_log2(float a) {
+    const uint32_t b = __float_as_uint(a);
+    const int e = (int)((b >> 23) & 0xFFu);
+    if (e != 0) return e - 127;
+    return (31 - __clz((int)(b & 0x7FFFFFu))) - 149;
+}
+
+// 2^e as fp32 for e in [-149, 127] (exact).
+__device__ __forceinline__ float exp2i(int e) {
+    if (e >= -126) return __uint_as_float((uint32_t)(e + 127) << 23);
+    return __uint_as_float(1u << (e + 149));
+}
+
+// Stochastic rounding of t > 0 onto powers of two; returns the E8M0 code.
+__device__ __forceinline__ uint32_t e8m0_sr(float t, float rho) {
+    int e = floor_log2(t);
+    const float lo = exp2i(e);
+    const float p = (t - lo) / lo;
+    if (rho < p) e += 1;
+    e = e < -127 ? -127 : (e > 127 ? 127 : e);
+    return (uint32_t)(e + 127);
+}
+
+// ---------------------------------------------------------------------------
+// shared-memory / barrier / TMA / tcgen05 wrappers
+__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+__device__ __forceinline__ void fence_mbarrier_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_shared() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Wait for the phase with the given parity to complete; false (and the
+// device error word set) when the wait exceeded kWaitLimitNs.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        for (int i = 0; i < 256; ++i)
+            if (mbar_try_wait(bar, parity)) return true;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            raise_device_error(DEV_ERR_TIMEOUT);
+            return false;
+        }
+    }
+}
+
+// 2D/5D tiled TMA load into shared memory, completing on an mbarrier.
+__device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, uint64_t* bar, int32_t x, int32_t y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
+            smem_u32(dst)),
+        "l"(tmap), "r"(smem_u32(bar)), "r"(x), "r"(y)
+        : "memory");
+}
+__device__ __forceinline__ void tma_load_5d(void* dst, const void* tmap, uint64_t* bar, int32_t c0, int32_t c1, int32_t c2,
+                                            int32_t c3, int32_t c4) {
+    asm volatile(
+        "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, %6, "
+        "%7}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(tmap), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4)
+        : "memory");
+}
+// Untiled bulk copy global -> shared (16-byte aligned addresses, size a multiple of 16).
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_u32(dst)),
+                 "l"(src), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+__device__ __forceinline__ void prefetch_tmap(const void* tmap) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");
+}
+
+// tcgen05 (5th-generation tensor core) wrappers
+__device__ __forceinline__ void tmem_alloc(uint32_t* slot_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(slot_smem)),
+                 "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+// Copy a 32-row x 128-bit shared-memory matrix (512 contiguous bytes) to TMEM
+// lanes 0-31 at 4 columns, replicated into the four 32-lane sub-partitions.
+__device__ __forceinline__ void tc_cp_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+__device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+}  // namespace qfp4

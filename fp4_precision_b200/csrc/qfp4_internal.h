@@ -1,0 +1,65 @@
+// qfp4_internal.h - declarations shared by the library's translation units
+// (not part of the public ABI; include/qfp4.h is).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+namespace qfp4 {
+
+constexpr int kNvfp4 = 0, kMxfp4 = 1;
+constexpr int kRtn = 0, kSr = 1, kQuartet2 = 2;
+constexpr int kTagElement = 0, kTagScale = 1, kTagSign = 2;
+
+// Upper bound on the number of per-CTA amax partials (the workspace holds them).
+constexpr int kMaxAmaxPartials = 1024;
+
+struct QuantParams {
+    const uint16_t* x;  // bf16 input, R x C, row stride ld
+    int64_t R, C, ld;
+    int64_t rows, k;  // quantized orientation
+    uint8_t* codes;
+    uint8_t* scales;
+    float* tensor_scale;
+    int64_t kb4;                  // scale columns padded to a multiple of 4
+    const float* amax_partials;   // NVFP4: partial maxima from the amax pass
+    int n_partials;
+    const float* amax_in;         // NVFP4: caller-provided amax (overrides partials)
+    float* amax_out;              // amax pass: partial maxima written here
+    uint32_t signs;               // random Hadamard sign bits (0 for deterministic / none)
+    uint64_t sr_seed;
+    uint32_t sr_tag_elem;         // kTagElement | stream << 4
+    uint32_t sr_tag_scale;        // kTagScale | stream << 4
+};
+
+// Launchers (quant.cu). Return cudaSuccess or the launch error.
+cudaError_t launch_amax(const QuantParams& p, int axis, int nh, const CUtensorMap* tmap_col, int n_partials,
+                        cudaStream_t s);
+cudaError_t launch_quant(const QuantParams& p, int fmt, int rnd, int nh, int axis, const CUtensorMap* tmap_col,
+                         cudaStream_t s);
+cudaError_t launch_reduce_max(const float* in, int n, float* out, cudaStream_t s);
+// Column-mode geometry: group G = max(block, n_h), tile = 4G rows x 128 columns.
+int col_group(int fmt_or_amax_block, int nh);
+
+struct GemmParams {
+    const uint8_t* sfa;
+    const uint8_t* sfb;
+    const float* ga;
+    const float* gb;
+    void* D;
+    int64_t ldd;
+    int out_f32;
+    int M, N, K;
+    int atoms_k;  // scale atoms per 128-row block along k: ceil(K / block / 4)
+};
+
+// gemm_sm100.cu
+cudaError_t launch_gemm(const GemmParams& p, int fmt, const CUtensorMap* tmapA, const CUtensorMap* tmapB,
+                        cudaStream_t s);
+constexpr int kGemmBM = 128, kGemmBN = 256, kGemmBK = 256;
+
+void count_launch();
+
+}  // namespace qfp4

@@ -1,0 +1,225 @@
+/*
+ * qfp4.h - C ABI of the B200 (sm_100a) FP4 quantized linear layer.
+ *
+ * What it computes (the pages are web articles on FP4 training; none prints
+ * code):
+ *  - Micro-scaled FP4 quantization of a bf16 tensor: E2M1 elements with one
+ *    E8M0 shared exponent per 32 elements (MXFP4; page "New AMD paper
+ *    overturns conventional wisdom: FP4 training...", section "Chto takoe
+ *    MXFP4") or one E4M3 scale per 16 elements plus an fp32 tensor scale
+ *    (NVFP4; page "Quartet II - obuchenie v NVFP4 s tochnymi nesmeshchyonnymi
+ *    gradientami": NVFP4 uses more precise FP8 scales).
+ *  - An optional block Hadamard rotation before quantization, deterministic or
+ *    with random signs, 16x16 or 32x32 (page "NVIDIA sozdala metod obucheniya
+ *    neyrosetey v 4-bit tochnosti", section "Kak eto rabotaet"; AMD page,
+ *    section "Poiskovaya eksperimental'naya rabota").
+ *  - Three rounding modes: round-to-nearest (AMD page, "Chto takoe MXFP4"),
+ *    per-element stochastic rounding (all three pages), and Quartet II, which
+ *    keeps round-to-nearest codes and stochastically rounds the per-block
+ *    renormalisation <u,u>/<u,q> (about 0.94-1.06) into the scale (Quartet II
+ *    page).
+ *  - Block-scaled FP4 GEMMs D = A . B^T, and the linear layer's three GEMMs
+ *    Fprop Y = X W^T, Dgrad dX = dY W, Wgrad dW = dY^T X (AMD page,
+ *    "Poiskovaya eksperimental'naya rabota").
+ *
+ * Conventions for every call:
+ *  - Pointers are DEVICE pointers unless stated otherwise; structs and
+ *    recipes are passed by HOST pointer. The library never allocates device
+ *    memory: the caller owns every buffer and the workspace.
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream). Calls are
+ *    asynchronous on it; the return value reports argument validation and
+ *    launch errors only. Device-side errors (a bounded wait that timed out)
+ *    are reported by qfp4_status().
+ *  - Errors are negative status codes; nothing aborts, traps or prints.
+ *  - Matrices are row-major. "rows x k" is the quantized orientation: k is the
+ *    axis the blocks run along, which is the reduction axis of the GEMM.
+ */
+#ifndef QFP4_H_
+#define QFP4_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ------------------------------------------------------ */
+#define QFP4_OK 0
+#define QFP4_ERR_INVALID_ARG (-1)      /* bad enum, negative or unsupported size, format mismatch */
+#define QFP4_ERR_MISALIGNED (-2)       /* a pointer or row stride breaks the stated alignment */
+#define QFP4_ERR_UNSUPPORTED_ARCH (-3) /* the current device is not sm_100 */
+#define QFP4_ERR_WORKSPACE (-4)        /* workspace missing or smaller than required */
+#define QFP4_ERR_CUDA (-5)             /* a CUDA runtime/driver call failed; see qfp4_last_cuda_error */
+#define QFP4_ERR_TIMEOUT (-6)          /* a device-side bounded wait expired (from qfp4_status) */
+
+/* ---- enums ---------------------------------------------------------------- */
+typedef enum { QFP4_NVFP4 = 0, QFP4_MXFP4 = 1 } qfp4_format;
+typedef enum { QFP4_RTN = 0, QFP4_SR = 1, QFP4_QUARTET2 = 2 } qfp4_rounding;
+typedef enum {
+    QFP4_HAD_NONE = 0,
+    QFP4_HAD_DET16 = 1,  /* deterministic 16x16 Hadamard (D = I) */
+    QFP4_HAD_DET32 = 2,  /* deterministic 32x32 Hadamard */
+    QFP4_HAD_RAND16 = 3, /* 16x16 Hadamard with a random sign vector */
+    QFP4_HAD_RAND32 = 4  /* 32x32 Hadamard with a random sign vector */
+} qfp4_hadamard;
+typedef enum { QFP4_AXIS_ROW = 0, QFP4_AXIS_COL = 1 } qfp4_axis;
+typedef enum { QFP4_OUT_BF16 = 0, QFP4_OUT_F32 = 1 } qfp4_dtype;
+typedef enum { QFP4_PRESET_NVIDIA_NVFP4 = 0, QFP4_PRESET_QUARTET2_NVFP4 = 1, QFP4_PRESET_AMD_MXFP4_H = 2 } qfp4_preset;
+
+/* ---- randomness -------------------------------------------------------------
+ * Every random bit is Philox4x32-10 (Salmon et al., SC'11) with key = a 64-bit
+ * seed and counter = (i/4 low 32 bits, i/4 high 32 bits, tag | stream << 4, 0);
+ * item i uses word i mod 4, and a uniform is (word >> 8) * 2^-24.
+ *   tag 0: element stochastic rounding, i = row * k + j in the quantized
+ *          orientation, key = sr;
+ *   tag 1: Quartet II scale rounding, i = row * (k / block) + block index, key = sr;
+ *   tag 2: the random Hadamard sign vector, i = 0, key = rot; bit b of the
+ *          word set flips position b of every Hadamard chunk.
+ * Reading: the pages name stochastic rounding and random sign flips but no
+ * generator; this layout makes every bit reproducible from (seed, position). */
+typedef struct {
+    uint64_t rot;        /* key of the sign vector */
+    uint64_t sr;         /* key of the rounding uniforms */
+    uint32_t rot_stream; /* stream id of the sign vector (< 2^28) */
+    uint32_t sr_stream;  /* stream id of the rounding uniforms (< 2^28) */
+} qfp4_seed;
+
+/* ---- quantized tensor -----------------------------------------------------
+ * codes:  rows * k / 2 bytes, row-major [rows][k/2]; element j of a row is the
+ *         low nibble of byte j/2 when j is even, the high nibble when odd. A
+ *         nibble is sign << 3 | index into {0, 0.5, 1, 1.5, 2, 3, 4, 6}.
+ *         16-byte aligned.
+ * scales: qfp4_scales_bytes(fmt, rows, k) bytes, 16-byte aligned, in the
+ *         tcgen05 block-scale layout: 512-byte atoms of 128 rows x 4 scale
+ *         columns (byte (r % 32) * 16 + ((r / 32) % 4) * 4 + c % 4 of atom
+ *         (r / 128) * ceil(k / block / 4) + c / 4); rows and scale columns
+ *         are padded to the atom with zero scales. E4M3 codes (NVFP4) or E8M0
+ *         codes (MXFP4). qfp4_scale_offset() gives the byte of (r, c).
+ * tensor_scale: one fp32, the NVFP4 decode multiplier g (1.0 for MXFP4).
+ * An element decodes as e2m1(code) * scale(row, j / block) * g, in the rotated
+ * domain when a Hadamard was applied.
+ * The caller sets codes, scales and tensor_scale; qfp4_quantize fills the rest. */
+typedef struct {
+    uint8_t* codes;
+    uint8_t* scales;
+    float* tensor_scale;
+    int64_t rows;
+    int64_t k;
+    int32_t fmt;         /* qfp4_format */
+    int32_t had;         /* qfp4_hadamard applied along k */
+    uint64_t rot_seed;   /* sign-vector key (random Hadamard only) */
+    uint32_t rot_stream; /* sign-vector stream (random Hadamard only) */
+    uint32_t reserved;
+} qfp4_tensor;
+
+/* ---- linear-layer recipe ------------------------------------------------- */
+typedef struct {
+    int32_t fmt;   /* qfp4_format of both operands */
+    int32_t rnd_a; /* qfp4_rounding of operand A (the left factor) */
+    int32_t rnd_b; /* qfp4_rounding of operand B */
+    int32_t had;   /* qfp4_hadamard along the GEMM's reduction axis, both operands */
+} qfp4_gemm_cfg;
+
+typedef struct {
+    qfp4_gemm_cfg fprop; /* Y  = X W^T:  A = X  (along K),  B = W (along K) */
+    qfp4_gemm_cfg dgrad; /* dX = dY W:   A = dY (along N),  B = W (along N) */
+    qfp4_gemm_cfg wgrad; /* dW = dY^T X: A = dY (along M),  B = X (along M) */
+    int32_t y_dtype, dx_dtype, dw_dtype; /* qfp4_dtype of the three outputs */
+    int32_t reserved;
+} qfp4_recipe;
+
+/* ---- errors -------------------------------------------------------------- */
+/* Static string for a status code. */
+const char* qfp4_strerror(int status);
+/* The cudaError_t behind the calling thread's last QFP4_ERR_CUDA. */
+int qfp4_last_cuda_error(void);
+
+/* ---- sizes and layouts (host-only, no device access) ---------------------- */
+/* Bytes of the codes of a rows x k tensor: rows * k / 2. */
+size_t qfp4_codes_bytes(int64_t rows, int64_t k);
+/* Bytes of the scale buffer: ceil(rows/128) * ceil(k/block/4) * 512. Returns 0 for a bad format. */
+size_t qfp4_scales_bytes(int32_t fmt, int64_t rows, int64_t k);
+/* Byte offset of the scale of (row r, scale column c) in the scale buffer,
+ * or -1 when out of range. */
+int64_t qfp4_scale_offset(int32_t fmt, int64_t rows, int64_t k, int64_t r, int64_t c);
+/* Workspace bytes qfp4_quantize / qfp4_amax need (fixed: 4096; 0 would do for
+ * MXFP4 or when the caller passes the amax). 16-byte aligned. */
+size_t qfp4_quantize_workspace_bytes(void);
+
+/* ---- quantization ----------------------------------------------------------
+ * qfp4_amax: the NVFP4 tensor amax, max |v| over the rotated tensor v in the
+ * given orientation (v = x when had is NONE), written to *amax (device fp32).
+ *
+ * qfp4_quantize: quantize x (bf16, R x C, row stride ld elements).
+ *   axis ROW: blocks run along C; the result is rows = R, k = C.
+ *   axis COL: blocks run along R; the result is the quantized transpose,
+ *             rows = C, k = R (the Wgrad operand: quantized along tokens).
+ * Steps per rows-x-k segment (k the quantized axis):
+ *   1. rotate (had != NONE): per n_h chunk v = fp32(1/sqrt(n_h)) * H (D x),
+ *      H the Sylvester matrix, D the sign vector (I for deterministic), the
+ *      butterflies in ascending half-width order, in fp32;
+ *   2. NVFP4: amax over v (or *amax_in when amax_in != NULL), s_enc = 2688 /
+ *      amax, g = amax / 2688 (both 1 when amax = 0);
+ *   3. block scale: NVFP4 S = E4M3_RN_sat(fp32(amax_b / 6) * s_enc),
+ *      r = s_enc / S (0 when S = 0); MXFP4 E = floor(log2 amax_b) - 2 clamped
+ *      to [-127, 127], code E + 127, r = 2^-E (code 0, r = 0 for a zero block);
+ *   4. u = v * r; codes by RTN (ties to even, saturating at 6, -0 -> +0), SR
+ *      (round up iff uniform < (|u| - lo) / gap), or Quartet II: RTN codes,
+ *      then alpha = T(u*u) / T(u*q) (T the halving-stride tree sum over the
+ *      block, 1 when the denominator is 0) and the scale becomes SR(S * alpha)
+ *      on the E4M3 (saturating at 448) or E8M0 grid.
+ * Requirements: R, C >= 0; k a multiple of the block (16 NVFP4, 32 MXFP4) and
+ *   of n_h; ld >= C and ld % 8 == 0; x, codes and scales 16-byte aligned;
+ *   for NVFP4 without amax_in, workspace >= qfp4_quantize_workspace_bytes(),
+ *   16-byte aligned (its contents on entry do not matter). The result depends
+ *   only on the inputs and seeds, never on the launch configuration.
+ * out: caller sets codes, scales and tensor_scale; the call sets the rest. */
+int qfp4_amax(const void* x, int64_t R, int64_t C, int64_t ld, int32_t had, int32_t axis, const qfp4_seed* seed,
+              float* amax, void* workspace, size_t workspace_bytes, void* stream);
+
+int qfp4_quantize(const void* x, int64_t R, int64_t C, int64_t ld, int32_t fmt, int32_t rounding, int32_t had,
+                  int32_t axis, const qfp4_seed* seed, const float* amax_in, qfp4_tensor* out, void* workspace,
+                  size_t workspace_bytes, void* stream);
+
+/* ---- GEMM -------------------------------------------------------------------
+ * D[i][j] = gA * gB * sum_k A(i,k) B(j,k) over the decoded FP4 operands, fp32
+ * accumulation on the tcgen05 tensor cores, D = A . B^T of shape
+ * A.rows x B.rows, written as bf16 or fp32 with row stride ldd elements.
+ * Requirements: same format, same k (a multiple of 64), same Hadamard (and for
+ * a random one, the same rot_seed and rot_stream, so the rotation cancels);
+ * D 16-byte aligned and ldd * element size a multiple of 16; ldd >= B.rows. */
+int qfp4_gemm(const qfp4_tensor* A, const qfp4_tensor* B, void* D, int64_t ldd, int32_t out_dtype, void* stream);
+
+/* ---- linear layer -------------------------------------------------------------
+ * X [M x K], W [N x K], dY [M x N] bf16 row-major (contiguous); Y [M x N],
+ * dX [M x K], dW [N x K] in the recipe's output types (contiguous).
+ * Seeds: the sign vector of GEMM g (0 Fprop, 1 Dgrad, 2 Wgrad) uses key
+ * seed->rot and stream g, shared by both operands; operand o (0 X and 1 W of
+ * Fprop, 2 dY and 3 W of Dgrad, 4 dY and 5 X of Wgrad) rounds with key
+ * seed->sr and stream o (the stream fields of *seed are ignored).
+ * Requirements: M, N, K multiples of 128; X, W, dY 16-byte aligned; the
+ * workspace holds the quantized operands. */
+int qfp4_recipe_preset(int32_t preset, qfp4_recipe* out);
+size_t qfp4_linear_workspace_bytes(int32_t backward, int64_t M, int64_t N, int64_t K, const qfp4_recipe* recipe);
+int qfp4_linear_fwd(const void* X, const void* W, void* Y, int64_t M, int64_t N, int64_t K, const qfp4_recipe* recipe,
+                    const qfp4_seed* seed, void* workspace, size_t workspace_bytes, void* stream);
+int qfp4_linear_bwd(const void* dY, const void* X, const void* W, void* dX, void* dW, int64_t M, int64_t N, int64_t K,
+                    const qfp4_recipe* recipe, const qfp4_seed* seed, void* workspace, size_t workspace_bytes,
+                    void* stream);
+
+/* ---- status ---------------------------------------------------------------
+ * Synchronizes `stream`, then reads and clears the library's device error word
+ * on the current device. Returns QFP4_OK, QFP4_ERR_TIMEOUT (a bounded wait in
+ * a kernel expired; that kernel skipped the rest of its work), or
+ * QFP4_ERR_CUDA. */
+int qfp4_status(void* stream);
+
+/* Number of kernels the library launched on the calling thread since the last
+ * reset (reset = 1 zeroes it after reading). */
+int64_t qfp4_launch_count(int32_t reset);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* QFP4_H_ */

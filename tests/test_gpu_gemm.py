@@ -1,0 +1,106 @@
+"""GPU block-scaled FP4 GEMMs vs the fp64 oracle, within
+|err| <= 2^-18 * sum_k |a_k b_k| per element (fp32 output; a bf16 output adds
+its own rounding, 2^-8 |D|). The GEMM is fed the oracle's own quantized
+operands (codes, scales and tensor scales laid out as include/qfp4.h states),
+so these tests isolate the GEMM from the quantizers."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from fp4_precision_b200 import inputs
+from fp4_precision_b200 import qfp4 as Q
+
+import helpers
+
+pytestmark = pytest.mark.gpu
+
+
+def upload(qo: O.QTensor, rot_seed=0, rot_stream=0) -> Q.QTensor:
+    """An oracle-quantized operand as a device QTensor."""
+    nb = O.BLOCK[qo.fmt]
+    kb = qo.k // nb
+    nbytes = max(Q.scales_bytes(qo.fmt, qo.rows, qo.k), 16)
+    flat = np.zeros(nbytes, dtype=np.uint8)
+    r = np.arange(qo.rows)[:, None]
+    c = np.arange(kb)[None, :]
+    flat[helpers.atom_offset(qo.rows, kb, r, c)] = qo.scales
+    codes = torch.from_numpy(qo.codes.copy()).cuda()
+    scales = torch.from_numpy(flat).cuda()
+    ts = torch.tensor([qo.g], dtype=torch.float32, device="cuda")
+    desc = Q.TensorDesc(codes.data_ptr(), scales.data_ptr(), ts.data_ptr(), qo.rows, qo.k, qo.fmt, qo.had,
+                        rot_seed, rot_stream, 0)
+    return Q.QTensor(codes, scales, ts, desc)
+
+
+def check_gemm(A_o, B_o, out_dtype, rows=None, cols=None, rot=(0, 0)):
+    A, B = upload(A_o, *rot), upload(B_o, *rot)
+    D = Q.gemm(A, B, out_dtype)
+    torch.cuda.synchronize()
+    Q.status()
+    Dg = D.float().cpu().numpy().astype(np.float64)
+    if rows is None:
+        ref, bound = O.gemm(A_o, B_o), O.gemm_bound(A_o, B_o)
+    else:
+        Ad, Bd = O.dequantize(A_o)[rows], O.dequantize(B_o)[cols]
+        ref = np.einsum("ik,ik->i", Ad, Bd)
+        bound = O.GEMM_REL_BOUND * np.einsum("ik,ik->i", np.abs(Ad), np.abs(Bd))
+        Dg = Dg[rows, cols]
+    tol = bound + (2.0 ** -8 * np.abs(ref) if out_dtype == torch.bfloat16 else 0.0)
+    err = np.abs(Dg - ref)
+    worst = np.max(err / np.maximum(bound / O.GEMM_REL_BOUND, 1e-300))
+    assert np.all(err <= tol), f"{np.sum(err > tol)} outputs out of bound; max err/sum|ab| = {worst:.3e}"
+    return worst
+
+
+@pytest.mark.parametrize("fmt", [O.NVFP4, O.MXFP4], ids=["nvfp4", "mxfp4"])
+@pytest.mark.parametrize("shape", [(128, 256, 256), (300, 200, 320), (512, 520, 1024), (130, 640, 64),
+                                   (1024, 768, 2048)], ids=lambda s: "x".join(map(str, s)))
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+def test_gemm_matches_oracle(fmt, shape, out_dtype):
+    M, N, K = shape
+    X = inputs.normal_with_outliers((M, K), 21, "ga")
+    W = inputs.normal((N, K), 0.02, 21, "gb")
+    A_o = O.quantize(X, fmt, O.RTN, O.HAD_NONE, O.ROW)
+    B_o = O.quantize(W, fmt, O.SR, O.HAD_NONE, O.ROW, 0, 0, 5, 1)
+    check_gemm(A_o, B_o, out_dtype)
+
+
+def test_gemm_rotated_operands():
+    """Random-Hadamard operands (same sign vector): the GEMM estimates X W^T."""
+    M, N, K = 256, 512, 512
+    X = inputs.normal((M, K), 1.0, 22, "ra")
+    W = inputs.normal((N, K), 1.0, 22, "rb")
+    A_o = O.quantize(X, O.NVFP4, O.QUARTET2, O.HAD_RAND16, O.ROW, 9, 1, 3, 0)
+    B_o = O.quantize(W, O.NVFP4, O.QUARTET2, O.HAD_RAND16, O.ROW, 9, 1, 3, 1)
+    check_gemm(A_o, B_o, torch.float32, rot=(9, 1))
+
+
+def test_gemm_qkv_shape_sampled():
+    """The QKV-projection Fprop shape, 8192 x 6144 x 4096, in the launch
+    configuration the benchmark times: 4096 sampled outputs plus two full
+    128 x 128 tiles against fp64 dot products."""
+    M, N, K = 8192, 6144, 4096
+    wl = inputs.workload("qkv")
+    A_o = O.quantize(wl["X"], O.NVFP4, O.RTN, O.HAD_DET16, O.ROW)
+    B_o = O.quantize(wl["W"], O.NVFP4, O.RTN, O.HAD_DET16, O.ROW)
+    rng = np.random.default_rng(0)
+    rows = rng.integers(0, M, 4096)
+    cols = rng.integers(0, N, 4096)
+    t = np.arange(128)
+    rows = np.concatenate([rows, np.repeat(t, 128), np.repeat(8064 + t, 128)])
+    cols = np.concatenate([cols, np.tile(t, 128), np.tile(6016 + t, 128)])
+    worst = check_gemm(A_o, B_o, torch.float32, rows=rows, cols=cols)
+    print(f"max err / sum|ab| = {worst:.3e}")
+
+
+def test_gemm_rejects_mismatched_operands():
+    X = inputs.normal((128, 256), 1.0, 23, "ma")
+    A = upload(O.quantize(X, O.NVFP4, O.RTN, O.HAD_RAND16, O.ROW, 1, 0), 1, 0)
+    B = upload(O.quantize(X, O.NVFP4, O.RTN, O.HAD_RAND16, O.ROW, 2, 0), 2, 0)
+    with pytest.raises(Q.QFP4Error) as e:
+        Q.gemm(A, B)
+    assert e.value.status == Q.ERR_INVALID_ARG
+    C = upload(O.quantize(X, O.MXFP4, O.RTN, O.HAD_RAND16, O.ROW, 1, 0), 1, 0)
+    with pytest.raises(Q.QFP4Error):
+        Q.gemm(A, C)

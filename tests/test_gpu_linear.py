@@ -1,0 +1,74 @@
+"""The FP4 linear layer (Fprop, Dgrad, Wgrad through the C ABI) vs the
+oracle's composition of the same quantizations and fp64 GEMMs."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from fp4_precision_b200 import inputs
+from fp4_precision_b200 import qfp4 as Q
+
+pytestmark = pytest.mark.gpu
+
+ROT, SRS = 0x1111_2222_3333_4444, 0x5555_6666_7777_8888
+
+
+def within(D_gpu, ref, bound, bf16_out):
+    Dg = D_gpu.float().cpu().numpy().astype(np.float64)
+    tol = bound + (2.0 ** -8 * np.abs(ref) if bf16_out else 0.0)
+    err = np.abs(Dg - ref)
+    assert np.all(err <= tol), f"{np.sum(err > tol)} of {err.size} out of bound"
+
+
+@pytest.mark.parametrize("preset", ["QUARTET2_NVFP4", "NVIDIA_NVFP4", "AMD_MXFP4_H"])
+def test_tiny_linear_fwd_bwd(preset):
+    """The tiny linear workload: X [512x256], W [256x256], dY [512x256]."""
+    wl = inputs.workload("tiny")
+    X, W, dY = wl["X"], wl["W"], wl["dY"]
+    rec = Q.recipe(preset)
+    seed = Q.make_seed(ROT, SRS)
+    Y = Q.linear_fwd(X.cuda(), W.cuda(), rec, seed)
+    dX, dW = Q.linear_bwd(dY.cuda(), X.cuda(), W.cuda(), rec, seed)
+    Q.status()
+    r = O.preset(preset)
+    y_ref, y_b = O.linear_fwd(X, W, r, ROT, SRS)
+    (dx_ref, dx_b), (dw_ref, dw_b) = O.linear_bwd(dY, X, W, r, ROT, SRS)
+    within(Y, y_ref, y_b, True)
+    within(dX, dx_ref, dx_b, True)
+    within(dW, dw_ref, dw_b, False)
+
+
+def test_autograd_function():
+    wl = inputs.workload("tiny")
+    X = wl["X"].cuda().requires_grad_(True)
+    W = wl["W"].cuda().requires_grad_(True)
+    rec = Q.recipe("QUARTET2_NVFP4")
+    seed = Q.make_seed(ROT, SRS)
+    Y = Q.Fp4Linear.apply(X, W, rec, seed)
+    Y.backward(wl["dY"].cuda())
+    Q.status()
+    r = O.preset("QUARTET2_NVFP4")
+    (dx_ref, dx_b), (dw_ref, dw_b) = O.linear_bwd(wl["dY"], wl["X"], wl["W"], r, ROT, SRS)
+    within(X.grad, dx_ref, dx_b, True)
+    within(W.grad, dw_ref, dw_b, True)
+
+
+def test_linear_estimates_bf16_product():
+    """Sanity (not parity): the FP4 layer's outputs track the bf16 products."""
+    wl = inputs.workload("tiny")
+    X, W, dY = (wl[k].cuda() for k in ("X", "W", "dY"))
+    rec = Q.recipe("QUARTET2_NVFP4")
+    seed = Q.make_seed(ROT, SRS)
+    Y = Q.linear_fwd(X, W, rec, seed).float()
+    dX, dW = Q.linear_bwd(dY, X, W, rec, seed)
+    for got, ref in ((Y, X.float() @ W.float().T), (dX.float(), dY.float() @ W.float()),
+                     (dW.float(), dY.float().T @ X.float())):
+        rel = (got - ref).norm() / ref.norm()
+        assert rel < 0.2, rel
+
+
+def test_linear_rejects_bad_shapes():
+    X = torch.zeros((100, 256), dtype=torch.bfloat16, device="cuda")
+    W = torch.zeros((256, 256), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(Q.QFP4Error):
+        Q.linear_fwd(X, W, Q.recipe("NVIDIA_NVFP4"), Q.make_seed())

@@ -1,0 +1,177 @@
+"""GPU quantizers vs the CPU oracle: codes, scales and the tensor scale must
+match bit for bit, for every format, rounding mode, Hadamard setting and
+orientation, on ragged shapes, at the sweep workload's full size, and on the
+degenerate inputs of the method."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from fp4_precision_b200 import inputs
+from fp4_precision_b200 import qfp4 as Q
+
+import helpers
+
+pytestmark = pytest.mark.gpu
+
+HADS = [Q.HAD_NONE, Q.HAD_DET16, Q.HAD_DET32, Q.HAD_RAND16, Q.HAD_RAND32]
+SEED = dict(rot=0x5EED_0001_2345_6789, sr=0xABCD_EF01_2345_6789, rot_stream=3, sr_stream=7)
+
+
+def gpu_quant(x_dev, fmt, rnd, had, axis, **kw):
+    seed = Q.make_seed(**SEED)
+    q = Q.quantize(x_dev, fmt, rnd, had, axis, seed, **kw)
+    torch.cuda.synchronize()
+    Q.status()
+    return q
+
+
+def oracle_quant(x_cpu, fmt, rnd, had, axis, amax=None):
+    return O.quantize(x_cpu, fmt, rnd, had, axis, SEED["rot"], SEED["rot_stream"], SEED["sr"], SEED["sr_stream"],
+                      amax=amax)
+
+
+def assert_same(q_gpu, q_ref, fmt):
+    nb = Q.BLOCK[fmt]
+    codes = helpers.to_numpy_u8(q_gpu.codes)
+    assert codes.shape == q_ref.codes.shape
+    bad = np.argwhere(codes != q_ref.codes)
+    assert bad.size == 0, f"{len(bad)} code bytes differ, first at {bad[:5].tolist()}"
+    flat = helpers.to_numpy_u8(q_gpu.scales)
+    sc = helpers.unswizzle_scales(flat, q_ref.rows, q_ref.k, nb)
+    bad = np.argwhere(sc != q_ref.scales)
+    assert bad.size == 0, f"{len(bad)} scales differ, first at {bad[:5].tolist()}"
+    assert helpers.padding_is_zero(flat, q_ref.rows, q_ref.k, nb)
+    g = float(q_gpu.tensor_scale.cpu()[0])
+    assert np.float32(g).tobytes() == np.float32(q_ref.g).tobytes(), (g, q_ref.g)
+
+
+def sweep_like(R, C, seed=1):
+    x = inputs.student_t_colgain((R, C), seed, "T")
+    # a few large outliers so some blocks saturate and the tensor amax is far from typical
+    x.view(-1)[:: 997] *= 40
+    return x
+
+
+@pytest.mark.parametrize("axis", [Q.ROW, Q.COL], ids=["row", "col"])
+@pytest.mark.parametrize("had", HADS, ids=["none", "det16", "det32", "rand16", "rand32"])
+@pytest.mark.parametrize("rnd", [Q.RTN, Q.SR, Q.QUARTET2], ids=["rtn", "sr", "q2"])
+@pytest.mark.parametrize("fmt", [Q.NVFP4, Q.MXFP4], ids=["nvfp4", "mxfp4"])
+def test_quantize_matches_oracle_ragged(fmt, rnd, had, axis):
+    # 352 x 416: several 128-tiles plus ragged tails in both directions
+    x = sweep_like(352, 416)
+    q = gpu_quant(x.cuda(), fmt, rnd, had, axis)
+    assert_same(q, oracle_quant(x, fmt, rnd, had, axis), fmt)
+
+
+@pytest.mark.parametrize("case", [
+    (Q.NVFP4, Q.RTN, Q.HAD_RAND16, Q.ROW), (Q.NVFP4, Q.QUARTET2, Q.HAD_RAND16, Q.COL),
+    (Q.MXFP4, Q.SR, Q.HAD_DET32, Q.COL), (Q.NVFP4, Q.SR, Q.HAD_NONE, Q.ROW),
+    (Q.MXFP4, Q.QUARTET2, Q.HAD_RAND32, Q.ROW), (Q.NVFP4, Q.RTN, Q.HAD_DET16, Q.COL),
+], ids=lambda c: f"{['nv', 'mx'][c[0]]}-{['rtn', 'sr', 'q2'][c[1]]}-h{c[2]}-{['row', 'col'][c[3]]}")
+def test_quantize_full_sweep_workload(case):
+    """The quantizer-sweep workload at its full size, [8192 x 4096]."""
+    fmt, rnd, had, axis = case
+    x_dev = inputs.workload("sweep", device="cuda")["T"]
+    q = gpu_quant(x_dev, fmt, rnd, had, axis)
+    assert_same(q, oracle_quant(x_dev.cpu(), fmt, rnd, had, axis), fmt)
+
+
+@pytest.mark.parametrize("fmt", [Q.NVFP4, Q.MXFP4])
+@pytest.mark.parametrize("shape", [(32, 32), (1, 64), (33, 96), (128, 128), (16, 4096), (4096, 32)])
+@pytest.mark.parametrize("axis", [Q.ROW, Q.COL])
+def test_small_and_thin_shapes(fmt, shape, axis):
+    R, C = shape
+    x = inputs.normal_with_outliers((R, C), 5, "thin")
+    rows_k = (R, C) if axis == Q.ROW else (C, R)
+    if rows_k[1] % 32:
+        pytest.skip("quantized axis must be a multiple of 32 for every Hadamard size")
+    for rnd, had in ((Q.RTN, Q.HAD_NONE), (Q.QUARTET2, Q.HAD_RAND32), (Q.SR, Q.HAD_DET16)):
+        q = gpu_quant(x.cuda(), fmt, rnd, had, axis)
+        assert_same(q, oracle_quant(x, fmt, rnd, had, axis), fmt)
+
+
+def test_strided_input():
+    """Row stride larger than the row (a column slice of a wider matrix)."""
+    big = sweep_like(256, 512)
+    x_dev = big.cuda()[:, 64:64 + 320]
+    assert x_dev.stride(0) == 512
+    for axis in (Q.ROW, Q.COL):
+        for fmt in (Q.NVFP4, Q.MXFP4):
+            q = gpu_quant(x_dev, fmt, Q.SR, Q.HAD_RAND16, axis)
+            assert_same(q, oracle_quant(x_dev.cpu().contiguous(), fmt, Q.SR, Q.HAD_RAND16, axis), fmt)
+
+
+def test_degenerate_inputs():
+    for fmt in (Q.NVFP4, Q.MXFP4):
+        for axis in (Q.ROW, Q.COL):
+            z = torch.zeros((160, 96), dtype=torch.bfloat16)
+            q = gpu_quant(z.cuda(), fmt, Q.QUARTET2, Q.HAD_RAND32, axis)
+            assert_same(q, oracle_quant(z, fmt, Q.QUARTET2, Q.HAD_RAND32, axis), fmt)
+            # huge and tiny magnitudes: saturation, E4M3 underflow to zero scales, subnormal E8M0 exponents
+            x = torch.zeros((128, 128), dtype=torch.float32)
+            x[0, 0] = 3.0e38
+            x[1, :] = torch.linspace(-1e-30, 1e-30, 128)
+            x[2, :] = 1e-38
+            x[3, :7] = -2.5
+            x = x.to(torch.bfloat16)
+            for rnd in (Q.RTN, Q.SR, Q.QUARTET2):
+                q = gpu_quant(x.cuda(), fmt, rnd, Q.HAD_NONE, axis)
+                assert_same(q, oracle_quant(x, fmt, rnd, Q.HAD_NONE, axis), fmt)
+            # empty tensors: nothing written but the tensor scale (1)
+            e = torch.zeros((0, 64), dtype=torch.bfloat16, device="cuda")
+            q = Q.quantize(e, fmt, Q.RTN, Q.HAD_NONE, axis)
+            torch.cuda.synchronize()
+            assert float(q.tensor_scale.cpu()[0]) == 1.0
+
+
+def test_rtn_ties_and_grid():
+    """Every E2M1 tie point and grid value, both signs, scaled into a block whose
+    scale is exactly 1 (the block max is 6 and the tensor max maps to 6 * 448)."""
+    vals = [0.0, 0.25, 0.5, 0.75, 1.0, 1.25, 1.5, 1.75, 2.0, 2.5, 3.0, 3.5, 4.0, 5.0, 6.0]
+    row = torch.tensor(vals + [6.0], dtype=torch.float32)
+    x = torch.cat([row, -row]).repeat(64, 1).reshape(64, 32).to(torch.bfloat16)
+    for fmt in (Q.NVFP4, Q.MXFP4):
+        q = gpu_quant(x.cuda(), fmt, Q.RTN, Q.HAD_NONE, Q.ROW)
+        assert_same(q, oracle_quant(x, fmt, Q.RTN, Q.HAD_NONE, Q.ROW), fmt)
+
+
+@pytest.mark.parametrize("axis", [Q.ROW, Q.COL])
+@pytest.mark.parametrize("had", [Q.HAD_NONE, Q.HAD_DET32, Q.HAD_RAND16])
+def test_amax_entry_point(axis, had):
+    x = sweep_like(384, 256)
+    seed = Q.make_seed(**SEED)
+    a = Q.amax(x.cuda(), had, axis, seed)
+    torch.cuda.synchronize()
+    v = O.rotate(x, had, axis, SEED["rot"], SEED["rot_stream"])
+    assert float(a.cpu()[0]) == float(np.abs(v).max())
+    # the caller-provided amax path gives the same result as the internal pass
+    q1 = gpu_quant(x.cuda(), Q.NVFP4, Q.RTN, had, axis, amax_in=a)
+    assert_same(q1, oracle_quant(x, Q.NVFP4, Q.RTN, had, axis), Q.NVFP4)
+
+
+def test_determinism_and_seed_sensitivity():
+    x = sweep_like(256, 256).cuda()
+    a = gpu_quant(x, Q.NVFP4, Q.SR, Q.HAD_RAND16, Q.COL)
+    b = gpu_quant(x, Q.NVFP4, Q.SR, Q.HAD_RAND16, Q.COL)
+    assert torch.equal(a.codes, b.codes) and torch.equal(a.scales, b.scales)
+    c = Q.quantize(x, Q.NVFP4, Q.SR, Q.HAD_RAND16, Q.COL, Q.make_seed(1, 2, 3, 4))
+    torch.cuda.synchronize()
+    assert not torch.equal(a.codes, c.codes)
+
+
+def test_argument_errors():
+    x = torch.zeros((64, 64), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(Q.QFP4Error) as e:
+        Q.quantize(x[:, :48], Q.MXFP4, Q.RTN, Q.HAD_NONE, Q.ROW)  # k = 48 not a multiple of 32
+    assert e.value.status == Q.ERR_INVALID_ARG
+    with pytest.raises(Q.QFP4Error) as e:
+        Q.quantize(x[:, 1:33], Q.NVFP4, Q.RTN, Q.HAD_NONE, Q.ROW)  # 2-byte offset: misaligned
+    assert e.value.status == Q.ERR_MISALIGNED
+    with pytest.raises(Q.QFP4Error) as e:
+        Q.quantize(x, Q.NVFP4, 9, Q.HAD_NONE, Q.ROW)
+    assert e.value.status == Q.ERR_INVALID_ARG
+    with pytest.raises(Q.QFP4Error) as e:
+        Q.quantize(x, Q.NVFP4, Q.RTN, Q.HAD_NONE, Q.ROW, workspace=torch.empty(16, dtype=torch.uint8, device="cuda"))
+    assert e.value.status == Q.ERR_WORKSPACE
+    Q.status()
