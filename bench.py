@@ -36,11 +36,13 @@ NOMINAL_FP4_OVER_BF16 = 4.0  # dense FP4 9 PF / dense BF16 2.25 PF (nominal rati
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--profile", choices=["gemm", "quant_row", "quant_col", "amax"],
+                    help="run only one kernel 3 times on a bounded case (for ncu captures), print nothing else")
     return ap.parse_args()
 
 
@@ -426,8 +428,44 @@ def run_reference(args, rank, world):
             "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def run_profile(kind: str):
+    """One kernel, three launches, on a case that exceeds L2 but holds about a
+    GB: the MLP up/gate Fprop GEMM (16384 x 28672 x 4096, NVFP4) or the
+    quantizers on the quantizer-sweep tensor [8192 x 4096]."""
+    import torch
+
+    from fp4_precision_b200 import inputs
+    from fp4_precision_b200 import qfp4 as Q
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    seed = Q.make_seed(3, 4)
+    if kind == "gemm":
+        wl = inputs.workload(WORKLOAD, device=dev)
+        A = Q.quantize(wl["X"], Q.NVFP4, Q.RTN, Q.HAD_DET16, Q.ROW, seed)
+        B = Q.quantize(wl["W"], Q.NVFP4, Q.RTN, Q.HAD_DET16, Q.ROW, seed)
+        del wl
+        D = torch.empty((A.rows, B.rows), dtype=torch.bfloat16, device=dev)
+        for _ in range(3):
+            Q.gemm(A, B, out=D)
+    else:
+        T = inputs.workload("sweep", device=dev)["T"]
+        if kind == "amax":
+            for _ in range(3):
+                Q.amax(T, Q.HAD_RAND16, Q.ROW, seed)
+        else:
+            axis = Q.ROW if kind == "quant_row" else Q.COL
+            am = Q.amax(T, Q.HAD_RAND16, axis, seed)
+            for _ in range(3):
+                Q.quantize(T, Q.NVFP4, Q.QUARTET2, Q.HAD_RAND16, axis, seed, amax_in=am)
+    torch.cuda.synchronize()
+    Q.status()
+
+
 def main():
     args = parse()
+    if args.profile:
+        run_profile(args.profile)
+        return 0
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

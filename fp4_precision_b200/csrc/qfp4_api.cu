@@ -33,6 +33,57 @@ int had_n(int had) {
 }
 bool had_random(int had) { return had == QFP4_HAD_RAND16 || had == QFP4_HAD_RAND32; }
 
+// Driver entry points are requested at a fixed ABI version (CUDA 12.0): a
+// later default can resolve a name to a newer signature (cuStreamGetCtx, for
+// one, gained a third argument in 12.5).
+template <typename Fn>
+Fn driver_fn(const char* name) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion(name, &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+        return reinterpret_cast<Fn>(p);
+    return nullptr;
+}
+
+// ---- context binding -----------------------------------------------------------
+// The library carries its own (static) CUDA runtime. A caller's thread may have
+// no current driver context (e.g. a framework's worker thread), and the right
+// GPU is the one the caller's stream lives on, so every entry point that
+// touches the device first makes the stream's context current.
+using GetCtxFn = CUresult (*)(CUstream, CUcontext*);
+using CurCtxFn = CUresult (*)(CUcontext*);
+using SetCtxFn = CUresult (*)(CUcontext);
+
+
+
+int bind_context(cudaStream_t stream) {
+    static GetCtxFn get_stream_ctx = nullptr;
+    static CurCtxFn get_cur = nullptr;
+    static SetCtxFn set_cur = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        get_stream_ctx = driver_fn<GetCtxFn>("cuStreamGetCtx");
+        get_cur = driver_fn<CurCtxFn>("cuCtxGetCurrent");
+        set_cur = driver_fn<SetCtxFn>("cuCtxSetCurrent");
+    });
+    if (!get_stream_ctx || !get_cur || !set_cur) return QFP4_OK;  // nothing to adjust
+    CUcontext want = nullptr, cur = nullptr;
+    const uintptr_t h = reinterpret_cast<uintptr_t>(stream);
+    if (h > 2 && get_stream_ctx(reinterpret_cast<CUstream>(stream), &want) != CUDA_SUCCESS) want = nullptr;
+    if (get_cur(&cur) != CUDA_SUCCESS) cur = nullptr;
+    if (want != nullptr && want != cur) {
+        if (set_cur(want) != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidResourceHandle);
+    } else if (want == nullptr && cur == nullptr) {
+        // default stream and no current context: the runtime's current device
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e == cudaSuccess) e = cudaSetDevice(dev);
+        if (e != cudaSuccess) return cuda_fail(e);
+    }
+    return QFP4_OK;
+}
+
 // ---- device check (sm_100), cached per device --------------------------------
 int check_device(int* sm_count) {
     int dev = 0;
@@ -55,6 +106,7 @@ int check_device(int* sm_count) {
         cached_sms[dev] = sms;
     }
     if (sm_count) *sm_count = cached_sms[dev];
+    set_sm_count(cached_sms[dev]);
     return cached_ok[dev] == 1 ? QFP4_OK : QFP4_ERR_UNSUPPORTED_ARCH;
 }
 
@@ -66,13 +118,7 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
 EncodeTiledFn encode_fn() {
     static EncodeTiledFn fn = nullptr;
     static std::once_flag once;
-    std::call_once(once, [] {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    });
+    std::call_once(once, [] { fn = driver_fn<EncodeTiledFn>("cuTensorMapEncodeTiled"); });
     return fn;
 }
 
@@ -93,6 +139,27 @@ int make_col_tmap(CUtensorMap* tm, const void* x, int64_t R, int64_t C, int64_t 
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
     return QFP4_OK;
+}
+
+// 2-D view of a bf16 R x C tensor for the row quantizer: box 64 columns x 256
+// rows (128 bytes per row), 128-byte swizzle.
+int make_row_tmap(CUtensorMap* tm, const void* x, int64_t R, int64_t C, int64_t ld) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return cuda_fail(cudaErrorNotSupported);
+    const cuuint64_t dims[2] = {(cuuint64_t)C, (cuuint64_t)R};
+    const cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
+    const cuuint32_t box[2] = {64, 256};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
+    return QFP4_OK;
+}
+
+// TMA view of x for a pass in the given orientation (G: column-mode group).
+int make_input_tmap(CUtensorMap* tm, const void* x, int64_t R, int64_t C, int64_t ld, int axis, int G) {
+    return axis == QFP4_AXIS_ROW ? make_row_tmap(tm, x, R, C, ld) : make_col_tmap(tm, x, R, C, ld, G);
 }
 
 // 2-D view of packed FP4 codes [rows][k/2] as bytes, box (128 bytes, box_rows),
@@ -118,7 +185,7 @@ int write_one(float* dst, cudaStream_t s) {
 }
 
 int amax_partial_count(int sms, int64_t tiles) {
-    int64_t n = 4 * (int64_t)sms;
+    int64_t n = 2 * (int64_t)sms;
     if (n > tiles) n = tiles;
     if (n > kMaxAmaxPartials) n = kMaxAmaxPartials;
     return n < 1 ? 1 : (int)n;
@@ -173,18 +240,11 @@ int run_amax(const void* x, int64_t R, int64_t C, int64_t ld, int32_t had, int32
     p.signs = signs;
     p.amax_out = partials;
     const int nh = had_n(had);
+    const int G = col_group(16, nh);
     CUtensorMap tm;
-    std::memset(&tm, 0, sizeof tm);
-    int64_t tiles;
-    if (axis == QFP4_AXIS_ROW) {
-        tiles = ((g.rows + 127) / 128) * ((g.k + 127) / 128);
-    } else {
-        const int G = col_group(16, nh);
-        int rc = make_col_tmap(&tm, x, R, C, ld, G);
-        if (rc) return rc;
-        tiles = ((g.rows + 127) / 128) * ((g.k + 4 * G - 1) / (4 * G));
-    }
-    *n_partials = amax_partial_count(sms, tiles);
+    int rc = make_input_tmap(&tm, x, R, C, ld, axis, G);
+    if (rc) return rc;
+    *n_partials = amax_partial_count(sms, quant_tiles(axis, g.rows, g.k, G));
     cudaError_t e = launch_amax(p, axis, nh, &tm, *n_partials, s);
     return e == cudaSuccess ? QFP4_OK : cuda_fail(e);
 }
@@ -193,7 +253,9 @@ int quantize_impl(const void* x, int64_t R, int64_t C, int64_t ld, int32_t fmt, 
                   int32_t axis, const qfp4_seed* seed, const float* amax_in, qfp4_tensor* out, void* workspace,
                   size_t workspace_bytes, cudaStream_t s) {
     int sms = 0;
-    int rc = check_device(&sms);
+    int rc = bind_context(s);
+    if (rc) return rc;
+    rc = check_device(&sms);
     if (rc) return rc;
     if (fmt != QFP4_NVFP4 && fmt != QFP4_MXFP4) return QFP4_ERR_INVALID_ARG;
     if (rounding < QFP4_RTN || rounding > QFP4_QUARTET2) return QFP4_ERR_INVALID_ARG;
@@ -246,16 +308,16 @@ int quantize_impl(const void* x, int64_t R, int64_t C, int64_t ld, int32_t fmt, 
         p.n_partials = n;
     }
     CUtensorMap tm;
-    std::memset(&tm, 0, sizeof tm);
-    if (axis == QFP4_AXIS_COL) {
-        if ((rc = make_col_tmap(&tm, x, R, C, ld, col_group(NB, nh)))) return rc;
-    }
+    if ((rc = make_input_tmap(&tm, x, R, C, ld, axis, col_group(NB, nh)))) return rc;
     cudaError_t e = launch_quant(p, fmt, rounding, nh, axis, &tm, s);
     return e == cudaSuccess ? QFP4_OK : cuda_fail(e);
 }
 
 int gemm_impl(const qfp4_tensor* A, const qfp4_tensor* B, void* D, int64_t ldd, int32_t out_dtype, cudaStream_t s) {
-    int rc = check_device(nullptr);
+    int rc = bind_context(s);
+    if (rc) return rc;
+    int sms = 0;
+    rc = check_device(&sms);
     if (rc) return rc;
     if (A == nullptr || B == nullptr) return QFP4_ERR_INVALID_ARG;
     if (out_dtype != QFP4_OUT_BF16 && out_dtype != QFP4_OUT_F32) return QFP4_ERR_INVALID_ARG;
@@ -293,7 +355,7 @@ int gemm_impl(const qfp4_tensor* A, const qfp4_tensor* B, void* D, int64_t ldd, 
     p.M = (int)M; p.N = (int)N; p.K = (int)K;
     const int NB = block_of(A->fmt);
     p.atoms_k = (int)((K / NB + 3) / 4);
-    cudaError_t e = launch_gemm(p, A->fmt, &tA, &tB, s);
+    cudaError_t e = launch_gemm(p, A->fmt, &tA, &tB, s, sms);
     return e == cudaSuccess ? QFP4_OK : cuda_fail(e);
 }
 
@@ -410,7 +472,9 @@ size_t qfp4_quantize_workspace_bytes(void) { return (size_t)kMaxAmaxPartials * s
 int qfp4_amax(const void* x, int64_t R, int64_t C, int64_t ld, int32_t had, int32_t axis, const qfp4_seed* seed,
               float* amax, void* workspace, size_t workspace_bytes, void* stream) {
     int sms = 0;
-    int rc = check_device(&sms);
+    int rc = bind_context(static_cast<cudaStream_t>(stream));
+    if (rc) return rc;
+    rc = check_device(&sms);
     if (rc) return rc;
     Geometry g;
     if ((rc = validate_input(x, R, C, ld, had, axis, &g))) return rc;
@@ -533,6 +597,8 @@ int qfp4_linear_bwd(const void* dY, const void* X, const void* W, void* dX, void
 }
 
 int qfp4_status(void* stream) {
+    const int rc = bind_context(static_cast<cudaStream_t>(stream));
+    if (rc) return rc;
     cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e);
     uint32_t v = 0;

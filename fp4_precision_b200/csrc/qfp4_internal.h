@@ -35,13 +35,18 @@ struct QuantParams {
 };
 
 // Launchers (quant.cu). Return cudaSuccess or the launch error.
-cudaError_t launch_amax(const QuantParams& p, int axis, int nh, const CUtensorMap* tmap_col, int n_partials,
+// `tmap` is the TMA view of x: 2-D (row mode) or the 5-D column view.
+cudaError_t launch_amax(const QuantParams& p, int axis, int nh, const CUtensorMap* tmap, int n_partials,
                         cudaStream_t s);
-cudaError_t launch_quant(const QuantParams& p, int fmt, int rnd, int nh, int axis, const CUtensorMap* tmap_col,
+cudaError_t launch_quant(const QuantParams& p, int fmt, int rnd, int nh, int axis, const CUtensorMap* tmap,
                          cudaStream_t s);
 cudaError_t launch_reduce_max(const float* in, int n, float* out, cudaStream_t s);
 // Column-mode geometry: group G = max(block, n_h), tile = 4G rows x 128 columns.
 int col_group(int fmt_or_amax_block, int nh);
+// Number of tiles a quantizer (or amax) pass walks (G: the column-mode group).
+int64_t quant_tiles(int axis, int64_t rows, int64_t k, int G);
+// SM count of the current device (sizes the persistent grids).
+void set_sm_count(int sms);
 
 struct GemmParams {
     const uint8_t* sfa;
@@ -57,7 +62,7 @@ struct GemmParams {
 
 // gemm_sm100.cu
 cudaError_t launch_gemm(const GemmParams& p, int fmt, const CUtensorMap* tmapA, const CUtensorMap* tmapB,
-                        cudaStream_t s);
+                        cudaStream_t s, int sms);
 constexpr int kGemmBM = 128, kGemmBN = 256, kGemmBK = 256;
 
 void count_launch();

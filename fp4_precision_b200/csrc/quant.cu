@@ -10,33 +10,31 @@
 // per 32 for MXFP4), then round-to-nearest, per-element stochastic rounding or
 // Quartet II (RTN codes, stochastically rounded renormalised scale).
 //
-// Row mode (blocks along the contiguous axis): a CTA owns 128 rows x 128
-// columns; each thread loads 16-byte chunks of 8 elements, coalesced across the
-// warp. The Hadamard butterflies of half-width < 8 run in registers, wider ones
-// and the block reductions with warp shuffles between the 2 or 4 lanes of a
-// block. Scales are staged in shared memory as whole 512-byte MMA atoms and
-// stored with 16-byte writes.
-//
-// Column mode (blocks along the strided axis; the output is the quantized
-// transpose): a CTA owns 4G rows x 128 columns (G = max(block, n_h)), brought
-// in by TMA as two 128-byte-swizzled boxes through a 5-D view of the tensor
-// whose row order makes the transposing ldmatrix reads conflict-free; each
-// thread then holds one whole group of one column in registers.
+// Structure: persistent CTAs of 8 compute warps and 1 producer warp. The
+// producer streams tiles of the bf16 tensor into a multi-stage shared-memory
+// ring with TMA; every compute thread owns whole groups (G = max(block, n_h)
+// consecutive elements of the quantized axis), so the rotation, the block
+// reductions and the rounding run in its registers without shuffles.
+//   Row mode (blocks along the contiguous axis): tiles of 256 rows x 64
+//     columns (128-byte swizzle); thread t takes row t, i.e. 64 / G groups.
+//   Column mode (blocks along the strided axis; the output is the quantized
+//     transpose): tiles of 4G rows x 128 columns through a 5-D view of the
+//     tensor whose row order makes the transposing ldmatrix reads
+//     conflict-free; thread (column c, q) takes rows [Gq, Gq + G) of c.
 //
 // Every fp32 operation is the one the method states, in its order, with no
-// fused multiply-add (the library is built with --fmad=false), so codes and
-// scales are exactly those of the definition.
-#include <cuda_fp16.h>
-
+// fused multiply-add (the library is built with --fmad=false; packed f32x2
+// adds and multiplies round each lane like the scalar instruction), so codes
+// and scales are exactly those of the definition.
 #include "qfp4_device.cuh"
 #include "qfp4_internal.h"
 
 namespace qfp4 {
-
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kRowTileRows = 128, kRowTileCols = 128;
+constexpr int kComputeWarps = 8;
+constexpr int kThreads = (kComputeWarps + 1) * 32;  // + one producer warp
+constexpr int kRowTileRows = 256, kRowTileCols = 64;
 constexpr int kColTileCols = 128;
 
 template <int NH>
@@ -44,36 +42,68 @@ __device__ __forceinline__ float had_norm() {
     return NH == 16 ? 0.25f : 0x1.6a09e6p-3f;  // fp32(1/sqrt(16)), fp32(1/sqrt(32))
 }
 
-// In-register butterflies of half-width 1, 2, 4 over 8 consecutive elements.
-__device__ __forceinline__ void fwht8(float* v) {
+__device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
+__device__ __forceinline__ float2 neg2(float2 a) { return make_float2(-a.x, -a.y); }
+
+// One butterfly stage of half-width H >= 2 over N elements, packed x2.
+template <int N, int H>
+__device__ __forceinline__ void fwht_stage(float* v) {
 #pragma unroll
-    for (int h = 1; h < 8; h <<= 1)
+    for (int j0 = 0; j0 < N; j0 += 2 * H)
 #pragma unroll
-        for (int j0 = 0; j0 < 8; j0 += 2 * h)
-#pragma unroll
-            for (int j = j0; j < j0 + h; ++j) {
-                const float a = v[j], b = v[j + h];
-                v[j] = __fadd_rn(a, b);
-                v[j + h] = __fsub_rn(a, b);
-            }
+        for (int j = j0; j < j0 + H; j += 2) {
+            const float2 a = f2(v[j], v[j + 1]), b = f2(v[j + H], v[j + H + 1]);
+            const float2 s = __fadd2_rn(a, b), d = __fadd2_rn(a, neg2(b));
+            v[j] = s.x; v[j + 1] = s.y;
+            v[j + H] = d.x; v[j + H + 1] = d.y;
+        }
 }
 
-// Butterflies of half-width 8 .. n/2 over n elements held by one thread.
+// Hadamard butterflies (ascending half-width, (a, b) -> (a + b, a - b)) over
+// n consecutive elements of v, in fp32: half-width 1 scalar, >= 2 packed x2.
 template <int N>
-__device__ __forceinline__ void fwht_wide(float* v) {
+__device__ __forceinline__ void fwht(float* v) {
 #pragma unroll
-    for (int h = 8; h < N; h <<= 1)
-#pragma unroll
-        for (int j0 = 0; j0 < N; j0 += 2 * h)
-#pragma unroll
-            for (int j = j0; j < j0 + h; ++j) {
-                const float a = v[j], b = v[j + h];
-                v[j] = __fadd_rn(a, b);
-                v[j + h] = __fsub_rn(a, b);
-            }
+    for (int j = 0; j < N; j += 2) {
+        const float a = v[j], b = v[j + 1];
+        v[j] = __fadd_rn(a, b);
+        v[j + 1] = __fsub_rn(a, b);
+    }
+    fwht_stage<N, 2>(v);
+    fwht_stage<N, 4>(v);
+    fwht_stage<N, 8>(v);
+    if constexpr (N == 32) fwht_stage<N, 16>(v);
 }
 
-// Reduce the CTA's amax partials (NVFP4) to s_enc and write g from CTA 0.
+// One stride of the halving tree: s[j] += s[j + ST] for j < ST, packed x2.
+template <int ST>
+__device__ __forceinline__ void tree_stage(float* s) {
+#pragma unroll
+    for (int j = 0; j < ST; j += 2) {
+        const float2 r = __fadd2_rn(f2(s[j], s[j + 1]), f2(s[j + ST], s[j + ST + 1]));
+        s[j] = r.x; s[j + 1] = r.y;
+    }
+}
+
+// Halving-stride tree sum of n fp32 terms (s[j] += s[j + stride], stride n/2 .. 1).
+template <int N>
+__device__ __forceinline__ float tree_sum(float* s) {
+    if constexpr (N == 32) tree_stage<16>(s);
+    tree_stage<8>(s);
+    tree_stage<4>(s);
+    tree_stage<2>(s);
+    return __fadd_rn(s[0], s[1]);
+}
+
+// E2M1 pair (one byte) -> two fp32 values (exact through f16).
+__device__ __forceinline__ float2 e2m1x2_decode(uint32_t byte) {
+    uint32_t h2;
+    const uint16_t b = (uint16_t)byte;
+    asm("{\n\t.reg .b8 t;\n\tcvt.u8.u16 t, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, t;\n\t}" : "=r"(h2) : "h"(b));
+    return __half22float2(*reinterpret_cast<__half2*>(&h2));
+}
+
+// Reduce the CTA's amax partials (NVFP4) to s_enc; CTA 0 writes g.
 __device__ float nvfp4_encode_scale(const QuantParams& p, float* red_smem, bool write_g) {
     float amax = 0.0f;
     if (p.amax_in != nullptr) {
@@ -104,229 +134,281 @@ __device__ float nvfp4_encode_scale(const QuantParams& p, float* red_smem, bool 
     return s_enc;
 }
 
-// Block scale of one block from its amax. Returns the scale code and sets the
-// element multiplier r and the decoded scale S.
-template <int FMT>
-__device__ __forceinline__ uint32_t block_scale(float amax_b, float s_enc, float& rmul, float& S) {
-    if constexpr (FMT == kNvfp4) {
-        const float d = __fdiv_rn(amax_b, 6.0f);
-        const float t = __fmul_rn(d, s_enc);
-        const uint32_t code = e4m3_rn(t);
-        S = e4m3_decode(code);
-        rmul = (S == 0.0f) ? 0.0f : __fdiv_rn(s_enc, S);
-        return code;
-    } else {
-        if (amax_b == 0.0f) {
-            S = exp2i(-127);
-            rmul = 0.0f;
-            return 0u;
+// The four Quartet II scale uniforms of one Philox quad, computed once per quad.
+struct ScaleRng {
+    uint64_t quad = ~0ull;
+    uint4 w;
+    __device__ __forceinline__ float uniform(const QuantParams& p, uint64_t block_index) {
+        const uint64_t q = block_index >> 2;
+        if (q != quad) {
+            w = philox_quad(p.sr_seed, p.sr_tag_scale, q);
+            quad = q;
         }
-        int E = floor_log2(amax_b) - 2;
-        E = E < -127 ? -127 : (E > 127 ? 127 : E);
-        S = exp2i(E);
-        rmul = exp2i(-E);
-        return (uint32_t)(E + 127);
+        const uint32_t i = (uint32_t)(block_index & 3);
+        return uniform24(i == 0 ? w.x : i == 1 ? w.y : i == 2 ? w.z : w.w);
     }
-}
+};
 
-// Quartet II scale: SR(S * alpha) onto the scale grid with the block's uniform.
-template <int FMT>
-__device__ __forceinline__ uint32_t quartet2_scale(float num, float den, float S, const QuantParams& p,
-                                                   uint64_t block_index) {
-    const float alpha = (den == 0.0f) ? 1.0f : __fdiv_rn(num, den);
-    const float t = __fmul_rn(S, alpha);
-    const uint4 w = philox_quad(p.sr_seed, p.sr_tag_scale, block_index >> 2);
-    const uint32_t word = (block_index & 3) == 0 ? w.x : (block_index & 3) == 1 ? w.y : (block_index & 3) == 2 ? w.z : w.w;
-    const float rho = uniform24(word);
-    if constexpr (FMT == kNvfp4)
-        return e4m3_sr(t, rho);
-    else
-        return e8m0_sr(t, rho);
-}
+// ---------------------------------------------------------------------------
+// One group of G consecutive elements of the quantized axis, in registers.
+//   v          : the G values (bf16 widened to fp32), consumed
+//   elem0      : index (row * k + j) of v[0] in the quantized orientation
+//   block0     : block index of v[0]
+//   codes      : G/8 words of packed E2M1 codes (element 0 lowest)
+//   scodes     : G/NB scale codes
+template <int FMT, int RND, int NH>
+struct Group {
+    static constexpr int NB = (FMT == kNvfp4) ? 16 : 32;
+    static constexpr int G = (NH > NB) ? NH : NB;
 
-// Write the CTA's staged scale atoms (n_atoms x 512 bytes, contiguous in the
-// global layout) unless they fall past the padded scale columns.
-__device__ __forceinline__ void store_atoms(const QuantParams& p, const uint8_t* stage, int n_atoms, int64_t row0,
-                                            int64_t first_kb) {
-    const int64_t atoms_k = p.kb4 / 4;
-    const int64_t atom_col = first_kb / 4;
-    for (int i = threadIdx.x; i < n_atoms * 32; i += blockDim.x) {
-        const int a = i >> 5;
-        if (atom_col + a >= atoms_k) continue;
-        const int64_t dst = ((row0 / 128) * atoms_k + atom_col + a) * 512 + (i & 31) * 16;
-        *reinterpret_cast<uint4*>(p.scales + dst) = *reinterpret_cast<const uint4*>(stage + a * 512 + (i & 31) * 16);
+    __device__ __forceinline__ static void rotate(float* v, uint32_t signs) {
+        if constexpr (NH > 0) {
+#pragma unroll
+            for (int hb = 0; hb < G / NH; ++hb) {
+                float* w = v + hb * NH;
+                if (signs != 0u) {
+#pragma unroll
+                    for (int e = 0; e < NH; ++e)
+                        w[e] = __uint_as_float(__float_as_uint(w[e]) ^ ((signs << (31 - e)) & 0x80000000u));
+                }
+                fwht<NH>(w);
+#pragma unroll
+                for (int e = 0; e < NH; e += 2) {
+                    const float2 r = __fmul2_rn(f2(w[e], w[e + 1]), f2(had_norm<NH>(), had_norm<NH>()));
+                    w[e] = r.x; w[e + 1] = r.y;
+                }
+            }
+        }
     }
+
+    __device__ __forceinline__ static void quantize(float* v, float s_enc, const QuantParams& p, uint64_t elem0,
+                                                    uint64_t block0, ScaleRng& srng, uint32_t* codes,
+                                                    uint32_t* scodes) {
+#pragma unroll
+        for (int b = 0; b < G / NB; ++b) {
+            float* vb = v + b * NB;
+            // block scale from the block amax
+            float am = 0.0f;
+#pragma unroll
+            for (int e = 0; e < NB; ++e) am = fmaxf(am, fabsf(vb[e]));
+            float rmul, S;
+            uint32_t scode;
+            if constexpr (FMT == kNvfp4) {
+                const float d = __fdiv_rn(am, 6.0f);
+                const float t = __fmul_rn(d, s_enc);
+                scode = e4m3_rn(t);
+                S = e4m3_decode(scode);
+                rmul = (S == 0.0f) ? 0.0f : __fdiv_rn(s_enc, S);
+            } else {
+                if (am == 0.0f) {
+                    scode = 0u;
+                    S = exp2i(-127);
+                    rmul = 0.0f;
+                } else {
+                    int E = floor_log2(am) - 2;
+                    E = E < -127 ? -127 : (E > 127 ? 127 : E);
+                    scode = (uint32_t)(E + 127);
+                    S = exp2i(E);
+                    rmul = exp2i(-E);
+                }
+            }
+            // scaled values
+#pragma unroll
+            for (int e = 0; e < NB; e += 2) {
+                const float2 r = __fmul2_rn(f2(vb[e], vb[e + 1]), f2(rmul, rmul));
+                vb[e] = r.x; vb[e + 1] = r.y;
+            }
+            // element rounding
+            uint32_t* cb = codes + b * (NB / 8);
+            if constexpr (RND == kSr) {
+                const uint64_t i0 = elem0 + (uint64_t)(b * NB);
+#pragma unroll
+                for (int e4 = 0; e4 < NB; e4 += 4) {
+                    const uint4 w = philox_quad(p.sr_seed, p.sr_tag_elem, (i0 + e4) >> 2);
+                    vb[e4 + 0] = e2m1_sr_value(vb[e4 + 0], uniform24(w.x));
+                    vb[e4 + 1] = e2m1_sr_value(vb[e4 + 1], uniform24(w.y));
+                    vb[e4 + 2] = e2m1_sr_value(vb[e4 + 2], uniform24(w.z));
+                    vb[e4 + 3] = e2m1_sr_value(vb[e4 + 3], uniform24(w.w));
+                }
+            }
+#pragma unroll
+            for (int e8 = 0; e8 < NB; e8 += 8) cb[e8 / 8] = e2m1x8_rn(vb + e8);
+            if constexpr (RND == kQuartet2) {
+                // alpha = T(u*u) / T(u*q), T the halving-stride tree sum
+                float sa[NB], sb[NB];
+#pragma unroll
+                for (int e = 0; e < NB; e += 2) {
+                    const float2 u = f2(vb[e], vb[e + 1]);
+                    const float2 q = e2m1x2_decode((cb[e / 8] >> (4 * (e & 7))) & 0xFFu);
+                    const float2 uu = __fmul2_rn(u, u), uq = __fmul2_rn(u, q);
+                    sa[e] = uu.x; sa[e + 1] = uu.y;
+                    sb[e] = uq.x; sb[e + 1] = uq.y;
+                }
+                const float num = tree_sum<NB>(sa);
+                const float den = tree_sum<NB>(sb);
+                const float alpha = (den == 0.0f) ? 1.0f : __fdiv_rn(num, den);
+                const float t = __fmul_rn(S, alpha);
+                const float rho = srng.uniform(p, block0 + b);
+                if constexpr (FMT == kNvfp4)
+                    scode = e4m3_sr(t, rho);
+                else
+                    scode = e8m0_sr(t, rho);
+            }
+            scodes[b] = scode;
+        }
+    }
+};
+
+// Ring of TMA stages: full[s] completes when the tile landed, empty[s] when all
+// compute warps finished with it.
+template <int STAGES>
+struct Ring {
+    uint64_t full[STAGES];
+    uint64_t empty[STAGES];
+};
+
+template <int STAGES>
+__device__ __forceinline__ void ring_init(Ring<STAGES>& ring) {
+    for (int s = 0; s < STAGES; ++s) {
+        mbar_init(&ring.full[s], 1);
+        mbar_init(&ring.empty[s], kComputeWarps);
+    }
+    fence_mbarrier_init();
 }
 
-__device__ __forceinline__ int atom_offset(int row_in_tile, int kb_local) {
-    return (kb_local >> 2) * 512 + (row_in_tile & 31) * 16 + ((row_in_tile >> 5) & 3) * 4 + (kb_local & 3);
+// CTA-wide max over the compute warps' values; thread 0 writes the partial.
+__device__ __forceinline__ void write_partial(float m, float* red, float* out) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+    asm volatile("bar.sync 1, %0;" ::"r"(kComputeWarps * 32));
+    if (threadIdx.x == 0) {
+        float r = 0.0f;
+        for (int w = 0; w < kComputeWarps; ++w) r = fmaxf(r, red[w]);
+        out[blockIdx.x] = r;
+    }
 }
 
 // ===========================================================================
 // Row mode
 // ===========================================================================
-template <int FMT, int RND, int NH, bool AMAX_ONLY>
-__global__ void __launch_bounds__(kThreads) quant_row_kernel(const QuantParams p) {
-    constexpr int NB = (FMT == kNvfp4) ? 16 : 32;
-    constexpr int CHUNKS = kRowTileRows * kRowTileCols / 8 / kThreads;  // 8 chunks per thread
-    __shared__ __align__(16) uint8_t scale_stage[1024];
+template <int FMT, int RND, int NH, bool AMAX_ONLY, int STAGES>
+__global__ void __launch_bounds__(kThreads, 2)
+    quant_row_kernel(const __grid_constant__ CUtensorMap tmap, const QuantParams p) {
+    using Grp = Group<FMT, RND, NH>;
+    constexpr int NB = Grp::NB;
+    constexpr int G = AMAX_ONLY ? ((NH > 16) ? NH : 16) : Grp::G;
+    constexpr int STAGE_BYTES = kRowTileRows * kRowTileCols * 2;  // 32 KiB
+    extern __shared__ __align__(1024) uint8_t dyn_smem[];
+    uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
+    __shared__ Ring<STAGES> ring;
     __shared__ float red[33];
 
-    const int tid = threadIdx.x;
-    const int cc = tid & 15;  // chunk column within the tile
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t tiles_c = (p.k + kRowTileCols - 1) / kRowTileCols;
     const int64_t tiles_total = tiles_c * ((p.rows + kRowTileRows - 1) / kRowTileRows);
 
+    if (tid == 0) {
+        prefetch_tmap(&tmap);
+        ring_init(ring);
+    }
+    __syncthreads();
     float s_enc = 1.0f;
     if constexpr (!AMAX_ONLY && FMT == kNvfp4) s_enc = nvfp4_encode_scale(p, red, blockIdx.x == 0);
     if constexpr (!AMAX_ONLY && FMT == kMxfp4) {
         if (blockIdx.x == 0 && tid == 0) *p.tensor_scale = 1.0f;
     }
+
+    if (warp == kComputeWarps) {
+        // ---------------- producer ----------------
+        if (lane == 0) {
+            int i = 0;
+            for (int64_t tile = blockIdx.x; tile < tiles_total; tile += gridDim.x, ++i) {
+                const int s = i % STAGES;
+                if (i >= STAGES && !mbar_wait(&ring.empty[s], ((i / STAGES) + 1) & 1)) break;
+                mbar_arrive_expect_tx(&ring.full[s], STAGE_BYTES);
+                tma_load_2d(tiles + s * STAGE_BYTES, &tmap, &ring.full[s],
+                            (int32_t)((tile % tiles_c) * kRowTileCols), (int32_t)((tile / tiles_c) * kRowTileRows));
+            }
+        }
+        return;
+    }
+
+    // ---------------- compute: thread = one row of the tile ----------------
+    const int64_t rows_pad = (p.rows + 127) / 128 * 128;
     float amax_acc = 0.0f;
-
-    for (int64_t tile = blockIdx.x; tile < tiles_total; tile += gridDim.x) {
-        const int64_t row0 = (tile / tiles_c) * kRowTileRows;
+    ScaleRng srng;
+    int i = 0;
+    for (int64_t tile = blockIdx.x; tile < tiles_total; tile += gridDim.x, ++i) {
+        const int s = i % STAGES;
+        if (!mbar_wait(&ring.full[s], (i / STAGES) & 1)) break;
+        const int64_t row = (tile / tiles_c) * kRowTileRows + tid;
         const int64_t col0 = (tile % tiles_c) * kRowTileCols;
-        const int64_t col = col0 + cc * 8;
-        const bool col_ok = col < p.k;
-
-        uint4 raw[CHUNKS];
+        const uint32_t sbase = smem_u32(tiles + s * STAGE_BYTES) + tid * 128;
+        uint32_t codes[kRowTileCols / 8];
+        uint32_t scodes[kRowTileCols / 16];
 #pragma unroll
-        for (int j = 0; j < CHUNKS; ++j) {
-            const int64_t row = row0 + 16 * j + (tid >> 4);
-            raw[j] = make_uint4(0u, 0u, 0u, 0u);
-            if (col_ok && row < p.rows) raw[j] = __ldg(reinterpret_cast<const uint4*>(p.x + row * p.ld + col));
-        }
-
+        for (int g = 0; g < kRowTileCols / G; ++g) {
+            float v[G];
 #pragma unroll
-        for (int j = 0; j < CHUNKS; ++j) {
-            const int r_in_tile = 16 * j + (tid >> 4);
-            const int64_t row = row0 + r_in_tile;
-            float v[8];
-            v[0] = bf16lo(raw[j].x); v[1] = bf16hi(raw[j].x);
-            v[2] = bf16lo(raw[j].y); v[3] = bf16hi(raw[j].y);
-            v[4] = bf16lo(raw[j].z); v[5] = bf16hi(raw[j].z);
-            v[6] = bf16lo(raw[j].w); v[7] = bf16hi(raw[j].w);
-
-            if constexpr (NH > 0) {
-                // 1. rotation: signs, butterflies h = 1, 2, 4 in registers, h = 8 (and
-                // 16) across lanes, then one fp32 multiply by 1/sqrt(n_h).
-                const uint32_t sbits = p.signs >> (uint32_t)(col % NH);
-#pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    if ((sbits >> e) & 1u) v[e] = -v[e];
-                fwht8(v);
-                {
-                    const bool lower = ((col >> 3) & 1) == 0;
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const float o = __shfl_xor_sync(0xffffffffu, v[e], 1);
-                        v[e] = lower ? __fadd_rn(v[e], o) : __fsub_rn(o, v[e]);
-                    }
-                }
-                if constexpr (NH == 32) {
-                    const bool lower = ((col >> 4) & 1) == 0;
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const float o = __shfl_xor_sync(0xffffffffu, v[e], 2);
-                        v[e] = lower ? __fadd_rn(v[e], o) : __fsub_rn(o, v[e]);
-                    }
-                }
-#pragma unroll
-                for (int e = 0; e < 8; ++e) v[e] = __fmul_rn(v[e], had_norm<NH>());
+            for (int c8 = 0; c8 < G / 8; ++c8) {
+                const int chunk = g * (G / 8) + c8;
+                uint32_t w0, w1, w2, w3;
+                asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                             : "=r"(w0), "=r"(w1), "=r"(w2), "=r"(w3)
+                             : "r"(sbase + ((chunk ^ (tid & 7)) << 4)));
+                v[8 * c8 + 0] = bf16lo(w0); v[8 * c8 + 1] = bf16hi(w0);
+                v[8 * c8 + 2] = bf16lo(w1); v[8 * c8 + 3] = bf16hi(w1);
+                v[8 * c8 + 4] = bf16lo(w2); v[8 * c8 + 5] = bf16hi(w2);
+                v[8 * c8 + 6] = bf16lo(w3); v[8 * c8 + 7] = bf16hi(w3);
             }
-
-            // 2-3. block amax (shuffles across the 2 or 4 lanes of the block)
-            float am = 0.0f;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) am = fmaxf(am, fabsf(v[e]));
             if constexpr (AMAX_ONLY) {
-                amax_acc = fmaxf(amax_acc, am);
-                continue;
+                Group<kNvfp4, kRtn, NH>::rotate(v, p.signs);
+#pragma unroll
+                for (int e = 0; e < G; ++e) amax_acc = fmaxf(amax_acc, fabsf(v[e]));
             } else {
-                am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
-                if constexpr (NB == 32) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 2));
-                float rmul, S;
-                uint32_t scode = block_scale<FMT>(am, s_enc, rmul, S);
-
-                // 4. scaled values and element rounding
-                float u[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) u[e] = __fmul_rn(v[e], rmul);
-                uint32_t codes;
-                if constexpr (RND == kSr) {
-                    const uint64_t i0 = (uint64_t)row * (uint64_t)p.k + (uint64_t)col;
-                    const uint4 w0 = philox_quad(p.sr_seed, p.sr_tag_elem, i0 >> 2);
-                    const uint4 w1 = philox_quad(p.sr_seed, p.sr_tag_elem, (i0 >> 2) + 1);
-                    float y[8];
-                    y[0] = e2m1_sr_value(u[0], uniform24(w0.x));
-                    y[1] = e2m1_sr_value(u[1], uniform24(w0.y));
-                    y[2] = e2m1_sr_value(u[2], uniform24(w0.z));
-                    y[3] = e2m1_sr_value(u[3], uniform24(w0.w));
-                    y[4] = e2m1_sr_value(u[4], uniform24(w1.x));
-                    y[5] = e2m1_sr_value(u[5], uniform24(w1.y));
-                    y[6] = e2m1_sr_value(u[6], uniform24(w1.z));
-                    y[7] = e2m1_sr_value(u[7], uniform24(w1.w));
-                    codes = e2m1x8_rn(y);
-                } else {
-                    codes = e2m1x8_rn(u);
-                }
-                if constexpr (RND == kQuartet2) {
-                    // alpha = T(u*u) / T(u*q): halving-stride tree, the widest strides
-                    // across lanes first, then within the thread.
-                    float sa[8], sb[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        sa[e] = __fmul_rn(u[e], u[e]);
-                        sb[e] = __fmul_rn(u[e], e2m1_decode((codes >> (4 * e)) & 15u));
-                    }
-                    if constexpr (NB == 32) {
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            sa[e] = __fadd_rn(sa[e], __shfl_xor_sync(0xffffffffu, sa[e], 2));
-                            sb[e] = __fadd_rn(sb[e], __shfl_xor_sync(0xffffffffu, sb[e], 2));
-                        }
-                    }
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        sa[e] = __fadd_rn(sa[e], __shfl_xor_sync(0xffffffffu, sa[e], 1));
-                        sb[e] = __fadd_rn(sb[e], __shfl_xor_sync(0xffffffffu, sb[e], 1));
-                    }
-#pragma unroll
-                    for (int st = 4; st >= 1; st >>= 1)
-#pragma unroll
-                        for (int e = 0; e < st; ++e) {
-                            sa[e] = __fadd_rn(sa[e], sa[e + st]);
-                            sb[e] = __fadd_rn(sb[e], sb[e + st]);
-                        }
-                    const uint64_t bidx = (uint64_t)row * (uint64_t)(p.k / NB) + (uint64_t)(col / NB);
-                    scode = quartet2_scale<FMT>(sa[0], sb[0], S, p, bidx);
-                }
-
-                // 5. pack + store (codes of padded rows/columns are not stored)
-                if (col_ok && row < p.rows)
-                    *reinterpret_cast<uint32_t*>(p.codes + row * (p.k / 2) + col / 2) = codes;
-                if ((cc & (NB / 8 - 1)) == 0) scale_stage[atom_offset(r_in_tile, (cc * 8) / NB)] = (uint8_t)scode;
+                Grp::rotate(v, p.signs);
+                const int64_t j0 = col0 + g * G;
+                Grp::quantize(v, s_enc, p, (uint64_t)row * (uint64_t)p.k + (uint64_t)j0,
+                              (uint64_t)row * (uint64_t)(p.k / NB) + (uint64_t)(j0 / NB), srng,
+                              codes + g * (G / 8), scodes + g * (G / NB));
             }
         }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ring.empty[s]);
         if constexpr (!AMAX_ONLY) {
-            __syncthreads();
-            store_atoms(p, scale_stage, kRowTileCols / (4 * NB), row0, col0 / NB);
-            __syncthreads();
-        }
-    }
-
-    if constexpr (AMAX_ONLY) {
+            if (row < p.rows) {
+                uint8_t* dst = p.codes + row * (p.k / 2) + col0 / 2;
+                if (col0 + kRowTileCols <= p.k) {
+                    reinterpret_cast<uint4*>(dst)[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+                    reinterpret_cast<uint4*>(dst)[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
+                } else {
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) amax_acc = fmaxf(amax_acc, __shfl_xor_sync(0xffffffffu, amax_acc, o));
-        if ((tid & 31) == 0) red[tid >> 5] = amax_acc;
-        __syncthreads();
-        if (tid == 0) {
-            float m = 0.0f;
-            for (int w = 0; w < kThreads / 32; ++w) m = fmaxf(m, red[w]);
-            p.amax_out[blockIdx.x] = m;
+                    for (int w = 0; w < 8; ++w)
+                        if (col0 + 8 * w < p.k) reinterpret_cast<uint32_t*>(dst)[w] = codes[w];
+                }
+            }
+            if (row < rows_pad) {
+                // this row's 64 / NB scale bytes: a whole 4-byte atom word (NVFP4) or
+                // half of one (MXFP4); past the last column tile the rest of the word
+                // is padding and is written as zero.
+                const int64_t kb0 = col0 / NB;
+                const int64_t off =
+                    ((row / 128) * (p.kb4 / 4) + kb0 / 4) * 512 + (row % 32) * 16 + ((row / 32) % 4) * 4;
+                if constexpr (NB == 16) {
+                    *reinterpret_cast<uint32_t*>(p.scales + off) =
+                        scodes[0] | (scodes[1] << 8) | (scodes[2] << 16) | (scodes[3] << 24);
+                } else {
+                    const uint32_t half = scodes[0] | (scodes[1] << 8);
+                    if ((kb0 & 3) == 0 && col0 + kRowTileCols >= p.k)
+                        *reinterpret_cast<uint32_t*>(p.scales + off) = half;
+                    else
+                        *reinterpret_cast<uint16_t*>(p.scales + off + (kb0 & 3)) = (uint16_t)half;
+                }
+            }
         }
     }
+    if constexpr (AMAX_ONLY) write_partial(amax_acc, red, p.amax_out);
 }
 
 // ===========================================================================
@@ -337,17 +419,21 @@ __global__ void __launch_bounds__(kThreads) quant_row_kernel(const QuantParams p
 // (columns, k, r/G, m, u) delivers rows in this order, so the 8 rows one
 // ldmatrix phase reads have s % 8 = k + 2q all distinct: with the 128-byte
 // swizzle (16-byte chunk index XOR s % 8) they hit 8 different bank groups.
-template <int FMT, int RND, int NH, bool AMAX_ONLY>
-__global__ void __launch_bounds__(kThreads) quant_col_kernel(const __grid_constant__ CUtensorMap tmap,
-                                                             const QuantParams p) {
-    constexpr int NB = AMAX_ONLY ? 16 : ((FMT == kNvfp4) ? 16 : 32);
-    constexpr int G = (NH > NB) ? NH : NB;
+// Lane l of an ldmatrix.x4 supplies row l % 8 of matrix l / 8, i.e. smem row
+// s = l + 32u; after the transposing load, lane (c = l / 4, q = l % 4) holds
+// x-rows Gq + 8u + [0, 8) of column c.
+template <int FMT, int RND, int NH, bool AMAX_ONLY, int STAGES>
+__global__ void __launch_bounds__(kThreads, 2)
+    quant_col_kernel(const __grid_constant__ CUtensorMap tmap, const QuantParams p) {
+    using Grp = Group<FMT, RND, NH>;
+    constexpr int NB = Grp::NB;
+    constexpr int G = AMAX_ONLY ? ((NH > 16) ? NH : 16) : Grp::G;
     constexpr int TILE_ROWS = 4 * G;
     constexpr int BOX_BYTES = TILE_ROWS * 64 * 2;
+    constexpr int STAGE_BYTES = 2 * BOX_BYTES;
     extern __shared__ __align__(1024) uint8_t dyn_smem[];
-    uint8_t* tile = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
-    __shared__ __align__(16) uint8_t scale_stage[1024];
-    __shared__ __align__(8) uint64_t bar;
+    uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
+    __shared__ Ring<STAGES> ring;
     __shared__ float red[33];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -356,210 +442,164 @@ __global__ void __launch_bounds__(kThreads) quant_col_kernel(const __grid_consta
 
     if (tid == 0) {
         prefetch_tmap(&tmap);
-        mbar_init(&bar, 1);
-        fence_mbarrier_init();
+        ring_init(ring);
     }
     __syncthreads();
-
     float s_enc = 1.0f;
     if constexpr (!AMAX_ONLY && FMT == kNvfp4) s_enc = nvfp4_encode_scale(p, red, blockIdx.x == 0);
     if constexpr (!AMAX_ONLY && FMT == kMxfp4) {
         if (blockIdx.x == 0 && tid == 0) *p.tensor_scale = 1.0f;
     }
-    float amax_acc = 0.0f;
-    uint32_t phase = 0;
-    bool ok = true;
 
-    for (int64_t tile_id = blockIdx.x; tile_id < tiles_total; tile_id += gridDim.x) {
-        const int64_t c0 = (tile_id % tiles_c) * kColTileCols;
-        const int64_t tr = tile_id / tiles_c;
-        const int64_t r0 = tr * TILE_ROWS;
-        if (tid == 0) {
-            mbar_arrive_expect_tx(&bar, 2 * BOX_BYTES);
-            tma_load_5d(tile, &tmap, &bar, (int32_t)c0, 0, (int32_t)(4 * tr), 0, 0);
-            tma_load_5d(tile + BOX_BYTES, &tmap, &bar, (int32_t)(c0 + 64), 0, (int32_t)(4 * tr), 0, 0);
+    if (warp == kComputeWarps) {
+        if (lane == 0) {
+            int i = 0;
+            for (int64_t tile = blockIdx.x; tile < tiles_total; tile += gridDim.x, ++i) {
+                const int s = i % STAGES;
+                if (i >= STAGES && !mbar_wait(&ring.empty[s], ((i / STAGES) + 1) & 1)) break;
+                const int64_t c0 = (tile % tiles_c) * kColTileCols;
+                const int32_t tr4 = (int32_t)(4 * (tile / tiles_c));
+                mbar_arrive_expect_tx(&ring.full[s], STAGE_BYTES);
+                tma_load_5d(tiles + s * STAGE_BYTES, &tmap, &ring.full[s], (int32_t)c0, 0, tr4, 0, 0);
+                tma_load_5d(tiles + s * STAGE_BYTES + BOX_BYTES, &tmap, &ring.full[s], (int32_t)(c0 + 64), 0, tr4, 0,
+                            0);
+            }
         }
-        ok = mbar_wait(&bar, phase);
-        phase ^= 1u;
-        if (!ok) break;
+        return;
+    }
 
-        // ldmatrix lane roles: matrix mm = lane / 8, matrix row pr = lane % 8 -> (q = pr / 2, k = pr % 2)
-        const int mm = lane >> 3, pr = lane & 7;
-        const int s_lane = (pr & 1) + 2 * (pr >> 1) + 8 * mm;  // + 32 u
+    const int64_t rows_pad = (p.rows + 127) / 128 * 128;
+    const int q = lane & 3;
+    float amax_acc = 0.0f;
+    ScaleRng srng;
+    int i = 0;
+    for (int64_t tile = blockIdx.x; tile < tiles_total; tile += gridDim.x, ++i) {
+        const int s = i % STAGES;
+        if (!mbar_wait(&ring.full[s], (i / STAGES) & 1)) break;
+        const int64_t c0 = (tile % tiles_c) * kColTileCols;
+        const int64_t r0 = (tile / tiles_c) * TILE_ROWS;
 #pragma unroll
         for (int ci = 0; ci < 2; ++ci) {
             const int chunk = 2 * warp + ci;  // 16 chunks of 8 columns
             const int box = chunk >> 3, ch = chunk & 7;
-            const uint32_t box_base = smem_u32(tile + box * BOX_BYTES);
+            const uint32_t box_base = smem_u32(tiles + s * STAGE_BYTES + box * BOX_BYTES);
             float v[G];
 #pragma unroll
             for (int u = 0; u < G / 8; ++u) {
-                const int s = s_lane + 32 * u;
-                const uint32_t addr = box_base + s * 128 + ((ch ^ (s & 7)) << 4);
-                uint32_t r0w, r1w, r2w, r3w;
+                const int srow = lane + 32 * u;
+                const uint32_t addr = box_base + srow * 128 + ((ch ^ (srow & 7)) << 4);
+                uint32_t a0, a1, a2, a3;
                 asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
-                             : "=r"(r0w), "=r"(r1w), "=r"(r2w), "=r"(r3w)
+                             : "=r"(a0), "=r"(a1), "=r"(a2), "=r"(a3)
                              : "r"(addr));
-                v[8 * u + 0] = bf16lo(r0w); v[8 * u + 1] = bf16hi(r0w);
-                v[8 * u + 2] = bf16lo(r1w); v[8 * u + 3] = bf16hi(r1w);
-                v[8 * u + 4] = bf16lo(r2w); v[8 * u + 5] = bf16hi(r2w);
-                v[8 * u + 6] = bf16lo(r3w); v[8 * u + 7] = bf16hi(r3w);
+                v[8 * u + 0] = bf16lo(a0); v[8 * u + 1] = bf16hi(a0);
+                v[8 * u + 2] = bf16lo(a1); v[8 * u + 3] = bf16hi(a1);
+                v[8 * u + 4] = bf16lo(a2); v[8 * u + 5] = bf16hi(a2);
+                v[8 * u + 6] = bf16lo(a3); v[8 * u + 7] = bf16hi(a3);
             }
-            // this thread: x column c, group of G consecutive x rows starting at r_grp
-            const int q = lane & 3;
-            const int64_t c = c0 + chunk * 8 + (lane >> 2);
-            const int64_t r_grp = r0 + (int64_t)G * q;
-
-            if constexpr (NH > 0) {
-#pragma unroll
-                for (int hb = 0; hb < G / NH; ++hb) {
-                    float* w = v + hb * NH;
-#pragma unroll
-                    for (int e = 0; e < NH; ++e)
-                        if ((p.signs >> e) & 1u) w[e] = -w[e];
-#pragma unroll
-                    for (int e8 = 0; e8 < NH; e8 += 8) fwht8(w + e8);
-                    fwht_wide<NH>(w);
-#pragma unroll
-                    for (int e = 0; e < NH; ++e) w[e] = __fmul_rn(w[e], had_norm<NH>());
-                }
-            }
-
+            const int64_t c = c0 + chunk * 8 + (lane >> 2);  // x column = output row
+            const int64_t r_grp = r0 + (int64_t)G * q;       // first k index of this group
             if constexpr (AMAX_ONLY) {
+                Group<kNvfp4, kRtn, NH>::rotate(v, p.signs);
 #pragma unroll
                 for (int e = 0; e < G; ++e) amax_acc = fmaxf(amax_acc, fabsf(v[e]));
             } else {
-                const bool store_codes = (c < p.rows) && (r_grp < p.k);
-                const int cl = (int)(c - c0);
-#pragma unroll
-                for (int b = 0; b < G / NB; ++b) {
-                    const float* vb = v + b * NB;
-                    float am = 0.0f;
-#pragma unroll
-                    for (int e = 0; e < NB; ++e) am = fmaxf(am, fabsf(vb[e]));
-                    float rmul, S;
-                    uint32_t scode = block_scale<FMT>(am, s_enc, rmul, S);
-                    float u[NB];
-#pragma unroll
-                    for (int e = 0; e < NB; ++e) u[e] = __fmul_rn(vb[e], rmul);
-                    const int64_t kbase = r_grp + b * NB;  // first k index of the block
-                    uint32_t codes[NB / 8];
-                    if constexpr (RND == kSr) {
-                        const uint64_t i0 = (uint64_t)c * (uint64_t)p.k + (uint64_t)kbase;
-#pragma unroll
-                        for (int e8 = 0; e8 < NB; e8 += 8) {
-                            const uint4 w0 = philox_quad(p.sr_seed, p.sr_tag_elem, (i0 + e8) >> 2);
-                            const uint4 w1 = philox_quad(p.sr_seed, p.sr_tag_elem, ((i0 + e8) >> 2) + 1);
-                            float y[8];
-                            y[0] = e2m1_sr_value(u[e8 + 0], uniform24(w0.x));
-                            y[1] = e2m1_sr_value(u[e8 + 1], uniform24(w0.y));
-                            y[2] = e2m1_sr_value(u[e8 + 2], uniform24(w0.z));
-                            y[3] = e2m1_sr_value(u[e8 + 3], uniform24(w0.w));
-                            y[4] = e2m1_sr_value(u[e8 + 4], uniform24(w1.x));
-                            y[5] = e2m1_sr_value(u[e8 + 5], uniform24(w1.y));
-                            y[6] = e2m1_sr_value(u[e8 + 6], uniform24(w1.z));
-                            y[7] = e2m1_sr_value(u[e8 + 7], uniform24(w1.w));
-                            codes[e8 / 8] = e2m1x8_rn(y);
-                        }
+                uint32_t codes[G / 8];
+                uint32_t scodes[G / NB];
+                Grp::rotate(v, p.signs);
+                Grp::quantize(v, s_enc, p, (uint64_t)c * (uint64_t)p.k + (uint64_t)r_grp,
+                              (uint64_t)c * (uint64_t)(p.k / NB) + (uint64_t)(r_grp / NB), srng, codes, scodes);
+                if (c < p.rows && r_grp < p.k) {
+                    uint8_t* dst = p.codes + c * (p.k / 2) + r_grp / 2;
+                    if constexpr (G == 16)
+                        *reinterpret_cast<uint2*>(dst) = make_uint2(codes[0], codes[1]);
+                    else
+                        *reinterpret_cast<uint4*>(dst) = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+                }
+                // Scales: the 4 lanes of column c (q = 0..3, consecutive lanes) hold
+                // scale columns kb0 + (G/NB) q + b; gather them into 4-byte atom words.
+                const int64_t kb0 = r0 / NB;
+                uint32_t mine = scodes[0];
+                if constexpr (G / NB == 2) mine |= scodes[1] << 8;
+                const uint32_t n1 = __shfl_down_sync(0xffffffffu, mine, 1);
+                const uint32_t n2 = __shfl_down_sync(0xffffffffu, mine, 2);
+                const uint32_t n3 = __shfl_down_sync(0xffffffffu, mine, 3);
+                if (c < rows_pad) {
+                    const int64_t rowoff = (c / 128) * (p.kb4 / 4) * 512 + (c % 32) * 16 + ((c / 32) % 4) * 4;
+                    if constexpr (G / NB == 1) {
+                        if (q == 0 && kb0 / 4 < p.kb4 / 4)
+                            *reinterpret_cast<uint32_t*>(p.scales + rowoff + (kb0 / 4) * 512) =
+                                mine | (n1 << 8) | (n2 << 16) | (n3 << 24);
                     } else {
-#pragma unroll
-                        for (int e8 = 0; e8 < NB; e8 += 8) codes[e8 / 8] = e2m1x8_rn(u + e8);
+                        if ((q == 0 || q == 2) && kb0 / 4 + q / 2 < p.kb4 / 4)
+                            *reinterpret_cast<uint32_t*>(p.scales + rowoff + (kb0 / 4 + q / 2) * 512) =
+                                mine | (n1 << 16);
                     }
-                    if constexpr (RND == kQuartet2) {
-                        float sa[NB], sb[NB];
-#pragma unroll
-                        for (int e = 0; e < NB; ++e) {
-                            sa[e] = __fmul_rn(u[e], u[e]);
-                            sb[e] = __fmul_rn(u[e], e2m1_decode((codes[e / 8] >> (4 * (e & 7))) & 15u));
-                        }
-#pragma unroll
-                        for (int st = NB / 2; st >= 1; st >>= 1)
-#pragma unroll
-                            for (int e = 0; e < st; ++e) {
-                                sa[e] = __fadd_rn(sa[e], sa[e + st]);
-                                sb[e] = __fadd_rn(sb[e], sb[e + st]);
-                            }
-                        const uint64_t bidx = (uint64_t)c * (uint64_t)(p.k / NB) + (uint64_t)(kbase / NB);
-                        scode = quartet2_scale<FMT>(sa[0], sb[0], S, p, bidx);
-                    }
-                    if (store_codes) {
-                        uint8_t* dst = p.codes + c * (p.k / 2) + kbase / 2;
-                        if constexpr (NB == 16)
-                            *reinterpret_cast<uint2*>(dst) = make_uint2(codes[0], codes[1]);
-                        else
-                            *reinterpret_cast<uint4*>(dst) = make_uint4(codes[0], codes[1], codes[2], codes[3]);
-                    }
-                    scale_stage[atom_offset(cl, (G * q) / NB + b)] = (uint8_t)scode;
                 }
             }
         }
-        __syncthreads();  // all ldmatrix reads done before the next TMA overwrites the tile
-        if constexpr (!AMAX_ONLY) {
-            store_atoms(p, scale_stage, G / NB, c0, r0 / NB);
-            __syncthreads();
-        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ring.empty[s]);
     }
-
-    if constexpr (AMAX_ONLY) {
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) amax_acc = fmaxf(amax_acc, __shfl_xor_sync(0xffffffffu, amax_acc, o));
-        if (lane == 0) red[warp] = amax_acc;
-        __syncthreads();
-        if (tid == 0) {
-            float m = 0.0f;
-            for (int w = 0; w < kThreads / 32; ++w) m = fmaxf(m, red[w]);
-            p.amax_out[blockIdx.x] = m;
-        }
-    }
+    if constexpr (AMAX_ONLY) write_partial(amax_acc, red, p.amax_out);
 }
 
-template <int FMT, int RND, int NH>
-cudaError_t launch_quant_t(const QuantParams& p, int axis, const CUtensorMap* tmap, cudaStream_t s) {
-    if (axis == 0) {
-        const int64_t tiles = ((p.rows + kRowTileRows - 1) / kRowTileRows) * ((p.k + kRowTileCols - 1) / kRowTileCols);
-        quant_row_kernel<FMT, RND, NH, false><<<(unsigned)tiles, kThreads, 0, s>>>(p);
-    } else {
-        constexpr int NB = (FMT == kNvfp4) ? 16 : 32;
-        constexpr int G = (NH > NB) ? NH : NB;
-        const int64_t tiles = ((p.rows + kColTileCols - 1) / kColTileCols) * ((p.k + 4 * G - 1) / (4 * G));
-        const int smem = 2 * (4 * G * 64 * 2) + 1024;
-        auto kern = quant_col_kernel<FMT, RND, NH, false>;
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
-        kern<<<(unsigned)tiles, kThreads, smem, s>>>(*tmap, p);
-    }
+int g_sm_count = 0;
+
+int persistent_grid(int64_t tiles, int per_sm) {
+    const int sms = g_sm_count > 0 ? g_sm_count : 148;
+    int64_t g = (int64_t)sms * per_sm;
+    if (g > tiles) g = tiles;
+    return g < 1 ? 1 : (int)g;
+}
+
+template <typename Kern>
+cudaError_t launch_persistent(Kern kern, int grid, int smem, const CUtensorMap& tmap, const QuantParams& p,
+                              cudaStream_t s) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, kThreads, smem, s>>>(tmap, p);
     count_launch();
     return cudaGetLastError();
+}
+
+constexpr int kRowStages = 3;
+template <int G>
+constexpr int col_stages() {
+    return G == 16 ? 4 : 3;
+}
+
+template <int FMT, int RND, int NH, bool AMAX_ONLY>
+cudaError_t launch_t(const QuantParams& p, int axis, const CUtensorMap* tmap, int grid, cudaStream_t s) {
+    if (axis == 0) {
+        const int64_t tiles =
+            ((p.rows + kRowTileRows - 1) / kRowTileRows) * ((p.k + kRowTileCols - 1) / kRowTileCols);
+        if (grid <= 0) grid = persistent_grid(tiles, 2);
+        const int smem = kRowStages * kRowTileRows * kRowTileCols * 2 + 1024;
+        return launch_persistent(quant_row_kernel<FMT, RND, NH, AMAX_ONLY, kRowStages>, grid, smem, *tmap, p, s);
+    } else {
+        constexpr int NB = (FMT == kNvfp4) ? 16 : 32;
+        constexpr int G = AMAX_ONLY ? ((NH > 16) ? NH : 16) : ((NH > NB) ? NH : NB);
+        constexpr int S = col_stages<G>();
+        const int64_t tiles = ((p.rows + kColTileCols - 1) / kColTileCols) * ((p.k + 4 * G - 1) / (4 * G));
+        if (grid <= 0) grid = persistent_grid(tiles, 2);
+        const int smem = S * 2 * (4 * G * 64 * 2) + 1024;
+        return launch_persistent(quant_col_kernel<FMT, RND, NH, AMAX_ONLY, S>, grid, smem, *tmap, p, s);
+    }
 }
 
 template <int FMT, int RND>
 cudaError_t dispatch_nh(const QuantParams& p, int nh, int axis, const CUtensorMap* tmap, cudaStream_t s) {
     switch (nh) {
-        case 0: return launch_quant_t<FMT, RND, 0>(p, axis, tmap, s);
-        case 16: return launch_quant_t<FMT, RND, 16>(p, axis, tmap, s);
-        default: return launch_quant_t<FMT, RND, 32>(p, axis, tmap, s);
+        case 0: return launch_t<FMT, RND, 0, false>(p, axis, tmap, 0, s);
+        case 16: return launch_t<FMT, RND, 16, false>(p, axis, tmap, 0, s);
+        default: return launch_t<FMT, RND, 32, false>(p, axis, tmap, 0, s);
     }
-}
-
-template <int NH>
-cudaError_t launch_amax_t(const QuantParams& p, int axis, const CUtensorMap* tmap, int n_partials, cudaStream_t s) {
-    if (axis == 0) {
-        quant_row_kernel<kNvfp4, kRtn, NH, true><<<n_partials, kThreads, 0, s>>>(p);
-    } else {
-        constexpr int G = (NH > 16) ? NH : 16;
-        const int smem = 2 * (4 * G * 64 * 2) + 1024;
-        auto kern = quant_col_kernel<kNvfp4, kRtn, NH, true>;
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
-        kern<<<n_partials, kThreads, smem, s>>>(*tmap, p);
-    }
-    count_launch();
-    return cudaGetLastError();
 }
 
 // Max of n partial maxima (one CTA).
-__global__ void __launch_bounds__(kThreads) reduce_max_kernel(const float* in, int n, float* out) {
-    __shared__ float red[33];
+__global__ void __launch_bounds__(256) reduce_max_kernel(const float* in, int n, float* out) {
+    __shared__ float red[8];
     float m = 0.0f;
     for (int i = threadIdx.x; i < n; i += blockDim.x) m = fmaxf(m, in[i]);
 #pragma unroll
@@ -567,15 +607,22 @@ __global__ void __launch_bounds__(kThreads) reduce_max_kernel(const float* in, i
     if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
     __syncthreads();
     if (threadIdx.x == 0) {
-        for (int w = 1; w < kThreads / 32; ++w) m = fmaxf(m, red[w]);
+        for (int w = 1; w < 8; ++w) m = fmaxf(m, red[w]);
         *out = fmaxf(m, red[0]);
     }
 }
 
 }  // namespace
 
+void set_sm_count(int sms) { g_sm_count = sms; }
+
+int64_t quant_tiles(int axis, int64_t rows, int64_t k, int G) {
+    if (axis == 0) return ((rows + kRowTileRows - 1) / kRowTileRows) * ((k + kRowTileCols - 1) / kRowTileCols);
+    return ((rows + kColTileCols - 1) / kColTileCols) * ((k + 4 * G - 1) / (4 * G));
+}
+
 cudaError_t launch_reduce_max(const float* in, int n, float* out, cudaStream_t s) {
-    reduce_max_kernel<<<1, kThreads, 0, s>>>(in, n, out);
+    reduce_max_kernel<<<1, 256, 0, s>>>(in, n, out);
     count_launch();
     return cudaGetLastError();
 }
@@ -597,9 +644,9 @@ cudaError_t launch_quant(const QuantParams& p, int fmt, int rnd, int nh, int axi
 cudaError_t launch_amax(const QuantParams& p, int axis, int nh, const CUtensorMap* tmap, int n_partials,
                         cudaStream_t s) {
     switch (nh) {
-        case 0: return launch_amax_t<0>(p, axis, tmap, n_partials, s);
-        case 16: return launch_amax_t<16>(p, axis, tmap, n_partials, s);
-        default: return launch_amax_t<32>(p, axis, tmap, n_partials, s);
+        case 0: return launch_t<kNvfp4, kRtn, 0, true>(p, axis, tmap, n_partials, s);
+        case 16: return launch_t<kNvfp4, kRtn, 16, true>(p, axis, tmap, n_partials, s);
+        default: return launch_t<kNvfp4, kRtn, 32, true>(p, axis, tmap, n_partials, s);
     }
 }
 

@@ -72,3 +72,35 @@ def test_linear_rejects_bad_shapes():
     W = torch.zeros((256, 256), dtype=torch.bfloat16, device="cuda")
     with pytest.raises(Q.QFP4Error):
         Q.linear_fwd(X, W, Q.recipe("NVIDIA_NVFP4"), Q.make_seed())
+
+
+def test_calls_from_a_worker_thread():
+    """A thread that never set a device (as a framework's worker thread may be)
+    still runs the library on the caller's stream's context."""
+    import threading
+    wl = inputs.workload("tiny")
+    X, W, dY = (wl[k].cuda() for k in ("X", "W", "dY"))
+    rec = Q.recipe("QUARTET2_NVFP4")
+    seed = Q.make_seed(ROT, SRS)
+    ref_dX, ref_dW = Q.linear_bwd(dY, X, W, rec, seed)
+    torch.cuda.synchronize()
+    out = {}
+
+    def worker():
+        try:
+            s = torch.cuda.Stream(device=X.device)
+            out["dX"], out["dW"] = Q.linear_bwd(dY, X, W, rec, seed, stream=s)
+            s.synchronize()
+            out["dX0"], out["dW0"] = Q.linear_bwd(dY, X, W, rec, seed)  # default stream
+            torch.cuda.synchronize()
+        except Exception as e:  # noqa: BLE001
+            out["err"] = e
+
+    t = threading.Thread(target=worker)
+    t.start()
+    t.join()
+    assert "err" not in out, out.get("err")
+    for k in ("dX", "dX0"):
+        assert torch.equal(out[k], ref_dX)
+    for k in ("dW", "dW0"):
+        assert torch.equal(out[k], ref_dW)
