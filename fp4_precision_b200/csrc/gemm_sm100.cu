@@ -6,22 +6,32 @@
 // "New AMD paper overturns conventional wisdom: FP4 training...", section
 // "Poiskovaya eksperimental'naya rabota").
 //
-// Persistent CTAs (one per SM) walk 128 x 256 tiles of D in a grouped order
-// (8 row-tiles at a time, so concurrent CTAs share A and B tiles in L2) with
-// tcgen05.mma (kind::mxf4nvf4 with scale_vec::4X for NVFP4, kind::mxf4 with
-// scale_vec::2X for MXFP4), M = 128, N = 256, K = 64 per instruction, fp32
-// accumulator in tensor memory:
-//   warp 0, one lane: TMA producer. Per 256-wide k-tile it loads the A and B
-//     tiles (128-byte swizzled) and, with plain bulk copies, the scale atoms,
-//     which the quantizers already store in the MMA's 512-byte atom layout,
-//     into a 4-stage shared-memory ring.
-//   warp 1, one lane: MMA issuer. Per k-tile it copies the scale atoms to
-//     tensor memory (tcgen05.cp 32x128b.warpx4), issues 4 MMAs and commits the
-//     stage back to the producer.
-//   warps 2-9: epilogue. Two warps per 32-lane quarter of tensor memory each
-//     drain 128 accumulator columns into registers (tcgen05.ld), hand the
-//     accumulator back to the MMA warp, then multiply by gA * gB and store
-//     bf16 or fp32 rows while the next tile's MMAs run.
+// Two kernels share one structure: persistent CTAs (one per SM) walk the
+// output tiles in a grouped order (a few row-tiles at a time, so CTAs running
+// together share A and B tiles in L2) and issue tcgen05.mma (kind::mxf4nvf4,
+// scale_vec::4X for NVFP4; kind::mxf4, scale_vec::2X for MXFP4) with K = 64 per
+// instruction and an fp32 accumulator in tensor memory.
+//   - single CTA: 128 x 256 tiles, M = 128, N = 256;
+//   - CTA pair (default): 256 x 256 tiles on the two SMs of a cluster with
+//     tcgen05.mma.cta_group::2, M = 256, N = 256; each CTA loads half of A and
+//     half of B, so an SM moves 32 KiB of operands per 256-wide k-tile.
+// Warp roles (14 warps):
+//   warp 0, one lane: TMA producer into a shared-memory ring (A and B tiles
+//     with 128-byte swizzle, and the scale atoms, which the quantizers store in
+//     the MMA's 512-byte atom layout).
+//   warp 1, one lane: MMA issuer: 4 MMAs per 256-wide k-tile, then commits the
+//     stage and the scale slot.
+//   warps 2-5: scale writers, one per 32-lane quarter of tensor memory. They
+//     read the k-tile's scale atoms from shared memory and write them into one
+//     of 4 rotating tensor-memory slots with tcgen05.st (each quarter holds the
+//     same 32 atom rows, as the MMA reads them). Measured on B200, the copy
+//     instruction for scales (tcgen05.cp) took ~110 cycles each in the tensor
+//     pipe, 12 per k-tile, more than the 512 cycles of MMA work; the store path
+//     runs beside the MMAs.
+//   warps 6-13: epilogue, two per lane quarter, 128 accumulator columns each:
+//     drain tensor memory to registers (tcgen05.ld), hand the accumulator back
+//     to the MMA warp, multiply by gA * gB and store bf16 or fp32 rows while
+//     the next tile's MMAs run.
 // Every wait is bounded (qfp4_device.cuh); on expiry the kernel raises the
 // device error word and skips the rest of its work.
 #include <cuda_fp16.h>
@@ -33,14 +43,18 @@ namespace qfp4 {
 namespace {
 
 constexpr int BM = kGemmBM, BN = kGemmBN, BK = kGemmBK;  // BK in elements
-constexpr int STAGES = 4;
-constexpr int A_STAGE = BM * BK / 2;  // 16 KiB
-constexpr int B_STAGE = BN * BK / 2;  // 32 KiB
-constexpr int SFA_STAGE = 2048;       // up to 4 atoms
-constexpr int SFB_STAGE = 4096;       // 2 row blocks x up to 4 atoms
 constexpr int TMEM_COLS = 512;
-constexpr int TMEM_D = 0, TMEM_SFA = 256, TMEM_SFB = 272;
-constexpr int SMEM_BYTES = STAGES * (A_STAGE + B_STAGE + SFA_STAGE + SFB_STAGE) + 1024 /*align*/ + 256 /*barriers*/;
+// Tensor-memory columns: the 128 x 256 fp32 accumulator, then NSLOT scale
+// slots of 48 columns (SFA 16, SFB 32).
+constexpr int TMEM_D = 0;
+constexpr int NSLOT = 4;
+__device__ __forceinline__ uint32_t sfa_col(int slot) { return 256u + 48u * (uint32_t)slot; }
+__device__ __forceinline__ uint32_t sfb_col(int slot) { return 256u + 48u * (uint32_t)slot + 16u; }
+
+constexpr int kScaleWarps = 4;
+constexpr int kEpiWarps = 8;
+constexpr int kFirstScaleWarp = 2, kFirstEpiWarp = 6;
+constexpr int kGemmThreads = (2 + kScaleWarps + kEpiWarps) * 32;
 
 // Shared-memory matrix descriptor (tcgen05): K-major, 128-byte swizzle, rows
 // 128 bytes apart, 8-row groups 1024 bytes apart, descriptor version 1.
@@ -54,52 +68,36 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
     return d;
 }
 
-// Descriptor of a 32-row x 16-byte contiguous matrix (a scale atom) for tcgen05.cp:
-// no swizzle, 8-row core matrices 128 bytes apart.
-__device__ __forceinline__ uint64_t atom_desc(uint32_t saddr) {
-    uint64_t d = 0;
-    d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
-    d |= (uint64_t)(128 >> 4) << 16;   // leading byte offset
-    d |= (uint64_t)(128 >> 4) << 32;   // stride byte offset
-    d |= (uint64_t)1 << 46;
-    return d;
-}
-
 // Instruction descriptor of the block-scaled MMA: E2M1 x E2M1, K-major
 // operands, M = 128, N = 256, scale type E4M3 (NVFP4) or E8M0 (MXFP4), and the
 // byte of the 32-bit scale column each operand's scales start at.
-template <int FMT>
-__device__ __forceinline__ uint32_t idesc(uint32_t a_sf_id, uint32_t b_sf_id) {
+template <int FMT, int MM, int NN>
+__device__ __forceinline__ uint32_t idesc_mn(uint32_t a_sf_id, uint32_t b_sf_id) {
     uint32_t d = 0;
     d |= (b_sf_id & 3u) << 4;
     d |= 1u << 7;                 // A: E2M1
     d |= 1u << 10;                // B: E2M1
-    d |= (uint32_t)(BN >> 3) << 17;
+    d |= (uint32_t)(NN >> 3) << 17;
     d |= (FMT == kMxfp4 ? 1u : 0u) << 23;
-    d |= (uint32_t)(BM >> 4) << 24;
+    d |= (uint32_t)(MM >> 4) << 24;
     d |= (a_sf_id & 3u) << 29;
     return d;
 }
-
-template <int FMT>
+// tcgen05.mma with block scaling, for one CTA or (PAIR) a CTA pair.
+#define QFP4_MMA_ASM(GROUP, KIND)                                                                                     \
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %6, 0;\n\t"                                                      \
+                 "tcgen05.mma.cta_group::" GROUP ".kind::" KIND " [%0], %1, %2, %3, [%4], [%5], p;\n\t}" ::"r"(d_tmem), \
+                 "l"(a_desc), "l"(b_desc), "r"(id), "r"(sfa), "r"(sfb), "r"(accumulate)                               \
+                 : "memory")
+template <int FMT, bool PAIR>
 __device__ __forceinline__ void mma_bs(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t id, uint32_t sfa,
                                        uint32_t sfb, uint32_t accumulate) {
-    if constexpr (FMT == kNvfp4) {
-        asm volatile(
-            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %6, 0;\n\t"
-            "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%4], [%5], p;\n\t}" ::"r"(
-                d_tmem),
-            "l"(a_desc), "l"(b_desc), "r"(id), "r"(sfa), "r"(sfb), "r"(accumulate)
-            : "memory");
-    } else {
-        asm volatile(
-            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %6, 0;\n\t"
-            "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.scale_vec::2X [%0], %1, %2, %3, [%4], [%5], p;\n\t}" ::"r"(
-                d_tmem),
-            "l"(a_desc), "l"(b_desc), "r"(id), "r"(sfa), "r"(sfb), "r"(accumulate)
-            : "memory");
-    }
+    if constexpr (FMT == kNvfp4 && !PAIR) QFP4_MMA_ASM("1", "mxf4nvf4.block_scale.scale_vec::4X");
+    if constexpr (FMT == kNvfp4 && PAIR) QFP4_MMA_ASM("2", "mxf4nvf4.block_scale.scale_vec::4X");
+    if constexpr (FMT == kMxfp4 && !PAIR) QFP4_MMA_ASM("1", "mxf4.block_scale.scale_vec::2X");
+    if constexpr (FMT == kMxfp4 && PAIR) QFP4_MMA_ASM("2", "mxf4.block_scale.scale_vec::2X");
 }
+#undef QFP4_MMA_ASM
 
 // 32 lanes x 32 consecutive fp32 columns of TMEM into registers (no wait).
 __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t* r) {
@@ -113,20 +111,151 @@ __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t* r) 
         : "r"(taddr));
 }
 
-// Persistent tile order: groups of GROUP_M row-tiles, walking down the group
-// first, so the CTAs running at one time share both A and B tiles in L2.
-constexpr int GROUP_M = 8;
+// Registers of 32 lanes into 8 / 16 / 32 consecutive 32-bit TMEM columns.
+__device__ __forceinline__ void tmem_st_x8(uint32_t taddr, const uint32_t* r) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr), "r"(r[0]),
+                 "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_st_x16(uint32_t taddr, const uint32_t* r) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+        "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_st_x32(uint32_t taddr, const uint32_t* r) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+        "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]),
+        "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]),
+        "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+__device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ uint4 lds128(uint32_t saddr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(saddr));
+    return v;
+}
+
+// Scale writer: lane i of the warp for lane quarter q copies row i of every
+// scale atom of the k-tile from shared memory into its TMEM lane 32q + i.
+// SFA atom a -> columns sfa_col + 4a; SFB atom a of row block rb -> columns
+// sfb_col + 8a + 4rb (the layout of tcgen05.cp 32x128b.warpx4).
+template <int ATOMS>
+__device__ __forceinline__ void write_scales(uint32_t tmem_lane, int slot, uint32_t sfa_smem, uint32_t sfb_smem,
+                                             int lane) {
+    uint32_t ra[4 * ATOMS], rb[8 * ATOMS];
+#pragma unroll
+    for (int a = 0; a < ATOMS; ++a) {
+        const uint4 v = lds128(sfa_smem + a * 512 + lane * 16);
+        ra[4 * a + 0] = v.x; ra[4 * a + 1] = v.y; ra[4 * a + 2] = v.z; ra[4 * a + 3] = v.w;
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            const uint4 w = lds128(sfb_smem + r * (ATOMS * 512) + a * 512 + lane * 16);
+            rb[8 * a + 4 * r + 0] = w.x; rb[8 * a + 4 * r + 1] = w.y;
+            rb[8 * a + 4 * r + 2] = w.z; rb[8 * a + 4 * r + 3] = w.w;
+        }
+    }
+    if constexpr (ATOMS == 4) {
+        tmem_st_x16(tmem_lane + sfa_col(slot), ra);
+        tmem_st_x32(tmem_lane + sfb_col(slot), rb);
+    } else {
+        tmem_st_x8(tmem_lane + sfa_col(slot), ra);
+        tmem_st_x16(tmem_lane + sfb_col(slot), rb);
+    }
+    tc_wait_st();
+}
+
+// Epilogue store of 64 accumulator columns of row `row` from column `n0`:
+// times gA * gB, as bf16 or fp32, with evict-first stores so the output stream
+// does not push the operand tiles out of L2.
+__device__ __forceinline__ void store64(const GemmParams& p, const uint32_t* acc, int row, int n0, float scale) {
+    if (row >= p.M) return;
+    if (p.out_f32) {
+        float* dst = reinterpret_cast<float*>(p.D) + (int64_t)row * p.ldd + n0;
+#pragma unroll
+        for (int c = 0; c < 64; c += 4) {
+            const float4 v4 = make_float4(__fmul_rn(__uint_as_float(acc[c]), scale),
+                                          __fmul_rn(__uint_as_float(acc[c + 1]), scale),
+                                          __fmul_rn(__uint_as_float(acc[c + 2]), scale),
+                                          __fmul_rn(__uint_as_float(acc[c + 3]), scale));
+            if (n0 + c + 4 <= p.N) {
+                __stcs(reinterpret_cast<float4*>(dst + c), v4);
+            } else {
+                if (n0 + c < p.N) dst[c] = v4.x;
+                if (n0 + c + 1 < p.N) dst[c + 1] = v4.y;
+                if (n0 + c + 2 < p.N) dst[c + 2] = v4.z;
+            }
+        }
+    } else {
+        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.D) + (int64_t)row * p.ldd + n0;
+#pragma unroll
+        for (int c = 0; c < 64; c += 8) {
+            uint32_t w[4];
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                __nv_bfloat162 b2 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(acc[c + 2 * h]), scale),
+                                                          __fmul_rn(__uint_as_float(acc[c + 2 * h + 1]), scale));
+                w[h] = *reinterpret_cast<uint32_t*>(&b2);
+            }
+            if (n0 + c + 8 <= p.N) {
+                __stcs(reinterpret_cast<uint4*>(dst + c), make_uint4(w[0], w[1], w[2], w[3]));
+            } else {
+#pragma unroll
+                for (int h = 0; h < 8; ++h)
+                    if (n0 + c + h < p.N) reinterpret_cast<uint16_t*>(dst)[c + h] = (uint16_t)(w[h >> 1] >> (16 * (h & 1)));
+            }
+        }
+    }
+}
+
+// Epilogue of one tile for one warp: drain 128 accumulator columns of its lane
+// quarter in two halves, releasing the accumulator (release()) as soon as the
+// second half is in registers.
+template <typename Release>
+__device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t taddr, int row, int n0, float scale,
+                                              Release release) {
+    uint32_t acc[64];
+    tmem_ld_32x32b_x32(taddr + 0, acc);
+    tmem_ld_32x32b_x32(taddr + 32, acc + 32);
+    tc_wait_ld();
+    store64(p, acc, row, n0, scale);
+    tmem_ld_32x32b_x32(taddr + 64, acc);
+    tmem_ld_32x32b_x32(taddr + 96, acc + 32);
+    tc_wait_ld();
+    tc_fence_before();
+    __syncwarp();
+    release();
+    store64(p, acc, row, n0 + 64, scale);
+}
+
+// Grouped tile order: GM row-tiles at a time, walking down the group first.
+template <int GM>
 __device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int& mb, int& nb) {
-    const int per_group = GROUP_M * num_n;
-    const int first_m = (t / per_group) * GROUP_M;
-    const int gm = min(num_m - first_m, GROUP_M);
+    const int per_group = GM * num_n;
+    const int first_m = (t / per_group) * GM;
+    const int gm = min(num_m - first_m, GM);
     const int r = t % per_group;
     mb = first_m + r % gm;
     nb = r / gm;
 }
 
-constexpr int kEpiWarps = 8;                      // 2 per TMEM lane quarter, 128 columns each
-constexpr int kGemmThreads = (2 + kEpiWarps) * 32;  // producer, MMA issuer, epilogue
+// ===========================================================================
+// Single-CTA kernel: 128 x 256 tiles.
+// ===========================================================================
+constexpr int STAGES = 4;
+constexpr int A_STAGE = BM * BK / 2;  // 16 KiB
+constexpr int B_STAGE = BN * BK / 2;  // 32 KiB
+constexpr int SFA_STAGE = 2048;       // up to 4 atoms
+constexpr int SFB_STAGE = 4096;       // 2 row blocks x up to 4 atoms
+constexpr int SMEM_BYTES = STAGES * (A_STAGE + B_STAGE + SFA_STAGE + SFB_STAGE) + 1024 + 256;
+constexpr int GROUP_M = 16;
 
 template <int FMT>
 __global__ void __launch_bounds__(kGemmThreads, 1)
@@ -142,7 +271,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint8_t* sSFB = sSFA + STAGES * SFA_STAGE;
     uint64_t* full = reinterpret_cast<uint64_t*>(sSFB + STAGES * SFB_STAGE);
     uint64_t* empty = full + STAGES;
-    uint64_t* acc_full = empty + STAGES;
+    uint64_t* sf_full = empty + STAGES;
+    uint64_t* sf_empty = sf_full + NSLOT;
+    uint64_t* acc_full = sf_empty + NSLOT;
     uint64_t* acc_empty = acc_full + 1;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
 
@@ -157,6 +288,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
+        }
+        for (int s = 0; s < NSLOT; ++s) {
+            mbar_init(&sf_full[s], kScaleWarps);
+            mbar_init(&sf_empty[s], 1);
         }
         mbar_init(acc_full, 1);
         mbar_init(acc_empty, kEpiWarps);
@@ -175,7 +310,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             bool ok = true;
             for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
                 int mb, nb;
-                tile_coords(t, num_m, num_n, mb, nb);
+                tile_coords<GROUP_M>(t, num_m, num_n, mb, nb);
                 const int n0 = nb * BN;
                 const int nrb = (n0 + 128 < p.N) ? 2 : 1;  // B row blocks present in the scale buffer
                 for (int kt = 0; kt < KT; ++kt, ++it) {
@@ -204,113 +339,73 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             int it = 0, lt = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++lt) {
-                // the epilogue has drained the previous tile's accumulator
                 if (lt > 0 && !mbar_wait(acc_empty, (lt - 1) & 1)) break;
                 tc_fence_after();
                 for (int kt = 0; kt < KT; ++kt, ++it) {
-                    const int s = it % STAGES;
-                    if (!mbar_wait(&full[s], (it / STAGES) & 1)) {
+                    const int s = it % STAGES, slot = it % NSLOT;
+                    if (!mbar_wait(&full[s], (it / STAGES) & 1) || !mbar_wait(&sf_full[slot], (it / NSLOT) & 1)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const int kelems = min(BK, p.K - kt * BK);
-                    const int atoms = (kelems + SF_K - 1) / SF_K;
-                    const uint32_t sfa_base = smem_u32(sSFA + s * SFA_STAGE);
-                    const uint32_t sfb_base = smem_u32(sSFB + s * SFB_STAGE);
-                    for (int a = 0; a < atoms; ++a) {
-                        tc_cp_32x128b_warpx4(tmem + TMEM_SFA + 4 * a, atom_desc(sfa_base + a * 512));
-                        tc_cp_32x128b_warpx4(tmem + TMEM_SFB + 8 * a, atom_desc(sfb_base + a * 512));
-                        tc_cp_32x128b_warpx4(tmem + TMEM_SFB + 8 * a + 4,
-                                             atom_desc(sfb_base + ATOMS_PER_KT * 512 + a * 512));
-                    }
+                    const int kblocks = min(BK, p.K - kt * BK) / 64;
                     const uint32_t a_base = smem_u32(sA + s * A_STAGE);
                     const uint32_t b_base = smem_u32(sB + s * B_STAGE);
-                    const int kblocks = kelems / 64;
                     for (int j = 0; j < kblocks; ++j) {
-                        const uint64_t ad = sw128_desc(a_base + j * 32);
-                        const uint64_t bd = sw128_desc(b_base + j * 32);
                         uint32_t sfa_t, sfb_t, id;
                         if constexpr (FMT == kNvfp4) {
-                            sfa_t = tmem + TMEM_SFA + 4 * j;
-                            sfb_t = tmem + TMEM_SFB + 8 * j;
-                            id = idesc<FMT>(0, 0);
+                            sfa_t = tmem + sfa_col(slot) + 4 * j;
+                            sfb_t = tmem + sfb_col(slot) + 8 * j;
+                            id = idesc_mn<FMT, BM, BN>(0, 0);
                         } else {
-                            sfa_t = tmem + TMEM_SFA + 4 * (j >> 1);
-                            sfb_t = tmem + TMEM_SFB + 8 * (j >> 1);
-                            id = idesc<FMT>(2 * (j & 1), 2 * (j & 1));
+                            sfa_t = tmem + sfa_col(slot) + 4 * (j >> 1);
+                            sfb_t = tmem + sfb_col(slot) + 8 * (j >> 1);
+                            id = idesc_mn<FMT, BM, BN>(2 * (j & 1), 2 * (j & 1));
                         }
-                        mma_bs<FMT>(tmem + TMEM_D, ad, bd, id, sfa_t, sfb_t, (kt > 0 || j > 0) ? 1u : 0u);
+                        mma_bs<FMT, false>(tmem + TMEM_D, sw128_desc(a_base + j * 32), sw128_desc(b_base + j * 32), id,
+                                           sfa_t, sfb_t, (kt > 0 || j > 0) ? 1u : 0u);
                     }
                     tc_commit(&empty[s]);
+                    tc_commit(&sf_empty[slot]);
                 }
-                tc_commit(acc_full);  // the tile's accumulator is complete
+                tc_commit(acc_full);
+            }
+        }
+    } else if (warp < kFirstEpiWarp) {
+        // ---------------- scale writers ----------------
+        const uint32_t tmem_lane = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+        int it = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+            for (int kt = 0; kt < KT; ++kt, ++it) {
+                const int s = it % STAGES, slot = it % NSLOT;
+                if (!mbar_wait(&full[s], (it / STAGES) & 1) ||
+                    (it >= NSLOT && !mbar_wait(&sf_empty[slot], ((it / NSLOT) + 1) & 1))) {
+                    ok = false;
+                    break;
+                }
+                write_scales<ATOMS_PER_KT>(tmem_lane, slot, smem_u32(sSFA + s * SFA_STAGE),
+                                           smem_u32(sSFB + s * SFB_STAGE), lane);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sf_full[slot]);
             }
         }
     } else {
-        // ---------------- epilogue: warps 2..9 ----------------
-        const int lq = warp & 3;          // TMEM lane quarter this warp may access
-        const int chalf = (warp - 2) >> 2;  // which 128 accumulator columns
+        // ---------------- epilogue ----------------
+        const int lq = warp & 3;
+        const int chalf = (warp - kFirstEpiWarp) >> 2;
         const float scale = __fmul_rn(__ldg(p.ga), __ldg(p.gb));
         int lt = 0;
         for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++lt) {
             int mb, nb;
-            tile_coords(t, num_m, num_n, mb, nb);
+            tile_coords<GROUP_M>(t, num_m, num_n, mb, nb);
             if (!mbar_wait(acc_full, lt & 1)) break;
             tc_fence_after();
-            uint32_t acc[128];
-            const uint32_t taddr = tmem + ((uint32_t)(lq * 32) << 16) + TMEM_D + chalf * 128;
-            tmem_ld_32x32b_x32(taddr + 0, acc + 0);
-            tmem_ld_32x32b_x32(taddr + 32, acc + 32);
-            tmem_ld_32x32b_x32(taddr + 64, acc + 64);
-            tmem_ld_32x32b_x32(taddr + 96, acc + 96);
-            tc_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(acc_empty);  // the MMA may start the next tile
-
-            const int row = mb * BM + lq * 32 + lane;
-            const int nbase = nb * BN + chalf * 128;
-            if (row < p.M) {
-                if (p.out_f32) {
-                    float* dst = reinterpret_cast<float*>(p.D) + (int64_t)row * p.ldd + nbase;
-#pragma unroll
-                    for (int c = 0; c < 128; c += 4) {
-                        const float4 v4 = make_float4(__fmul_rn(__uint_as_float(acc[c]), scale),
-                                                      __fmul_rn(__uint_as_float(acc[c + 1]), scale),
-                                                      __fmul_rn(__uint_as_float(acc[c + 2]), scale),
-                                                      __fmul_rn(__uint_as_float(acc[c + 3]), scale));
-                        if (nbase + c + 4 <= p.N) {
-                            *reinterpret_cast<float4*>(dst + c) = v4;
-                        } else {
-                            if (nbase + c < p.N) dst[c] = v4.x;
-                            if (nbase + c + 1 < p.N) dst[c + 1] = v4.y;
-                            if (nbase + c + 2 < p.N) dst[c + 2] = v4.z;
-                        }
-                    }
-                } else {
-                    __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.D) + (int64_t)row * p.ldd + nbase;
-#pragma unroll
-                    for (int c = 0; c < 128; c += 8) {
-                        uint32_t w[4];
-#pragma unroll
-                        for (int h = 0; h < 4; ++h) {
-                            __nv_bfloat162 b2 =
-                                __floats2bfloat162_rn(__fmul_rn(__uint_as_float(acc[c + 2 * h]), scale),
-                                                      __fmul_rn(__uint_as_float(acc[c + 2 * h + 1]), scale));
-                            w[h] = *reinterpret_cast<uint32_t*>(&b2);
-                        }
-                        if (nbase + c + 8 <= p.N) {
-                            *reinterpret_cast<uint4*>(dst + c) = make_uint4(w[0], w[1], w[2], w[3]);
-                        } else {
-#pragma unroll
-                            for (int h = 0; h < 8; ++h)
-                                if (nbase + c + h < p.N)
-                                    reinterpret_cast<uint16_t*>(dst)[c + h] = (uint16_t)(w[h >> 1] >> (16 * (h & 1)));
-                        }
-                    }
-                }
-            }
+            epilogue_tile(p, tmem + ((uint32_t)(lq * 32) << 16) + TMEM_D + chalf * 128, mb * BM + lq * 32 + lane,
+                          nb * BN + chalf * 128, scale, [&] {
+                              if (lane == 0) mbar_arrive(acc_empty);
+                          });
         }
     }
 
@@ -320,6 +415,189 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tc_fence_after();
         tmem_dealloc(tmem, TMEM_COLS);
         tmem_relinquish();
+    }
+}
+
+// ===========================================================================
+// CTA-pair kernel: 256 x 256 tiles, tcgen05.mma.cta_group::2.
+// The leader (rank 0) issues the MMAs. The A and B loads of both CTAs complete
+// on the leader's stage barrier; each CTA's scale atoms (its own 128 rows of
+// SFA, all 256 rows of SFB; a 3-D view, out-of-range atoms read as zero)
+// complete on a barrier of its own, which its scale writers wait on before
+// they fill its tensor memory and arrive on the leader's scale-slot barrier.
+// The leader's commits arrive on the barriers of both CTAs.
+// ===========================================================================
+constexpr int P_STAGES = 5;
+constexpr int P_A = 128 * BK / 2;   // 16 KiB: this CTA's A rows
+constexpr int P_B = 128 * BK / 2;   // 16 KiB: this CTA's B rows
+constexpr int P_SFA = 4 * 512;      // up to 4 atoms of this CTA's rows
+constexpr int P_SFB = 2 * 4 * 512;  // 2 row blocks x up to 4 atoms
+constexpr int P_STAGE = P_A + P_B + P_SFA + P_SFB;
+constexpr int P_SMEM = P_STAGES * P_STAGE + 1024 + 512;
+constexpr int P_GROUP_M = 4;  // 256-row tiles per group of the tile order
+
+template <int FMT>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+    gemm_bs_fp4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                            const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
+                            const GemmParams p) {
+    constexpr int SF_K = (FMT == kNvfp4) ? 64 : 128;
+    constexpr int ATOMS_PER_KT = BK / SF_K;  // 4 or 2
+    constexpr uint32_t AB_TX = 2u * (P_A + P_B);            // both CTAs, on the leader
+    constexpr uint32_t SF_TX = 3u * ATOMS_PER_KT * 512u;    // this CTA's scale boxes
+    extern __shared__ __align__(1024) uint8_t dyn_smem[];
+    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
+    uint8_t* sA = base;
+    uint8_t* sB = sA + P_STAGES * P_A;
+    uint8_t* sSFA = sB + P_STAGES * P_B;
+    uint8_t* sSFB = sSFA + P_STAGES * P_SFA;
+    uint64_t* full = reinterpret_cast<uint64_t*>(sSFB + P_STAGES * P_SFB);
+    uint64_t* empty = full + P_STAGES;
+    uint64_t* sf_load = empty + P_STAGES;
+    uint64_t* sf_full = sf_load + P_STAGES;
+    uint64_t* sf_empty = sf_full + NSLOT;
+    uint64_t* acc_full = sf_empty + NSLOT;
+    uint64_t* acc_empty = acc_full + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const int KT = (p.K + BK - 1) / BK;
+    const int num_m = (p.M + 2 * BM - 1) / (2 * BM), num_n = (p.N + BN - 1) / BN;
+    const int tiles = num_m * num_n;
+    const int cid = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
+
+    if (threadIdx.x == 0) {
+        prefetch_tmap(&tmA);
+        prefetch_tmap(&tmB);
+        prefetch_tmap(&tmSFA);
+        prefetch_tmap(&tmSFB);
+        for (int s = 0; s < P_STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+            mbar_init(&sf_load[s], 1);
+        }
+        for (int s = 0; s < NSLOT; ++s) {
+            mbar_init(&sf_full[s], 2 * kScaleWarps);
+            mbar_init(&sf_empty[s], 1);
+        }
+        mbar_init(acc_full, 1);
+        mbar_init(acc_empty, 2 * kEpiWarps);
+        fence_mbarrier_init();
+    }
+    if (warp == 0) tmem_alloc_pair(tmem_slot, TMEM_COLS);
+    tc_fence_before();
+    cluster_sync();  // barriers of both CTAs initialised, tensor memory allocated
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ---------------- TMA producer (both CTAs) ----------------
+        if (lane == 0) {
+            int it = 0;
+            bool ok = true;
+            for (int t = cid; t < tiles && ok; t += nclusters) {
+                int mb, nb;
+                tile_coords<P_GROUP_M>(t, num_m, num_n, mb, nb);
+                for (int kt = 0; kt < KT; ++kt, ++it) {
+                    const int s = it % P_STAGES;
+                    if (it >= P_STAGES && !mbar_wait_cluster(&empty[s], ((it / P_STAGES) + 1) & 1)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t bar_leader = mapa_shared(smem_u32(&full[s]), 0);
+                    if (rank == 0) mbar_arrive_expect_tx(&full[s], AB_TX);
+                    tma_load_2d_pair(sA + s * P_A, &tmA, bar_leader, kt * (BK / 2), mb * 2 * BM + (int)rank * BM);
+                    tma_load_2d_pair(sB + s * P_B, &tmB, bar_leader, kt * (BK / 2), nb * BN + (int)rank * 128);
+                    mbar_arrive_expect_tx(&sf_load[s], SF_TX);
+                    tma_load_3d(sSFA + s * P_SFA, &tmSFA, &sf_load[s], 0, kt * ATOMS_PER_KT, 2 * mb + (int)rank);
+                    tma_load_3d(sSFB + s * P_SFB, &tmSFB, &sf_load[s], 0, kt * ATOMS_PER_KT, 2 * nb);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer (leader CTA only) ----------------
+        if (lane == 0 && rank == 0) {
+            int it = 0, lt = 0;
+            bool ok = true;
+            for (int t = cid; t < tiles && ok; t += nclusters, ++lt) {
+                if (lt > 0 && !mbar_wait_cluster(acc_empty, (lt - 1) & 1)) break;
+                tc_fence_after();
+                for (int kt = 0; kt < KT; ++kt, ++it) {
+                    const int s = it % P_STAGES, slot = it % NSLOT;
+                    if (!mbar_wait_cluster(&full[s], (it / P_STAGES) & 1) || !mbar_wait_cluster(&sf_full[slot], (it / NSLOT) & 1)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const int kblocks = min(BK, p.K - kt * BK) / 64;
+                    const uint32_t a_base = smem_u32(sA + s * P_A);
+                    const uint32_t b_base = smem_u32(sB + s * P_B);
+                    for (int j = 0; j < kblocks; ++j) {
+                        uint32_t sfa_t, sfb_t, id;
+                        if constexpr (FMT == kNvfp4) {
+                            sfa_t = tmem + sfa_col(slot) + 4 * j;
+                            sfb_t = tmem + sfb_col(slot) + 8 * j;
+                            id = idesc_mn<FMT, 2 * BM, BN>(0, 0);
+                        } else {
+                            sfa_t = tmem + sfa_col(slot) + 4 * (j >> 1);
+                            sfb_t = tmem + sfb_col(slot) + 8 * (j >> 1);
+                            id = idesc_mn<FMT, 2 * BM, BN>(2 * (j & 1), 2 * (j & 1));
+                        }
+                        mma_bs<FMT, true>(tmem + TMEM_D, sw128_desc(a_base + j * 32), sw128_desc(b_base + j * 32), id,
+                                          sfa_t, sfb_t, (kt > 0 || j > 0) ? 1u : 0u);
+                    }
+                    tc_commit_pair(&empty[s]);       // frees stage s in both CTAs
+                    tc_commit_pair(&sf_empty[slot]);  // frees the scale slot in both CTAs
+                }
+                tc_commit_pair(acc_full);  // both CTAs' accumulators are complete
+            }
+        }
+    } else if (warp < kFirstEpiWarp) {
+        // ---------------- scale writers (both CTAs) ----------------
+        const uint32_t tmem_lane = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+        int it = 0;
+        bool ok = true;
+        for (int t = cid; t < tiles && ok; t += nclusters) {
+            for (int kt = 0; kt < KT; ++kt, ++it) {
+                const int s = it % P_STAGES, slot = it % NSLOT;
+                if (!mbar_wait_cluster(&sf_load[s], (it / P_STAGES) & 1) ||
+                    (it >= NSLOT && !mbar_wait_cluster(&sf_empty[slot], ((it / NSLOT) + 1) & 1))) {
+                    ok = false;
+                    break;
+                }
+                write_scales<ATOMS_PER_KT>(tmem_lane, slot, smem_u32(sSFA + s * P_SFA), smem_u32(sSFB + s * P_SFB),
+                                           lane);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&sf_full[slot]), 0));
+            }
+        }
+    } else {
+        // ---------------- epilogue (both CTAs) ----------------
+        const int lq = warp & 3;
+        const int chalf = (warp - kFirstEpiWarp) >> 2;
+        const float scale = __fmul_rn(__ldg(p.ga), __ldg(p.gb));
+        const uint32_t acc_empty_leader = mapa_shared(smem_u32(acc_empty), 0);
+        int lt = 0;
+        for (int t = cid; t < tiles; t += nclusters, ++lt) {
+            int mb, nb;
+            tile_coords<P_GROUP_M>(t, num_m, num_n, mb, nb);
+            if (!mbar_wait_cluster(acc_full, lt & 1)) break;
+            tc_fence_after();
+            epilogue_tile(p, tmem + ((uint32_t)(lq * 32) << 16) + TMEM_D + chalf * 128,
+                          mb * 2 * BM + (int)rank * BM + lq * 32 + lane, nb * BN + chalf * 128, scale, [&] {
+                              if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
+                          });
+        }
+    }
+
+    tc_fence_before();
+    cluster_sync();  // no CTA leaves while its peer may still signal it
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem, TMEM_COLS);
+        tmem_relinquish_pair();
     }
 }
 
@@ -338,6 +616,28 @@ cudaError_t launch_gemm(const GemmParams& p, int fmt, const CUtensorMap* tmapA, 
         e = cudaFuncSetAttribute(gemm_bs_fp4_kernel<kMxfp4>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
         if (e != cudaSuccess) return e;
         gemm_bs_fp4_kernel<kMxfp4><<<grid, kGemmThreads, SMEM_BYTES, s>>>(*tmapA, *tmapB, p);
+    }
+    count_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gemm_pair(const GemmParams& p, int fmt, const CUtensorMap* tmapA, const CUtensorMap* tmapB,
+                             const CUtensorMap* tmapSFA, const CUtensorMap* tmapSFB, cudaStream_t s, int sms) {
+    const int tiles = ((p.M + 2 * BM - 1) / (2 * BM)) * ((p.N + BN - 1) / BN);
+    int clusters = sms / 2;
+    if (clusters > tiles) clusters = tiles;
+    if (clusters < 1) clusters = 1;
+    cudaError_t e;
+    if (fmt == kNvfp4) {
+        e = cudaFuncSetAttribute(gemm_bs_fp4_pair_kernel<kNvfp4>, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM);
+        if (e != cudaSuccess) return e;
+        gemm_bs_fp4_pair_kernel<kNvfp4><<<2 * clusters, kGemmThreads, P_SMEM, s>>>(*tmapA, *tmapB, *tmapSFA,
+                                                                                   *tmapSFB, p);
+    } else {
+        e = cudaFuncSetAttribute(gemm_bs_fp4_pair_kernel<kMxfp4>, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM);
+        if (e != cudaSuccess) return e;
+        gemm_bs_fp4_pair_kernel<kMxfp4><<<2 * clusters, kGemmThreads, P_SMEM, s>>>(*tmapA, *tmapB, *tmapSFA,
+                                                                                   *tmapSFB, p);
     }
     count_launch();
     return cudaGetLastError();

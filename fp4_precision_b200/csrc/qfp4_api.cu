@@ -7,6 +7,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -178,6 +179,31 @@ int make_codes_tmap(CUtensorMap* tm, const void* codes, int64_t rows, int64_t k,
     return QFP4_OK;
 }
 
+// 3-D view of a scale buffer as uint32 words: (128 words = one 512-byte atom,
+// atoms along k, 128-row blocks), box (128, atoms_per_box, depth). Atoms past
+// the buffer read as zero scales.
+int make_scale_tmap(CUtensorMap* tm, const void* scales, int64_t rows, int64_t atoms_k, int atoms_per_box,
+                    int depth) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return cuda_fail(cudaErrorNotSupported);
+    const cuuint64_t dims[3] = {128, (cuuint64_t)atoms_k, (cuuint64_t)((rows + 127) / 128)};
+    const cuuint64_t strides[2] = {512, (cuuint64_t)atoms_k * 512};
+    const cuuint32_t box[3] = {128, (cuuint32_t)atoms_per_box, (cuuint32_t)depth};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<void*>(scales), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
+    return QFP4_OK;
+}
+
+// The single-CTA GEMM is the default (measured faster on B200); QFP4_GEMM_PAIR=1
+// in the environment (read at each call) selects the CTA-pair kernel.
+bool use_pair_gemm() {
+    const char* e = std::getenv("QFP4_GEMM_PAIR");
+    return e != nullptr && e[0] == '1';
+}
+
 int write_one(float* dst, cudaStream_t s) {
     static const float one = 1.0f;
     cudaError_t e = cudaMemcpyAsync(dst, &one, sizeof(float), cudaMemcpyHostToDevice, s);
@@ -341,9 +367,10 @@ int gemm_impl(const qfp4_tensor* A, const qfp4_tensor* B, void* D, int64_t ldd, 
         return QFP4_ERR_INVALID_ARG;
     if (!aligned16(A->codes) || !aligned16(B->codes) || !aligned16(A->scales) || !aligned16(B->scales))
         return QFP4_ERR_MISALIGNED;
+    const bool pair = use_pair_gemm();
     CUtensorMap tA, tB;
     if ((rc = make_codes_tmap(&tA, A->codes, M, K, kGemmBM))) return rc;
-    if ((rc = make_codes_tmap(&tB, B->codes, N, K, kGemmBN))) return rc;
+    if ((rc = make_codes_tmap(&tB, B->codes, N, K, pair ? 128 : kGemmBN))) return rc;
     GemmParams p{};
     p.sfa = A->scales;
     p.sfb = B->scales;
@@ -355,7 +382,16 @@ int gemm_impl(const qfp4_tensor* A, const qfp4_tensor* B, void* D, int64_t ldd, 
     p.M = (int)M; p.N = (int)N; p.K = (int)K;
     const int NB = block_of(A->fmt);
     p.atoms_k = (int)((K / NB + 3) / 4);
-    cudaError_t e = launch_gemm(p, A->fmt, &tA, &tB, s, sms);
+    cudaError_t e;
+    if (pair) {
+        const int atoms_per_kt = kGemmBK / (4 * NB);
+        CUtensorMap tSFA, tSFB;
+        if ((rc = make_scale_tmap(&tSFA, A->scales, M, p.atoms_k, atoms_per_kt, 1))) return rc;
+        if ((rc = make_scale_tmap(&tSFB, B->scales, N, p.atoms_k, atoms_per_kt, 2))) return rc;
+        e = launch_gemm_pair(p, A->fmt, &tA, &tB, &tSFA, &tSFB, s, sms);
+    } else {
+        e = launch_gemm(p, A->fmt, &tA, &tB, s, sms);
+    }
     return e == cudaSuccess ? QFP4_OK : cuda_fail(e);
 }
 

@@ -63,6 +63,10 @@ struct GemmParams {
 // gemm_sm100.cu
 cudaError_t launch_gemm(const GemmParams& p, int fmt, const CUtensorMap* tmapA, const CUtensorMap* tmapB,
                         cudaStream_t s, int sms);
+// 2-SM (CTA pair) variant; tmapSFA / tmapSFB are 3-D views of the scale
+// buffers (see make_scale_tmap in qfp4_api.cu).
+cudaError_t launch_gemm_pair(const GemmParams& p, int fmt, const CUtensorMap* tmapA, const CUtensorMap* tmapB,
+                             const CUtensorMap* tmapSFA, const CUtensorMap* tmapSFB, cudaStream_t s, int sms);
 constexpr int kGemmBM = 128, kGemmBN = 256, kGemmBK = 256;
 
 void count_launch();

@@ -161,16 +161,19 @@ struct Group {
     static constexpr int NB = (FMT == kNvfp4) ? 16 : 32;
     static constexpr int G = (NH > NB) ? NH : NB;
 
-    __device__ __forceinline__ static void rotate(float* v, uint32_t signs) {
+    // Sign-flip mask of packed bf16 word i of a group (elements 2i, 2i+1 at
+    // bits 15 and 31): the random Hadamard's D applied before widening.
+    __device__ __forceinline__ static uint32_t sign_mask(uint32_t signs, int i) {
+        const int e = (2 * i) % (NH > 0 ? NH : 32);
+        return ((signs >> e) & 1u) << 15 | ((signs >> (e + 1)) & 1u) << 31;
+    }
+
+    // v = c * H * (D x) per n_h chunk; D was applied to the packed words.
+    __device__ __forceinline__ static void rotate(float* v) {
         if constexpr (NH > 0) {
 #pragma unroll
             for (int hb = 0; hb < G / NH; ++hb) {
                 float* w = v + hb * NH;
-                if (signs != 0u) {
-#pragma unroll
-                    for (int e = 0; e < NH; ++e)
-                        w[e] = __uint_as_float(__float_as_uint(w[e]) ^ ((signs << (31 - e)) & 0x80000000u));
-                }
                 fwht<NH>(w);
 #pragma unroll
                 for (int e = 0; e < NH; e += 2) {
@@ -357,17 +360,23 @@ __global__ void __launch_bounds__(kThreads, 2)
                 asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
                              : "=r"(w0), "=r"(w1), "=r"(w2), "=r"(w3)
                              : "r"(sbase + ((chunk ^ (tid & 7)) << 4)));
+                if (NH > 0 && p.signs != 0u) {
+                    w0 ^= Grp::sign_mask(p.signs, 4 * c8 + 0);
+                    w1 ^= Grp::sign_mask(p.signs, 4 * c8 + 1);
+                    w2 ^= Grp::sign_mask(p.signs, 4 * c8 + 2);
+                    w3 ^= Grp::sign_mask(p.signs, 4 * c8 + 3);
+                }
                 v[8 * c8 + 0] = bf16lo(w0); v[8 * c8 + 1] = bf16hi(w0);
                 v[8 * c8 + 2] = bf16lo(w1); v[8 * c8 + 3] = bf16hi(w1);
                 v[8 * c8 + 4] = bf16lo(w2); v[8 * c8 + 5] = bf16hi(w2);
                 v[8 * c8 + 6] = bf16lo(w3); v[8 * c8 + 7] = bf16hi(w3);
             }
             if constexpr (AMAX_ONLY) {
-                Group<kNvfp4, kRtn, NH>::rotate(v, p.signs);
+                Group<kNvfp4, kRtn, NH>::rotate(v);
 #pragma unroll
                 for (int e = 0; e < G; ++e) amax_acc = fmaxf(amax_acc, fabsf(v[e]));
             } else {
-                Grp::rotate(v, p.signs);
+                Grp::rotate(v);
                 const int64_t j0 = col0 + g * G;
                 Grp::quantize(v, s_enc, p, (uint64_t)row * (uint64_t)p.k + (uint64_t)j0,
                               (uint64_t)row * (uint64_t)(p.k / NB) + (uint64_t)(j0 / NB), srng,
@@ -492,6 +501,12 @@ __global__ void __launch_bounds__(kThreads, 2)
                 asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
                              : "=r"(a0), "=r"(a1), "=r"(a2), "=r"(a3)
                              : "r"(addr));
+                if (NH > 0 && p.signs != 0u) {
+                    a0 ^= Grp::sign_mask(p.signs, 4 * u + 0);
+                    a1 ^= Grp::sign_mask(p.signs, 4 * u + 1);
+                    a2 ^= Grp::sign_mask(p.signs, 4 * u + 2);
+                    a3 ^= Grp::sign_mask(p.signs, 4 * u + 3);
+                }
                 v[8 * u + 0] = bf16lo(a0); v[8 * u + 1] = bf16hi(a0);
                 v[8 * u + 2] = bf16lo(a1); v[8 * u + 3] = bf16hi(a1);
                 v[8 * u + 4] = bf16lo(a2); v[8 * u + 5] = bf16hi(a2);
@@ -500,13 +515,13 @@ __global__ void __launch_bounds__(kThreads, 2)
             const int64_t c = c0 + chunk * 8 + (lane >> 2);  // x column = output row
             const int64_t r_grp = r0 + (int64_t)G * q;       // first k index of this group
             if constexpr (AMAX_ONLY) {
-                Group<kNvfp4, kRtn, NH>::rotate(v, p.signs);
+                Group<kNvfp4, kRtn, NH>::rotate(v);
 #pragma unroll
                 for (int e = 0; e < G; ++e) amax_acc = fmaxf(amax_acc, fabsf(v[e]));
             } else {
                 uint32_t codes[G / 8];
                 uint32_t scodes[G / NB];
-                Grp::rotate(v, p.signs);
+                Grp::rotate(v);
                 Grp::quantize(v, s_enc, p, (uint64_t)c * (uint64_t)p.k + (uint64_t)r_grp,
                               (uint64_t)c * (uint64_t)(p.k / NB) + (uint64_t)(r_grp / NB), srng, codes, scodes);
                 if (c < p.rows && r_grp < p.k) {

@@ -188,7 +188,10 @@ int qfp4_quantize(const void* x, int64_t R, int64_t C, int64_t ld, int32_t fmt, 
  * A.rows x B.rows, written as bf16 or fp32 with row stride ldd elements.
  * Requirements: same format, same k (a multiple of 64), same Hadamard (and for
  * a random one, the same rot_seed and rot_stream, so the rotation cancels);
- * D 16-byte aligned and ldd * element size a multiple of 16; ldd >= B.rows. */
+ * D 16-byte aligned and ldd * element size a multiple of 16; ldd >= B.rows.
+ * Kernel: persistent single-CTA 128 x 256 tiles; setting the environment
+ * variable QFP4_GEMM_PAIR=1 selects a CTA-pair kernel (256 x 256 tiles,
+ * tcgen05 cta_group::2) instead (same results within the bound). */
 int qfp4_gemm(const qfp4_tensor* A, const qfp4_tensor* B, void* D, int64_t ldd, int32_t out_dtype, void* stream);
 
 /* ---- linear layer -------------------------------------------------------------

@@ -53,11 +53,21 @@ def check_gemm(A_o, B_o, out_dtype, rows=None, cols=None, rot=(0, 0)):
     return worst
 
 
+@pytest.fixture(params=["pair", "single"])
+def kernel_variant(request, monkeypatch):
+    """Both GEMM kernels: the single-CTA default and the CTA-pair one."""
+    if request.param == "pair":
+        monkeypatch.setenv("QFP4_GEMM_PAIR", "1")
+    else:
+        monkeypatch.delenv("QFP4_GEMM_PAIR", raising=False)
+    return request.param
+
+
 @pytest.mark.parametrize("fmt", [O.NVFP4, O.MXFP4], ids=["nvfp4", "mxfp4"])
 @pytest.mark.parametrize("shape", [(128, 256, 256), (300, 200, 320), (512, 520, 1024), (130, 640, 64),
-                                   (1024, 768, 2048)], ids=lambda s: "x".join(map(str, s)))
+                                   (1024, 768, 2048), (100, 136, 192)], ids=lambda s: "x".join(map(str, s)))
 @pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
-def test_gemm_matches_oracle(fmt, shape, out_dtype):
+def test_gemm_matches_oracle(fmt, shape, out_dtype, kernel_variant):
     M, N, K = shape
     X = inputs.normal_with_outliers((M, K), 21, "ga")
     W = inputs.normal((N, K), 0.02, 21, "gb")
@@ -66,7 +76,7 @@ def test_gemm_matches_oracle(fmt, shape, out_dtype):
     check_gemm(A_o, B_o, out_dtype)
 
 
-def test_gemm_rotated_operands():
+def test_gemm_rotated_operands(kernel_variant):
     """Random-Hadamard operands (same sign vector): the GEMM estimates X W^T."""
     M, N, K = 256, 512, 512
     X = inputs.normal((M, K), 1.0, 22, "ra")
@@ -76,7 +86,7 @@ def test_gemm_rotated_operands():
     check_gemm(A_o, B_o, torch.float32, rot=(9, 1))
 
 
-def test_gemm_qkv_shape_sampled():
+def test_gemm_qkv_shape_sampled(kernel_variant):
     """The QKV-projection Fprop shape, 8192 x 6144 x 4096, in the launch
     configuration the benchmark times: 4096 sampled outputs plus two full
     128 x 128 tiles against fp64 dot products."""
