@@ -475,6 +475,7 @@ const char* qfp4_strerror(int status) {
         case QFP4_ERR_WORKSPACE: return "workspace missing or too small";
         case QFP4_ERR_CUDA: return "CUDA error";
         case QFP4_ERR_TIMEOUT: return "device-side bounded wait expired";
+        case QFP4_ERR_TOO_LARGE: return "problem exceeds the fixed scratch of qfp4_linear_fwd_noalloc (32 MiB)";
         default: return "unknown status";
     }
 }
@@ -645,6 +646,42 @@ int qfp4_status(void* stream) {
         return QFP4_ERR_TIMEOUT;
     }
     return QFP4_OK;
+}
+
+// ---- forward pass without allocation ------------------------------------------
+// The scratch of qfp4_linear_fwd_noalloc: a fixed device array (every GPU that
+// loads the library holds it until the process exits). Host code cannot use
+// the array's name as a device address; its address is looked up once per
+// device with cudaGetSymbolAddress, with that device current.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[QFP4_NOALLOC_SCRATCH_BYTES];
+
+static int noalloc_scratch(void** out) {
+    static std::mutex mu;
+    static void* addr[64] = {nullptr};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (dev < 0 || dev >= 64) return QFP4_ERR_UNSUPPORTED_ARCH;
+    std::lock_guard<std::mutex> lock(mu);
+    if (addr[dev] == nullptr) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return cuda_fail(e);
+        addr[dev] = p;
+    }
+    *out = addr[dev];
+    return QFP4_OK;
+}
+
+int qfp4_linear_fwd_noalloc(const void* X, const void* W, void* Y, int64_t M, int64_t N, int64_t K,
+                            const qfp4_recipe* recipe, const qfp4_seed* seed, void* stream) {
+    int rc = check_linear_args(M, N, K, recipe, seed);
+    if (rc) return rc;
+    if (qfp4_linear_workspace_bytes(0, M, N, K, recipe) > QFP4_NOALLOC_SCRATCH_BYTES) return QFP4_ERR_TOO_LARGE;
+    if ((rc = bind_context(static_cast<cudaStream_t>(stream)))) return rc;
+    void* scratch = nullptr;
+    if ((rc = noalloc_scratch(&scratch))) return rc;
+    return qfp4_linear_fwd(X, W, Y, M, N, K, recipe, seed, scratch, QFP4_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 }  // extern "C"

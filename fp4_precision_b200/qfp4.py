@@ -25,6 +25,8 @@ PRESETS = {"NVIDIA_NVFP4": 0, "QUARTET2_NVFP4": 1, "AMD_MXFP4_H": 2}
 BLOCK = {NVFP4: 16, MXFP4: 32}
 
 OK, ERR_INVALID_ARG, ERR_MISALIGNED, ERR_UNSUPPORTED_ARCH, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT = 0, -1, -2, -3, -4, -5, -6
+ERR_TOO_LARGE = -7
+NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
 class Seed(ctypes.Structure):
@@ -76,6 +78,8 @@ _SIGNATURES = {
                                        ctypes.POINTER(Seed), _VOID, _SZ, _VOID]),
     "qfp4_linear_bwd": (ctypes.c_int, [_VOID, _VOID, _VOID, _VOID, _VOID, _I64, _I64, _I64, ctypes.POINTER(Recipe),
                                        ctypes.POINTER(Seed), _VOID, _SZ, _VOID]),
+    "qfp4_linear_fwd_noalloc": (ctypes.c_int, [_VOID, _VOID, _VOID, _I64, _I64, _I64, ctypes.POINTER(Recipe),
+                                               ctypes.POINTER(Seed), _VOID]),
     "qfp4_status": (ctypes.c_int, [_VOID]),
     "qfp4_launch_count": (_I64, [_I32]),
 }
@@ -232,6 +236,17 @@ def linear_fwd(X, W, rec: Recipe, seed: Seed, Y=None, workspace=None, stream=Non
         workspace = torch.empty((linear_workspace_bytes(False, M, N, K, rec),), dtype=torch.uint8, device=X.device)
     _check(lib().qfp4_linear_fwd(_ptr(X), _ptr(W), _ptr(Y), M, N, K, ctypes.byref(rec), ctypes.byref(seed),
                                  _ptr(workspace), workspace.numel(), _stream(stream)), "qfp4_linear_fwd")
+    return Y
+
+
+def linear_fwd_noalloc(X, W, rec: Recipe, seed: Seed, Y=None, stream=None) -> torch.Tensor:
+    """qfp4_linear_fwd_noalloc: the forward pass with the library's fixed
+    scratch instead of a workspace (the binding allocates Y only if not given)."""
+    M, K = X.shape
+    N = W.shape[0]
+    Y = torch.empty((M, N), dtype=_dtype(rec.y_dtype), device=X.device) if Y is None else Y
+    _check(lib().qfp4_linear_fwd_noalloc(_ptr(X), _ptr(W), _ptr(Y), M, N, K, ctypes.byref(rec), ctypes.byref(seed),
+                                         _stream(stream)), "qfp4_linear_fwd_noalloc")
     return Y
 
 

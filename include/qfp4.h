@@ -52,6 +52,7 @@ extern "C" {
 #define QFP4_ERR_WORKSPACE (-4)        /* workspace missing or smaller than required */
 #define QFP4_ERR_CUDA (-5)             /* a CUDA runtime/driver call failed; see qfp4_last_cuda_error */
 #define QFP4_ERR_TIMEOUT (-6)          /* a device-side bounded wait expired (from qfp4_status) */
+#define QFP4_ERR_TOO_LARGE (-7)        /* the problem needs more than qfp4_linear_fwd_noalloc's fixed scratch */
 
 /* ---- enums ---------------------------------------------------------------- */
 typedef enum { QFP4_NVFP4 = 0, QFP4_MXFP4 = 1 } qfp4_format;
@@ -210,6 +211,32 @@ int qfp4_linear_fwd(const void* X, const void* W, void* Y, int64_t M, int64_t N,
 int qfp4_linear_bwd(const void* dY, const void* X, const void* W, void* dX, void* dW, int64_t M, int64_t N, int64_t K,
                     const qfp4_recipe* recipe, const qfp4_seed* seed, void* workspace, size_t workspace_bytes,
                     void* stream);
+
+/* ---- forward pass without any allocation ----------------------------------
+ * qfp4_linear_fwd_noalloc: the same computation as qfp4_linear_fwd, for
+ * callers that cannot allocate device memory at all: code running under a
+ * memory plan fixed at start-up (a serving runtime or an embedded system that
+ * forbids device allocation after initialisation), a plugin inside a host
+ * framework that owns the allocator and exposes no way to reach it, or a
+ * latency-critical path where a cudaMalloc (which may synchronise the device)
+ * is not acceptable. The caller passes only X, W and Y. The library's own
+ * scratch (the quantized operands and the amax partials) lives in a fixed
+ * array of QFP4_NOALLOC_SCRATCH_BYTES (32 MiB) of device memory that every GPU
+ * loading the library keeps until the process exits; a layer whose
+ * qfp4_linear_workspace_bytes(0, ...) exceeds it is rejected with
+ * QFP4_ERR_TOO_LARGE before anything is launched. The call makes no
+ * cudaMalloc / cudaFree or other allocation.
+ * Set-up: the first call on a device looks up the array's device address (once
+ * per device, with the stream's device current); make that first call before
+ * any stream capture. All calls share the one array and it keeps the last
+ * call's contents; every byte a call reads there it has written first, so
+ * nothing needs clearing, but calls that overlap on the GPU (on different
+ * streams, or from different threads) race on it: serialise them.
+ * The pages have no counterpart to this entry point; it is part of the
+ * library's interface only. */
+#define QFP4_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+int qfp4_linear_fwd_noalloc(const void* X, const void* W, void* Y, int64_t M, int64_t N, int64_t K,
+                            const qfp4_recipe* recipe, const qfp4_seed* seed, void* stream);
 
 /* ---- status ---------------------------------------------------------------
  * Synchronizes `stream`, then reads and clears the library's device error word
