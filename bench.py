@@ -41,7 +41,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--profile", choices=["gemm", "quant_row", "quant_col", "amax"],
+    ap.add_argument("--profile", choices=["gemm_fprop", "gemm_dgrad", "gemm_wgrad", "quant_row", "quant_col",
+                                          "amax_row", "amax_col"],
                     help="run only one kernel 3 times on a bounded case (for ncu captures), print nothing else")
     return ap.parse_args()
 
@@ -52,6 +53,29 @@ def measured_peaks():
             return json.load(f), "measured"
     except OSError:
         return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def measured_gemm_traffic():
+    """DRAM bytes per GEMM launch (dram__bytes_read.sum + dram__bytes_write.sum)
+    from the committed ncu summary of this workload, or None when the GEMM
+    kernel's source has changed since those counters were taken."""
+    import hashlib
+    import re
+    try:
+        with open(os.path.join(ROOT, "profiles", "gemm_bs_fp4_mlp_up.md")) as f:
+            text = f.read()
+    except OSError:
+        return None
+    csrc = os.path.join(ROOT, "fp4_precision_b200", "csrc")
+    for key, fname in (("gemm_source_sha256", "gemm_sm100.cu"), ("device_header_sha256", "qfp4_device.cuh")):
+        m = re.search(key + r"\s+([0-9a-f]{64})", text)
+        with open(os.path.join(csrc, fname), "rb") as f:
+            if m is None or hashlib.sha256(f.read()).hexdigest() != m.group(1):
+                return None
+    m = re.search(r"traffic_bytes_per_launch fprop=(\d+) dgrad=(\d+) wgrad=(\d+)", text)
+    if m is None:
+        return None
+    return dict(zip(("fprop", "dgrad", "wgrad"), (int(v) for v in m.groups())))
 
 
 # ---------------------------------------------------------------------------
@@ -209,6 +233,7 @@ def run_ours(args, rank, world, local_rank):
     peaks, src = measured_peaks()
     fp4_peak = peaks["bf16_tflops_sustained"] * NOMINAL_FP4_OVER_BF16
     gemm_achieved = sum(gemm_flops) / (sum(gemm_ms) * 1e-3) / 1e12
+    traffic = measured_gemm_traffic()
 
     # quantizer sweep workload (GB/s of algorithmic bytes), L2 flushed between launches
     quant = quant_sweep(Q, inputs, dev, stream, peaks)
@@ -229,7 +254,14 @@ def run_ours(args, rank, world, local_rank):
         "roofline": {"bound": "tensor", "kernel": "gemm_bs_fp4 (tcgen05 kind::mxf4nvf4)",
                      "achieved": round(gemm_achieved, 1),
                      "peak": round(fp4_peak, 1), "unit": "TFLOP/s", "frac": round(gemm_achieved / fp4_peak, 4),
-                     "traffic": None,
+                     "traffic": None if traffic is None else int(statistics.mean(traffic.values())),
+                     "traffic_unit": "DRAM bytes per GEMM launch (mean of Fprop, Dgrad, Wgrad; ncu, "
+                                     "profiles/gemm_bs_fp4_mlp_up.md)",
+                     "traffic_per_gemm": traffic,
+                     "algorithmic_bytes_per_gemm": {
+                         "fprop": (M + N) * (K // 2 + K // 16) + M * N * 2,
+                         "dgrad": (M + K) * (N // 2 + N // 16) + M * K * 2,
+                         "wgrad": (N + K) * (M // 2 + M // 16) + N * K * 4},
                      "peak_source": f"{src}: bf16_tflops_sustained {peaks['bf16_tflops_sustained']} x nominal FP4/BF16 "
                                     f"ratio {NOMINAL_FP4_OVER_BF16}",
                      "per_gemm_ms": {"fprop": round(gemm_ms[0], 4), "dgrad": round(gemm_ms[1], 4),
@@ -397,7 +429,7 @@ def oracle_sample(m_rows: int, n_rows: int, steps: int = 1):
     return dt, 6.0 * M * N * K, os.cpu_count()
 
 
-def cpu_baseline_obj(m_rows=128, n_rows=8192):
+def cpu_baseline_obj(m_rows=256, n_rows=16384):
     dt, flops, cores = oracle_sample(m_rows, n_rows)
     return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
             "sample": f"linear fwd+bwd of the first {m_rows} tokens x {n_rows} output features (full K = 4096) of "
@@ -429,9 +461,10 @@ def run_reference(args, rank, world):
 
 
 def run_profile(kind: str):
-    """One kernel, three launches, on a case that exceeds L2 but holds about a
-    GB: the MLP up/gate Fprop GEMM (16384 x 28672 x 4096, NVFP4) or the
-    quantizers on the quantizer-sweep tensor [8192 x 4096]."""
+    """One kernel, three launches, on a case larger than L2 that holds a few GB
+    at most: each of the MLP up/gate layer's three GEMMs (Fprop, Dgrad, Wgrad
+    operands quantized as in the step), or a quantizer / amax pass (Quartet II
+    NVFP4, random 16x16 Hadamard) over a [16384 x 8192] bf16 tensor (268 MB)."""
     import torch
 
     from fp4_precision_b200 import inputs
@@ -439,21 +472,33 @@ def run_profile(kind: str):
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     seed = Q.make_seed(3, 4)
-    if kind == "gemm":
+    if kind.startswith("gemm"):
         wl = inputs.workload(WORKLOAD, device=dev)
-        A = Q.quantize(wl["X"], Q.NVFP4, Q.RTN, Q.HAD_DET16, Q.ROW, seed)
-        B = Q.quantize(wl["W"], Q.NVFP4, Q.RTN, Q.HAD_DET16, Q.ROW, seed)
-        del wl
-        D = torch.empty((A.rows, B.rows), dtype=torch.bfloat16, device=dev)
-        for _ in range(3):
-            Q.gemm(A, B, out=D)
-    else:
-        T = inputs.workload("sweep", device=dev)["T"]
-        if kind == "amax":
-            for _ in range(3):
-                Q.amax(T, Q.HAD_RAND16, Q.ROW, seed)
+        rec = Q.recipe(RECIPE)
+        c = {"gemm_fprop": rec.fprop, "gemm_dgrad": rec.dgrad, "gemm_wgrad": rec.wgrad}[kind]
+        if kind == "gemm_fprop":
+            A = Q.quantize(wl["X"], c.fmt, c.rnd_a, c.had, Q.ROW, seed)
+            B = Q.quantize(wl["W"], c.fmt, c.rnd_b, c.had, Q.ROW, seed)
+            out_dtype = torch.bfloat16
+        elif kind == "gemm_dgrad":
+            A = Q.quantize(wl["dY"], c.fmt, c.rnd_a, c.had, Q.ROW, seed)
+            B = Q.quantize(wl["W"], c.fmt, c.rnd_b, c.had, Q.COL, seed)
+            out_dtype = torch.bfloat16
         else:
-            axis = Q.ROW if kind == "quant_row" else Q.COL
+            A = Q.quantize(wl["dY"], c.fmt, c.rnd_a, c.had, Q.COL, seed)
+            B = Q.quantize(wl["X"], c.fmt, c.rnd_b, c.had, Q.COL, seed)
+            out_dtype = torch.float32
+        del wl
+        D = torch.empty((A.rows, B.rows), dtype=out_dtype, device=dev)
+        for _ in range(3):
+            Q.gemm(A, B, out_dtype, out=D)
+    else:
+        T = inputs.normal((16384, 8192), 1e-3, 5, "prof", device=dev)
+        axis = Q.ROW if kind.endswith("row") else Q.COL
+        if kind.startswith("amax"):
+            for _ in range(3):
+                Q.amax(T, Q.HAD_RAND16, axis, seed)
+        else:
             am = Q.amax(T, Q.HAD_RAND16, axis, seed)
             for _ in range(3):
                 Q.quantize(T, Q.NVFP4, Q.QUARTET2, Q.HAD_RAND16, axis, seed, amax_in=am)
