@@ -11,27 +11,33 @@
 // together share A and B tiles in L2) and issue tcgen05.mma (kind::mxf4nvf4,
 // scale_vec::4X for NVFP4; kind::mxf4, scale_vec::2X for MXFP4) with K = 64 per
 // instruction and an fp32 accumulator in tensor memory.
-//   - single CTA: 128 x 256 tiles, M = 128, N = 256;
-//   - CTA pair (default): 256 x 256 tiles on the two SMs of a cluster with
+//   - single CTA (default): 128 x 256 tiles, M = 128, N = 256;
+//   - CTA pair: 256 x 256 tiles on the two SMs of a cluster with
 //     tcgen05.mma.cta_group::2, M = 256, N = 256; each CTA loads half of A and
 //     half of B, so an SM moves 32 KiB of operands per 256-wide k-tile.
 // Warp roles (14 warps):
 //   warp 0, one lane: TMA producer into a shared-memory ring (A and B tiles
 //     with 128-byte swizzle, and the scale atoms, which the quantizers store in
 //     the MMA's 512-byte atom layout).
-//   warp 1, one lane: MMA issuer: 4 MMAs per 256-wide k-tile, then commits the
-//     stage and the scale slot.
+//   warp 1, one lane: MMA issuer: 4 MMAs per 256-wide k-tile and ONE commit,
+//     which frees both the ring stage and its tensor-memory scale slot.
 //   warps 2-5: scale writers, one per 32-lane quarter of tensor memory. They
-//     read the k-tile's scale atoms from shared memory and write them into one
-//     of 4 rotating tensor-memory slots with tcgen05.st (each quarter holds the
-//     same 32 atom rows, as the MMA reads them). Measured on B200, the copy
-//     instruction for scales (tcgen05.cp) took ~110 cycles each in the tensor
-//     pipe, 12 per k-tile, more than the 512 cycles of MMA work; the store path
-//     runs beside the MMAs.
+//     read the k-tile's scale atoms from shared memory and write them with
+//     tcgen05.st into the scale slot of the same index as the ring stage (each
+//     quarter holds the same 32 atom rows, as the MMA reads them).
 //   warps 6-13: epilogue, two per lane quarter, 128 accumulator columns each:
 //     drain tensor memory to registers (tcgen05.ld), hand the accumulator back
-//     to the MMA warp, multiply by gA * gB and store bf16 or fp32 rows while
-//     the next tile's MMAs run.
+//     to the MMA warp before the global stores (bf16) or after the first 32
+//     columns (fp32), multiply by gA * gB and store rows while the next tile's
+//     MMAs run.
+// The tensor pipe queues only a few MMAs, so the issuing thread's work between
+// k-tiles shows up directly as idle tensor cycles. Measured on B200: a second
+// commit per k-tile cost ~90 cycles per k-tile, a runtime-trip-count MMA loop
+// ~160 and descriptors rebuilt from addresses ~50, against 512 cycles of MMA
+// work. Hence the single commit, the unrolled 4-MMA k-tile and descriptors
+// advanced by adding to a base. (An earlier design copied the scales with
+// tcgen05.cp from the MMA thread; at ~110 cycles per copy and 12 per k-tile
+// that serialised the tensor pipe.)
 // Every wait is bounded (qfp4_device.cuh); on expiry the kernel raises the
 // device error word and skips the rest of its work.
 #include <cuda_fp16.h>
@@ -44,10 +50,10 @@ namespace {
 
 constexpr int BM = kGemmBM, BN = kGemmBN, BK = kGemmBK;  // BK in elements
 constexpr int TMEM_COLS = 512;
-// Tensor-memory columns: the 128 x 256 fp32 accumulator, then NSLOT scale
-// slots of 48 columns (SFA 16, SFB 32).
+// Tensor-memory columns: the 128 x 256 fp32 accumulator, then one scale slot
+// of 48 columns (SFA 16, SFB 32) per ring stage (4 stages single, 5 pair: at
+// most 256 + 5 * 48 = 496 columns).
 constexpr int TMEM_D = 0;
-constexpr int NSLOT = 4;
 __device__ __forceinline__ uint32_t sfa_col(int slot) { return 256u + 48u * (uint32_t)slot; }
 __device__ __forceinline__ uint32_t sfb_col(int slot) { return 256u + 48u * (uint32_t)slot + 16u; }
 
@@ -99,6 +105,47 @@ __device__ __forceinline__ void mma_bs(uint32_t d_tmem, uint64_t a_desc, uint64_
 }
 #undef QFP4_MMA_ASM
 
+// One K = 64 block j (0-3) of a k-tile: operand descriptors advance 32 bytes
+// (2 in the 16-byte address field) per block; NVFP4 scales take one 4-column
+// group per block, MXFP4 scales one per two blocks, the odd block reading the
+// upper two bytes of each scale word (scale-factor id 2).
+template <int FMT, bool PAIR, int MM>
+__device__ __forceinline__ void mma_kblock(uint32_t d, uint64_t ad, uint64_t bd, uint32_t sfa, uint32_t sfb, int j,
+                                           bool overwrite) {
+    uint32_t sa, sb, id;
+    if constexpr (FMT == kNvfp4) {
+        sa = sfa + 4u * (uint32_t)j;
+        sb = sfb + 8u * (uint32_t)j;
+        id = idesc_mn<FMT, MM, BN>(0, 0);
+    } else {
+        sa = sfa + 4u * (uint32_t)(j >> 1);
+        sb = sfb + 8u * (uint32_t)(j >> 1);
+        id = idesc_mn<FMT, MM, BN>(2u * (j & 1), 2u * (j & 1));
+    }
+    mma_bs<FMT, PAIR>(d, ad + 2u * (uint32_t)j, bd + 2u * (uint32_t)j, id, sa, sb, overwrite ? 0u : 1u);
+}
+// The MMAs of one k-tile of kb K = 64 blocks; a full k-tile (kb = 4) is
+// unrolled so the issuing thread does no loop work between MMAs.
+template <int FMT, bool PAIR, int MM>
+__device__ __forceinline__ void mma_ktile(uint32_t d, uint64_t ad, uint64_t bd, uint32_t sfa, uint32_t sfb, int kb,
+                                          bool first) {
+    if (kb == 4) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) mma_kblock<FMT, PAIR, MM>(d, ad, bd, sfa, sfb, j, first && j == 0);
+    } else {
+        for (int j = 0; j < kb; ++j) mma_kblock<FMT, PAIR, MM>(d, ad, bd, sfa, sfb, j, first && j == 0);
+    }
+}
+
+// 32 lanes x 16 consecutive fp32 columns of TMEM into registers (no wait).
+__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t* r) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, "
+        "[%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+          "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
 // 32 lanes x 32 consecutive fp32 columns of TMEM into registers (no wait).
 __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t* r) {
     asm volatile(
@@ -112,6 +159,14 @@ __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t* r) 
 }
 
 // Registers of 32 lanes into 8 / 16 / 32 consecutive 32-bit TMEM columns.
+__device__ __forceinline__ void tmem_st_x1(uint32_t taddr, uint32_t r) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(r) : "memory");
+}
+__device__ __forceinline__ uint32_t lds32(uint32_t saddr) {
+    uint32_t v;
+    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(saddr));
+    return v;
+}
 __device__ __forceinline__ void tmem_st_x8(uint32_t taddr, const uint32_t* r) {
     asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr), "r"(r[0]),
                  "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
@@ -143,18 +198,22 @@ __device__ __forceinline__ uint4 lds128(uint32_t saddr) {
     return v;
 }
 
-// Scale writer: lane i of the warp for lane quarter q copies row i of every
-// scale atom of the k-tile from shared memory into its TMEM lane 32q + i.
-// SFA atom a -> columns sfa_col + 4a; SFB atom a of row block rb -> columns
-// sfb_col + 8a + 4rb (the layout of tcgen05.cp 32x128b.warpx4).
+// Scale writer for TMEM lane quarter q (lanes 32q..32q+31): lane i copies
+// line i of the k-tile's scale atoms from shared memory into TMEM lane 32q + i.
+// Line i of an atom holds four words, word w the four scales of row i + 32w;
+// in tensor memory word w goes to column base + w (the layout
+// tcgen05.cp.32x128b.warpx4 produces). The MMA computes output row 32q + i in
+// lane quarter q, so for A it reads only word q of each line: only that
+// column is written. Every quarter needs all B rows: SFB gets all four words
+// of both 128-row blocks. SFA atom a -> column sfa_col + 4a + q; SFB atom a of
+// row block rb -> columns sfb_col + 8a + 4rb .. +3.
 template <int ATOMS>
 __device__ __forceinline__ void write_scales(uint32_t tmem_lane, int slot, uint32_t sfa_smem, uint32_t sfb_smem,
-                                             int lane) {
-    uint32_t ra[4 * ATOMS], rb[8 * ATOMS];
+                                             int lane, int q) {
+    uint32_t ra[ATOMS], rb[8 * ATOMS];
 #pragma unroll
     for (int a = 0; a < ATOMS; ++a) {
-        const uint4 v = lds128(sfa_smem + a * 512 + lane * 16);
-        ra[4 * a + 0] = v.x; ra[4 * a + 1] = v.y; ra[4 * a + 2] = v.z; ra[4 * a + 3] = v.w;
+        ra[a] = lds32(sfa_smem + a * 512 + lane * 16 + q * 4);
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
             const uint4 w = lds128(sfb_smem + r * (ATOMS * 512) + a * 512 + lane * 16);
@@ -162,77 +221,121 @@ __device__ __forceinline__ void write_scales(uint32_t tmem_lane, int slot, uint3
             rb[8 * a + 4 * r + 2] = w.z; rb[8 * a + 4 * r + 3] = w.w;
         }
     }
+#pragma unroll
+    for (int a = 0; a < ATOMS; ++a) tmem_st_x1(tmem_lane + sfa_col(slot) + 4u * a + (uint32_t)q, ra[a]);
     if constexpr (ATOMS == 4) {
-        tmem_st_x16(tmem_lane + sfa_col(slot), ra);
         tmem_st_x32(tmem_lane + sfb_col(slot), rb);
     } else {
-        tmem_st_x8(tmem_lane + sfa_col(slot), ra);
         tmem_st_x16(tmem_lane + sfb_col(slot), rb);
     }
     tc_wait_st();
 }
 
-// Epilogue store of 64 accumulator columns of row `row` from column `n0`:
-// times gA * gB, as bf16 or fp32, with evict-first stores so the output stream
-// does not push the operand tiles out of L2.
-__device__ __forceinline__ void store64(const GemmParams& p, const uint32_t* acc, int row, int n0, float scale) {
+// Scaled accumulator pair as two packed bf16.
+__device__ __forceinline__ uint32_t pack_bf16(uint32_t a, uint32_t b, float scale) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(a), scale), __fmul_rn(__uint_as_float(b), scale));
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Epilogue stores of one row's NC columns from column n0, with evict-first
+// stores so the output stream does not push the operand tiles out of L2.
+// bf16: NC / 2 packed words; fp32: NC accumulator words times gA * gB.
+template <int NC>
+__device__ __forceinline__ void store_bf16(const GemmParams& p, const uint32_t* w, int row, int n0) {
     if (row >= p.M) return;
-    if (p.out_f32) {
-        float* dst = reinterpret_cast<float*>(p.D) + (int64_t)row * p.ldd + n0;
+    __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.D) + (int64_t)row * p.ldd + n0;
 #pragma unroll
-        for (int c = 0; c < 64; c += 4) {
-            const float4 v4 = make_float4(__fmul_rn(__uint_as_float(acc[c]), scale),
-                                          __fmul_rn(__uint_as_float(acc[c + 1]), scale),
-                                          __fmul_rn(__uint_as_float(acc[c + 2]), scale),
-                                          __fmul_rn(__uint_as_float(acc[c + 3]), scale));
-            if (n0 + c + 4 <= p.N) {
-                __stcs(reinterpret_cast<float4*>(dst + c), v4);
-            } else {
-                if (n0 + c < p.N) dst[c] = v4.x;
-                if (n0 + c + 1 < p.N) dst[c + 1] = v4.y;
-                if (n0 + c + 2 < p.N) dst[c + 2] = v4.z;
-            }
-        }
-    } else {
-        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.D) + (int64_t)row * p.ldd + n0;
+    for (int c = 0; c < NC; c += 8)
+        __stcs(reinterpret_cast<uint4*>(dst + c), make_uint4(w[c / 2], w[c / 2 + 1], w[c / 2 + 2], w[c / 2 + 3]));
+}
+// Ragged right edge: the first nv (< NC) of NC bf16 columns, element by element.
+template <int NC>
+__device__ __forceinline__ void store_bf16_edge(const GemmParams& p, const uint32_t* w, int row, int n0) {
+    if (row >= p.M) return;
+    uint16_t* d16 = reinterpret_cast<uint16_t*>(p.D) + (int64_t)row * p.ldd + n0;
+    const int nv = p.N - n0;
 #pragma unroll
-        for (int c = 0; c < 64; c += 8) {
-            uint32_t w[4];
+    for (int c = 0; c < NC; ++c)
+        if (c < nv) d16[c] = (uint16_t)(w[c >> 1] >> (16 * (c & 1)));
+}
+template <int NC>
+__device__ __forceinline__ void store_f32(const GemmParams& p, uint32_t* acc, int row, int n0, float scale) {
+    if (row >= p.M) return;
+    float* dst = reinterpret_cast<float*>(p.D) + (int64_t)row * p.ldd + n0;
 #pragma unroll
-            for (int h = 0; h < 4; ++h) {
-                __nv_bfloat162 b2 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(acc[c + 2 * h]), scale),
-                                                          __fmul_rn(__uint_as_float(acc[c + 2 * h + 1]), scale));
-                w[h] = *reinterpret_cast<uint32_t*>(&b2);
-            }
-            if (n0 + c + 8 <= p.N) {
-                __stcs(reinterpret_cast<uint4*>(dst + c), make_uint4(w[0], w[1], w[2], w[3]));
-            } else {
+    for (int c = 0; c < NC; ++c) acc[c] = __float_as_uint(__fmul_rn(__uint_as_float(acc[c]), scale));
+    if (n0 + NC <= p.N) {
 #pragma unroll
-                for (int h = 0; h < 8; ++h)
-                    if (n0 + c + h < p.N) reinterpret_cast<uint16_t*>(dst)[c + h] = (uint16_t)(w[h >> 1] >> (16 * (h & 1)));
+        for (int c = 0; c < NC; c += 4)
+            __stcs(reinterpret_cast<uint4*>(dst + c), make_uint4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]));
+    } else {  // ragged right edge: nv < NC valid columns, whole 4-column chunks first
+        const int nv = p.N - n0, nfull = nv >> 2, rem = nv & 3;
+        uint32_t* d32 = reinterpret_cast<uint32_t*>(dst);
+#pragma unroll
+        for (int c = 0; c < NC; c += 4) {
+            if ((c >> 2) < nfull) {
+                __stcs(reinterpret_cast<uint4*>(dst + c), make_uint4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]));
+            } else if ((c >> 2) == nfull && rem != 0) {
+#pragma unroll
+                for (int h = 0; h < 3; ++h)
+                    if (h < rem) d32[c + h] = acc[c + h];
             }
         }
     }
 }
 
-// Epilogue of one tile for one warp: drain 128 accumulator columns of its lane
-// quarter in two halves, releasing the accumulator (release()) as soon as the
-// second half is in registers.
+// Epilogue of one tile for one warp: 128 accumulator columns of its lane
+// quarter. The accumulator goes back to the MMA warp (release()) as soon as
+// the values are in registers: all 128 columns for bf16 output (packed, 64
+// registers), the last 96 for fp32 after the first 32 are stored.
 template <typename Release>
 __device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t taddr, int row, int n0, float scale,
                                               Release release) {
-    uint32_t acc[64];
-    tmem_ld_32x32b_x32(taddr + 0, acc);
-    tmem_ld_32x32b_x32(taddr + 32, acc + 32);
-    tc_wait_ld();
-    store64(p, acc, row, n0, scale);
-    tmem_ld_32x32b_x32(taddr + 64, acc);
-    tmem_ld_32x32b_x32(taddr + 96, acc + 32);
-    tc_wait_ld();
-    tc_fence_before();
-    __syncwarp();
-    release();
-    store64(p, acc, row, n0 + 64, scale);
+    if (!p.out_f32 && n0 + 128 > p.N) {
+        // ragged right edge (rare): 16 columns at a time, released after the last load
+#pragma unroll 1
+        for (int h = 0; h < 8; ++h) {
+            uint32_t acc[16], w[8];
+            tmem_ld_32x32b_x16(taddr + 16 * h, acc);
+            tc_wait_ld();
+            if (h == 7) {
+                tc_fence_before();
+                __syncwarp();
+                release();
+            }
+#pragma unroll
+            for (int c = 0; c < 8; ++c) w[c] = pack_bf16(acc[2 * c], acc[2 * c + 1], scale);
+            if (n0 + 16 * h < p.N) store_bf16_edge<16>(p, w, row, n0 + 16 * h);
+        }
+    } else if (!p.out_f32) {
+        uint32_t w[64];
+#pragma unroll
+        for (int h = 0; h < 8; ++h) {
+            uint32_t acc[16];
+            tmem_ld_32x32b_x16(taddr + 16 * h, acc);
+            tc_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 8; ++c) w[8 * h + c] = pack_bf16(acc[2 * c], acc[2 * c + 1], scale);
+        }
+        tc_fence_before();
+        __syncwarp();
+        release();
+        store_bf16<128>(p, w, row, n0);
+    } else {
+        uint32_t acc[80];
+        tmem_ld_32x32b_x16(taddr, acc);
+        tmem_ld_32x32b_x32(taddr + 16, acc + 16);
+        tc_wait_ld();
+        store_f32<48>(p, acc, row, n0, scale);
+        tmem_ld_32x32b_x16(taddr + 48, acc);
+        tmem_ld_32x32b_x32(taddr + 64, acc + 16);
+        tmem_ld_32x32b_x32(taddr + 96, acc + 48);
+        tc_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        release();
+        store_f32<80>(p, acc, row, n0 + 48, scale);
+    }
 }
 
 // Grouped tile order: GM row-tiles at a time, walking down the group first.
@@ -269,11 +372,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint8_t* sB = sA + STAGES * A_STAGE;
     uint8_t* sSFA = sB + STAGES * B_STAGE;
     uint8_t* sSFB = sSFA + STAGES * SFA_STAGE;
-    uint64_t* full = reinterpret_cast<uint64_t*>(sSFB + STAGES * SFB_STAGE);
-    uint64_t* empty = full + STAGES;
-    uint64_t* sf_full = empty + STAGES;
-    uint64_t* sf_empty = sf_full + NSLOT;
-    uint64_t* acc_full = sf_empty + NSLOT;
+    uint64_t* full = reinterpret_cast<uint64_t*>(sSFB + STAGES * SFB_STAGE);  // A and B of stage s landed
+    uint64_t* empty = full + STAGES;      // stage s and scale slot s free again
+    uint64_t* sf_load = empty + STAGES;   // scale atoms of stage s landed
+    uint64_t* sf_full = sf_load + STAGES; // scale slot s written
+    uint64_t* acc_full = sf_full + STAGES;
     uint64_t* acc_empty = acc_full + 1;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
 
@@ -288,10 +391,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
-        }
-        for (int s = 0; s < NSLOT; ++s) {
+            mbar_init(&sf_load[s], 1);
             mbar_init(&sf_full[s], kScaleWarps);
-            mbar_init(&sf_empty[s], 1);
         }
         mbar_init(acc_full, 1);
         mbar_init(acc_empty, kEpiWarps);
@@ -321,74 +422,74 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     }
                     const int kelems = min(BK, p.K - kt * BK);
                     const int atoms = (kelems + SF_K - 1) / SF_K;
-                    mbar_arrive_expect_tx(&full[s], A_STAGE + B_STAGE + atoms * 512 * (1 + nrb));
-                    tma_load_2d(sA + s * A_STAGE, &tmA, &full[s], kt * (BK / 2), mb * BM);
-                    tma_load_2d(sB + s * B_STAGE, &tmB, &full[s], kt * (BK / 2), n0);
+                    // scale atoms first, on their own barrier: the scale writers
+                    // start while the operand tiles are still in flight
+                    mbar_arrive_expect_tx(&sf_load[s], atoms * 512 * (1 + nrb));
                     const int64_t katom = (int64_t)kt * ATOMS_PER_KT;
                     bulk_load(sSFA + s * SFA_STAGE, p.sfa + ((int64_t)mb * p.atoms_k + katom) * 512, atoms * 512,
-                              &full[s]);
+                              &sf_load[s]);
                     for (int rb = 0; rb < nrb; ++rb)
                         bulk_load(sSFB + s * SFB_STAGE + rb * (ATOMS_PER_KT * 512),
-                                  p.sfb + ((int64_t)(n0 / 128 + rb) * p.atoms_k + katom) * 512, atoms * 512, &full[s]);
+                                  p.sfb + ((int64_t)(n0 / 128 + rb) * p.atoms_k + katom) * 512, atoms * 512,
+                                  &sf_load[s]);
+                    mbar_arrive_expect_tx(&full[s], A_STAGE + B_STAGE);
+                    tma_load_2d(sA + s * A_STAGE, &tmA, &full[s], kt * (BK / 2), mb * BM);
+                    tma_load_2d(sB + s * B_STAGE, &tmB, &full[s], kt * (BK / 2), n0);
                 }
             }
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
         if (lane == 0) {
-            int it = 0, lt = 0;
+            const uint64_t a_desc0 = sw128_desc(smem_u32(sA)), b_desc0 = sw128_desc(smem_u32(sB));
+            int s = 0, lt = 0;
+            uint32_t ph = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++lt) {
                 if (lt > 0 && !mbar_wait(acc_empty, (lt - 1) & 1)) break;
                 tc_fence_after();
-                for (int kt = 0; kt < KT; ++kt, ++it) {
-                    const int s = it % STAGES, slot = it % NSLOT;
-                    if (!mbar_wait(&full[s], (it / STAGES) & 1) || !mbar_wait(&sf_full[slot], (it / NSLOT) & 1)) {
+                for (int kt = 0; kt < KT; ++kt) {
+                    if (!mbar_wait(&full[s], ph) || !mbar_wait(&sf_full[s], ph)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const int kblocks = min(BK, p.K - kt * BK) / 64;
-                    const uint32_t a_base = smem_u32(sA + s * A_STAGE);
-                    const uint32_t b_base = smem_u32(sB + s * B_STAGE);
-                    for (int j = 0; j < kblocks; ++j) {
-                        uint32_t sfa_t, sfb_t, id;
-                        if constexpr (FMT == kNvfp4) {
-                            sfa_t = tmem + sfa_col(slot) + 4 * j;
-                            sfb_t = tmem + sfb_col(slot) + 8 * j;
-                            id = idesc_mn<FMT, BM, BN>(0, 0);
-                        } else {
-                            sfa_t = tmem + sfa_col(slot) + 4 * (j >> 1);
-                            sfb_t = tmem + sfb_col(slot) + 8 * (j >> 1);
-                            id = idesc_mn<FMT, BM, BN>(2 * (j & 1), 2 * (j & 1));
-                        }
-                        mma_bs<FMT, false>(tmem + TMEM_D, sw128_desc(a_base + j * 32), sw128_desc(b_base + j * 32), id,
-                                           sfa_t, sfb_t, (kt > 0 || j > 0) ? 1u : 0u);
+                    mma_ktile<FMT, false, BM>(tmem + TMEM_D, a_desc0 + (uint64_t)(s * (A_STAGE >> 4)),
+                                              b_desc0 + (uint64_t)(s * (B_STAGE >> 4)), tmem + sfa_col(s),
+                                              tmem + sfb_col(s), min(BK, p.K - kt * BK) / 64, kt == 0);
+                    tc_commit(&empty[s]);  // stage s and scale slot s are free once these MMAs finish
+                    if (++s == STAGES) {
+                        s = 0;
+                        ph ^= 1;
                     }
-                    tc_commit(&empty[s]);
-                    tc_commit(&sf_empty[slot]);
                 }
                 tc_commit(acc_full);
             }
         }
     } else if (warp < kFirstEpiWarp) {
         // ---------------- scale writers ----------------
+        // Stage s's scale atoms arriving (sf_load[s]) implies the MMAs that
+        // last read scale slot s have finished: the producer refills a stage
+        // only after their commit.
         const uint32_t tmem_lane = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-        int it = 0;
+        int s = 0;
+        uint32_t ph = 0;
         bool ok = true;
         for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
-            for (int kt = 0; kt < KT; ++kt, ++it) {
-                const int s = it % STAGES, slot = it % NSLOT;
-                if (!mbar_wait(&full[s], (it / STAGES) & 1) ||
-                    (it >= NSLOT && !mbar_wait(&sf_empty[slot], ((it / NSLOT) + 1) & 1))) {
+            for (int kt = 0; kt < KT; ++kt) {
+                if (!mbar_wait(&sf_load[s], ph)) {
                     ok = false;
                     break;
                 }
-                write_scales<ATOMS_PER_KT>(tmem_lane, slot, smem_u32(sSFA + s * SFA_STAGE),
-                                           smem_u32(sSFB + s * SFB_STAGE), lane);
+                write_scales<ATOMS_PER_KT>(tmem_lane, s, smem_u32(sSFA + s * SFA_STAGE), smem_u32(sSFB + s * SFB_STAGE),
+                                           lane, warp & 3);
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&sf_full[slot]);
+                if (lane == 0) mbar_arrive(&sf_full[s]);
+                if (++s == STAGES) {
+                    s = 0;
+                    ph ^= 1;
+                }
             }
         }
     } else {
@@ -453,10 +554,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     uint8_t* sSFB = sSFA + P_STAGES * P_SFA;
     uint64_t* full = reinterpret_cast<uint64_t*>(sSFB + P_STAGES * P_SFB);
     uint64_t* empty = full + P_STAGES;
-    uint64_t* sf_load = empty + P_STAGES;
-    uint64_t* sf_full = sf_load + P_STAGES;
-    uint64_t* sf_empty = sf_full + NSLOT;
-    uint64_t* acc_full = sf_empty + NSLOT;
+    uint64_t* sf_load = empty + P_STAGES;   // this CTA's scale atoms of stage s landed
+    uint64_t* sf_full = sf_load + P_STAGES;  // scale slot s written in both CTAs (leader's)
+    uint64_t* acc_full = sf_full + P_STAGES;
     uint64_t* acc_empty = acc_full + 1;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
 
@@ -476,10 +576,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
             mbar_init(&sf_load[s], 1);
-        }
-        for (int s = 0; s < NSLOT; ++s) {
             mbar_init(&sf_full[s], 2 * kScaleWarps);
-            mbar_init(&sf_empty[s], 1);
         }
         mbar_init(acc_full, 1);
         mbar_init(acc_empty, 2 * kEpiWarps);
@@ -518,59 +615,55 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     } else if (warp == 1) {
         // ---------------- MMA issuer (leader CTA only) ----------------
         if (lane == 0 && rank == 0) {
-            int it = 0, lt = 0;
+            const uint64_t a_desc0 = sw128_desc(smem_u32(sA)), b_desc0 = sw128_desc(smem_u32(sB));
+            int s = 0, lt = 0;
+            uint32_t ph = 0;
             bool ok = true;
             for (int t = cid; t < tiles && ok; t += nclusters, ++lt) {
                 if (lt > 0 && !mbar_wait_cluster(acc_empty, (lt - 1) & 1)) break;
                 tc_fence_after();
-                for (int kt = 0; kt < KT; ++kt, ++it) {
-                    const int s = it % P_STAGES, slot = it % NSLOT;
-                    if (!mbar_wait_cluster(&full[s], (it / P_STAGES) & 1) || !mbar_wait_cluster(&sf_full[slot], (it / NSLOT) & 1)) {
+                for (int kt = 0; kt < KT; ++kt) {
+                    if (!mbar_wait_cluster(&full[s], ph) || !mbar_wait_cluster(&sf_full[s], ph)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const int kblocks = min(BK, p.K - kt * BK) / 64;
-                    const uint32_t a_base = smem_u32(sA + s * P_A);
-                    const uint32_t b_base = smem_u32(sB + s * P_B);
-                    for (int j = 0; j < kblocks; ++j) {
-                        uint32_t sfa_t, sfb_t, id;
-                        if constexpr (FMT == kNvfp4) {
-                            sfa_t = tmem + sfa_col(slot) + 4 * j;
-                            sfb_t = tmem + sfb_col(slot) + 8 * j;
-                            id = idesc_mn<FMT, 2 * BM, BN>(0, 0);
-                        } else {
-                            sfa_t = tmem + sfa_col(slot) + 4 * (j >> 1);
-                            sfb_t = tmem + sfb_col(slot) + 8 * (j >> 1);
-                            id = idesc_mn<FMT, 2 * BM, BN>(2 * (j & 1), 2 * (j & 1));
-                        }
-                        mma_bs<FMT, true>(tmem + TMEM_D, sw128_desc(a_base + j * 32), sw128_desc(b_base + j * 32), id,
-                                          sfa_t, sfb_t, (kt > 0 || j > 0) ? 1u : 0u);
+                    mma_ktile<FMT, true, 2 * BM>(tmem + TMEM_D, a_desc0 + (uint64_t)(s * (P_A >> 4)),
+                                                 b_desc0 + (uint64_t)(s * (P_B >> 4)), tmem + sfa_col(s),
+                                                 tmem + sfb_col(s), min(BK, p.K - kt * BK) / 64, kt == 0);
+                    tc_commit_pair(&empty[s]);  // frees stage s and scale slot s in both CTAs
+                    if (++s == P_STAGES) {
+                        s = 0;
+                        ph ^= 1;
                     }
-                    tc_commit_pair(&empty[s]);       // frees stage s in both CTAs
-                    tc_commit_pair(&sf_empty[slot]);  // frees the scale slot in both CTAs
                 }
                 tc_commit_pair(acc_full);  // both CTAs' accumulators are complete
             }
         }
     } else if (warp < kFirstEpiWarp) {
         // ---------------- scale writers (both CTAs) ----------------
+        // The producer loads stage s's scale atoms only after the commit of
+        // the MMAs that last read scale slot s, so sf_load[s] implies the slot
+        // is free.
         const uint32_t tmem_lane = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-        int it = 0;
+        int s = 0;
+        uint32_t ph = 0;
         bool ok = true;
         for (int t = cid; t < tiles && ok; t += nclusters) {
-            for (int kt = 0; kt < KT; ++kt, ++it) {
-                const int s = it % P_STAGES, slot = it % NSLOT;
-                if (!mbar_wait_cluster(&sf_load[s], (it / P_STAGES) & 1) ||
-                    (it >= NSLOT && !mbar_wait_cluster(&sf_empty[slot], ((it / NSLOT) + 1) & 1))) {
+            for (int kt = 0; kt < KT; ++kt) {
+                if (!mbar_wait_cluster(&sf_load[s], ph)) {
                     ok = false;
                     break;
                 }
-                write_scales<ATOMS_PER_KT>(tmem_lane, slot, smem_u32(sSFA + s * P_SFA), smem_u32(sSFB + s * P_SFB),
-                                           lane);
+                write_scales<ATOMS_PER_KT>(tmem_lane, s, smem_u32(sSFA + s * P_SFA), smem_u32(sSFB + s * P_SFB), lane,
+                                           warp & 3);
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&sf_full[slot]), 0));
+                if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&sf_full[s]), 0));
+                if (++s == P_STAGES) {
+                    s = 0;
+                    ph ^= 1;
+                }
             }
         }
     } else {
