@@ -11,10 +11,14 @@
 // together share A and B tiles in L2) and issue tcgen05.mma (kind::mxf4nvf4,
 // scale_vec::4X for NVFP4; kind::mxf4, scale_vec::2X for MXFP4) with K = 64 per
 // instruction and an fp32 accumulator in tensor memory.
-//   - single CTA (default): 128 x 256 tiles, M = 128, N = 256;
-//   - CTA pair: 256 x 256 tiles on the two SMs of a cluster with
-//     tcgen05.mma.cta_group::2, M = 256, N = 256; each CTA loads half of A and
-//     half of B, so an SM moves 32 KiB of operands per 256-wide k-tile.
+//   - CTA pair (default for more than 128 rows of A): 256 x 256 tiles on the
+//     two SMs of a cluster with tcgen05.mma.cta_group::2, M = 256, N = 256;
+//     each CTA loads half of A and half of B, so an SM moves 32 KiB of
+//     operands (+ 6 KiB of scales) per 256-wide k-tile;
+//   - single CTA: 128 x 256 tiles, M = 128, N = 256, 48 KiB (+ 6 KiB) per SM
+//     per k-tile. Measured on B200, one SM's TMA fill tops out near 106 bytes
+//     per cycle, so 54 KiB per 512 cycles of MMA leaves the single-CTA
+//     kernel no headroom; the pair kernel's 38 KiB leaves ~30 %.
 // Warp roles (14 warps):
 //   warp 0, one lane: TMA producer into a shared-memory ring (A and B tiles
 //     with 128-byte swizzle, and the scale atoms, which the quantizers store in
@@ -602,13 +606,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                         ok = false;
                         break;
                     }
+                    // scale atoms first: the scale writers start while the
+                    // operand tiles are still in flight
+                    mbar_arrive_expect_tx(&sf_load[s], SF_TX);
+                    tma_load_3d(sSFA + s * P_SFA, &tmSFA, &sf_load[s], 0, kt * ATOMS_PER_KT, 2 * mb + (int)rank);
+                    tma_load_3d(sSFB + s * P_SFB, &tmSFB, &sf_load[s], 0, kt * ATOMS_PER_KT, 2 * nb);
                     const uint32_t bar_leader = mapa_shared(smem_u32(&full[s]), 0);
                     if (rank == 0) mbar_arrive_expect_tx(&full[s], AB_TX);
                     tma_load_2d_pair(sA + s * P_A, &tmA, bar_leader, kt * (BK / 2), mb * 2 * BM + (int)rank * BM);
                     tma_load_2d_pair(sB + s * P_B, &tmB, bar_leader, kt * (BK / 2), nb * BN + (int)rank * 128);
-                    mbar_arrive_expect_tx(&sf_load[s], SF_TX);
-                    tma_load_3d(sSFA + s * P_SFA, &tmSFA, &sf_load[s], 0, kt * ATOMS_PER_KT, 2 * mb + (int)rank);
-                    tma_load_3d(sSFB + s * P_SFB, &tmSFB, &sf_load[s], 0, kt * ATOMS_PER_KT, 2 * nb);
                 }
             }
         }

@@ -199,9 +199,12 @@ int make_scale_tmap(CUtensorMap* tm, const void* scales, int64_t rows, int64_t a
 
 // The single-CTA GEMM is the default (measured faster on B200); QFP4_GEMM_PAIR=1
 // in the environment (read at each call) selects the CTA-pair kernel.
-bool use_pair_gemm() {
+// CTA-pair kernel unless A has at most 128 rows (one pair tile would be half
+// empty); QFP4_GEMM_PAIR=1 / =0 forces one kernel (read on every call).
+bool use_pair_gemm(int64_t M) {
     const char* e = std::getenv("QFP4_GEMM_PAIR");
-    return e != nullptr && e[0] == '1';
+    if (e != nullptr && (e[0] == '0' || e[0] == '1')) return e[0] == '1';
+    return M > kGemmBM;
 }
 
 int write_one(float* dst, cudaStream_t s) {
@@ -367,7 +370,7 @@ int gemm_impl(const qfp4_tensor* A, const qfp4_tensor* B, void* D, int64_t ldd, 
         return QFP4_ERR_INVALID_ARG;
     if (!aligned16(A->codes) || !aligned16(B->codes) || !aligned16(A->scales) || !aligned16(B->scales))
         return QFP4_ERR_MISALIGNED;
-    const bool pair = use_pair_gemm();
+    const bool pair = use_pair_gemm(M);
     CUtensorMap tA, tB;
     if ((rc = make_codes_tmap(&tA, A->codes, M, K, kGemmBM))) return rc;
     if ((rc = make_codes_tmap(&tB, B->codes, N, K, pair ? 128 : kGemmBN))) return rc;

@@ -312,9 +312,15 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
 __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
-// Arrive on an mbarrier given by its shared::cluster address (possibly the peer's).
+// Arrive on an mbarrier given by its shared::cluster address (possibly the
+// peer's), with the default (CTA-scope release) semantics. The arriving
+// threads have already waited for their own tensor-memory operations
+// (tcgen05.wait::st / ::ld) and fenced them (tcgen05.fence::before_thread_sync),
+// which is all the peer's tensor-core work needs. Measured on B200: the
+// .release.cluster form cost ~1500 cycles per arrive, longer than a k-tile's
+// MMAs.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 // TMA loads into this CTA's shared memory whose completion is counted on the
 // pair's leader barrier (`bar_cluster`, a shared::cluster address).

@@ -190,9 +190,10 @@ int qfp4_quantize(const void* x, int64_t R, int64_t C, int64_t ld, int32_t fmt, 
  * Requirements: same format, same k (a multiple of 64), same Hadamard (and for
  * a random one, the same rot_seed and rot_stream, so the rotation cancels);
  * D 16-byte aligned and ldd * element size a multiple of 16; ldd >= B.rows.
- * Kernel: persistent single-CTA 128 x 256 tiles; setting the environment
- * variable QFP4_GEMM_PAIR=1 selects a CTA-pair kernel (256 x 256 tiles,
- * tcgen05 cta_group::2) instead (same results within the bound). */
+ * Kernel: persistent CTA pairs on 256 x 256 tiles (tcgen05 cta_group::2) when
+ * A has more than 128 rows, else single CTAs on 128 x 256 tiles; the
+ * environment variable QFP4_GEMM_PAIR=1 or =0 forces the pair or the single
+ * kernel (same results within the bound). */
 int qfp4_gemm(const qfp4_tensor* A, const qfp4_tensor* B, void* D, int64_t ldd, int32_t out_dtype, void* stream);
 
 /* ---- linear layer -------------------------------------------------------------

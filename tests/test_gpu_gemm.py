@@ -53,11 +53,14 @@ def check_gemm(A_o, B_o, out_dtype, rows=None, cols=None, rot=(0, 0)):
     return worst
 
 
-@pytest.fixture(params=["pair", "single"])
+@pytest.fixture(params=["pair", "single", "default"])
 def kernel_variant(request, monkeypatch):
-    """Both GEMM kernels: the single-CTA default and the CTA-pair one."""
+    """Both GEMM kernels, forced (the CTA pair, the single CTA), and the
+    library's own choice (the pair when A has more than 128 rows)."""
     if request.param == "pair":
         monkeypatch.setenv("QFP4_GEMM_PAIR", "1")
+    elif request.param == "single":
+        monkeypatch.setenv("QFP4_GEMM_PAIR", "0")
     else:
         monkeypatch.delenv("QFP4_GEMM_PAIR", raising=False)
     return request.param
