@@ -235,10 +235,12 @@ __device__ __forceinline__ void write_scales(uint32_t tmem_lane, int slot, uint3
     tc_wait_st();
 }
 
-// Scaled accumulator pair as two packed bf16.
+// Scaled accumulator pair as two packed bf16 (one packed fp32x2 multiply, one
+// conversion).
 __device__ __forceinline__ uint32_t pack_bf16(uint32_t a, uint32_t b, float scale) {
-    __nv_bfloat162 v = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(a), scale), __fmul_rn(__uint_as_float(b), scale));
-    return *reinterpret_cast<uint32_t*>(&v);
+    const float2 v = __fmul2_rn(make_float2(__uint_as_float(a), __uint_as_float(b)), make_float2(scale, scale));
+    __nv_bfloat162 h = __float22bfloat162_rn(v);
+    return *reinterpret_cast<uint32_t*>(&h);
 }
 
 // Epilogue stores of one row's NC columns from column n0, with evict-first
@@ -267,7 +269,12 @@ __device__ __forceinline__ void store_f32(const GemmParams& p, uint32_t* acc, in
     if (row >= p.M) return;
     float* dst = reinterpret_cast<float*>(p.D) + (int64_t)row * p.ldd + n0;
 #pragma unroll
-    for (int c = 0; c < NC; ++c) acc[c] = __float_as_uint(__fmul_rn(__uint_as_float(acc[c]), scale));
+    for (int c = 0; c < NC; c += 2) {
+        const float2 v = __fmul2_rn(make_float2(__uint_as_float(acc[c]), __uint_as_float(acc[c + 1])),
+                                    make_float2(scale, scale));
+        acc[c] = __float_as_uint(v.x);
+        acc[c + 1] = __float_as_uint(v.y);
+    }
     if (n0 + NC <= p.N) {
 #pragma unroll
         for (int c = 0; c < NC; c += 4)
@@ -314,12 +321,13 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tadd
     } else if (!p.out_f32) {
         uint32_t w[64];
 #pragma unroll
-        for (int h = 0; h < 8; ++h) {
-            uint32_t acc[16];
-            tmem_ld_32x32b_x16(taddr + 16 * h, acc);
+        for (int h = 0; h < 2; ++h) {  // two round trips of 64 columns
+            uint32_t acc[64];
+            tmem_ld_32x32b_x32(taddr + 64 * h, acc);
+            tmem_ld_32x32b_x32(taddr + 64 * h + 32, acc + 32);
             tc_wait_ld();
 #pragma unroll
-            for (int c = 0; c < 8; ++c) w[8 * h + c] = pack_bf16(acc[2 * c], acc[2 * c + 1], scale);
+            for (int c = 0; c < 32; ++c) w[32 * h + c] = pack_bf16(acc[2 * c], acc[2 * c + 1], scale);
         }
         tc_fence_before();
         __syncwarp();

@@ -197,8 +197,6 @@ int make_scale_tmap(CUtensorMap* tm, const void* scales, int64_t rows, int64_t a
     return QFP4_OK;
 }
 
-// The single-CTA GEMM is the default (measured faster on B200); QFP4_GEMM_PAIR=1
-// in the environment (read at each call) selects the CTA-pair kernel.
 // CTA-pair kernel unless A has at most 128 rows (one pair tile would be half
 // empty); QFP4_GEMM_PAIR=1 / =0 forces one kernel (read on every call).
 bool use_pair_gemm(int64_t M) {

@@ -43,6 +43,34 @@ __device__ __forceinline__ float had_norm() {
 }
 
 __device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
+
+// max(a, b, c) in one instruction (IEEE maxNum semantics, like fmaxf).
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// Largest |v[e]| of N values, starting from m.
+template <int N>
+__device__ __forceinline__ float abs_max(float m, const float* v) {
+#pragma unroll
+    for (int e = 0; e < N; e += 2) m = max3(m, fabsf(v[e]), fabsf(v[e + 1]));
+    return m;
+}
+
+// x / 6 correctly rounded. For finite x >= 2^-125: one product with RN(1/6)
+// and one fused correction (the division-by-a-known-divisor method of
+// Brisebarre, Muller and Raina, IEEE Trans. Computers 53(8), 2004), checked
+// against the division for every such fp32 x; below 2^-125 (subnormal
+// quotients), and for inf or NaN, the division itself.
+__device__ __forceinline__ float div6(float x) {
+    if (!(x >= 0x1p-125f && x <= 0x1.fffffep127f)) return __fdiv_rn(x, 6.0f);
+    constexpr float C = 1.0f / 6.0f;
+    const float q = __fmul_rn(x, C);
+    const float r = __fmaf_rn(-q, 6.0f, x);
+    return __fmaf_rn(r, C, q);
+}
 __device__ __forceinline__ float2 neg2(float2 a) { return make_float2(-a.x, -a.y); }
 
 // One butterfly stage of half-width H >= 2 over N elements, packed x2.
@@ -134,6 +162,15 @@ __device__ float nvfp4_encode_scale(const QuantParams& p, float* red_smem, bool 
     return s_enc;
 }
 
+// rtab[c] = s_enc / S(c) for every E4M3 code c the saturating conversion can
+// produce (1-126; S(0) = 0 gives 0), the same divisions as per block, once per
+// CTA. Ends with a CTA barrier.
+__device__ void fill_rtab(float* rtab, float s_enc) {
+    for (int c = threadIdx.x; c < 128; c += blockDim.x)
+        rtab[c] = (c == 0 || c == 127) ? 0.0f : __fdiv_rn(s_enc, e4m3_decode((uint32_t)c));
+    __syncthreads();
+}
+
 // The four Quartet II scale uniforms of one Philox quad, computed once per quad.
 struct ScaleRng {
     uint64_t quad = ~0ull;
@@ -169,39 +206,43 @@ struct Group {
     }
 
     // v = c * H * (D x) per n_h chunk; D was applied to the packed words.
+    // SCALE = false leaves out the factor c (the amax pass applies it once to
+    // the maximum: rounding c * y is monotone in y).
+    template <bool SCALE = true>
     __device__ __forceinline__ static void rotate(float* v) {
         if constexpr (NH > 0) {
 #pragma unroll
             for (int hb = 0; hb < G / NH; ++hb) {
                 float* w = v + hb * NH;
                 fwht<NH>(w);
+                if constexpr (SCALE) {
 #pragma unroll
-                for (int e = 0; e < NH; e += 2) {
-                    const float2 r = __fmul2_rn(f2(w[e], w[e + 1]), f2(had_norm<NH>(), had_norm<NH>()));
-                    w[e] = r.x; w[e + 1] = r.y;
+                    for (int e = 0; e < NH; e += 2) {
+                        const float2 r = __fmul2_rn(f2(w[e], w[e + 1]), f2(had_norm<NH>(), had_norm<NH>()));
+                        w[e] = r.x; w[e + 1] = r.y;
+                    }
                 }
             }
         }
     }
 
-    __device__ __forceinline__ static void quantize(float* v, float s_enc, const QuantParams& p, uint64_t elem0,
-                                                    uint64_t block0, ScaleRng& srng, uint32_t* codes,
-                                                    uint32_t* scodes) {
+    // rtab[c] = s_enc / (E4M3 value of c) for codes 1-126, 0 for code 0.
+    __device__ __forceinline__ static void quantize(float* v, float s_enc, const float* rtab, const QuantParams& p,
+                                                    uint64_t elem0, uint64_t block0, ScaleRng& srng,
+                                                    uint32_t* codes, uint32_t* scodes) {
 #pragma unroll
         for (int b = 0; b < G / NB; ++b) {
             float* vb = v + b * NB;
             // block scale from the block amax
-            float am = 0.0f;
-#pragma unroll
-            for (int e = 0; e < NB; ++e) am = fmaxf(am, fabsf(vb[e]));
+            const float am = abs_max<NB>(0.0f, vb);
             float rmul, S;
             uint32_t scode;
             if constexpr (FMT == kNvfp4) {
-                const float d = __fdiv_rn(am, 6.0f);
+                const float d = div6(am);
                 const float t = __fmul_rn(d, s_enc);
-                scode = e4m3_rn(t);
+                scode = e4m3_rn(t);  // saturating: codes 0-126
                 S = e4m3_decode(scode);
-                rmul = (S == 0.0f) ? 0.0f : __fdiv_rn(s_enc, S);
+                rmul = rtab[scode];
             } else {
                 if (am == 0.0f) {
                     scode = 0u;
@@ -316,8 +357,12 @@ __global__ void __launch_bounds__(kThreads, 2)
         ring_init(ring);
     }
     __syncthreads();
+    __shared__ float rtab[128];
     float s_enc = 1.0f;
-    if constexpr (!AMAX_ONLY && FMT == kNvfp4) s_enc = nvfp4_encode_scale(p, red, blockIdx.x == 0);
+    if constexpr (!AMAX_ONLY && FMT == kNvfp4) {
+        s_enc = nvfp4_encode_scale(p, red, blockIdx.x == 0);
+        fill_rtab(rtab, s_enc);
+    }
     if constexpr (!AMAX_ONLY && FMT == kMxfp4) {
         if (blockIdx.x == 0 && tid == 0) *p.tensor_scale = 1.0f;
     }
@@ -372,13 +417,12 @@ __global__ void __launch_bounds__(kThreads, 2)
                 v[8 * c8 + 6] = bf16lo(w3); v[8 * c8 + 7] = bf16hi(w3);
             }
             if constexpr (AMAX_ONLY) {
-                Group<kNvfp4, kRtn, NH>::rotate(v);
-#pragma unroll
-                for (int e = 0; e < G; ++e) amax_acc = fmaxf(amax_acc, fabsf(v[e]));
+                Group<kNvfp4, kRtn, NH>::template rotate<false>(v);
+                amax_acc = abs_max<G>(amax_acc, v);
             } else {
                 Grp::rotate(v);
                 const int64_t j0 = col0 + g * G;
-                Grp::quantize(v, s_enc, p, (uint64_t)row * (uint64_t)p.k + (uint64_t)j0,
+                Grp::quantize(v, s_enc, rtab, p, (uint64_t)row * (uint64_t)p.k + (uint64_t)j0,
                               (uint64_t)row * (uint64_t)(p.k / NB) + (uint64_t)(j0 / NB), srng,
                               codes + g * (G / 8), scodes + g * (G / NB));
             }
@@ -417,7 +461,10 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
         }
     }
-    if constexpr (AMAX_ONLY) write_partial(amax_acc, red, p.amax_out);
+    if constexpr (AMAX_ONLY) {
+        if constexpr (NH > 0) amax_acc = __fmul_rn(amax_acc, had_norm<NH>());  // c * max |y| = max |c * y|
+        write_partial(amax_acc, red, p.amax_out);
+    }
 }
 
 // ===========================================================================
@@ -454,8 +501,12 @@ __global__ void __launch_bounds__(kThreads, 2)
         ring_init(ring);
     }
     __syncthreads();
+    __shared__ float rtab[128];
     float s_enc = 1.0f;
-    if constexpr (!AMAX_ONLY && FMT == kNvfp4) s_enc = nvfp4_encode_scale(p, red, blockIdx.x == 0);
+    if constexpr (!AMAX_ONLY && FMT == kNvfp4) {
+        s_enc = nvfp4_encode_scale(p, red, blockIdx.x == 0);
+        fill_rtab(rtab, s_enc);
+    }
     if constexpr (!AMAX_ONLY && FMT == kMxfp4) {
         if (blockIdx.x == 0 && tid == 0) *p.tensor_scale = 1.0f;
     }
@@ -515,14 +566,13 @@ __global__ void __launch_bounds__(kThreads, 2)
             const int64_t c = c0 + chunk * 8 + (lane >> 2);  // x column = output row
             const int64_t r_grp = r0 + (int64_t)G * q;       // first k index of this group
             if constexpr (AMAX_ONLY) {
-                Group<kNvfp4, kRtn, NH>::rotate(v);
-#pragma unroll
-                for (int e = 0; e < G; ++e) amax_acc = fmaxf(amax_acc, fabsf(v[e]));
+                Group<kNvfp4, kRtn, NH>::template rotate<false>(v);
+                amax_acc = abs_max<G>(amax_acc, v);
             } else {
                 uint32_t codes[G / 8];
                 uint32_t scodes[G / NB];
                 Grp::rotate(v);
-                Grp::quantize(v, s_enc, p, (uint64_t)c * (uint64_t)p.k + (uint64_t)r_grp,
+                Grp::quantize(v, s_enc, rtab, p, (uint64_t)c * (uint64_t)p.k + (uint64_t)r_grp,
                               (uint64_t)c * (uint64_t)(p.k / NB) + (uint64_t)(r_grp / NB), srng, codes, scodes);
                 if (c < p.rows && r_grp < p.k) {
                     uint8_t* dst = p.codes + c * (p.k / 2) + r_grp / 2;
@@ -556,7 +606,10 @@ __global__ void __launch_bounds__(kThreads, 2)
         __syncwarp();
         if (lane == 0) mbar_arrive(&ring.empty[s]);
     }
-    if constexpr (AMAX_ONLY) write_partial(amax_acc, red, p.amax_out);
+    if constexpr (AMAX_ONLY) {
+        if constexpr (NH > 0) amax_acc = __fmul_rn(amax_acc, had_norm<NH>());  // c * max |y| = max |c * y|
+        write_partial(amax_acc, red, p.amax_out);
+    }
 }
 
 int g_sm_count = 0;
