@@ -235,8 +235,10 @@ def run_ours(args, rank, world, local_rank):
     gemm_achieved = sum(gemm_flops) / (sum(gemm_ms) * 1e-3) / 1e12
     traffic = measured_gemm_traffic()
 
-    # quantizer sweep workload (GB/s of algorithmic bytes), L2 flushed between launches
+    # quantizer sweep workload (GB/s of algorithmic bytes), L2 flushed between launches,
+    # and the same kernels on dY [16384 x 28672] (940 MB, steady state)
     quant = quant_sweep(Q, inputs, dev, stream, peaks)
+    quant["large"] = quant_large(Q, dY, stream, peaks)
 
     # linear API (device-resident) and end to end with host buffers
     api_ms = linear_api_time(Q, X, W, dY, rec, seed, args, stream, dev)
@@ -332,6 +334,49 @@ def quant_sweep(Q, inputs, dev, stream, peaks):
     return {"workload": "quantizer sweep tensor [8192x4096] bf16, Student-t(3)*0.02*LogNormal(0,1) column gains",
             "bytes_per_elem": "2 read + 0.5 codes + 1/16 (NVFP4) or 1/32 (MXFP4) scales; amax pass 2 read",
             "l2": "256 MiB buffer written before every launch", "unit": "GB/s", "cases": res}
+
+
+def quant_large(Q, T, stream, peaks):
+    """Quantizer and amax kernels on a tensor far larger than L2 (the layer's
+    dY, [16384 x 28672] bf16, 940 MB): steady-state GB/s of algorithmic bytes
+    (2 B read + 0.5 B codes + 1/16 B scales per element; amax: 2 B read)."""
+    import torch
+    R, C = T.shape
+    dev = T.device
+    ws = torch.empty((Q.quantize_workspace_bytes(),), dtype=torch.uint8, device=dev)
+    seed = Q.make_seed(7, 8)
+    res = {}
+
+    def timeit(fn, n=5):
+        for _ in range(2):
+            fn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / n
+
+    for name, rnd, had, axis in (("nvfp4_rtn_none_row", Q.RTN, Q.HAD_NONE, Q.ROW),
+                                 ("nvfp4_q2_rand16_row", Q.QUARTET2, Q.HAD_RAND16, Q.ROW),
+                                 ("nvfp4_q2_rand16_col", Q.QUARTET2, Q.HAD_RAND16, Q.COL)):
+        rows, k = (R, C) if axis == Q.ROW else (C, R)
+        q = Q.empty_qtensor(Q.NVFP4, rows, k, dev)
+        am = Q.amax(T, had, axis, seed, workspace=ws, stream=stream)
+        ms = timeit(lambda: Q.quantize(T, Q.NVFP4, rnd, had, axis, seed, amax_in=am, out=q, workspace=ws,
+                                       stream=stream))
+        gbs = R * C * (2 + 0.5 + 1 / 16) / (ms * 1e-3) / 1e9
+        res[name] = {"ms": round(ms, 4), "GB/s": round(gbs, 1), "frac_of_measured_hbm": round(gbs / peaks["hbm_gbs"], 3)}
+        del q
+    for name, axis in (("amax_rand16_row", Q.ROW), ("amax_rand16_col", Q.COL)):
+        am = torch.empty((1,), dtype=torch.float32, device=dev)
+        ms = timeit(lambda: Q.amax(T, Q.HAD_RAND16, axis, seed, out=am, workspace=ws, stream=stream))
+        gbs = R * C * 2 / (ms * 1e-3) / 1e9
+        res[name] = {"ms": round(ms, 4), "GB/s": round(gbs, 1), "frac_of_measured_hbm": round(gbs / peaks["hbm_gbs"], 3)}
+    Q.status()
+    return {"workload": f"dY [{R}x{C}] bf16 N(0,1e-3), 940 MB (larger than L2; no flush)", "unit": "GB/s",
+            "cases": res}
 
 
 def linear_api_time(Q, X, W, dY, rec, seed, args, stream, dev):

@@ -23,12 +23,14 @@
 //   warp 0, one lane: TMA producer into a shared-memory ring (A and B tiles
 //     with 128-byte swizzle, and the scale atoms, which the quantizers store in
 //     the MMA's 512-byte atom layout).
-//   warp 1, one lane: MMA issuer: 4 MMAs per 256-wide k-tile and ONE commit,
-//     which frees both the ring stage and its tensor-memory scale slot.
+//   warp 1, one lane: MMA issuer: one barrier wait, 4 MMAs per 256-wide
+//     k-tile and ONE commit, which frees both the ring stage and its
+//     tensor-memory scale slot.
 //   warps 2-5: scale writers, one per 32-lane quarter of tensor memory. They
 //     read the k-tile's scale atoms from shared memory and write them with
 //     tcgen05.st into the scale slot of the same index as the ring stage (each
-//     quarter holds the same 32 atom rows, as the MMA reads them).
+//     quarter holds the same 32 atom rows, as the MMA reads them), then wait
+//     for the stage's operand tiles before signalling the MMA warp.
 //   warps 6-13: epilogue, two per lane quarter, 128 accumulator columns each:
 //     drain tensor memory to registers (tcgen05.ld), hand the accumulator back
 //     to the MMA warp before the global stores (bf16) or after the first 32
@@ -461,7 +463,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 if (lt > 0 && !mbar_wait(acc_empty, (lt - 1) & 1)) break;
                 tc_fence_after();
                 for (int kt = 0; kt < KT; ++kt) {
-                    if (!mbar_wait(&full[s], ph) || !mbar_wait(&sf_full[s], ph)) {
+                    // sf_full[s] completes after the scale writers saw full[s]:
+                    // one wait covers the operand tiles and the scales
+                    if (!mbar_wait(&sf_full[s], ph)) {
                         ok = false;
                         break;
                     }
@@ -495,6 +499,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 }
                 write_scales<ATOMS_PER_KT>(tmem_lane, s, smem_u32(sSFA + s * SFA_STAGE), smem_u32(sSFB + s * SFB_STAGE),
                                            lane, warp & 3);
+                if (!mbar_wait(&full[s], ph)) {  // the operand tiles too, so the MMA waits once
+                    ok = false;
+                    break;
+                }
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sf_full[s]);
@@ -637,7 +645,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                 if (lt > 0 && !mbar_wait_cluster(acc_empty, (lt - 1) & 1)) break;
                 tc_fence_after();
                 for (int kt = 0; kt < KT; ++kt) {
-                    if (!mbar_wait_cluster(&full[s], ph) || !mbar_wait_cluster(&sf_full[s], ph)) {
+                    // sf_full[s] completes after the leader's scale writers saw
+                    // full[s] (both CTAs' operand tiles): one wait covers all
+                    if (!mbar_wait_cluster(&sf_full[s], ph)) {
                         ok = false;
                         break;
                     }
@@ -671,6 +681,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                 }
                 write_scales<ATOMS_PER_KT>(tmem_lane, s, smem_u32(sSFA + s * P_SFA), smem_u32(sSFB + s * P_SFB), lane,
                                            warp & 3);
+                // the leader's writers also wait for both CTAs' operand tiles
+                // (they complete on the leader's full[s]), so the MMA waits once
+                if (rank == 0 && !mbar_wait_cluster(&full[s], ph)) {
+                    ok = false;
+                    break;
+                }
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&sf_full[s]), 0));
