@@ -359,6 +359,9 @@ def quant_large(Q, T, stream, peaks):
         return e0.elapsed_time(e1) / n
 
     for name, rnd, had, axis in (("nvfp4_rtn_none_row", Q.RTN, Q.HAD_NONE, Q.ROW),
+                                 ("nvfp4_rtn_rand16_row", Q.RTN, Q.HAD_RAND16, Q.ROW),
+                                 ("nvfp4_rtn_rand16_col", Q.RTN, Q.HAD_RAND16, Q.COL),
+                                 ("nvfp4_sr_rand16_row", Q.SR, Q.HAD_RAND16, Q.ROW),
                                  ("nvfp4_q2_rand16_row", Q.QUARTET2, Q.HAD_RAND16, Q.ROW),
                                  ("nvfp4_q2_rand16_col", Q.QUARTET2, Q.HAD_RAND16, Q.COL)):
         rows, k = (R, C) if axis == Q.ROW else (C, R)

@@ -127,18 +127,25 @@ __device__ __forceinline__ float e4m3_decode(uint32_t code) {
     return __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
 }
 
-// Stochastic rounding of t >= 0 onto the E4M3 grid (saturating at 448).
-__device__ __forceinline__ uint32_t e4m3_sr(float t, float rho) {
+// Stochastic rounding of t >= 0 onto the E4M3 grid (saturating at 448) with
+// the Philox word w (uniform rho = (w >> 8) * 2^-24): code of the largest
+// E4M3 value lo <= t, plus one iff rho < (t - lo) / gap.
+// For t in [2^-6, 448) (normal E4M3 values, 3 mantissa bits) lo is t with its
+// fp32 mantissa cut to 3 bits, the code is the fp32 exponent and top 3
+// mantissa bits rebased (bias 127 -> 7), and (t - lo) / gap is exactly the
+// cut-off 20 mantissa bits over 2^20, so the comparison is an integer one:
+// (w >> 8) < (those 20 bits) * 16. Below 2^-6 (subnormal E4M3, gap 2^-9):
+// t * 2^9 split into integer code and fraction.
+__device__ __forceinline__ uint32_t e4m3_sr(float t, uint32_t w) {
     if (!(t < 448.0f)) return 0x7Eu;
-    uint32_t c = e4m3_rn(t);
-    if (e4m3_decode(c) > t) c -= 1u;  // c = largest code with value <= t
-    const float lo = e4m3_decode(c);
-    const float hi = e4m3_decode(c + 1u);
-    // the gap is a power of two in [2^-9, 32]: multiplying by its exact
-    // reciprocal equals the division
-    const uint32_t gap_exp = (__float_as_uint(hi - lo) >> 23) & 0xFFu;
-    const float p = (t - lo) * __uint_as_float((254u - gap_exp) << 23);
-    return rho < p ? c + 1u : c;
+    if (t >= 0x1p-6f) {
+        const uint32_t b = __float_as_uint(t);
+        const uint32_t lo = (b >> 20) - (120u << 3);
+        return lo + ((w >> 8) < ((b & 0xFFFFFu) << 4) ? 1u : 0u);
+    }
+    const float x = t * 512.0f;  // exact
+    const float fl = floorf(x);
+    return (uint32_t)fl + (uniform24(w) < x - fl ? 1u : 0u);
 }
 
 // floor(log2(a)) of a positive finite fp32, exact (subnormals included).

@@ -175,14 +175,15 @@ __device__ void fill_rtab(float* rtab, float s_enc) {
 struct ScaleRng {
     uint64_t quad = ~0ull;
     uint4 w;
-    __device__ __forceinline__ float uniform(const QuantParams& p, uint64_t block_index) {
+    // Philox word of the block (its uniform is (word >> 8) * 2^-24).
+    __device__ __forceinline__ uint32_t word(const QuantParams& p, uint64_t block_index) {
         const uint64_t q = block_index >> 2;
         if (q != quad) {
             w = philox_quad(p.sr_seed, p.sr_tag_scale, q);
             quad = q;
         }
         const uint32_t i = (uint32_t)(block_index & 3);
-        return uniform24(i == 0 ? w.x : i == 1 ? w.y : i == 2 ? w.z : w.w);
+        return i == 0 ? w.x : i == 1 ? w.y : i == 2 ? w.z : w.w;
     }
 };
 
@@ -292,11 +293,11 @@ struct Group {
                 const float den = tree_sum<NB>(sb);
                 const float alpha = (den == 0.0f) ? 1.0f : __fdiv_rn(num, den);
                 const float t = __fmul_rn(S, alpha);
-                const float rho = srng.uniform(p, block0 + b);
+                const uint32_t rw = srng.word(p, block0 + b);
                 if constexpr (FMT == kNvfp4)
-                    scode = e4m3_sr(t, rho);
+                    scode = e4m3_sr(t, rw);
                 else
-                    scode = e8m0_sr(t, rho);
+                    scode = e8m0_sr(t, uniform24(rw));
             }
             scodes[b] = scode;
         }
