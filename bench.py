@@ -240,6 +240,9 @@ def run_ours(args, rank, world, local_rank):
     quant = quant_sweep(Q, inputs, dev, stream, peaks)
     quant["large"] = quant_large(Q, dY, stream, peaks)
 
+    # the other configurations of the MLP shapes (not part of the headline value)
+    layers = more_layers(Q, inputs, X, W, dY, seed, stream, dev)
+
     # linear API (device-resident) and end to end with host buffers
     api_ms = linear_api_time(Q, X, W, dY, rec, seed, args, stream, dev)
     e2e = None if args.no_e2e else e2e_time(Q, X, W, dY, rec, seed, args, stream, dev, world)
@@ -270,11 +273,84 @@ def run_ours(args, rank, world, local_rank):
                                      "wgrad": round(gemm_ms[2], 4)}},
         "step_breakdown_ms": {"quantize": [round(v, 4) for v in quant_ms], "gemm": [round(v, 4) for v in gemm_ms]},
         "quantize": quant,
+        "layers": layers,
         "linear_api_ms_per_step": round(api_ms, 4),
         "e2e": e2e,
         "gpu_launches": launches,
         "clocks": clk.summary(),
     }
+    return out
+
+
+def layer_step(Q, X, W, dY, rec, seed, steps, stream, dev):
+    """One linear layer's fwd+bwd through the six quantize and three GEMM calls
+    (the same sequence as the headline step), timed with CUDA events on the
+    launching stream: ms per step and per GEMM."""
+    import torch
+    M, K = X.shape
+    N = W.shape[0]
+    ws = torch.empty((Q.quantize_workspace_bytes(),), dtype=torch.uint8, device=dev)
+    c = rec.fprop, rec.dgrad, rec.wgrad
+    ops = [(X, c[0].fmt, c[0].rnd_a, c[0].had, Q.ROW, Q.make_seed(seed.rot, seed.sr, 0, 0)),
+           (W, c[0].fmt, c[0].rnd_b, c[0].had, Q.ROW, Q.make_seed(seed.rot, seed.sr, 0, 1)),
+           (dY, c[1].fmt, c[1].rnd_a, c[1].had, Q.ROW, Q.make_seed(seed.rot, seed.sr, 1, 2)),
+           (W, c[1].fmt, c[1].rnd_b, c[1].had, Q.COL, Q.make_seed(seed.rot, seed.sr, 1, 3)),
+           (dY, c[2].fmt, c[2].rnd_a, c[2].had, Q.COL, Q.make_seed(seed.rot, seed.sr, 2, 4)),
+           (X, c[2].fmt, c[2].rnd_b, c[2].had, Q.COL, Q.make_seed(seed.rot, seed.sr, 2, 5))]
+    qs = []
+    for (t, fmt, rnd, had, axis, sd) in ops:
+        rows, k = (t.shape[0], t.shape[1]) if axis == Q.ROW else (t.shape[1], t.shape[0])
+        qs.append(Q.empty_qtensor(fmt, rows, k, dev))
+    dw_dtype = torch.float32 if rec.dw_dtype == Q.OUT_F32 else torch.bfloat16
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    dX = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+    dW = torch.empty((N, K), dtype=dw_dtype, device=dev)
+    outs = [(0, 1, Y, torch.bfloat16), (2, 3, dX, torch.bfloat16), (4, 5, dW, dw_dtype)]
+
+    def step(ev):
+        for i, (t, fmt, rnd, had, axis, sd) in enumerate(ops):
+            Q.quantize(t, fmt, rnd, had, axis, sd, out=qs[i], workspace=ws, stream=stream)
+            if i % 2 == 1:
+                a, b, D, odt = outs[i // 2]
+                if ev is not None:
+                    ev[i // 2][0].record(stream)
+                Q.gemm(qs[a], qs[b], odt, out=D, stream=stream)
+                if ev is not None:
+                    ev[i // 2][1].record(stream)
+
+    for _ in range(3):
+        step(None)
+    torch.cuda.synchronize()
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(3)] for _ in range(steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for st in range(steps):
+        step(evs[st])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    Q.status()
+    ms = t0.elapsed_time(t1) / steps
+    gemm_ms = [statistics.mean(evs[st][g][0].elapsed_time(evs[st][g][1]) for st in range(steps)) for g in range(3)]
+    flops = 2.0 * M * N * K
+    return {"ms_per_step": round(ms, 4), "TFLOP/s": round(3 * flops / (ms * 1e-3) / 1e12, 1),
+            "gemm_ms": {"fprop": round(gemm_ms[0], 4), "dgrad": round(gemm_ms[1], 4), "wgrad": round(gemm_ms[2], 4)},
+            "gemm_TFLOP/s": round(3 * flops / (sum(gemm_ms) * 1e-3) / 1e12, 1)}
+
+
+def more_layers(Q, inputs, X, W, dY, seed, stream, dev):
+    """The other arm of the MLP up/gate configuration (MXFP4, deterministic
+    32x32 Hadamard on Wgrad) and the MLP down layer at 16384 tokens with the
+    Quartet II and the per-element SR NVFP4 recipes."""
+    import torch
+    out = {"mlp_up_AMD_MXFP4_H": layer_step(Q, X, W, dY, Q.recipe("AMD_MXFP4_H"), seed, 10, stream, dev)}
+    wl = inputs.workload("mlp_down", device=dev, M=16384)
+    for rec in ("QUARTET2_NVFP4", "NVIDIA_NVFP4"):
+        out["mlp_down_" + rec] = layer_step(Q, wl["X"], wl["W"], wl["dY"], Q.recipe(rec), seed, 10, stream, dev)
+    out["workloads"] = {"mlp_up": "X[16384x4096] W[28672x4096] dY[16384x28672]",
+                        "mlp_down": "X[16384x14336] = SiLU(N(0,1))*N(0,1), W[4096x14336] N(0,0.02), "
+                                    "dY[16384x4096] N(0,1e-3)"}
+    del wl
+    torch.cuda.empty_cache()
     return out
 
 

@@ -352,6 +352,90 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tadd
     }
 }
 
+// Epilogue of one tile for one warp with TMA stores (bf16 output): its 32
+// rows x 128 columns of the accumulator go to registers (packed bf16), the
+// accumulator is released, then each 64-column half is written row by row into
+// the warp's 4 KiB shared-memory box in the 128-byte swizzled layout (chunk j
+// of row r at chunk j ^ (r % 8): conflict-free) and stored by one TMA bulk
+// store, which writes whole lines and clips rows >= M and columns >= N. The
+// box is rewritten only after the previous store has read it.
+template <typename Release>
+__device__ __forceinline__ void epilogue_tile_tma(const GemmParams& p, const CUtensorMap* tmD, uint32_t taddr, int row0,
+                                                  int n0, float scale, uint32_t obox, int lane, Release release) {
+    uint32_t w[64];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        uint32_t acc[64];
+        tmem_ld_32x32b_x32(taddr + 64 * h, acc);
+        tmem_ld_32x32b_x32(taddr + 64 * h + 32, acc + 32);
+        tc_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 32; ++c) w[32 * h + c] = pack_bf16(acc[2 * c], acc[2 * c + 1], scale);
+    }
+    tc_fence_before();
+    __syncwarp();
+    release();
+    const uint32_t rbase = obox + (uint32_t)lane * 128u;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        if (lane == 0) bulk_wait_group_read0();
+        __syncwarp();
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            sts128(rbase + ((uint32_t)(j ^ (lane & 7)) << 4), w[32 * h + 4 * j], w[32 * h + 4 * j + 1],
+                   w[32 * h + 4 * j + 2], w[32 * h + 4 * j + 3]);
+        fence_proxy_async_shared();
+        __syncwarp();
+        if (lane == 0 && row0 < p.M && n0 + 64 * h < p.N) {  // boxes wholly outside D are skipped
+            tma_store_2d(tmD, obox, n0 + 64 * h, row0);
+            bulk_commit_group();
+        }
+    }
+}
+
+// fp32 output: the same with boxes of 32 rows x 32 columns (128-byte rows),
+// four per warp and tile. The first 32 columns are boxed and stored before the
+// accumulator is released, the other 96 are held in registers across it.
+__device__ __forceinline__ void box_f32(const GemmParams& p, const CUtensorMap* tmD, uint32_t obox, int lane,
+                                        const uint32_t* acc, int row0, int x, float scale) {
+    if (lane == 0) bulk_wait_group_read0();
+    __syncwarp();
+    const uint32_t rbase = obox + (uint32_t)lane * 128u;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const float2 a = __fmul2_rn(make_float2(__uint_as_float(acc[4 * j]), __uint_as_float(acc[4 * j + 1])),
+                                    make_float2(scale, scale));
+        const float2 b = __fmul2_rn(make_float2(__uint_as_float(acc[4 * j + 2]), __uint_as_float(acc[4 * j + 3])),
+                                    make_float2(scale, scale));
+        sts128(rbase + ((uint32_t)(j ^ (lane & 7)) << 4), __float_as_uint(a.x), __float_as_uint(a.y),
+               __float_as_uint(b.x), __float_as_uint(b.y));
+    }
+    fence_proxy_async_shared();
+    __syncwarp();
+    if (lane == 0 && row0 < p.M && x < p.N) {
+        tma_store_2d(tmD, obox, x, row0);
+        bulk_commit_group();
+    }
+}
+template <typename Release>
+__device__ __forceinline__ void epilogue_tile_tma_f32(const GemmParams& p, const CUtensorMap* tmD, uint32_t taddr,
+                                                      int row0, int n0, float scale, uint32_t obox, int lane,
+                                                      Release release) {
+    uint32_t acc[96];
+    tmem_ld_32x32b_x32(taddr, acc);
+    tc_wait_ld();
+    box_f32(p, tmD, obox, lane, acc, row0, n0, scale);
+    tmem_ld_32x32b_x32(taddr + 32, acc);
+    tmem_ld_32x32b_x32(taddr + 64, acc + 32);
+    tmem_ld_32x32b_x32(taddr + 96, acc + 64);
+    tc_wait_ld();
+    tc_fence_before();
+    __syncwarp();
+    release();
+#pragma unroll
+    for (int b = 0; b < 3; ++b) box_f32(p, tmD, obox, lane, acc + 32 * b, row0, n0 + 32 * (b + 1), scale);
+}
+
 // Grouped tile order: GM row-tiles at a time, walking down the group first.
 template <int GM>
 __device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int& mb, int& nb) {
@@ -554,14 +638,15 @@ constexpr int P_B = 128 * BK / 2;   // 16 KiB: this CTA's B rows
 constexpr int P_SFA = 4 * 512;      // up to 4 atoms of this CTA's rows
 constexpr int P_SFB = 2 * 4 * 512;  // 2 row blocks x up to 4 atoms
 constexpr int P_STAGE = P_A + P_B + P_SFA + P_SFB;
-constexpr int P_SMEM = P_STAGES * P_STAGE + 1024 + 512;
+constexpr int P_OUT_BOX = 4096;      // one epilogue warp's TMA-store box (32 rows x 128 B)
+constexpr int P_SMEM = P_STAGES * P_STAGE + kEpiWarps * P_OUT_BOX + 1024 + 512;
 constexpr int P_GROUP_M = 4;  // 256-row tiles per group of the tile order
 
 template <int FMT>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     gemm_bs_fp4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                             const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
-                            const GemmParams p) {
+                            const __grid_constant__ CUtensorMap tmD, const GemmParams p) {
     constexpr int SF_K = (FMT == kNvfp4) ? 64 : 128;
     constexpr int ATOMS_PER_KT = BK / SF_K;  // 4 or 2
     constexpr uint32_t AB_TX = 2u * (P_A + P_B);            // both CTAs, on the leader
@@ -572,7 +657,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     uint8_t* sB = sA + P_STAGES * P_A;
     uint8_t* sSFA = sB + P_STAGES * P_B;
     uint8_t* sSFB = sSFA + P_STAGES * P_SFA;
-    uint64_t* full = reinterpret_cast<uint64_t*>(sSFB + P_STAGES * P_SFB);
+    uint8_t* sOut = sSFB + P_STAGES * P_SFB;  // kEpiWarps boxes, 1024-byte aligned
+    uint64_t* full = reinterpret_cast<uint64_t*>(sOut + kEpiWarps * P_OUT_BOX);
     uint64_t* empty = full + P_STAGES;
     uint64_t* sf_load = empty + P_STAGES;   // this CTA's scale atoms of stage s landed
     uint64_t* sf_full = sf_load + P_STAGES;  // scale slot s written in both CTAs (leader's)
@@ -592,6 +678,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         prefetch_tmap(&tmB);
         prefetch_tmap(&tmSFA);
         prefetch_tmap(&tmSFB);
+        prefetch_tmap(&tmD);
         for (int s = 0; s < P_STAGES; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
@@ -702,17 +789,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         const int chalf = (warp - kFirstEpiWarp) >> 2;
         const float scale = __fmul_rn(__ldg(p.ga), __ldg(p.gb));
         const uint32_t acc_empty_leader = mapa_shared(smem_u32(acc_empty), 0);
+        const uint32_t obox = smem_u32(sOut) + (uint32_t)(warp - kFirstEpiWarp) * P_OUT_BOX;
         int lt = 0;
         for (int t = cid; t < tiles; t += nclusters, ++lt) {
             int mb, nb;
             tile_coords<P_GROUP_M>(t, num_m, num_n, mb, nb);
             if (!mbar_wait_cluster(acc_full, lt & 1)) break;
             tc_fence_after();
-            epilogue_tile(p, tmem + ((uint32_t)(lq * 32) << 16) + TMEM_D + chalf * 128,
-                          mb * 2 * BM + (int)rank * BM + lq * 32 + lane, nb * BN + chalf * 128, scale, [&] {
-                              if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
-                          });
+            const uint32_t taddr = tmem + ((uint32_t)(lq * 32) << 16) + TMEM_D + chalf * 128;
+            const int row0 = mb * 2 * BM + (int)rank * BM + lq * 32;
+            auto release = [&] {
+                if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
+            };
+            if (p.out_f32)
+                epilogue_tile_tma_f32(p, &tmD, taddr, row0, nb * BN + chalf * 128, scale, obox, lane, release);
+            else
+                epilogue_tile_tma(p, &tmD, taddr, row0, nb * BN + chalf * 128, scale, obox, lane, release);
         }
+        if (lane == 0) bulk_wait_group0();  // this warp's stores are complete
     }
 
     tc_fence_before();
@@ -745,7 +839,8 @@ cudaError_t launch_gemm(const GemmParams& p, int fmt, const CUtensorMap* tmapA, 
 }
 
 cudaError_t launch_gemm_pair(const GemmParams& p, int fmt, const CUtensorMap* tmapA, const CUtensorMap* tmapB,
-                             const CUtensorMap* tmapSFA, const CUtensorMap* tmapSFB, cudaStream_t s, int sms) {
+                             const CUtensorMap* tmapSFA, const CUtensorMap* tmapSFB, const CUtensorMap* tmapD,
+                             cudaStream_t s, int sms) {
     const int tiles = ((p.M + 2 * BM - 1) / (2 * BM)) * ((p.N + BN - 1) / BN);
     int clusters = sms / 2;
     if (clusters > tiles) clusters = tiles;
@@ -755,12 +850,12 @@ cudaError_t launch_gemm_pair(const GemmParams& p, int fmt, const CUtensorMap* tm
         e = cudaFuncSetAttribute(gemm_bs_fp4_pair_kernel<kNvfp4>, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM);
         if (e != cudaSuccess) return e;
         gemm_bs_fp4_pair_kernel<kNvfp4><<<2 * clusters, kGemmThreads, P_SMEM, s>>>(*tmapA, *tmapB, *tmapSFA,
-                                                                                   *tmapSFB, p);
+                                                                                   *tmapSFB, *tmapD, p);
     } else {
         e = cudaFuncSetAttribute(gemm_bs_fp4_pair_kernel<kMxfp4>, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM);
         if (e != cudaSuccess) return e;
         gemm_bs_fp4_pair_kernel<kMxfp4><<<2 * clusters, kGemmThreads, P_SMEM, s>>>(*tmapA, *tmapB, *tmapSFA,
-                                                                                   *tmapSFB, p);
+                                                                                   *tmapSFB, *tmapD, p);
     }
     count_launch();
     return cudaGetLastError();

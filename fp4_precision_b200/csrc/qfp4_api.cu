@@ -179,6 +179,23 @@ int make_codes_tmap(CUtensorMap* tm, const void* codes, int64_t rows, int64_t k,
     return QFP4_OK;
 }
 
+// 2-D view of the GEMM output D [M][N] (row stride ldd elements, bf16 or fp32)
+// for TMA stores: box of 128 bytes x 32 rows, 128-byte swizzle.
+int make_out_tmap(CUtensorMap* tm, void* D, int64_t M, int64_t N, int64_t ldd, bool f32) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return cuda_fail(cudaErrorNotSupported);
+    const cuuint32_t esz = f32 ? 4 : 2;
+    const cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)M};
+    const cuuint64_t strides[1] = {(cuuint64_t)ldd * esz};
+    const cuuint32_t box[2] = {128 / esz, 32};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(tm, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, dims, strides,
+                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
+    return QFP4_OK;
+}
+
 // 3-D view of a scale buffer as uint32 words: (128 words = one 512-byte atom,
 // atoms along k, 128-row blocks), box (128, atoms_per_box, depth). Atoms past
 // the buffer read as zero scales.
@@ -386,10 +403,11 @@ int gemm_impl(const qfp4_tensor* A, const qfp4_tensor* B, void* D, int64_t ldd, 
     cudaError_t e;
     if (pair) {
         const int atoms_per_kt = kGemmBK / (4 * NB);
-        CUtensorMap tSFA, tSFB;
+        CUtensorMap tSFA, tSFB, tD;
         if ((rc = make_scale_tmap(&tSFA, A->scales, M, p.atoms_k, atoms_per_kt, 1))) return rc;
         if ((rc = make_scale_tmap(&tSFB, B->scales, N, p.atoms_k, atoms_per_kt, 2))) return rc;
-        e = launch_gemm_pair(p, A->fmt, &tA, &tB, &tSFA, &tSFB, s, sms);
+        if ((rc = make_out_tmap(&tD, D, M, N, ldd, p.out_f32))) return rc;
+        e = launch_gemm_pair(p, A->fmt, &tA, &tB, &tSFA, &tSFB, &tD, s, sms);
     } else {
         e = launch_gemm(p, A->fmt, &tA, &tB, s, sms);
     }

@@ -64,9 +64,11 @@ struct GemmParams {
 cudaError_t launch_gemm(const GemmParams& p, int fmt, const CUtensorMap* tmapA, const CUtensorMap* tmapB,
                         cudaStream_t s, int sms);
 // 2-SM (CTA pair) variant; tmapSFA / tmapSFB are 3-D views of the scale
-// buffers (see make_scale_tmap in qfp4_api.cu).
+// buffers, tmapD a 2-D view of D for TMA stores (see make_scale_tmap and
+// make_out_tmap in qfp4_api.cu).
 cudaError_t launch_gemm_pair(const GemmParams& p, int fmt, const CUtensorMap* tmapA, const CUtensorMap* tmapB,
-                             const CUtensorMap* tmapSFA, const CUtensorMap* tmapSFB, cudaStream_t s, int sms);
+                             const CUtensorMap* tmapSFA, const CUtensorMap* tmapSFB, const CUtensorMap* tmapD,
+                             cudaStream_t s, int sms);
 constexpr int kGemmBM = 128, kGemmBN = 256, kGemmBK = 256;
 
 void count_launch();
