@@ -304,6 +304,33 @@ struct Group {
     }
 };
 
+// This CTA's tiles of a tiles_r x tiles_c grid (blockIdx.x, + gridDim.x, ...)
+// as (tr, tc), advanced without divisions, with the TMA ring stage and phase
+// of each.
+template <int STAGES>
+struct TileWalk {
+    int tr, tc, tiles_c, step_r, step_c, stage = 0;
+    uint32_t phase = 0;
+    __device__ __forceinline__ explicit TileWalk(int tiles_c_) : tiles_c(tiles_c_) {
+        tr = (int)blockIdx.x / tiles_c;
+        tc = (int)blockIdx.x % tiles_c;
+        step_r = (int)gridDim.x / tiles_c;
+        step_c = (int)gridDim.x % tiles_c;
+    }
+    __device__ __forceinline__ void next() {
+        tc += step_c;
+        tr += step_r;
+        if (tc >= tiles_c) {
+            tc -= tiles_c;
+            ++tr;
+        }
+        if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+        }
+    }
+};
+
 // Ring of TMA stages: full[s] completes when the tile landed, empty[s] when all
 // compute warps finished with it.
 template <int STAGES>
@@ -350,8 +377,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     __shared__ float red[33];
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int64_t tiles_c = (p.k + kRowTileCols - 1) / kRowTileCols;
-    const int64_t tiles_total = tiles_c * ((p.rows + kRowTileRows - 1) / kRowTileRows);
+    const int tiles_c = (int)((p.k + kRowTileCols - 1) / kRowTileCols);
+    const int tiles_r = (int)((p.rows + kRowTileRows - 1) / kRowTileRows);
 
     if (tid == 0) {
         prefetch_tmap(&tmap);
@@ -372,12 +399,11 @@ __global__ void __launch_bounds__(kThreads, 2)
         // ---------------- producer ----------------
         if (lane == 0) {
             int i = 0;
-            for (int64_t tile = blockIdx.x; tile < tiles_total; tile += gridDim.x, ++i) {
-                const int s = i % STAGES;
-                if (i >= STAGES && !mbar_wait(&ring.empty[s], ((i / STAGES) + 1) & 1)) break;
+            for (TileWalk<STAGES> w(tiles_c); w.tr < tiles_r; w.next(), ++i) {
+                const int s = w.stage;
+                if (i >= STAGES && !mbar_wait(&ring.empty[s], w.phase ^ 1u)) break;
                 mbar_arrive_expect_tx(&ring.full[s], STAGE_BYTES);
-                tma_load_2d(tiles + s * STAGE_BYTES, &tmap, &ring.full[s],
-                            (int32_t)((tile % tiles_c) * kRowTileCols), (int32_t)((tile / tiles_c) * kRowTileRows));
+                tma_load_2d(tiles + s * STAGE_BYTES, &tmap, &ring.full[s], w.tc * kRowTileCols, w.tr * kRowTileRows);
             }
         }
         return;
@@ -387,12 +413,11 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int64_t rows_pad = (p.rows + 127) / 128 * 128;
     float amax_acc = 0.0f;
     ScaleRng srng;
-    int i = 0;
-    for (int64_t tile = blockIdx.x; tile < tiles_total; tile += gridDim.x, ++i) {
-        const int s = i % STAGES;
-        if (!mbar_wait(&ring.full[s], (i / STAGES) & 1)) break;
-        const int64_t row = (tile / tiles_c) * kRowTileRows + tid;
-        const int64_t col0 = (tile % tiles_c) * kRowTileCols;
+    for (TileWalk<STAGES> w(tiles_c); w.tr < tiles_r; w.next()) {
+        const int s = w.stage;
+        if (!mbar_wait(&ring.full[s], w.phase)) break;
+        const int64_t row = (int64_t)w.tr * kRowTileRows + tid;
+        const int64_t col0 = (int64_t)w.tc * kRowTileCols;
         const uint32_t sbase = smem_u32(tiles + s * STAGE_BYTES) + tid * 128;
         uint32_t codes[kRowTileCols / 8];
         uint32_t scodes[kRowTileCols / 16];
@@ -494,8 +519,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     __shared__ float red[33];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int64_t tiles_c = (p.rows + kColTileCols - 1) / kColTileCols;  // output rows = x columns
-    const int64_t tiles_total = tiles_c * ((p.k + TILE_ROWS - 1) / TILE_ROWS);
+    const int tiles_c = (int)((p.rows + kColTileCols - 1) / kColTileCols);  // output rows = x columns
+    const int tiles_r = (int)((p.k + TILE_ROWS - 1) / TILE_ROWS);
 
     if (tid == 0) {
         prefetch_tmap(&tmap);
@@ -515,11 +540,11 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (warp == kComputeWarps) {
         if (lane == 0) {
             int i = 0;
-            for (int64_t tile = blockIdx.x; tile < tiles_total; tile += gridDim.x, ++i) {
-                const int s = i % STAGES;
-                if (i >= STAGES && !mbar_wait(&ring.empty[s], ((i / STAGES) + 1) & 1)) break;
-                const int64_t c0 = (tile % tiles_c) * kColTileCols;
-                const int32_t tr4 = (int32_t)(4 * (tile / tiles_c));
+            for (TileWalk<STAGES> w(tiles_c); w.tr < tiles_r; w.next(), ++i) {
+                const int s = w.stage;
+                if (i >= STAGES && !mbar_wait(&ring.empty[s], w.phase ^ 1u)) break;
+                const int32_t c0 = w.tc * kColTileCols;
+                const int32_t tr4 = 4 * w.tr;
                 mbar_arrive_expect_tx(&ring.full[s], STAGE_BYTES);
                 tma_load_5d(tiles + s * STAGE_BYTES, &tmap, &ring.full[s], (int32_t)c0, 0, tr4, 0, 0);
                 tma_load_5d(tiles + s * STAGE_BYTES + BOX_BYTES, &tmap, &ring.full[s], (int32_t)(c0 + 64), 0, tr4, 0,
@@ -533,12 +558,26 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int q = lane & 3;
     float amax_acc = 0.0f;
     ScaleRng srng;
-    int i = 0;
-    for (int64_t tile = blockIdx.x; tile < tiles_total; tile += gridDim.x, ++i) {
-        const int s = i % STAGES;
-        if (!mbar_wait(&ring.full[s], (i / STAGES) & 1)) break;
-        const int64_t c0 = (tile % tiles_c) * kColTileCols;
-        const int64_t r0 = (tile / tiles_c) * TILE_ROWS;
+    // Quartet II with 16-element groups: the 4 lanes of a column hold the 4
+    // blocks of one Philox quad (when k is a multiple of 64), so each lane
+    // computes the quad of one (chunk, column) of the warp per tile (lanes 2j
+    // and 2j + 1 the same one) and the 4 lanes that use it take its words by
+    // shuffles, instead of every lane computing it.
+    constexpr bool kSharedQuads = (RND == kQuartet2 && !AMAX_ONLY && G == 16 && NB == 16);
+    const bool shared_quads = kSharedQuads && (p.k % 64) == 0;
+    for (TileWalk<STAGES> w(tiles_c); w.tr < tiles_r; w.next()) {
+        const int s = w.stage;
+        if (!mbar_wait(&ring.full[s], w.phase)) break;
+        const int64_t c0 = (int64_t)w.tc * kColTileCols;
+        const int64_t r0 = (int64_t)w.tr * TILE_ROWS;
+        uint4 lane_quad = make_uint4(0u, 0u, 0u, 0u);
+        if constexpr (kSharedQuads) {
+            if (shared_quads) {
+                const int64_t cq = c0 + (2 * warp + (lane >> 4)) * 8 + ((lane >> 1) & 7);
+                lane_quad = philox_quad(p.sr_seed, p.sr_tag_scale,
+                                        ((uint64_t)cq * (uint64_t)(p.k / NB) + (uint64_t)(r0 / NB)) >> 2);
+            }
+        }
 #pragma unroll
         for (int ci = 0; ci < 2; ++ci) {
             const int chunk = 2 * warp + ci;  // 16 chunks of 8 columns
@@ -573,8 +612,19 @@ __global__ void __launch_bounds__(kThreads, 2)
                 uint32_t codes[G / 8];
                 uint32_t scodes[G / NB];
                 Grp::rotate(v);
-                Grp::quantize(v, s_enc, rtab, p, (uint64_t)c * (uint64_t)p.k + (uint64_t)r_grp,
-                              (uint64_t)c * (uint64_t)(p.k / NB) + (uint64_t)(r_grp / NB), srng, codes, scodes);
+                const uint64_t blk = (uint64_t)c * (uint64_t)(p.k / NB) + (uint64_t)(r_grp / NB);
+                if constexpr (kSharedQuads) {
+                    if (shared_quads) {  // this group's quad: computed by lane (ci, column) * 2
+                        const int src = (ci << 4) | ((lane >> 2) << 1);
+                        srng.w = make_uint4(__shfl_sync(0xffffffffu, lane_quad.x, src),
+                                            __shfl_sync(0xffffffffu, lane_quad.y, src),
+                                            __shfl_sync(0xffffffffu, lane_quad.z, src),
+                                            __shfl_sync(0xffffffffu, lane_quad.w, src));
+                        srng.quad = blk >> 2;
+                    }
+                }
+                Grp::quantize(v, s_enc, rtab, p, (uint64_t)c * (uint64_t)p.k + (uint64_t)r_grp, blk, srng, codes,
+                              scodes);
                 if (c < p.rows && r_grp < p.k) {
                     uint8_t* dst = p.codes + c * (p.k / 2) + r_grp / 2;
                     if constexpr (G == 16)
