@@ -168,12 +168,23 @@ def run_ours(args, rank, world, local_rank):
     gemm_flops = [2.0 * M * N * K] * 3
     quant_elems = [t.numel() for (t, *_rest) in ops]
 
+    # dY is quantized along both axes; with NVFP4 and the same Hadamard for Dgrad
+    # and Wgrad one pass gives both tensor amaxes (as qfp4_linear_bwd does)
+    fused_dy_amax = (c[1].fmt == Q.NVFP4 and c[2].fmt == Q.NVFP4 and c[1].had == c[2].had
+                     and c[1].had in (Q.HAD_NONE, Q.HAD_DET16, Q.HAD_RAND16))
+    dy_amax = torch.empty((2,), dtype=torch.float32, device=dev)
+
     def step(ev=None):
         # ev: list of (start, end) event pairs per kernel group, or None
         for i, (t, fmt, rnd, had, axis, sd) in enumerate(ops):
             if ev is not None:
                 ev[i][0].record(stream)
-            Q.quantize(t, fmt, rnd, had, axis, sd, out=qs[i], workspace=ws, stream=stream)
+            am = None
+            if fused_dy_amax and i == 2:
+                Q.amax_rowcol(dY, had, ops[2][5], ops[4][5], out=dy_amax, workspace=ws, stream=stream)
+            if fused_dy_amax and i in (2, 4):
+                am = dy_amax[0:1] if i == 2 else dy_amax[1:2]
+            Q.quantize(t, fmt, rnd, had, axis, sd, amax_in=am, out=qs[i], workspace=ws, stream=stream)
             if ev is not None:
                 ev[i][1].record(stream)
             if i == 1:
@@ -307,9 +318,18 @@ def layer_step(Q, X, W, dY, rec, seed, steps, stream, dev):
     dW = torch.empty((N, K), dtype=dw_dtype, device=dev)
     outs = [(0, 1, Y, torch.bfloat16), (2, 3, dX, torch.bfloat16), (4, 5, dW, dw_dtype)]
 
+    fused_dy_amax = (c[1].fmt == Q.NVFP4 and c[2].fmt == Q.NVFP4 and c[1].had == c[2].had
+                     and c[1].had in (Q.HAD_NONE, Q.HAD_DET16, Q.HAD_RAND16))
+    dy_amax = torch.empty((2,), dtype=torch.float32, device=dev)
+
     def step(ev):
         for i, (t, fmt, rnd, had, axis, sd) in enumerate(ops):
-            Q.quantize(t, fmt, rnd, had, axis, sd, out=qs[i], workspace=ws, stream=stream)
+            am = None
+            if fused_dy_amax and i == 2:
+                Q.amax_rowcol(dY, had, ops[2][5], ops[4][5], out=dy_amax, workspace=ws, stream=stream)
+            if fused_dy_amax and i in (2, 4):
+                am = dy_amax[0:1] if i == 2 else dy_amax[1:2]
+            Q.quantize(t, fmt, rnd, had, axis, sd, amax_in=am, out=qs[i], workspace=ws, stream=stream)
             if i % 2 == 1:
                 a, b, D, odt = outs[i // 2]
                 if ev is not None:

@@ -442,9 +442,13 @@ bool valid_cfg(const qfp4_gemm_cfg& g) {
 bool valid_dtype(int32_t d) { return d == QFP4_OUT_BF16 || d == QFP4_OUT_F32; }
 
 int linear_layout(int backward, int64_t M, int64_t N, int64_t K, const qfp4_recipe* r, uint8_t* ws, qfp4_tensor* t,
-                  float** partials, size_t* total) {
+                  float** partials, size_t* total, float** dy_amax = nullptr) {
     Carver c{ws, 0};
     *partials = static_cast<float*>(c.take(qfp4_quantize_workspace_bytes()));
+    if (backward) {
+        float* a = static_cast<float*>(c.take(2 * sizeof(float)));  // dY's row and column amax
+        if (dy_amax) *dy_amax = a;
+    }
     if (!backward) {
         carve_operand(c, &t[0], r->fprop.fmt, M, K);  // X along K
         carve_operand(c, &t[1], r->fprop.fmt, N, K);  // W along K
@@ -473,6 +477,59 @@ qfp4_seed op_seed(const qfp4_seed* s, uint32_t gemm, uint32_t operand) {
     o.rot_stream = gemm;
     o.sr_stream = operand;
     return o;
+}
+
+// Both orientations' rotated amax. n_h <= 16: one read of x by the column
+// kernel (its tile serves 16-element groups of both axes); n_h = 32: two passes.
+int amax_rowcol_impl(const void* x, int64_t R, int64_t C, int64_t ld, int32_t had, const qfp4_seed* seed_row,
+                     const qfp4_seed* seed_col, float* amax_row, float* amax_col, void* workspace,
+                     size_t workspace_bytes, cudaStream_t s) {
+    int rc = bind_context(s);  // callers may run on threads without a current context
+    if (rc) return rc;
+    int sms = 0;
+    if ((rc = check_device(&sms))) return rc;
+    Geometry gr, gc;
+    if ((rc = validate_input(x, R, C, ld, had, QFP4_AXIS_ROW, &gr))) return rc;
+    if ((rc = validate_input(x, R, C, ld, had, QFP4_AXIS_COL, &gc))) return rc;
+    if (amax_row == nullptr || amax_col == nullptr) return QFP4_ERR_INVALID_ARG;
+    if (had_random(had) && (seed_row == nullptr || seed_col == nullptr)) return QFP4_ERR_INVALID_ARG;
+    if (workspace == nullptr || workspace_bytes < qfp4_quantize_workspace_bytes()) return QFP4_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return QFP4_ERR_MISALIGNED;
+    if (R == 0 || C == 0) {
+        cudaError_t e = cudaMemsetAsync(amax_row, 0, sizeof(float), s);
+        if (e == cudaSuccess) e = cudaMemsetAsync(amax_col, 0, sizeof(float), s);
+        return e == cudaSuccess ? QFP4_OK : cuda_fail(e);
+    }
+    const uint32_t signs_row = had_random(had) ? host_sign_bits(seed_row->rot, seed_row->rot_stream) : 0u;
+    const uint32_t signs_col = had_random(had) ? host_sign_bits(seed_col->rot, seed_col->rot_stream) : 0u;
+    float* partials = static_cast<float*>(workspace);
+    const int nh = had_n(had);
+    cudaError_t e;
+    if (nh <= 16) {
+        QuantParams p{};
+        p.x = static_cast<const uint16_t*>(x);
+        p.R = R; p.C = C; p.ld = ld;
+        p.rows = gc.rows; p.k = gc.k;
+        p.signs = signs_col;
+        p.signs_row = signs_row;
+        const int n = amax_partial_count(sms, quant_tiles(QFP4_AXIS_COL, gc.rows, gc.k, 16));
+        if (2 * n > kMaxAmaxPartials) return QFP4_ERR_WORKSPACE;
+        p.amax_out = partials;
+        p.amax_out_row = partials + n;
+        CUtensorMap tm;
+        if ((rc = make_input_tmap(&tm, x, R, C, ld, QFP4_AXIS_COL, 16))) return rc;
+        e = launch_amax_rowcol(p, nh, &tm, n, s);
+        if (e == cudaSuccess) e = launch_reduce_max(partials, n, amax_col, s);
+        if (e == cudaSuccess) e = launch_reduce_max(partials + n, n, amax_row, s);
+    } else {
+        int n = 0;
+        if ((rc = run_amax(x, R, C, ld, had, QFP4_AXIS_ROW, signs_row, gr, partials, &n, sms, s))) return rc;
+        e = launch_reduce_max(partials, n, amax_row, s);
+        if (e != cudaSuccess) return cuda_fail(e);
+        if ((rc = run_amax(x, R, C, ld, had, QFP4_AXIS_COL, signs_col, gc, partials, &n, sms, s))) return rc;
+        e = launch_reduce_max(partials, n, amax_col, s);
+    }
+    return e == cudaSuccess ? QFP4_OK : cuda_fail(e);
 }
 
 }  // namespace
@@ -548,6 +605,13 @@ int qfp4_amax(const void* x, int64_t R, int64_t C, int64_t ld, int32_t had, int3
     if ((rc = run_amax(x, R, C, ld, had, axis, signs, g, partials, &n, sms, s))) return rc;
     cudaError_t e = launch_reduce_max(partials, n, amax, s);
     return e == cudaSuccess ? QFP4_OK : cuda_fail(e);
+}
+
+int qfp4_amax_rowcol(const void* x, int64_t R, int64_t C, int64_t ld, int32_t had, const qfp4_seed* seed_row,
+                     const qfp4_seed* seed_col, float* amax_row, float* amax_col, void* workspace,
+                     size_t workspace_bytes, void* stream) {
+    return amax_rowcol_impl(x, R, C, ld, had, seed_row, seed_col, amax_row, amax_col, workspace, workspace_bytes,
+                            static_cast<cudaStream_t>(stream));
 }
 
 int qfp4_quantize(const void* x, int64_t R, int64_t C, int64_t ld, int32_t fmt, int32_t rounding, int32_t had,
@@ -631,21 +695,32 @@ int qfp4_linear_bwd(const void* dY, const void* X, const void* W, void* dX, void
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     qfp4_tensor t[4];
     float* partials;
+    float* dy_amax;
     size_t total;
-    linear_layout(1, M, N, K, recipe, static_cast<uint8_t*>(workspace), t, &partials, &total);
+    linear_layout(1, M, N, K, recipe, static_cast<uint8_t*>(workspace), t, &partials, &total, &dy_amax);
     const size_t pws = qfp4_quantize_workspace_bytes();
     const qfp4_gemm_cfg& d = recipe->dgrad;
     const qfp4_gemm_cfg& w = recipe->wgrad;
-    // Dgrad dX[M,K] = dY[M,N] . W[N,K]: reduce over N.
     qfp4_seed s0 = op_seed(seed, 1, 2), s1 = op_seed(seed, 1, 3);
-    if ((rc = quantize_impl(dY, M, N, N, d.fmt, d.rnd_a, d.had, QFP4_AXIS_ROW, &s0, nullptr, &t[0], partials, pws, s)))
+    qfp4_seed s2 = op_seed(seed, 2, 4), s3 = op_seed(seed, 2, 5);
+    // dY is quantized along both axes (Dgrad: along N; Wgrad: along M). When
+    // both are NVFP4 with the same Hadamard (size <= 16; the sign vectors
+    // differ per GEMM), one read of dY gives both tensor amaxes.
+    const float* am_row = nullptr;
+    const float* am_col = nullptr;
+    if (d.fmt == QFP4_NVFP4 && w.fmt == QFP4_NVFP4 && d.had == w.had && had_n(d.had) <= 16) {
+        if ((rc = amax_rowcol_impl(dY, M, N, N, d.had, &s0, &s2, dy_amax, dy_amax + 1, partials, pws, s))) return rc;
+        am_row = dy_amax;
+        am_col = dy_amax + 1;
+    }
+    // Dgrad dX[M,K] = dY[M,N] . W[N,K]: reduce over N.
+    if ((rc = quantize_impl(dY, M, N, N, d.fmt, d.rnd_a, d.had, QFP4_AXIS_ROW, &s0, am_row, &t[0], partials, pws, s)))
         return rc;
     if ((rc = quantize_impl(W, N, K, K, d.fmt, d.rnd_b, d.had, QFP4_AXIS_COL, &s1, nullptr, &t[1], partials, pws, s)))
         return rc;
     if ((rc = gemm_impl(&t[0], &t[1], dX, K, recipe->dx_dtype, s))) return rc;
     // Wgrad dW[N,K] = dY^T[N,M] . X[M,K]: reduce over M (tokens).
-    qfp4_seed s2 = op_seed(seed, 2, 4), s3 = op_seed(seed, 2, 5);
-    if ((rc = quantize_impl(dY, M, N, N, w.fmt, w.rnd_a, w.had, QFP4_AXIS_COL, &s2, nullptr, &t[2], partials, pws, s)))
+    if ((rc = quantize_impl(dY, M, N, N, w.fmt, w.rnd_a, w.had, QFP4_AXIS_COL, &s2, am_col, &t[2], partials, pws, s)))
         return rc;
     if ((rc = quantize_impl(X, M, K, K, w.fmt, w.rnd_b, w.had, QFP4_AXIS_COL, &s3, nullptr, &t[3], partials, pws, s)))
         return rc;

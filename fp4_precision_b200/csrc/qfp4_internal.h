@@ -29,6 +29,10 @@ struct QuantParams {
     const float* amax_in;         // NVFP4: caller-provided amax (overrides partials)
     float* amax_out;              // amax pass: partial maxima written here
     uint32_t signs;               // random Hadamard sign bits (0 for deterministic / none)
+    // Row-and-column amax pass (column kernel): the row orientation's sign bits
+    // and partial maxima.
+    uint32_t signs_row;
+    float* amax_out_row;
     uint64_t sr_seed;
     uint32_t sr_tag_elem;         // kTagElement | stream << 4
     uint32_t sr_tag_scale;        // kTagScale | stream << 4
@@ -40,6 +44,10 @@ cudaError_t launch_amax(const QuantParams& p, int axis, int nh, const CUtensorMa
                         cudaStream_t s);
 cudaError_t launch_quant(const QuantParams& p, int fmt, int rnd, int nh, int axis, const CUtensorMap* tmap,
                          cudaStream_t s);
+// One pass of the column kernel (tmap: its 5-D view, group 16) that writes the
+// column orientation's partial maxima to p.amax_out and the row orientation's
+// to p.amax_out_row (n_partials each). nh: 0 or 16.
+cudaError_t launch_amax_rowcol(const QuantParams& p, int nh, const CUtensorMap* tmap, int n_partials, cudaStream_t s);
 cudaError_t launch_reduce_max(const float* in, int n, float* out, cudaStream_t s);
 // Column-mode geometry: group G = max(block, n_h), tile = 4G rows x 128 columns.
 int col_group(int fmt_or_amax_block, int nh);

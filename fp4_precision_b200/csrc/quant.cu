@@ -504,7 +504,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 // Lane l of an ldmatrix.x4 supplies row l % 8 of matrix l / 8, i.e. smem row
 // s = l + 32u; after the transposing load, lane (c = l / 4, q = l % 4) holds
 // x-rows Gq + 8u + [0, 8) of column c.
-template <int FMT, int RND, int NH, bool AMAX_ONLY, int STAGES>
+template <int FMT, int RND, int NH, bool AMAX_ONLY, int STAGES, bool DUAL = false>
 __global__ void __launch_bounds__(kThreads, 2)
     quant_col_kernel(const __grid_constant__ CUtensorMap tmap, const QuantParams p) {
     using Grp = Group<FMT, RND, NH>;
@@ -556,7 +556,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 
     const int64_t rows_pad = (p.rows + 127) / 128 * 128;
     const int q = lane & 3;
-    float amax_acc = 0.0f;
+    float amax_acc = 0.0f, amax_row_acc = 0.0f;
     ScaleRng srng;
     // Quartet II with 16-element groups: the 4 lanes of a column hold the 4
     // blocks of one Philox quad (when k is a multiple of 64), so each lane
@@ -608,6 +608,38 @@ __global__ void __launch_bounds__(kThreads, 2)
             if constexpr (AMAX_ONLY) {
                 Group<kNvfp4, kRtn, NH>::template rotate<false>(v);
                 amax_acc = abs_max<G>(amax_acc, v);
+                if constexpr (DUAL) {
+                    // Row orientation from the same tile: thread t takes shared-
+                    // memory row t % 64 (some x-row of the tile; the max does not
+                    // care which) and its 16-column group 2 (t / 64) + ci, two
+                    // 16-byte chunks of a 128-byte swizzled row (8 consecutive
+                    // lanes: 8 distinct rows mod 8, conflict-free).
+                    static_assert(G == 16, "the row-and-column amax pass uses 16-row groups");
+                    const int srow = tid & 63;
+                    const int g16 = 2 * (tid >> 6) + ci;  // 0..7 over the tile's 128 columns
+                    const uint32_t rb = smem_u32(tiles + s * STAGE_BYTES + (g16 >> 2) * BOX_BYTES) + srow * 128;
+                    float vr[16];
+#pragma unroll
+                    for (int c8 = 0; c8 < 2; ++c8) {
+                        const int chunk = 2 * (g16 & 3) + c8;
+                        uint32_t w0, w1, w2, w3;
+                        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                                     : "=r"(w0), "=r"(w1), "=r"(w2), "=r"(w3)
+                                     : "r"(rb + ((chunk ^ (srow & 7)) << 4)));
+                        if (NH > 0 && p.signs_row != 0u) {
+                            w0 ^= Grp::sign_mask(p.signs_row, 4 * c8 + 0);
+                            w1 ^= Grp::sign_mask(p.signs_row, 4 * c8 + 1);
+                            w2 ^= Grp::sign_mask(p.signs_row, 4 * c8 + 2);
+                            w3 ^= Grp::sign_mask(p.signs_row, 4 * c8 + 3);
+                        }
+                        vr[8 * c8 + 0] = bf16lo(w0); vr[8 * c8 + 1] = bf16hi(w0);
+                        vr[8 * c8 + 2] = bf16lo(w1); vr[8 * c8 + 3] = bf16hi(w1);
+                        vr[8 * c8 + 4] = bf16lo(w2); vr[8 * c8 + 5] = bf16hi(w2);
+                        vr[8 * c8 + 6] = bf16lo(w3); vr[8 * c8 + 7] = bf16hi(w3);
+                    }
+                    Group<kNvfp4, kRtn, NH>::template rotate<false>(vr);
+                    amax_row_acc = abs_max<16>(amax_row_acc, vr);
+                }
             } else {
                 uint32_t codes[G / 8];
                 uint32_t scodes[G / NB];
@@ -660,6 +692,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     if constexpr (AMAX_ONLY) {
         if constexpr (NH > 0) amax_acc = __fmul_rn(amax_acc, had_norm<NH>());  // c * max |y| = max |c * y|
         write_partial(amax_acc, red, p.amax_out);
+        if constexpr (DUAL) {
+            if constexpr (NH > 0) amax_row_acc = __fmul_rn(amax_row_acc, had_norm<NH>());
+            write_partial(amax_row_acc, red + 16, p.amax_out_row);
+        }
     }
 }
 
@@ -758,6 +794,15 @@ cudaError_t launch_quant(const QuantParams& p, int fmt, int rnd, int nh, int axi
     if (rnd == kRtn) return dispatch_nh<kMxfp4, kRtn>(p, nh, axis, tmap, s);
     if (rnd == kSr) return dispatch_nh<kMxfp4, kSr>(p, nh, axis, tmap, s);
     return dispatch_nh<kMxfp4, kQuartet2>(p, nh, axis, tmap, s);
+}
+
+cudaError_t launch_amax_rowcol(const QuantParams& p, int nh, const CUtensorMap* tmap, int n_partials,
+                               cudaStream_t s) {
+    constexpr int G = 16, S = col_stages<G>();
+    const int smem = S * 2 * (4 * G * 64 * 2) + 1024;
+    if (nh == 16)
+        return launch_persistent(quant_col_kernel<kNvfp4, kRtn, 16, true, S, true>, n_partials, smem, *tmap, p, s);
+    return launch_persistent(quant_col_kernel<kNvfp4, kRtn, 0, true, S, true>, n_partials, smem, *tmap, p, s);
 }
 
 cudaError_t launch_amax(const QuantParams& p, int axis, int nh, const CUtensorMap* tmap, int n_partials,

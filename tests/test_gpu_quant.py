@@ -150,6 +150,24 @@ def test_amax_entry_point(axis, had):
     assert_same(q1, oracle_quant(x, Q.NVFP4, Q.RTN, had, axis), Q.NVFP4)
 
 
+@pytest.mark.parametrize("had", [Q.HAD_NONE, Q.HAD_DET16, Q.HAD_RAND16, Q.HAD_RAND32],
+                         ids=["none", "det16", "rand16", "rand32"])
+@pytest.mark.parametrize("shape", [(352, 416), (384, 256), (64, 128), (8192, 4096)], ids=lambda s: "x".join(map(str, s)))
+def test_amax_rowcol_matches_oracle(had, shape):
+    """Both orientations' amax from one call (one read of x for n_h <= 16, with
+    different sign vectors per orientation) equal the oracle's max |rotated x|."""
+    R, C = shape
+    x = sweep_like(R, C)
+    s_row = Q.make_seed(SEED["rot"], SEED["sr"], 1, 2)
+    s_col = Q.make_seed(SEED["rot"], SEED["sr"], 2, 4)
+    a = Q.amax_rowcol(x.cuda(), had, s_row, s_col).cpu().numpy()
+    Q.status()
+    v_row = O.rotate(x, had, O.ROW, SEED["rot"], 1)
+    v_col = O.rotate(x, had, O.COL, SEED["rot"], 2)
+    assert np.float32(a[0]) == np.float32(np.abs(v_row).max())
+    assert np.float32(a[1]) == np.float32(np.abs(v_col).max())
+
+
 def test_determinism_and_seed_sensitivity():
     x = sweep_like(256, 256).cuda()
     a = gpu_quant(x, Q.NVFP4, Q.SR, Q.HAD_RAND16, Q.COL)
