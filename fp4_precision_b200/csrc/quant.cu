@@ -565,11 +565,34 @@ __global__ void __launch_bounds__(kThreads, 2)
     // shuffles, instead of every lane computing it.
     constexpr bool kSharedQuads = (RND == kQuartet2 && !AMAX_ONLY && G == 16 && NB == 16);
     const bool shared_quads = kSharedQuads && (p.k % 64) == 0;
+    // Tile-invariant per thread (chunk ci = 0, 1): the column within the tile
+    // (tiles start at multiples of 128 columns), the ldmatrix offsets within a
+    // stage, the scale byte offset within a 128-row atom block, and the code
+    // row offset.
+    int cc[2];
+    uint32_t lm_off[2][G / 8];
+    int64_t sc_off[2], code_off[2], blk_off[2];
+#pragma unroll
+    for (int ci = 0; ci < 2; ++ci) {
+        const int chunk = 2 * warp + ci;  // 16 chunks of 8 columns
+        const int box = chunk >> 3, ch = chunk & 7;
+        cc[ci] = chunk * 8 + (lane >> 2);
+#pragma unroll
+        for (int u = 0; u < G / 8; ++u) {
+            const int srow = lane + 32 * u;
+            lm_off[ci][u] = (uint32_t)(box * BOX_BYTES + srow * 128 + ((ch ^ (srow & 7)) << 4));
+        }
+        sc_off[ci] = (cc[ci] % 32) * 16 + ((cc[ci] / 32) % 4) * 4;
+        code_off[ci] = (int64_t)cc[ci] * (p.k / 2);
+        blk_off[ci] = (int64_t)cc[ci] * (p.k / NB);
+    }
+    const int64_t atom_row_bytes = (p.kb4 / 4) * 512;  // one 128-row block of scale atoms
     for (TileWalk<STAGES> w(tiles_c); w.tr < tiles_r; w.next()) {
         const int s = w.stage;
         if (!mbar_wait(&ring.full[s], w.phase)) break;
         const int64_t c0 = (int64_t)w.tc * kColTileCols;
         const int64_t r0 = (int64_t)w.tr * TILE_ROWS;
+        const uint32_t stage_base = smem_u32(tiles) + (uint32_t)(s * STAGE_BYTES);
         uint4 lane_quad = make_uint4(0u, 0u, 0u, 0u);
         if constexpr (kSharedQuads) {
             if (shared_quads) {
@@ -580,14 +603,10 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
 #pragma unroll
         for (int ci = 0; ci < 2; ++ci) {
-            const int chunk = 2 * warp + ci;  // 16 chunks of 8 columns
-            const int box = chunk >> 3, ch = chunk & 7;
-            const uint32_t box_base = smem_u32(tiles + s * STAGE_BYTES + box * BOX_BYTES);
             float v[G];
 #pragma unroll
             for (int u = 0; u < G / 8; ++u) {
-                const int srow = lane + 32 * u;
-                const uint32_t addr = box_base + srow * 128 + ((ch ^ (srow & 7)) << 4);
+                const uint32_t addr = stage_base + lm_off[ci][u];
                 uint32_t a0, a1, a2, a3;
                 asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
                              : "=r"(a0), "=r"(a1), "=r"(a2), "=r"(a3)
@@ -603,8 +622,8 @@ __global__ void __launch_bounds__(kThreads, 2)
                 v[8 * u + 4] = bf16lo(a2); v[8 * u + 5] = bf16hi(a2);
                 v[8 * u + 6] = bf16lo(a3); v[8 * u + 7] = bf16hi(a3);
             }
-            const int64_t c = c0 + chunk * 8 + (lane >> 2);  // x column = output row
-            const int64_t r_grp = r0 + (int64_t)G * q;       // first k index of this group
+            const int64_t c = c0 + cc[ci];              // x column = output row
+            const int64_t r_grp = r0 + (int64_t)G * q;  // first k index of this group
             if constexpr (AMAX_ONLY) {
                 Group<kNvfp4, kRtn, NH>::template rotate<false>(v);
                 amax_acc = abs_max<G>(amax_acc, v);
@@ -644,7 +663,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 uint32_t codes[G / 8];
                 uint32_t scodes[G / NB];
                 Grp::rotate(v);
-                const uint64_t blk = (uint64_t)c * (uint64_t)(p.k / NB) + (uint64_t)(r_grp / NB);
+                const uint64_t blk = (uint64_t)(c0 * (p.k / NB) + blk_off[ci] + r_grp / NB);
                 if constexpr (kSharedQuads) {
                     if (shared_quads) {  // this group's quad: computed by lane (ci, column) * 2
                         const int src = (ci << 4) | ((lane >> 2) << 1);
@@ -658,7 +677,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 Grp::quantize(v, s_enc, rtab, p, (uint64_t)c * (uint64_t)p.k + (uint64_t)r_grp, blk, srng, codes,
                               scodes);
                 if (c < p.rows && r_grp < p.k) {
-                    uint8_t* dst = p.codes + c * (p.k / 2) + r_grp / 2;
+                    uint8_t* dst = p.codes + c0 * (p.k / 2) + code_off[ci] + r_grp / 2;
                     if constexpr (G == 16)
                         *reinterpret_cast<uint2*>(dst) = make_uint2(codes[0], codes[1]);
                     else
@@ -673,7 +692,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 const uint32_t n2 = __shfl_down_sync(0xffffffffu, mine, 2);
                 const uint32_t n3 = __shfl_down_sync(0xffffffffu, mine, 3);
                 if (c < rows_pad) {
-                    const int64_t rowoff = (c / 128) * (p.kb4 / 4) * 512 + (c % 32) * 16 + ((c / 32) % 4) * 4;
+                    const int64_t rowoff = (c0 / 128) * atom_row_bytes + sc_off[ci];
                     if constexpr (G / NB == 1) {
                         if (q == 0 && kb0 / 4 < p.kb4 / 4)
                             *reinterpret_cast<uint32_t*>(p.scales + rowoff + (kb0 / 4) * 512) =
