@@ -55,6 +55,19 @@ def measured_peaks():
         return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The largest of the ranks' values, on every rank (a multi-GPU job's time
+    is its slowest rank's): one all-reduce of a one-element tensor on `device`
+    (the rank's GPU under NCCL, the CPU under gloo)."""
+    if world <= 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def measured_gemm_traffic():
     """DRAM bytes per GEMM launch (dram__bytes_read.sum + dram__bytes_write.sum)
     from the committed ncu summary of this workload, or None when the GEMM
@@ -229,11 +242,7 @@ def run_ours(args, rank, world, local_rank):
         barrier()
     launches = Q.launch_count(reset=True)
     Q.status()
-    ms = t0.elapsed_time(t1)
-    if world > 1:
-        tt = torch.tensor([ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
     ms_step = ms / args.steps
     per = [[evs[s][j][0].elapsed_time(evs[s][j][1]) for s in range(args.steps)] for j in range(9)]
     gemm_ms = [statistics.mean(per[6 + g]) for g in range(3)]
@@ -563,12 +572,7 @@ def e2e_time(Q, X, W, dY, rec, seed, args, stream, dev, world):
     e1.record(s_out)
     torch.cuda.synchronize()
     Q.status()
-    ms = e0.elapsed_time(e1) / n
-    if world > 1:
-        import torch.distributed as dist
-        tt = torch.tensor([ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(e0.elapsed_time(e1) / n, world, dev)
     h2d = (M * K + N * K + M * N) * 2
     d2h = M * N * 2 + M * K * 2 + N * K * 4
     return {"value": round(world * 6.0 * M * N * K / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
