@@ -742,6 +742,34 @@ int qfp4_status(void* stream) {
     return QFP4_OK;
 }
 
+// ---- failure-detection self-test ------------------------------------------------
+namespace qfp4 {
+namespace {
+// One CTA: an mbarrier that nothing arrives on, waited on with the library's
+// bounded wait; the wait gives up after limit_ns, raises the device error word
+// and the kernel returns.
+__global__ void wait_timeout_kernel(uint64_t limit_ns) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbarrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) (void)mbar_wait_for(&bar, 0, limit_ns);
+}
+}  // namespace
+}  // namespace qfp4
+
+int qfp4_selftest_wait_timeout(int64_t limit_ns, void* stream) {
+    const int rc = bind_context(static_cast<cudaStream_t>(stream));
+    if (rc) return rc;
+    if (limit_ns <= 0 || limit_ns > (int64_t)kWaitLimitNs) return QFP4_ERR_INVALID_ARG;
+    qfp4::wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>((uint64_t)limit_ns);
+    count_launch();
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? QFP4_OK : cuda_fail(e);
+}
+
 // ---- forward pass without allocation ------------------------------------------
 // The scratch of qfp4_linear_fwd_noalloc: a fixed device array (every GPU that
 // loads the library holds it until the process exits). Host code cannot use

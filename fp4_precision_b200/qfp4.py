@@ -83,6 +83,7 @@ _SIGNATURES = {
     "qfp4_linear_fwd_noalloc": (ctypes.c_int, [_VOID, _VOID, _VOID, _I64, _I64, _I64, ctypes.POINTER(Recipe),
                                                ctypes.POINTER(Seed), _VOID]),
     "qfp4_status": (ctypes.c_int, [_VOID]),
+    "qfp4_selftest_wait_timeout": (ctypes.c_int, [_I64, _VOID]),
     "qfp4_launch_count": (_I64, [_I32]),
 }
 

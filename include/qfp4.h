@@ -264,6 +264,16 @@ int qfp4_status(void* stream);
  * reset (reset = 1 zeroes it after reading). */
 int64_t qfp4_launch_count(int32_t reset);
 
+/* Self-test of the failure-detection path (no counterpart on the pages):
+ * launches one small kernel whose shared-memory mbarrier wait nothing
+ * satisfies, waited on with the same bounded wait as the library's kernels
+ * but with limit_ns (0 < limit_ns <= 2 s) instead of 2 s. The wait gives up,
+ * sets the device error word and the kernel returns: the next qfp4_status on
+ * the stream returns QFP4_ERR_TIMEOUT and clears the word, and the context
+ * stays usable. Nothing faults, traps or spins without a limit.
+ * Returns QFP4_OK (launched), QFP4_ERR_INVALID_ARG or QFP4_ERR_CUDA. */
+int qfp4_selftest_wait_timeout(int64_t limit_ns, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
