@@ -413,12 +413,26 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int64_t rows_pad = (p.rows + 127) / 128 * 128;
     float amax_acc = 0.0f;
     ScaleRng srng;
+    // Tile-invariant per thread: the swizzled 16-byte chunk offsets of its row
+    // and the scale byte offset of its row within a 128-row atom block (tiles
+    // start at multiples of 256 rows). Held in registers except by the
+    // per-element SR kernels, which need those registers for Philox words.
+    constexpr bool kHoist = (RND != kSr);
+    uint32_t chunk_off[kRowTileCols / 8];
+#pragma unroll
+    for (int c = 0; c < kRowTileCols / 8; ++c) chunk_off[c] = (uint32_t)(tid * 128 + ((c ^ (tid & 7)) << 4));
+    const int64_t atom_row_bytes = (p.kb4 / 4) * 512;  // one 128-row block of scale atoms
+    const int64_t sc_row_off = (tid / 128) * atom_row_bytes + (tid % 32) * 16 + ((tid / 32) % 4) * 4;
+    // the random Hadamard's sign-flip masks of the packed bf16 words of a group
+    uint32_t smask[G / 2];
+#pragma unroll
+    for (int i = 0; i < G / 2; ++i) smask[i] = Grp::sign_mask(p.signs, i);
     for (TileWalk<STAGES> w(tiles_c); w.tr < tiles_r; w.next()) {
         const int s = w.stage;
         if (!mbar_wait(&ring.full[s], w.phase)) break;
         const int64_t row = (int64_t)w.tr * kRowTileRows + tid;
         const int64_t col0 = (int64_t)w.tc * kRowTileCols;
-        const uint32_t sbase = smem_u32(tiles + s * STAGE_BYTES) + tid * 128;
+        const uint32_t sbase = smem_u32(tiles) + (uint32_t)(s * STAGE_BYTES) + (kHoist ? 0u : (uint32_t)tid * 128u);
         uint32_t codes[kRowTileCols / 8];
         uint32_t scodes[kRowTileCols / 16];
 #pragma unroll
@@ -428,14 +442,15 @@ __global__ void __launch_bounds__(kThreads, 2)
             for (int c8 = 0; c8 < G / 8; ++c8) {
                 const int chunk = g * (G / 8) + c8;
                 uint32_t w0, w1, w2, w3;
+                const uint32_t addr = kHoist ? sbase + chunk_off[chunk] : sbase + ((chunk ^ (tid & 7)) << 4);
                 asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
                              : "=r"(w0), "=r"(w1), "=r"(w2), "=r"(w3)
-                             : "r"(sbase + ((chunk ^ (tid & 7)) << 4)));
+                             : "r"(addr));
                 if (NH > 0 && p.signs != 0u) {
-                    w0 ^= Grp::sign_mask(p.signs, 4 * c8 + 0);
-                    w1 ^= Grp::sign_mask(p.signs, 4 * c8 + 1);
-                    w2 ^= Grp::sign_mask(p.signs, 4 * c8 + 2);
-                    w3 ^= Grp::sign_mask(p.signs, 4 * c8 + 3);
+                    w0 ^= kHoist ? smask[4 * c8 + 0] : Grp::sign_mask(p.signs, 4 * c8 + 0);
+                    w1 ^= kHoist ? smask[4 * c8 + 1] : Grp::sign_mask(p.signs, 4 * c8 + 1);
+                    w2 ^= kHoist ? smask[4 * c8 + 2] : Grp::sign_mask(p.signs, 4 * c8 + 2);
+                    w3 ^= kHoist ? smask[4 * c8 + 3] : Grp::sign_mask(p.signs, 4 * c8 + 3);
                 }
                 v[8 * c8 + 0] = bf16lo(w0); v[8 * c8 + 1] = bf16hi(w0);
                 v[8 * c8 + 2] = bf16lo(w1); v[8 * c8 + 3] = bf16hi(w1);
@@ -473,7 +488,8 @@ __global__ void __launch_bounds__(kThreads, 2)
                 // is padding and is written as zero.
                 const int64_t kb0 = col0 / NB;
                 const int64_t off =
-                    ((row / 128) * (p.kb4 / 4) + kb0 / 4) * 512 + (row % 32) * 16 + ((row / 32) % 4) * 4;
+                    kHoist ? (2 * (int64_t)w.tr) * atom_row_bytes + (kb0 / 4) * 512 + sc_row_off
+                           : ((row / 128) * (p.kb4 / 4) + kb0 / 4) * 512 + (row % 32) * 16 + ((row / 32) % 4) * 4;
                 if constexpr (NB == 16) {
                     *reinterpret_cast<uint32_t*>(p.scales + off) =
                         scodes[0] | (scodes[1] << 8) | (scodes[2] << 16) | (scodes[3] << 24);
@@ -587,6 +603,9 @@ __global__ void __launch_bounds__(kThreads, 2)
         blk_off[ci] = (int64_t)cc[ci] * (p.k / NB);
     }
     const int64_t atom_row_bytes = (p.kb4 / 4) * 512;  // one 128-row block of scale atoms
+    uint32_t smask[G / 2];  // the random Hadamard's sign-flip masks of a group's packed words
+#pragma unroll
+    for (int i = 0; i < G / 2; ++i) smask[i] = Grp::sign_mask(p.signs, i);
     for (TileWalk<STAGES> w(tiles_c); w.tr < tiles_r; w.next()) {
         const int s = w.stage;
         if (!mbar_wait(&ring.full[s], w.phase)) break;
@@ -612,10 +631,10 @@ __global__ void __launch_bounds__(kThreads, 2)
                              : "=r"(a0), "=r"(a1), "=r"(a2), "=r"(a3)
                              : "r"(addr));
                 if (NH > 0 && p.signs != 0u) {
-                    a0 ^= Grp::sign_mask(p.signs, 4 * u + 0);
-                    a1 ^= Grp::sign_mask(p.signs, 4 * u + 1);
-                    a2 ^= Grp::sign_mask(p.signs, 4 * u + 2);
-                    a3 ^= Grp::sign_mask(p.signs, 4 * u + 3);
+                    a0 ^= smask[4 * u + 0];
+                    a1 ^= smask[4 * u + 1];
+                    a2 ^= smask[4 * u + 2];
+                    a3 ^= smask[4 * u + 3];
                 }
                 v[8 * u + 0] = bf16lo(a0); v[8 * u + 1] = bf16hi(a0);
                 v[8 * u + 2] = bf16lo(a1); v[8 * u + 3] = bf16hi(a1);
