@@ -42,7 +42,7 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--profile", choices=["gemm_fprop", "gemm_dgrad", "gemm_wgrad", "quant_row", "quant_col",
-                                          "amax_row", "amax_col"],
+                                          "quant_sr_row", "quant_sr_col", "amax_row", "amax_col"],
                     help="run only one kernel 3 times on a bounded case (for ncu captures), print nothing else")
     return ap.parse_args()
 
@@ -636,8 +636,9 @@ def run_reference(args, rank, world):
 def run_profile(kind: str):
     """One kernel, three launches, on a case larger than L2 that holds a few GB
     at most: each of the MLP up/gate layer's three GEMMs (Fprop, Dgrad, Wgrad
-    operands quantized as in the step), or a quantizer / amax pass (Quartet II
-    NVFP4, random 16x16 Hadamard) over a [16384 x 8192] bf16 tensor (268 MB)."""
+    operands quantized as in the step), or a quantizer / amax pass (NVFP4 with
+    Quartet II rounding, or per-element SR for the ``quant_sr_*`` cases, after a
+    random 16x16 Hadamard) over a [16384 x 8192] bf16 tensor (268 MB)."""
     import torch
 
     from fp4_precision_b200 import inputs
@@ -673,8 +674,9 @@ def run_profile(kind: str):
                 Q.amax(T, Q.HAD_RAND16, axis, seed)
         else:
             am = Q.amax(T, Q.HAD_RAND16, axis, seed)
+            rnd = Q.SR if kind.startswith("quant_sr") else Q.QUARTET2
             for _ in range(3):
-                Q.quantize(T, Q.NVFP4, Q.QUARTET2, Q.HAD_RAND16, axis, seed, amax_in=am)
+                Q.quantize(T, Q.NVFP4, rnd, Q.HAD_RAND16, axis, seed, amax_in=am)
     torch.cuda.synchronize()
     Q.status()
 
