@@ -31,13 +31,13 @@ _BUILD_DIR = os.path.join(_HERE, "_build")
 _LIB_PATH = os.path.join(_BUILD_DIR, "liboracle.so")
 _lib = None
 
-NVFP4, MXFP4 = 0, 1
+NVFP4, MXFP4, MXFP4_RU = 0, 1, 2
 RTN, SR, QUARTET2 = 0, 1, 2
 HAD_NONE, HAD_DET16, HAD_DET32, HAD_RAND16, HAD_RAND32 = 0, 1, 2, 3, 4
 ROW, COL = 0, 1
 TAG_ELEMENT, TAG_SCALE, TAG_SIGN = 0, 1, 2
 
-BLOCK = {NVFP4: 16, MXFP4: 32}
+BLOCK = {NVFP4: 16, MXFP4: 32, MXFP4_RU: 32}
 HAD_N = {HAD_NONE: 0, HAD_DET16: 16, HAD_DET32: 32, HAD_RAND16: 16, HAD_RAND32: 32}
 
 # Error bound of a GEMM output against the fp64 oracle, relative to sum_k |a_k b_k|.

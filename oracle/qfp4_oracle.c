@@ -31,7 +31,7 @@
 #include <stdlib.h>
 #include <string.h>
 
-enum { FMT_NVFP4 = 0, FMT_MXFP4 = 1 };
+enum { FMT_NVFP4 = 0, FMT_MXFP4 = 1, FMT_MXFP4_RU = 2 };
 enum { RND_RTN = 0, RND_SR = 1, RND_QUARTET2 = 2 };
 enum { HAD_NONE = 0, HAD_DET16 = 1, HAD_DET32 = 2, HAD_RAND16 = 3, HAD_RAND32 = 4 };
 enum { AXIS_ROW = 0, AXIS_COL = 1 };
@@ -297,7 +297,7 @@ static void load_segment(const uint16_t* x, int64_t ld, int axis, int64_t row, i
 int oracle_quantize(const uint16_t* x, int64_t R, int64_t C, int64_t ld, int fmt, int rnd, int had,
                     int axis, uint64_t rot_seed, uint32_t rot_stream, uint64_t sr_seed, uint32_t sr_stream,
                     const float* amax_in, uint8_t* codes, uint8_t* scales, float* g_out, float* alpha_out) {
-    if (fmt != FMT_NVFP4 && fmt != FMT_MXFP4) return -1;
+    if (fmt != FMT_NVFP4 && fmt != FMT_MXFP4 && fmt != FMT_MXFP4_RU) return -1;
     if (rnd < RND_RTN || rnd > RND_QUARTET2) return -1;
     if (had < HAD_NONE || had > HAD_RAND32) return -1;
     if (axis != AXIS_ROW && axis != AXIS_COL) return -1;
@@ -378,6 +378,15 @@ int oracle_quantize(const uint16_t* x, int64_t R, int64_t C, int64_t ld, int fmt
                         rmul = 0.0f;
                     } else {
                         int E = floor_log2f(amax_b) - 2;
+                        if (fmt == FMT_MXFP4_RU) {
+                            /* Round-up variant, not on the pages (they give the
+                             * shared exponent only as the block's largest one):
+                             * the smallest E with amax_b <= 6 * 2^E, so that no
+                             * element of the block clips; searched upward from one
+                             * below the floor rule's E, 6 * 2^E exact in double. */
+                            E -= 1;
+                            while ((double)amax_b > 6.0 * ldexp(1.0, E)) E += 1;
+                        }
                         if (E < -127) E = -127;
                         if (E > 127) E = 127;
                         s_code = (uint8_t)(E + 127);

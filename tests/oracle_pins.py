@@ -413,6 +413,47 @@ def check_mxfp4_scales():
     assert np.all(np.abs(xhat[~nc]) == 6.0 * Se[~nc])
 
 
+def check_mxfp4_round_up():
+    """MXFP4 with the round-up shared exponent (a variant the pages leave open:
+    [AMD MXFP4] "Chto takoe MXFP4" gives the shared exponent only as the
+    block's largest one): E is the smallest exponent with amax_b <= 6 * 2^E, so
+    the block max scaled by 2^-E lies in (3, 6] and no element clips. Where the
+    floor rule already leaves the block max at or below 6 the two rules agree
+    on the block's scale and codes; elsewhere the round-up exponent is one
+    above the floor one. Worked blocks: max 7 (the floor rule clips it to 6)
+    gets E = 1 and 7 / 2 = 3.5 rounds, ties to even, to code 6 (value 4, so 8
+    after scaling), 1 / 2 = 0.5 to code 1; a block whose max is exactly 6 keeps
+    E = 0 (and -0.75 rounds, ties to even, to code 2 with the sign bit)."""
+    x = inputs.workload("sweep")["T"][:128, :512]
+    qf = O.quantize(x, O.MXFP4, O.RTN, O.HAD_NONE, O.ROW)
+    qr = O.quantize(x, O.MXFP4_RU, O.RTN, O.HAD_NONE, O.ROW)
+    v = x.float().numpy().astype(np.float64)
+    amax_b = np.abs(v).reshape(128, -1, 32).max(axis=2)
+    nz = amax_b > 0
+    ratio = amax_b[nz] / O.scale_values(qr)[nz]
+    assert np.all((ratio > 3.0) & (ratio <= 6.0))
+    fits = (amax_b <= 6.0 * O.scale_values(qf)) & nz
+    assert fits.any() and (nz & ~fits).any()
+    ef, er = qf.scales.astype(np.int64), qr.scales.astype(np.int64)
+    assert np.all(er[fits] == ef[fits])
+    assert np.all(er[nz & ~fits] == ef[nz & ~fits] + 1)
+    cf = O.unpack_codes(qf.codes).reshape(128, -1, 32)
+    cr = O.unpack_codes(qr.codes).reshape(128, -1, 32)
+    assert np.array_equal(cf[fits], cr[fits])
+    # no element clips: every reconstruction is within half a grid gap
+    S = np.repeat(O.scale_values(qr), 32, axis=1)
+    u = np.abs(v) / S
+    gap = np.where(u < 2, 0.5, np.where(u < 4, 1.0, 2.0))
+    assert np.all(u <= 6.0)
+    assert np.all(np.abs(O.dequantize(qr) - v) <= gap / 2 * S)
+    # worked blocks
+    b = torch.zeros((1, 96), dtype=torch.float32)
+    b[0, 0], b[0, 1], b[0, 32], b[0, 33] = 7.0, 1.0, 6.0, -0.75
+    q = O.quantize(b.to(torch.bfloat16), O.MXFP4_RU, O.RTN, O.HAD_NONE, O.ROW)
+    assert list(q.scales[0]) == [128, 127, 0]
+    assert int(q.codes[0, 0]) == 0x16 and int(q.codes[0, 16]) == 0xA7 and not q.codes[0, 32:].any()
+
+
 def check_zero_and_degenerate():
     """All-zero input: zero codes, zero NVFP4 scales, g = 1; E8M0 code 0."""
     z = torch.zeros((32, 64), dtype=torch.bfloat16)
@@ -499,6 +540,6 @@ ALL_CHECKS = [
     check_philox_matches_torch_engine, check_sylvester_matches_scipy, check_fwht_is_matrix_product,
     check_rotation_orthonormal, check_sr_threshold_exact, check_e4m3_sr_threshold_exact,
     check_sr_unbiased_rtn_biased, check_quartet2_projection_unbiased, check_quartet2_alpha_range,
-    check_nvfp4_scales, check_mxfp4_scales, check_zero_and_degenerate, check_col_is_row_of_transpose,
+    check_nvfp4_scales, check_mxfp4_scales, check_mxfp4_round_up, check_zero_and_degenerate, check_col_is_row_of_transpose,
     check_seed_determinism, check_gemm_brute_force, check_hadamard_cancels_in_gemm,
 ]

@@ -21,6 +21,10 @@ MUTATIONS = [
     ("nvfp4_tensor_scale", "s_enc = 2688.0f / amax;", "s_enc = 2048.0f / amax;"),
     ("nvfp4_block_top", "float d = amax_b / 6.0f;", "float d = amax_b / 4.0f;"),
     ("mxfp4_exponent_offset", "int E = floor_log2f(amax_b) - 2;", "int E = floor_log2f(amax_b) - 1;"),
+    ("mxfp4_ru_floor_rule", "while ((double)amax_b > 6.0 * ldexp(1.0, E)) E += 1;",
+     "while ((double)amax_b >= 8.0 * ldexp(1.0, E)) E += 1;"),
+    ("mxfp4_ru_not_strict", "while ((double)amax_b > 6.0 * ldexp(1.0, E)) E += 1;",
+     "while ((double)amax_b >= 6.0 * ldexp(1.0, E)) E += 1;"),
     ("sr_compare_flipped", "idx = (rho < p) ? lo + 1 : lo;", "idx = (rho > p) ? lo + 1 : lo;"),
     ("philox_multiplier", "(uint64_t)0xD2511F53u", "(uint64_t)0xD2511F55u"),
     ("philox_key_bump", "k1 += 0xBB67AE85u;", "k1 += 0xBB67AE86u;"),
