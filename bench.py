@@ -263,6 +263,9 @@ def run_ours(args, rank, world, local_rank):
     # the other configurations of the MLP shapes (not part of the headline value)
     layers = more_layers(Q, inputs, X, W, dY, seed, stream, dev)
 
+    # MXFP4 variants on the Wgrad product of this layer (quality, not speed)
+    study = mxfp4_wgrad_study(Q, X, dY, stream)
+
     # linear API (device-resident) and end to end with host buffers
     api_ms = linear_api_time(Q, X, W, dY, rec, seed, args, stream, dev)
     e2e = None if args.no_e2e else e2e_time(Q, X, W, dY, rec, seed, args, stream, dev, world)
@@ -294,6 +297,7 @@ def run_ours(args, rank, world, local_rank):
         "step_breakdown_ms": {"quantize": [round(v, 4) for v in quant_ms], "gemm": [round(v, 4) for v in gemm_ms]},
         "quantize": quant,
         "layers": layers,
+        "study": study,
         "linear_api_ms_per_step": round(api_ms, 4),
         "e2e": e2e,
         "gpu_launches": launches,
@@ -399,7 +403,8 @@ def quant_sweep(Q, inputs, dev, stream, peaks):
              ("nvfp4_sr_rand16_row", Q.NVFP4, Q.SR, Q.HAD_RAND16, Q.ROW),
              ("nvfp4_q2_rand16_col", Q.NVFP4, Q.QUARTET2, Q.HAD_RAND16, Q.COL),
              ("mxfp4_rtn_det32_col", Q.MXFP4, Q.RTN, Q.HAD_DET32, Q.COL),
-             ("mxfp4_rtn_none_row", Q.MXFP4, Q.RTN, Q.HAD_NONE, Q.ROW)]
+             ("mxfp4_rtn_none_row", Q.MXFP4, Q.RTN, Q.HAD_NONE, Q.ROW),
+             ("mxfp4ru_rtn_det32_col", Q.MXFP4_RU, Q.RTN, Q.HAD_DET32, Q.COL)]
     seed = Q.make_seed(5, 6)
     for name, fmt, rnd, had, axis in cases:
         rows, k = (R, C) if axis == Q.ROW else (C, R)
@@ -444,7 +449,8 @@ def quant_sweep(Q, inputs, dev, stream, peaks):
 def quant_large(Q, T, stream, peaks):
     """Quantizer and amax kernels on a tensor far larger than L2 (the layer's
     dY, [16384 x 28672] bf16, 940 MB): steady-state GB/s of algorithmic bytes
-    (2 B read + 0.5 B codes + 1/16 B scales per element; amax: 2 B read)."""
+    (2 B read + 0.5 B codes + 1/16 B (NVFP4) or 1/32 B (MXFP4) scales per
+    element; amax: 2 B read)."""
     import torch
     R, C = T.shape
     dev = T.device
@@ -463,18 +469,20 @@ def quant_large(Q, T, stream, peaks):
         torch.cuda.synchronize()
         return e0.elapsed_time(e1) / n
 
-    for name, rnd, had, axis in (("nvfp4_rtn_none_row", Q.RTN, Q.HAD_NONE, Q.ROW),
-                                 ("nvfp4_rtn_rand16_row", Q.RTN, Q.HAD_RAND16, Q.ROW),
-                                 ("nvfp4_rtn_rand16_col", Q.RTN, Q.HAD_RAND16, Q.COL),
-                                 ("nvfp4_sr_rand16_row", Q.SR, Q.HAD_RAND16, Q.ROW),
-                                 ("nvfp4_q2_rand16_row", Q.QUARTET2, Q.HAD_RAND16, Q.ROW),
-                                 ("nvfp4_q2_rand16_col", Q.QUARTET2, Q.HAD_RAND16, Q.COL)):
+    for name, fmt, rnd, had, axis in (("nvfp4_rtn_none_row", Q.NVFP4, Q.RTN, Q.HAD_NONE, Q.ROW),
+                                      ("nvfp4_rtn_rand16_row", Q.NVFP4, Q.RTN, Q.HAD_RAND16, Q.ROW),
+                                      ("nvfp4_rtn_rand16_col", Q.NVFP4, Q.RTN, Q.HAD_RAND16, Q.COL),
+                                      ("nvfp4_sr_rand16_row", Q.NVFP4, Q.SR, Q.HAD_RAND16, Q.ROW),
+                                      ("nvfp4_q2_rand16_row", Q.NVFP4, Q.QUARTET2, Q.HAD_RAND16, Q.ROW),
+                                      ("nvfp4_q2_rand16_col", Q.NVFP4, Q.QUARTET2, Q.HAD_RAND16, Q.COL),
+                                      ("mxfp4_rtn_det32_col", Q.MXFP4, Q.RTN, Q.HAD_DET32, Q.COL),
+                                      ("mxfp4ru_rtn_det32_col", Q.MXFP4_RU, Q.RTN, Q.HAD_DET32, Q.COL)):
         rows, k = (R, C) if axis == Q.ROW else (C, R)
-        q = Q.empty_qtensor(Q.NVFP4, rows, k, dev)
-        am = Q.amax(T, had, axis, seed, workspace=ws, stream=stream)
-        ms = timeit(lambda: Q.quantize(T, Q.NVFP4, rnd, had, axis, seed, amax_in=am, out=q, workspace=ws,
+        q = Q.empty_qtensor(fmt, rows, k, dev)
+        am = Q.amax(T, had, axis, seed, workspace=ws, stream=stream) if fmt == Q.NVFP4 else None
+        ms = timeit(lambda: Q.quantize(T, fmt, rnd, had, axis, seed, amax_in=am, out=q, workspace=ws,
                                        stream=stream))
-        gbs = R * C * (2 + 0.5 + 1 / 16) / (ms * 1e-3) / 1e9
+        gbs = R * C * (2 + 0.5 + (1 / 16 if fmt == Q.NVFP4 else 1 / 32)) / (ms * 1e-3) / 1e9
         res[name] = {"ms": round(ms, 4), "GB/s": round(gbs, 1), "frac_of_measured_hbm": round(gbs / peaks["hbm_gbs"], 3)}
         del q
     for name, axis in (("amax_rand16_row", Q.ROW), ("amax_rand16_col", Q.COL)):
@@ -485,6 +493,34 @@ def quant_large(Q, T, stream, peaks):
     Q.status()
     return {"workload": f"dY [{R}x{C}] bf16 N(0,1e-3), 940 MB (larger than L2; no flush)", "unit": "GB/s",
             "cases": res}
+
+
+def mxfp4_wgrad_study(Q, X, dY, stream):
+    """Relative Frobenius error of the MXFP4 Wgrad product dY^T X (both
+    operands quantized along the tokens, RTN) against the fp32 product of the
+    bf16 inputs, for the Hadamard sizes the AMD MXFP4 page's experiments use
+    (none, 16, 32; deterministic) and for the floor and the round-up shared
+    exponent. A quality figure of the variants, not part of the timed path."""
+    import torch
+    prev = torch.backends.cuda.matmul.allow_tf32
+    torch.backends.cuda.matmul.allow_tf32 = False
+    ref = dY.t().float() @ X.float()
+    torch.backends.cuda.matmul.allow_tf32 = prev
+    nref = torch.linalg.vector_norm(ref).item()
+    seed = Q.make_seed(9, 10)
+    res = {}
+    for hname, had in (("none", Q.HAD_NONE), ("det16", Q.HAD_DET16), ("det32", Q.HAD_DET32)):
+        for ename, fmt in (("floor", Q.MXFP4), ("round_up", Q.MXFP4_RU)):
+            A = Q.quantize(dY, fmt, Q.RTN, had, Q.COL, seed, stream=stream)
+            B = Q.quantize(X, fmt, Q.RTN, had, Q.COL, seed, stream=stream)
+            D = Q.gemm(A, B, torch.float32, stream=stream)
+            res[f"{hname}_{ename}"] = round(torch.linalg.vector_norm(D - ref).item() / nref, 5)
+            del A, B, D
+    Q.status()
+    del ref
+    return {"mxfp4_wgrad_rel_err": res,
+            "what": "||dW_fp4 - dW_fp32|| / ||dW_fp32||, dW = dY^T X of the MLP up/gate workload, MXFP4 RTN along "
+                    "the tokens, deterministic Hadamard none/16/32, floor vs round-up shared exponent"}
 
 
 def linear_api_time(Q, X, W, dY, rec, seed, args, stream, dev):

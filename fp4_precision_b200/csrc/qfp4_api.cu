@@ -27,6 +27,7 @@ int cuda_fail(cudaError_t e) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 int block_of(int fmt) { return fmt == kNvfp4 ? 16 : 32; }
+bool valid_fmt(int fmt) { return fmt == QFP4_NVFP4 || fmt == QFP4_MXFP4 || fmt == QFP4_MXFP4_RU; }
 int had_n(int had) {
     return (had == QFP4_HAD_DET16 || had == QFP4_HAD_RAND16)   ? 16
            : (had == QFP4_HAD_DET32 || had == QFP4_HAD_RAND32) ? 32
@@ -301,7 +302,7 @@ int quantize_impl(const void* x, int64_t R, int64_t C, int64_t ld, int32_t fmt, 
     if (rc) return rc;
     rc = check_device(&sms);
     if (rc) return rc;
-    if (fmt != QFP4_NVFP4 && fmt != QFP4_MXFP4) return QFP4_ERR_INVALID_ARG;
+    if (!valid_fmt(fmt)) return QFP4_ERR_INVALID_ARG;
     if (rounding < QFP4_RTN || rounding > QFP4_QUARTET2) return QFP4_ERR_INVALID_ARG;
     if (out == nullptr || seed == nullptr) return QFP4_ERR_INVALID_ARG;
     if (seed->rot_stream >= (1u << 28) || seed->sr_stream >= (1u << 28)) return QFP4_ERR_INVALID_ARG;
@@ -322,7 +323,10 @@ int quantize_impl(const void* x, int64_t R, int64_t C, int64_t ld, int32_t fmt, 
     }
     out->rows = g.rows;
     out->k = g.k;
-    out->fmt = fmt;
+    // the round-up MXFP4 variant only chooses the exponent differently: the
+    // result is an ordinary MXFP4 tensor
+    const int sfmt = (fmt == QFP4_MXFP4_RU) ? QFP4_MXFP4 : fmt;
+    out->fmt = sfmt;
     out->had = had;
     out->rot_seed = had_random(had) ? seed->rot : 0;
     out->rot_stream = had_random(had) ? seed->rot_stream : 0;
@@ -344,6 +348,7 @@ int quantize_impl(const void* x, int64_t R, int64_t C, int64_t ld, int32_t fmt, 
     p.sr_tag_elem = (uint32_t)kTagElement | (seed->sr_stream << 4);
     p.sr_tag_scale = (uint32_t)kTagScale | (seed->sr_stream << 4);
     p.amax_in = amax_in;
+    p.mx_round_up = (fmt == QFP4_MXFP4_RU) ? 1u : 0u;
     if (need_ws) {
         int n = 0;
         float* partials = static_cast<float*>(workspace);
@@ -353,7 +358,7 @@ int quantize_impl(const void* x, int64_t R, int64_t C, int64_t ld, int32_t fmt, 
     }
     CUtensorMap tm;
     if ((rc = make_input_tmap(&tm, x, R, C, ld, axis, col_group(NB, nh)))) return rc;
-    cudaError_t e = launch_quant(p, fmt, rounding, nh, axis, &tm, s);
+    cudaError_t e = launch_quant(p, sfmt, rounding, nh, axis, &tm, s);
     return e == cudaSuccess ? QFP4_OK : cuda_fail(e);
 }
 
@@ -436,7 +441,7 @@ void carve_operand(Carver& c, qfp4_tensor* t, int fmt, int64_t rows, int64_t k) 
 }
 
 bool valid_cfg(const qfp4_gemm_cfg& g) {
-    return (g.fmt == QFP4_NVFP4 || g.fmt == QFP4_MXFP4) && g.rnd_a >= QFP4_RTN && g.rnd_a <= QFP4_QUARTET2 &&
+    return valid_fmt(g.fmt) && g.rnd_a >= QFP4_RTN && g.rnd_a <= QFP4_QUARTET2 &&
            g.rnd_b >= QFP4_RTN && g.rnd_b <= QFP4_QUARTET2 && g.had >= QFP4_HAD_NONE && g.had <= QFP4_HAD_RAND32;
 }
 bool valid_dtype(int32_t d) { return d == QFP4_OUT_BF16 || d == QFP4_OUT_F32; }
@@ -567,13 +572,13 @@ int64_t qfp4_launch_count(int32_t reset) {
 size_t qfp4_codes_bytes(int64_t rows, int64_t k) { return (rows <= 0 || k <= 0) ? 0 : (size_t)(rows * k / 2); }
 
 size_t qfp4_scales_bytes(int32_t fmt, int64_t rows, int64_t k) {
-    if ((fmt != QFP4_NVFP4 && fmt != QFP4_MXFP4) || rows <= 0 || k <= 0) return 0;
+    if (!valid_fmt(fmt) || rows <= 0 || k <= 0) return 0;
     const int64_t kb = (k + block_of(fmt) - 1) / block_of(fmt);
     return (size_t)(((rows + 127) / 128) * ((kb + 3) / 4) * 512);
 }
 
 int64_t qfp4_scale_offset(int32_t fmt, int64_t rows, int64_t k, int64_t r, int64_t c) {
-    if ((fmt != QFP4_NVFP4 && fmt != QFP4_MXFP4) || rows <= 0 || k <= 0) return -1;
+    if (!valid_fmt(fmt) || rows <= 0 || k <= 0) return -1;
     const int64_t kb = (k + block_of(fmt) - 1) / block_of(fmt);
     const int64_t rows_p = (rows + 127) / 128 * 128, kb4 = (kb + 3) / 4 * 4;
     if (r < 0 || c < 0 || r >= rows_p || c >= kb4) return -1;

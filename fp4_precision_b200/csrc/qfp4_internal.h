@@ -36,6 +36,7 @@ struct QuantParams {
     uint64_t sr_seed;
     uint32_t sr_tag_elem;         // kTagElement | stream << 4
     uint32_t sr_tag_scale;        // kTagScale | stream << 4
+    uint32_t mx_round_up;         // MXFP4: 1 = the smallest E with amax_b <= 6 * 2^E (no clipping)
 };
 
 // Launchers (quant.cu). Return cudaSuccess or the launch error.

@@ -250,7 +250,14 @@ struct Group {
                     S = exp2i(-127);
                     rmul = 0.0f;
                 } else {
-                    int E = floor_log2(am) - 2;
+                    const int e = floor_log2(am);
+                    int E = e - 2;
+                    if (p.mx_round_up) {
+                        // the smallest E with am <= 6 * 2^E: one more when
+                        // am > 1.5 * 2^e, i.e. 2 (am - 2^e) > 2^e (both exact)
+                        const float lo = exp2i(e);
+                        if (__fmul_rn(2.0f, __fsub_rn(am, lo)) > lo) ++E;
+                    }
                     E = E < -127 ? -127 : (E > 127 ? 127 : E);
                     scode = (uint32_t)(E + 127);
                     S = exp2i(E);

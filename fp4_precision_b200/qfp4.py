@@ -16,13 +16,13 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libqfp4.so")
 
-NVFP4, MXFP4 = 0, 1
+NVFP4, MXFP4, MXFP4_RU = 0, 1, 2
 RTN, SR, QUARTET2 = 0, 1, 2
 HAD_NONE, HAD_DET16, HAD_DET32, HAD_RAND16, HAD_RAND32 = 0, 1, 2, 3, 4
 ROW, COL = 0, 1
 OUT_BF16, OUT_F32 = 0, 1
 PRESETS = {"NVIDIA_NVFP4": 0, "QUARTET2_NVFP4": 1, "AMD_MXFP4_H": 2}
-BLOCK = {NVFP4: 16, MXFP4: 32}
+BLOCK = {NVFP4: 16, MXFP4: 32, MXFP4_RU: 32}
 
 OK, ERR_INVALID_ARG, ERR_MISALIGNED, ERR_UNSUPPORTED_ARCH, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT = 0, -1, -2, -3, -4, -5, -6
 ERR_TOO_LARGE = -7

@@ -55,7 +55,13 @@ extern "C" {
 #define QFP4_ERR_TOO_LARGE (-7)        /* the problem needs more than qfp4_linear_fwd_noalloc's fixed scratch */
 
 /* ---- enums ---------------------------------------------------------------- */
-typedef enum { QFP4_NVFP4 = 0, QFP4_MXFP4 = 1 } qfp4_format;
+/* QFP4_MXFP4_RU: MXFP4 whose shared exponent is rounded up instead of down,
+ * E = the smallest exponent with amax_b <= 6 * 2^E, so that no element of a
+ * block clips (a reading the AMD MXFP4 page, "Chto takoe MXFP4", leaves open:
+ * it gives the shared exponent only as the block's largest one). Accepted by
+ * qfp4_quantize and in recipes; the tensor it writes is an ordinary MXFP4
+ * tensor (fmt = QFP4_MXFP4), since only the choice of E differs. */
+typedef enum { QFP4_NVFP4 = 0, QFP4_MXFP4 = 1, QFP4_MXFP4_RU = 2 } qfp4_format;
 typedef enum { QFP4_RTN = 0, QFP4_SR = 1, QFP4_QUARTET2 = 2 } qfp4_rounding;
 typedef enum {
     QFP4_HAD_NONE = 0,
@@ -163,8 +169,9 @@ size_t qfp4_quantize_workspace_bytes(void);
  *   2. NVFP4: amax over v (or *amax_in when amax_in != NULL), s_enc = 2688 /
  *      amax, g = amax / 2688 (both 1 when amax = 0);
  *   3. block scale: NVFP4 S = E4M3_RN_sat(fp32(amax_b / 6) * s_enc),
- *      r = s_enc / S (0 when S = 0); MXFP4 E = floor(log2 amax_b) - 2 clamped
- *      to [-127, 127], code E + 127, r = 2^-E (code 0, r = 0 for a zero block);
+ *      r = s_enc / S (0 when S = 0); MXFP4 E = floor(log2 amax_b) - 2 (plus
+ *      one for QFP4_MXFP4_RU when amax_b > 6 * 2^E) clamped to [-127, 127],
+ *      code E + 127, r = 2^-E (code 0, r = 0 for a zero block);
  *   4. u = v * r; codes by RTN (ties to even, saturating at 6, -0 -> +0), SR
  *      (round up iff uniform < (|u| - lo) / gap), or Quartet II: RTN codes,
  *      then alpha = T(u*u) / T(u*q) (T the halving-stride tree sum over the

@@ -3,8 +3,21 @@ the oracle. Written from the layout stated in include/qfp4.h, independently of
 the library's own index function (which a test checks against this one)."""
 from __future__ import annotations
 
+import os
+import tempfile
+
 import numpy as np
 import torch
+
+# Scratch space of the tests that compile C helpers (kept inside the
+# repository, git-ignored).
+SCRATCH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_scratch")
+
+
+def scratch_dir(prefix: str) -> str:
+    """A fresh directory under the tests' scratch space."""
+    os.makedirs(SCRATCH, exist_ok=True)
+    return tempfile.mkdtemp(prefix=prefix, dir=SCRATCH)
 
 
 def atom_offset(rows: int, kb: int, r, c):

@@ -17,12 +17,12 @@ from __future__ import annotations
 import json
 import os
 import subprocess
-import tempfile
 from fractions import Fraction
 
 import numpy as np
 import torch
 
+import helpers
 import oracle as O
 from fp4_precision_b200 import inputs
 
@@ -138,7 +138,7 @@ def _torch_philox(cases):
     (offset lo, offset hi, subsequence lo, subsequence hi))."""
     global _philox_ref_bin
     if _philox_ref_bin is None:
-        d = tempfile.mkdtemp(prefix="philox_ref_")
+        d = helpers.scratch_dir("philox_ref_")
         src = os.path.join(d, "ref.cpp")
         with open(src, "w") as f:
             f.write(_PHILOX_HARNESS)

@@ -44,7 +44,7 @@ def test_strerror(lib):
     assert lib.qfp4_strerror(12345) == b"unknown status"
 
 
-@pytest.mark.parametrize("fmt", [Q.NVFP4, Q.MXFP4])
+@pytest.mark.parametrize("fmt", [Q.NVFP4, Q.MXFP4, Q.MXFP4_RU])
 @pytest.mark.parametrize("rows,k", [(1, 64), (128, 128), (300, 320), (512, 4096), (129, 96)])
 def test_scale_layout(lib, fmt, rows, k):
     nb = Q.BLOCK[fmt]
@@ -73,6 +73,7 @@ def test_sizes(lib):
     assert Q.codes_bytes(10, 64) == 320
     assert Q.codes_bytes(0, 64) == 0
     assert Q.scales_bytes(7, 10, 64) == 0
+    assert Q.scales_bytes(Q.MXFP4_RU, 128, 256) == Q.scales_bytes(Q.MXFP4, 128, 256)
     assert Q.quantize_workspace_bytes() >= 4 * 148
 
 

@@ -7,9 +7,11 @@ fp32 in that range, that the two steps give the correctly rounded quotient
 and divisions the kernel's __fmul_rn / __fmaf_rn / __fdiv_rn perform)."""
 import os
 import subprocess
-import tempfile
+import shutil
 
 import pytest
+
+import helpers
 
 SRC = r"""
 #include <math.h>
@@ -41,7 +43,8 @@ int main(void) {
 
 
 def test_divide_by_six_is_correctly_rounded_above_2_pow_minus_125():
-    with tempfile.TemporaryDirectory() as d:
+    d = helpers.scratch_dir("div6_")
+    try:
         c, exe = os.path.join(d, "div6.c"), os.path.join(d, "div6")
         with open(c, "w") as f:
             f.write(SRC)
@@ -51,4 +54,6 @@ def test_divide_by_six_is_correctly_rounded_above_2_pow_minus_125():
         except (OSError, subprocess.CalledProcessError):
             pytest.skip("no host C compiler with OpenMP")
         out = subprocess.check_output([exe], text=True, timeout=600)
+    finally:
+        shutil.rmtree(d, ignore_errors=True)
     assert int(out.strip()) == 0

@@ -38,6 +38,28 @@ def test_tiny_linear_fwd_bwd(preset):
     within(dW, dw_ref, dw_b, False)
 
 
+def test_tiny_linear_mxfp4_round_up():
+    """The AMD MXFP4 recipe with the round-up shared exponent on all six
+    operands (the tiny linear workload)."""
+    import dataclasses
+    wl = inputs.workload("tiny")
+    X, W, dY = wl["X"], wl["W"], wl["dY"]
+    rec = Q.recipe("AMD_MXFP4_H")
+    for c in (rec.fprop, rec.dgrad, rec.wgrad):
+        c.fmt = Q.MXFP4_RU
+    seed = Q.make_seed(ROT, SRS)
+    Y = Q.linear_fwd(X.cuda(), W.cuda(), rec, seed)
+    dX, dW = Q.linear_bwd(dY.cuda(), X.cuda(), W.cuda(), rec, seed)
+    Q.status()
+    r0 = O.preset("AMD_MXFP4_H")
+    r = O.Recipe(*(dataclasses.replace(c, fmt=O.MXFP4_RU) for c in (r0.fprop, r0.dgrad, r0.wgrad)))
+    y_ref, y_b = O.linear_fwd(X, W, r, ROT, SRS)
+    (dx_ref, dx_b), (dw_ref, dw_b) = O.linear_bwd(dY, X, W, r, ROT, SRS)
+    within(Y, y_ref, y_b, True)
+    within(dX, dx_ref, dx_b, True)
+    within(dW, dw_ref, dw_b, False)
+
+
 def test_autograd_function():
     wl = inputs.workload("tiny")
     X = wl["X"].cuda().requires_grad_(True)

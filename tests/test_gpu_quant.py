@@ -56,7 +56,7 @@ def sweep_like(R, C, seed=1):
 @pytest.mark.parametrize("axis", [Q.ROW, Q.COL], ids=["row", "col"])
 @pytest.mark.parametrize("had", HADS, ids=["none", "det16", "det32", "rand16", "rand32"])
 @pytest.mark.parametrize("rnd", [Q.RTN, Q.SR, Q.QUARTET2], ids=["rtn", "sr", "q2"])
-@pytest.mark.parametrize("fmt", [Q.NVFP4, Q.MXFP4], ids=["nvfp4", "mxfp4"])
+@pytest.mark.parametrize("fmt", [Q.NVFP4, Q.MXFP4, Q.MXFP4_RU], ids=["nvfp4", "mxfp4", "mxfp4ru"])
 def test_quantize_matches_oracle_ragged(fmt, rnd, had, axis):
     # 352 x 416: several 128-tiles plus ragged tails in both directions
     x = sweep_like(352, 416)
@@ -68,7 +68,8 @@ def test_quantize_matches_oracle_ragged(fmt, rnd, had, axis):
     (Q.NVFP4, Q.RTN, Q.HAD_RAND16, Q.ROW), (Q.NVFP4, Q.QUARTET2, Q.HAD_RAND16, Q.COL),
     (Q.MXFP4, Q.SR, Q.HAD_DET32, Q.COL), (Q.NVFP4, Q.SR, Q.HAD_NONE, Q.ROW),
     (Q.MXFP4, Q.QUARTET2, Q.HAD_RAND32, Q.ROW), (Q.NVFP4, Q.RTN, Q.HAD_DET16, Q.COL),
-], ids=lambda c: f"{['nv', 'mx'][c[0]]}-{['rtn', 'sr', 'q2'][c[1]]}-h{c[2]}-{['row', 'col'][c[3]]}")
+    (Q.MXFP4_RU, Q.RTN, Q.HAD_DET32, Q.COL), (Q.MXFP4_RU, Q.SR, Q.HAD_NONE, Q.ROW),
+], ids=lambda c: f"{['nv', 'mx', 'mxru'][c[0]]}-{['rtn', 'sr', 'q2'][c[1]]}-h{c[2]}-{['row', 'col'][c[3]]}")
 def test_quantize_full_sweep_workload(case):
     """The quantizer-sweep workload at its full size, [8192 x 4096]."""
     fmt, rnd, had, axis = case
@@ -91,6 +92,26 @@ def test_small_and_thin_shapes(fmt, shape, axis):
         assert_same(q, oracle_quant(x, fmt, rnd, had, axis), fmt)
 
 
+def test_mxfp4_round_up_writes_an_mxfp4_tensor():
+    """The round-up variant only changes the shared exponent: the tensor it
+    writes is an ordinary MXFP4 tensor (format field, scale layout), its
+    exponents are the floor rule's or one more, and a GEMM takes it."""
+    x_dev = sweep_like(256, 512).cuda()
+    qf = gpu_quant(x_dev, Q.MXFP4, Q.RTN, Q.HAD_NONE, Q.ROW)
+    qr = gpu_quant(x_dev, Q.MXFP4_RU, Q.RTN, Q.HAD_NONE, Q.ROW)
+    assert qr.fmt == Q.MXFP4
+    ef = helpers.unswizzle_scales(helpers.to_numpy_u8(qf.scales), 256, 512, 32).astype(np.int64)
+    er = helpers.unswizzle_scales(helpers.to_numpy_u8(qr.scales), 256, 512, 32).astype(np.int64)
+    d = er - ef
+    assert set(np.unique(d).tolist()) == {0, 1}
+    D = Q.gemm(qr, qr, torch.float32)
+    torch.cuda.synchronize()
+    Q.status()
+    A = oracle_quant(x_dev.cpu(), Q.MXFP4_RU, Q.RTN, Q.HAD_NONE, Q.ROW)
+    err = np.abs(D.cpu().numpy().astype(np.float64) - O.gemm(A, A))
+    assert np.all(err <= O.gemm_bound(A, A))
+
+
 def test_strided_input():
     """Row stride larger than the row (a column slice of a wider matrix)."""
     big = sweep_like(256, 512)
@@ -103,7 +124,7 @@ def test_strided_input():
 
 
 def test_degenerate_inputs():
-    for fmt in (Q.NVFP4, Q.MXFP4):
+    for fmt in (Q.NVFP4, Q.MXFP4, Q.MXFP4_RU):
         for axis in (Q.ROW, Q.COL):
             z = torch.zeros((160, 96), dtype=torch.bfloat16)
             q = gpu_quant(z.cuda(), fmt, Q.QUARTET2, Q.HAD_RAND32, axis)

@@ -3,10 +3,10 @@ at least one pin fails on it (CPU only). A pin set that passes a mutant would
 not protect the oracle against that mistake."""
 import os
 import shutil
-import tempfile
 
 import pytest
 
+import helpers
 import oracle as O
 import oracle_pins as P
 
@@ -40,7 +40,7 @@ MUTATIONS = [
 
 @pytest.fixture(scope="module")
 def tmpdir_mut():
-    d = tempfile.mkdtemp(prefix="oracle_mut_")
+    d = helpers.scratch_dir("oracle_mut_")
     yield d
     shutil.rmtree(d, ignore_errors=True)
 
