@@ -255,6 +255,29 @@ def run_ours(args, rank, world, local_rank):
     gemm_achieved = sum(gemm_flops) / (sum(gemm_ms) * 1e-3) / 1e12
     traffic = measured_gemm_traffic()
 
+    # Wgrad accumulating into an fp32 main gradient (dW += dY^T X) on the step's operands
+    def wgrad(acc):
+        if acc:
+            Q.gemm_accumulate(qs[4], qs[5], dW, stream=stream)
+        else:
+            Q.gemm(qs[4], qs[5], torch.float32, out=dW, stream=stream)
+    wg = {}
+    for acc in (False, True, False, True):
+        for _ in range(2):
+            wgrad(acc)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(10):
+            wgrad(acc)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        wg[acc] = e0.elapsed_time(e1) / 10
+    Q.status()
+    wgrad_acc = {"store_ms": round(wg[False], 4), "accumulate_ms": round(wg[True], 4),
+                 "accumulate_TFLOP/s": round(gemm_flops[2] / (wg[True] * 1e-3) / 1e12, 1),
+                 "what": "Wgrad of the step, dW = dY^T X vs dW += dY^T X (TMA reduce-add epilogue), fp32 dW "
+                         f"[{N}x{K}]; 10 back-to-back launches each"}
+
     # quantizer sweep workload (GB/s of algorithmic bytes), L2 flushed between launches,
     # and the same kernels on dY [16384 x 28672] (940 MB, steady state)
     quant = quant_sweep(Q, inputs, dev, stream, peaks)
@@ -298,6 +321,7 @@ def run_ours(args, rank, world, local_rank):
         "quantize": quant,
         "layers": layers,
         "study": study,
+        "wgrad_accumulate": wgrad_acc,
         "linear_api_ms_per_step": round(api_ms, 4),
         "e2e": e2e,
         "gpu_launches": launches,

@@ -277,7 +277,12 @@ __device__ __forceinline__ void store_f32(const GemmParams& p, uint32_t* acc, in
         acc[c] = __float_as_uint(v.x);
         acc[c + 1] = __float_as_uint(v.y);
     }
-    if (n0 + NC <= p.N) {
+    if (p.accumulate) {  // D += result: one fp32 add per element (each element has one owner)
+        const int nv = p.N - n0;
+#pragma unroll
+        for (int c = 0; c < NC; ++c)
+            if (c < nv) dst[c] = __fadd_rn(dst[c], __uint_as_float(acc[c]));
+    } else if (n0 + NC <= p.N) {
 #pragma unroll
         for (int c = 0; c < NC; c += 4)
             __stcs(reinterpret_cast<uint4*>(dst + c), make_uint4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]));
@@ -413,7 +418,10 @@ __device__ __forceinline__ void box_f32(const GemmParams& p, const CUtensorMap* 
     fence_proxy_async_shared();
     __syncwarp();
     if (lane == 0 && row0 < p.M && x < p.N) {
-        tma_store_2d(tmD, obox, x, row0);
+        if (p.accumulate)
+            tma_reduce_add_2d(tmD, obox, x, row0);
+        else
+            tma_store_2d(tmD, obox, x, row0);
         bulk_commit_group();
     }
 }

@@ -362,7 +362,8 @@ int quantize_impl(const void* x, int64_t R, int64_t C, int64_t ld, int32_t fmt, 
     return e == cudaSuccess ? QFP4_OK : cuda_fail(e);
 }
 
-int gemm_impl(const qfp4_tensor* A, const qfp4_tensor* B, void* D, int64_t ldd, int32_t out_dtype, cudaStream_t s) {
+int gemm_impl(const qfp4_tensor* A, const qfp4_tensor* B, void* D, int64_t ldd, int32_t out_dtype, bool accumulate,
+              cudaStream_t s) {
     int rc = bind_context(s);
     if (rc) return rc;
     int sms = 0;
@@ -370,6 +371,7 @@ int gemm_impl(const qfp4_tensor* A, const qfp4_tensor* B, void* D, int64_t ldd, 
     if (rc) return rc;
     if (A == nullptr || B == nullptr) return QFP4_ERR_INVALID_ARG;
     if (out_dtype != QFP4_OUT_BF16 && out_dtype != QFP4_OUT_F32) return QFP4_ERR_INVALID_ARG;
+    if (accumulate && out_dtype != QFP4_OUT_F32) return QFP4_ERR_INVALID_ARG;
     if (A->fmt != B->fmt || (A->fmt != QFP4_NVFP4 && A->fmt != QFP4_MXFP4)) return QFP4_ERR_INVALID_ARG;
     if (A->k != B->k || A->k < 0 || A->rows < 0 || B->rows < 0) return QFP4_ERR_INVALID_ARG;
     if (A->had != B->had) return QFP4_ERR_INVALID_ARG;
@@ -383,6 +385,7 @@ int gemm_impl(const qfp4_tensor* A, const qfp4_tensor* B, void* D, int64_t ldd, 
     if (D == nullptr || ldd < N) return QFP4_ERR_INVALID_ARG;
     if (!aligned16(D) || (ldd * (int64_t)esz) % 16 != 0) return QFP4_ERR_MISALIGNED;
     if (K == 0) {
+        if (accumulate) return QFP4_OK;  // D += 0
         cudaError_t e = cudaMemset2DAsync(D, (size_t)ldd * esz, 0, (size_t)N * esz, (size_t)M, s);
         return e == cudaSuccess ? QFP4_OK : cuda_fail(e);
     }
@@ -402,6 +405,7 @@ int gemm_impl(const qfp4_tensor* A, const qfp4_tensor* B, void* D, int64_t ldd, 
     p.D = D;
     p.ldd = ldd;
     p.out_f32 = out_dtype == QFP4_OUT_F32;
+    p.accumulate = accumulate ? 1 : 0;
     p.M = (int)M; p.N = (int)N; p.K = (int)K;
     const int NB = block_of(A->fmt);
     p.atoms_k = (int)((K / NB + 3) / 4);
@@ -472,6 +476,7 @@ int check_linear_args(int64_t M, int64_t N, int64_t K, const qfp4_recipe* r, con
     if (M <= 0 || N <= 0 || K <= 0 || (M % 128) || (N % 128) || (K % 128)) return QFP4_ERR_INVALID_ARG;
     if (!valid_cfg(r->fprop) || !valid_cfg(r->dgrad) || !valid_cfg(r->wgrad)) return QFP4_ERR_INVALID_ARG;
     if (!valid_dtype(r->y_dtype) || !valid_dtype(r->dx_dtype) || !valid_dtype(r->dw_dtype)) return QFP4_ERR_INVALID_ARG;
+    if (r->dw_accumulate != 0 && (r->dw_accumulate != 1 || r->dw_dtype != QFP4_OUT_F32)) return QFP4_ERR_INVALID_ARG;
     return QFP4_OK;
 }
 
@@ -627,7 +632,11 @@ int qfp4_quantize(const void* x, int64_t R, int64_t C, int64_t ld, int32_t fmt, 
 }
 
 int qfp4_gemm(const qfp4_tensor* A, const qfp4_tensor* B, void* D, int64_t ldd, int32_t out_dtype, void* stream) {
-    return gemm_impl(A, B, D, ldd, out_dtype, static_cast<cudaStream_t>(stream));
+    return gemm_impl(A, B, D, ldd, out_dtype, false, static_cast<cudaStream_t>(stream));
+}
+
+int qfp4_gemm_accumulate(const qfp4_tensor* A, const qfp4_tensor* B, float* D, int64_t ldd, void* stream) {
+    return gemm_impl(A, B, D, ldd, QFP4_OUT_F32, true, static_cast<cudaStream_t>(stream));
 }
 
 int qfp4_recipe_preset(int32_t preset, qfp4_recipe* out) {
@@ -685,7 +694,7 @@ int qfp4_linear_fwd(const void* X, const void* W, void* Y, int64_t M, int64_t N,
         return rc;
     if ((rc = quantize_impl(W, N, K, K, c.fmt, c.rnd_b, c.had, QFP4_AXIS_ROW, &sw, nullptr, &t[1], partials, pws, s)))
         return rc;
-    return gemm_impl(&t[0], &t[1], Y, N, recipe->y_dtype, s);
+    return gemm_impl(&t[0], &t[1], Y, N, recipe->y_dtype, false, s);
 }
 
 int qfp4_linear_bwd(const void* dY, const void* X, const void* W, void* dX, void* dW, int64_t M, int64_t N, int64_t K,
@@ -723,13 +732,13 @@ int qfp4_linear_bwd(const void* dY, const void* X, const void* W, void* dX, void
         return rc;
     if ((rc = quantize_impl(W, N, K, K, d.fmt, d.rnd_b, d.had, QFP4_AXIS_COL, &s1, nullptr, &t[1], partials, pws, s)))
         return rc;
-    if ((rc = gemm_impl(&t[0], &t[1], dX, K, recipe->dx_dtype, s))) return rc;
+    if ((rc = gemm_impl(&t[0], &t[1], dX, K, recipe->dx_dtype, false, s))) return rc;
     // Wgrad dW[N,K] = dY^T[N,M] . X[M,K]: reduce over M (tokens).
     if ((rc = quantize_impl(dY, M, N, N, w.fmt, w.rnd_a, w.had, QFP4_AXIS_COL, &s2, am_col, &t[2], partials, pws, s)))
         return rc;
     if ((rc = quantize_impl(X, M, K, K, w.fmt, w.rnd_b, w.had, QFP4_AXIS_COL, &s3, nullptr, &t[3], partials, pws, s)))
         return rc;
-    return gemm_impl(&t[2], &t[3], dW, K, recipe->dw_dtype, s);
+    return gemm_impl(&t[2], &t[3], dW, K, recipe->dw_dtype, recipe->dw_accumulate != 0, s);
 }
 
 int qfp4_status(void* stream) {

@@ -261,6 +261,14 @@ __device__ __forceinline__ void tma_store_2d(const void* tmap, uint32_t src_smem
                  "r"(src_smem), "r"(x), "r"(y)
                  : "memory");
 }
+// Element-wise fp32 add of a shared-memory box into global memory (TMA
+// reduce; the tensor map's element type is fp32).
+__device__ __forceinline__ void tma_reduce_add_2d(const void* tmap, uint32_t src_smem, int32_t x, int32_t y) {
+    asm volatile("cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                     tmap),
+                 "r"(src_smem), "r"(x), "r"(y)
+                 : "memory");
+}
 __device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // This thread's committed bulk stores have finished reading shared memory.
 __device__ __forceinline__ void bulk_wait_group_read0() {

@@ -65,6 +65,7 @@ struct GemmParams {
     void* D;
     int64_t ldd;
     int out_f32;
+    int accumulate;  // fp32 output only: D += result (one fp32 add per element)
     int M, N, K;
     int atoms_k;  // scale atoms per 128-row block along k: ceil(K / block / 4)
 };

@@ -46,7 +46,7 @@ class GemmCfg(ctypes.Structure):
 
 class Recipe(ctypes.Structure):
     _fields_ = [("fprop", GemmCfg), ("dgrad", GemmCfg), ("wgrad", GemmCfg), ("y_dtype", ctypes.c_int32),
-                ("dx_dtype", ctypes.c_int32), ("dw_dtype", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+                ("dx_dtype", ctypes.c_int32), ("dw_dtype", ctypes.c_int32), ("dw_accumulate", ctypes.c_int32)]
 
 
 class QFP4Error(RuntimeError):
@@ -74,6 +74,8 @@ _SIGNATURES = {
     "qfp4_quantize": (ctypes.c_int, [_VOID, _I64, _I64, _I64, _I32, _I32, _I32, _I32, ctypes.POINTER(Seed), _VOID,
                                      ctypes.POINTER(TensorDesc), _VOID, _SZ, _VOID]),
     "qfp4_gemm": (ctypes.c_int, [ctypes.POINTER(TensorDesc), ctypes.POINTER(TensorDesc), _VOID, _I64, _I32, _VOID]),
+    "qfp4_gemm_accumulate": (ctypes.c_int, [ctypes.POINTER(TensorDesc), ctypes.POINTER(TensorDesc), _VOID, _I64,
+                                            _VOID]),
     "qfp4_recipe_preset": (ctypes.c_int, [_I32, ctypes.POINTER(Recipe)]),
     "qfp4_linear_workspace_bytes": (_SZ, [_I32, _I64, _I64, _I64, ctypes.POINTER(Recipe)]),
     "qfp4_linear_fwd": (ctypes.c_int, [_VOID, _VOID, _VOID, _I64, _I64, _I64, ctypes.POINTER(Recipe),
@@ -232,6 +234,14 @@ def gemm(A: QTensor, B: QTensor, out_dtype=torch.bfloat16, out: torch.Tensor | N
     return out
 
 
+def gemm_accumulate(A: QTensor, B: QTensor, out: torch.Tensor, stream=None) -> torch.Tensor:
+    """out += gA gB A . B^T in fp32 (A.rows x B.rows); see qfp4_gemm_accumulate."""
+    assert out.dtype == torch.float32 and out.dim() == 2 and out.stride(1) == 1
+    _check(lib().qfp4_gemm_accumulate(ctypes.byref(A.desc), ctypes.byref(B.desc), _ptr(out), out.stride(0),
+                                      _stream(stream)), "qfp4_gemm_accumulate")
+    return out
+
+
 def recipe(name: str, dw_fp32: bool = True) -> Recipe:
     r = Recipe()
     _check(lib().qfp4_recipe_preset(PRESETS[name], ctypes.byref(r)), "qfp4_recipe_preset")
@@ -273,6 +283,8 @@ def linear_bwd(dY, X, W, rec: Recipe, seed: Seed, dX=None, dW=None, workspace=No
     M, K = X.shape
     N = W.shape[0]
     dX = torch.empty((M, K), dtype=_dtype(rec.dx_dtype), device=X.device) if dX is None else dX
+    if rec.dw_accumulate and dW is None:
+        raise ValueError("a recipe with dw_accumulate adds into dW: pass the buffer")
     dW = torch.empty((N, K), dtype=_dtype(rec.dw_dtype), device=X.device) if dW is None else dW
     if workspace is None:
         workspace = torch.empty((linear_workspace_bytes(True, M, N, K, rec),), dtype=torch.uint8, device=X.device)

@@ -133,7 +133,7 @@ typedef struct {
     qfp4_gemm_cfg dgrad; /* dX = dY W:   A = dY (along N),  B = W (along N) */
     qfp4_gemm_cfg wgrad; /* dW = dY^T X: A = dY (along M),  B = X (along M) */
     int32_t y_dtype, dx_dtype, dw_dtype; /* qfp4_dtype of the three outputs */
-    int32_t reserved;
+    int32_t dw_accumulate; /* 1: dW += dY^T X (fp32 dW only, e.g. a main-grad buffer), 0: dW = dY^T X */
 } qfp4_recipe;
 
 /* ---- errors -------------------------------------------------------------- */
@@ -216,6 +216,14 @@ int qfp4_quantize(const void* x, int64_t R, int64_t C, int64_t ld, int32_t fmt, 
  * environment variable QFP4_GEMM_PAIR=1 or =0 forces the pair or the single
  * kernel (same results within the bound). */
 int qfp4_gemm(const qfp4_tensor* A, const qfp4_tensor* B, void* D, int64_t ldd, int32_t out_dtype, void* stream);
+/* qfp4_gemm_accumulate: D[i][j] += gA * gB * sum_k A(i,k) B(j,k) into an fp32
+ * D (beta = 1: the Wgrad accumulation into an fp32 main gradient across
+ * micro-batches). The product is formed exactly as by qfp4_gemm with an fp32
+ * output, then added to D with one fp32 add (round to nearest) per element;
+ * the pair kernel adds through TMA reduce-add stores, the single-CTA kernel
+ * by a read-modify-write of the element it owns. D must not be written by
+ * anything else until the call completes. Requirements as qfp4_gemm. */
+int qfp4_gemm_accumulate(const qfp4_tensor* A, const qfp4_tensor* B, float* D, int64_t ldd, void* stream);
 
 /* ---- linear layer -------------------------------------------------------------
  * X [M x K], W [N x K], dY [M x N] bf16 row-major (contiguous); Y [M x N],

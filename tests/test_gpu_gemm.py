@@ -67,6 +67,53 @@ def kernel_variant(request, monkeypatch):
 
 
 @pytest.mark.parametrize("fmt", [O.NVFP4, O.MXFP4], ids=["nvfp4", "mxfp4"])
+@pytest.mark.parametrize("shape", [(128, 256, 256), (300, 200, 320), (512, 520, 1024), (100, 136, 192)],
+                         ids=lambda s: "x".join(map(str, s)))
+def test_gemm_accumulate_matches_oracle(fmt, shape, kernel_variant):
+    """D += A . B^T into an fp32 buffer (beta = 1): the product within the
+    GEMM bound, then one fp32 add per element; untouched outside A.rows x
+    B.rows (a wider row stride leaves the padding columns as they were)."""
+    M, N, K = shape
+    X = inputs.normal_with_outliers((M, K), 23, "aa")
+    W = inputs.normal((N, K), 0.02, 23, "ab")
+    A_o = O.quantize(X, fmt, O.RTN, O.HAD_NONE, O.ROW)
+    B_o = O.quantize(W, fmt, O.SR, O.HAD_NONE, O.ROW, 0, 0, 5, 1)
+    A, B = upload(A_o), upload(B_o)
+    ld = N + 4 - N % 4 + 8
+    D0 = inputs.normal((M, ld), 3.0, 23, "d0").float().cuda()
+    D = D0.clone()
+    Q.gemm_accumulate(A, B, D[:, :N])
+    torch.cuda.synchronize()
+    Q.status()
+    ref = O.gemm(A_o, B_o)
+    d0 = D0[:, :N].cpu().numpy().astype(np.float64)
+    tol = O.gemm_bound(A_o, B_o) + 2.0 ** -23 * (np.abs(d0) + np.abs(ref))
+    err = np.abs(D[:, :N].cpu().numpy().astype(np.float64) - (d0 + ref))
+    assert np.all(err <= tol), f"{np.sum(err > tol)} outputs out of bound"
+    assert torch.equal(D[:, N:], D0[:, N:])
+    # twice: the second call adds the same product again
+    Q.gemm_accumulate(A, B, D[:, :N])
+    torch.cuda.synchronize()
+    err2 = np.abs(D[:, :N].cpu().numpy().astype(np.float64) - (d0 + 2 * ref))
+    assert np.all(err2 <= 2 * tol + 2.0 ** -23 * np.abs(d0 + 2 * ref))
+
+
+def test_linear_dw_accumulate_needs_fp32_dw():
+    """A recipe that accumulates into dW must have an fp32 dW: the call is
+    rejected on the host, before anything is launched."""
+    rec = Q.recipe("QUARTET2_NVFP4", dw_fp32=False)
+    rec.dw_accumulate = 1
+    X = torch.zeros((128, 128), dtype=torch.bfloat16, device="cuda")
+    dW = torch.zeros((128, 128), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(Q.QFP4Error):
+        Q.linear_bwd(X, X, X, rec, Q.make_seed(), dW=dW)
+    acc = Q.recipe("QUARTET2_NVFP4")
+    acc.dw_accumulate = 1
+    with pytest.raises(ValueError):  # nothing to add into
+        Q.linear_bwd(X, X, X, acc, Q.make_seed())
+
+
+@pytest.mark.parametrize("fmt", [O.NVFP4, O.MXFP4], ids=["nvfp4", "mxfp4"])
 @pytest.mark.parametrize("shape", [(128, 256, 256), (300, 200, 320), (512, 520, 1024), (130, 640, 64),
                                    (1024, 768, 2048), (100, 136, 192)], ids=lambda s: "x".join(map(str, s)))
 @pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])

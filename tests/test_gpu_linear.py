@@ -60,6 +60,25 @@ def test_tiny_linear_mxfp4_round_up():
     within(dW, dw_ref, dw_b, False)
 
 
+def test_tiny_linear_dw_accumulate():
+    """dw_accumulate = 1: dW += dY^T X into the caller's fp32 buffer (a main
+    gradient across micro-batches); dX as without it."""
+    wl = inputs.workload("tiny")
+    X, W, dY = wl["X"], wl["W"], wl["dY"]
+    rec = Q.recipe("QUARTET2_NVFP4")
+    rec.dw_accumulate = 1
+    seed = Q.make_seed(ROT, SRS)
+    dW0 = inputs.normal(tuple(W.shape), 1.0, 3, "main_grad").float()
+    dW = dW0.cuda()
+    dX, dW = Q.linear_bwd(dY.cuda(), X.cuda(), W.cuda(), rec, seed, dW=dW)
+    Q.status()
+    r = O.preset("QUARTET2_NVFP4")
+    (dx_ref, dx_b), (dw_ref, dw_b) = O.linear_bwd(dY, X, W, r, ROT, SRS)
+    within(dX, dx_ref, dx_b, True)
+    d0 = dW0.numpy().astype(np.float64)
+    within(dW, d0 + dw_ref, dw_b + 2.0 ** -23 * (np.abs(d0) + np.abs(dw_ref)), False)
+
+
 def test_autograd_function():
     wl = inputs.workload("tiny")
     X = wl["X"].cuda().requires_grad_(True)
