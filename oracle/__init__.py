@@ -111,6 +111,10 @@ def load(path: str) -> ctypes.CDLL:
                                   ctypes.c_int, u64, u32, u64, u32, f32p, ctypes.c_void_p, ctypes.c_void_p,
                                   f32p, f32p]
     L.oracle_quantize.restype = ctypes.c_int
+    L.oracle_quantize_rows.argtypes = [ctypes.c_void_p, i64, i64, i64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                       ctypes.c_int, u64, u32, u64, u32, f32p, ctypes.c_void_p, i64,
+                                       ctypes.c_void_p, ctypes.c_void_p, f32p, f32p]
+    L.oracle_quantize_rows.restype = ctypes.c_int
     L.oracle_rotate.argtypes = [ctypes.c_void_p, i64, i64, i64, ctypes.c_int, ctypes.c_int, u64, u32,
                                 ctypes.c_void_p]
     L.oracle_rotate.restype = ctypes.c_int
@@ -207,21 +211,28 @@ class QTensor:
 
 
 def quantize(x, fmt: int, rnd: int, had: int, axis: int, rot_seed: int = 0, rot_stream: int = 0,
-             sr_seed: int = 0, sr_stream: int = 0, amax: float | None = None) -> QTensor:
+             sr_seed: int = 0, sr_stream: int = 0, amax: float | None = None, rows_sel=None) -> QTensor:
+    """Quantize x (bf16 [R, C]). rows_sel (optional): only these rows of the
+    quantized orientation, in that order (the tensor amax and the random words
+    stay those of the whole tensor); the result then has len(rows_sel) rows."""
     xb = _as_bf16_bits(x)
     R, C = xb.shape
     rows, k = (R, C) if axis == ROW else (C, R)
     nb = BLOCK[fmt]
-    codes = np.zeros((rows, k // 2), dtype=np.uint8)
-    scales = np.zeros((rows, k // nb), dtype=np.uint8)
-    alpha = np.ones((rows, k // nb), dtype=np.float32)
+    sel = None if rows_sel is None else np.ascontiguousarray(np.asarray(rows_sel, dtype=np.int64))
+    n_out = rows if sel is None else len(sel)
+    codes = np.zeros((n_out, k // 2), dtype=np.uint8)
+    scales = np.zeros((n_out, k // nb), dtype=np.uint8)
+    alpha = np.ones((n_out, k // nb), dtype=np.float32)
     g = np.zeros(1, dtype=np.float32)
     am = None if amax is None else np.array([amax], dtype=np.float32)
-    rc = lib().oracle_quantize(_ptr(xb), R, C, C, fmt, rnd, had, axis, rot_seed, rot_stream, sr_seed, sr_stream,
-                               None if am is None else _ptr(am), _ptr(codes), _ptr(scales), _ptr(g), _ptr(alpha))
+    rc = lib().oracle_quantize_rows(_ptr(xb), R, C, C, fmt, rnd, had, axis, rot_seed, rot_stream, sr_seed,
+                                    sr_stream, None if am is None else _ptr(am),
+                                    None if sel is None else _ptr(sel), 0 if sel is None else len(sel),
+                                    _ptr(codes), _ptr(scales), _ptr(g), _ptr(alpha))
     if rc != 0:
         raise ValueError("oracle_quantize: invalid arguments")
-    return QTensor(codes, scales, float(g[0]), fmt, had, rows, k, alpha)
+    return QTensor(codes, scales, float(g[0]), fmt, had, n_out, k, alpha)
 
 
 def rotate(x, had: int, axis: int, rot_seed: int = 0, rot_stream: int = 0) -> np.ndarray:

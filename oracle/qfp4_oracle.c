@@ -292,11 +292,16 @@ static void load_segment(const uint16_t* x, int64_t ld, int axis, int64_t row, i
  * (E4M3 for NVFP4, E8M0 for MXFP4), *g_out the NVFP4 per-tensor scale (1 for
  * MXFP4), alpha_out (optional) [rows][k/nb] the Quartet II renormalisation.
  * amax_in (optional) replaces the tensor amax of step 2.
+ * sel (optional, nsel entries): quantize only these rows of the quantized
+ * orientation; row sel[i] goes to output row i. Everything else is as for the
+ * whole tensor: the tensor amax is over all rows, and the random words are
+ * those of the row's own index.
  * Returns 0, or -1 on an invalid argument.
  */
-int oracle_quantize(const uint16_t* x, int64_t R, int64_t C, int64_t ld, int fmt, int rnd, int had,
-                    int axis, uint64_t rot_seed, uint32_t rot_stream, uint64_t sr_seed, uint32_t sr_stream,
-                    const float* amax_in, uint8_t* codes, uint8_t* scales, float* g_out, float* alpha_out) {
+int oracle_quantize_rows(const uint16_t* x, int64_t R, int64_t C, int64_t ld, int fmt, int rnd, int had,
+                         int axis, uint64_t rot_seed, uint32_t rot_stream, uint64_t sr_seed, uint32_t sr_stream,
+                         const float* amax_in, const int64_t* sel, int64_t nsel, uint8_t* codes, uint8_t* scales,
+                         float* g_out, float* alpha_out) {
     if (fmt != FMT_NVFP4 && fmt != FMT_MXFP4 && fmt != FMT_MXFP4_RU) return -1;
     if (rnd < RND_RTN || rnd > RND_QUARTET2) return -1;
     if (had < HAD_NONE || had > HAD_RAND32) return -1;
@@ -309,6 +314,12 @@ int oracle_quantize(const uint16_t* x, int64_t R, int64_t C, int64_t ld, int fmt
     if (k % nb != 0 || (nh && k % nh != 0)) return -1;
     const uint32_t signs = (had == HAD_RAND16 || had == HAD_RAND32) ? oracle_sign_bits(rot_seed, rot_stream) : 0u;
     const int64_t nblk = k / nb;
+    if (sel) {
+        if (nsel < 0) return -1;
+        for (int64_t i = 0; i < nsel; ++i)
+            if (sel[i] < 0 || sel[i] >= rows) return -1;
+    }
+    const int64_t n_out = sel ? nsel : rows;
 
     /* Step 1-2: the NVFP4 per-tensor scale from the amax of the rotated tensor.
      * Reading (NVFP4 two-level scaling, FP32 tensor scale): amax maps to 6 * 448,
@@ -349,12 +360,14 @@ int oracle_quantize(const uint16_t* x, int64_t R, int64_t C, int64_t ld, int fmt
         float u[32], prod[32];
         uint8_t q[32];
 #pragma omp for schedule(static)
-        for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t ro = 0; ro < n_out; ++ro) {
+            const int64_t r = sel ? sel[ro] : ro; /* row of the quantized orientation */
             load_segment(x, ld, axis, r, k, seg);
             rotate_segment(seg, k, nh, signs);
             for (int64_t b = 0; b < nblk; ++b) {
                 const float* v = seg + b * nb;
                 const int64_t blk_index = r * nblk + b; /* block index in the quantized orientation */
+                const int64_t blk_out = ro * nblk + b;  /* where it is stored */
                 /* Step 3: block scale from the block amax. */
                 float amax_b = 0.0f;
                 for (int j = 0; j < nb; ++j) amax_b = fmaxf(amax_b, fabsf(v[j]));
@@ -420,16 +433,23 @@ int oracle_quantize(const uint16_t* x, int64_t R, int64_t C, int64_t ld, int fmt
                     float rho = uniform24(random_word(sr_seed, TAG_SCALE, sr_stream, (uint64_t)blk_index));
                     s_code = (fmt == FMT_NVFP4) ? oracle_e4m3_sr(t, rho) : e8m0_sr(t, rho);
                 }
-                if (alpha_out) alpha_out[blk_index] = alpha;
-                scales[blk_index] = s_code;
+                if (alpha_out) alpha_out[blk_out] = alpha;
+                scales[blk_out] = s_code;
                 /* Step 6: pack two codes per byte, the lower index in the low nibble. */
-                uint8_t* out = codes + r * (k / 2) + b * (nb / 2);
+                uint8_t* out = codes + ro * (k / 2) + b * (nb / 2);
                 for (int j = 0; j < nb; j += 2) out[j / 2] = (uint8_t)(q[j] | (q[j + 1] << 4));
             }
         }
         free(seg);
     }
     return 0;
+}
+
+int oracle_quantize(const uint16_t* x, int64_t R, int64_t C, int64_t ld, int fmt, int rnd, int had,
+                    int axis, uint64_t rot_seed, uint32_t rot_stream, uint64_t sr_seed, uint32_t sr_stream,
+                    const float* amax_in, uint8_t* codes, uint8_t* scales, float* g_out, float* alpha_out) {
+    return oracle_quantize_rows(x, R, C, ld, fmt, rnd, had, axis, rot_seed, rot_stream, sr_seed, sr_stream, amax_in,
+                                NULL, 0, codes, scales, g_out, alpha_out);
 }
 
 /* The rotated, unquantized values v of the quantized orientation, [rows][k]
