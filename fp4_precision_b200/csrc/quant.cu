@@ -582,12 +582,14 @@ __global__ void __launch_bounds__(kThreads, 2)
     float amax_acc = 0.0f, amax_row_acc = 0.0f;
     ScaleRng srng;
     // Quartet II with 16-element groups: the 4 lanes of a column hold the 4
-    // blocks of one Philox quad (when k is a multiple of 64), so each lane
-    // computes the quad of one (chunk, column) of the warp per tile (lanes 2j
-    // and 2j + 1 the same one) and the 4 lanes that use it take its words by
-    // shuffles, instead of every lane computing it.
+    // blocks of one Philox quad (when k is a multiple of 64), and a warp needs
+    // 16 quads per tile (2 chunks x 8 columns). Every other tile, lanes 0-15
+    // compute this tile's quads and lanes 16-31 those of the CTA's next tile;
+    // the 4 lanes that use a quad take its words by shuffles.
     constexpr bool kSharedQuads = (RND == kQuartet2 && !AMAX_ONLY && G == 16 && NB == 16);
     const bool shared_quads = kSharedQuads && (p.k % 64) == 0;
+    uint4 lane_quad = make_uint4(0u, 0u, 0u, 0u);
+    uint32_t quad_half = 0;  // 0: compute this and the next tile's quads; 1: use the next tile's
     // Tile-invariant per thread (chunk ci = 0, 1): the column within the tile
     // (tiles start at multiples of 128 columns), the ldmatrix offsets within a
     // stage, the scale byte offset within a 128-row atom block, and the code
@@ -619,12 +621,21 @@ __global__ void __launch_bounds__(kThreads, 2)
         const int64_t c0 = (int64_t)w.tc * kColTileCols;
         const int64_t r0 = (int64_t)w.tr * TILE_ROWS;
         const uint32_t stage_base = smem_u32(tiles) + (uint32_t)(s * STAGE_BYTES);
-        uint4 lane_quad = make_uint4(0u, 0u, 0u, 0u);
         if constexpr (kSharedQuads) {
-            if (shared_quads) {
-                const int64_t cq = c0 + (2 * warp + (lane >> 4)) * 8 + ((lane >> 1) & 7);
+            if (shared_quads && quad_half == 0) {
+                int qtr = w.tr, qtc = w.tc;
+                if (lane >= 16) {  // the next tile of this CTA's walk (TileWalk::next)
+                    qtc += w.step_c;
+                    qtr += w.step_r;
+                    if (qtc >= w.tiles_c) {
+                        qtc -= w.tiles_c;
+                        ++qtr;
+                    }
+                }
+                const int64_t cq = (int64_t)qtc * kColTileCols + (2 * warp + ((lane >> 3) & 1)) * 8 + (lane & 7);
+                const int64_t rq = (int64_t)qtr * TILE_ROWS;
                 lane_quad = philox_quad(p.sr_seed, p.sr_tag_scale,
-                                        ((uint64_t)cq * (uint64_t)(p.k / NB) + (uint64_t)(r0 / NB)) >> 2);
+                                        ((uint64_t)cq * (uint64_t)(p.k / NB) + (uint64_t)(rq / NB)) >> 2);
             }
         }
 #pragma unroll
@@ -691,8 +702,8 @@ __global__ void __launch_bounds__(kThreads, 2)
                 Grp::rotate(v);
                 const uint64_t blk = (uint64_t)(c0 * (p.k / NB) + blk_off[ci] + r_grp / NB);
                 if constexpr (kSharedQuads) {
-                    if (shared_quads) {  // this group's quad: computed by lane (ci, column) * 2
-                        const int src = (ci << 4) | ((lane >> 2) << 1);
+                    if (shared_quads) {  // this group's quad: lane 16 * half + 8 * ci + column
+                        const int src = (int)(quad_half << 4) | (ci << 3) | (lane >> 2);
                         srng.w = make_uint4(__shfl_sync(0xffffffffu, lane_quad.x, src),
                                             __shfl_sync(0xffffffffu, lane_quad.y, src),
                                             __shfl_sync(0xffffffffu, lane_quad.z, src),
@@ -733,6 +744,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&ring.empty[s]);
+        if constexpr (kSharedQuads) quad_half ^= 1u;
     }
     if constexpr (AMAX_ONLY) {
         if constexpr (NH > 0) amax_acc = __fmul_rn(amax_acc, had_norm<NH>());  // c * max |y| = max |c * y|
