@@ -143,6 +143,25 @@ int make_col_tmap(CUtensorMap* tm, const void* x, int64_t R, int64_t C, int64_t 
     return QFP4_OK;
 }
 
+// 4-D view of a bf16 R x C tensor (R a multiple of 64) for the column
+// quantizer over 64-row bands: dimensions (column, r % 2, r / 64, (r / 2) % 32),
+// box (64, 2, 4, 32), 128-byte swizzle. The box lands in shared memory with
+// x-row r = k + 2 v + 64 q at 128-byte row s = k + 2 q + 8 v. The band count
+// bounds the view, so no address past row R - 1 is formed.
+int make_col64_tmap(CUtensorMap* tm, const void* x, int64_t R, int64_t C, int64_t ld) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return cuda_fail(cudaErrorNotSupported);
+    const cuuint64_t dims[4] = {(cuuint64_t)C, 2, (cuuint64_t)(R / 64), 32};
+    const cuuint64_t strides[3] = {(cuuint64_t)ld * 2, (cuuint64_t)64 * ld * 2, (cuuint64_t)2 * ld * 2};
+    const cuuint32_t box[4] = {64, 2, 4, 32};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(x), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
+    return QFP4_OK;
+}
+
 // 2-D view of a bf16 R x C tensor for the row quantizer: box 64 columns x 256
 // rows (128 bytes per row), 128-byte swizzle.
 int make_row_tmap(CUtensorMap* tm, const void* x, int64_t R, int64_t C, int64_t ld) {
@@ -213,6 +232,14 @@ int make_scale_tmap(CUtensorMap* tm, const void* scales, int64_t rows, int64_t a
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
     return QFP4_OK;
+}
+
+// The band-walking column quantizer is used whenever the quantized axis is a
+// multiple of 64; QFP4_COL_BANDS=0 selects the group-walking one instead (same
+// results; read on every call).
+bool col_bands_enabled() {
+    const char* e = std::getenv("QFP4_COL_BANDS");
+    return !(e != nullptr && e[0] == '0');
 }
 
 // CTA-pair kernel unless A has at most 128 rows (one pair tile would be half
@@ -357,8 +384,14 @@ int quantize_impl(const void* x, int64_t R, int64_t C, int64_t ld, int32_t fmt, 
         p.n_partials = n;
     }
     CUtensorMap tm;
-    if ((rc = make_input_tmap(&tm, x, R, C, ld, axis, col_group(NB, nh)))) return rc;
-    cudaError_t e = launch_quant(p, sfmt, rounding, nh, axis, &tm, s);
+    // the column quantizer walks 64-row bands when the quantized axis allows it
+    const bool bands = axis == QFP4_AXIS_COL && g.k % 64 == 0 && col_bands_enabled();
+    if (bands)
+        rc = make_col64_tmap(&tm, x, R, C, ld);
+    else
+        rc = make_input_tmap(&tm, x, R, C, ld, axis, col_group(NB, nh));
+    if (rc) return rc;
+    cudaError_t e = launch_quant(p, sfmt, rounding, nh, bands ? 2 : axis, &tm, s);
     return e == cudaSuccess ? QFP4_OK : cuda_fail(e);
 }
 

@@ -43,6 +43,8 @@ struct QuantParams {
 // `tmap` is the TMA view of x: 2-D (row mode) or the 5-D column view.
 cudaError_t launch_amax(const QuantParams& p, int axis, int nh, const CUtensorMap* tmap, int n_partials,
                         cudaStream_t s);
+// axis: 0 row, 1 column (5-D group view), 2 column over 64-row bands (the
+// 4-D band view; quantized axis a multiple of 64).
 cudaError_t launch_quant(const QuantParams& p, int fmt, int rnd, int nh, int axis, const CUtensorMap* tmap,
                          cudaStream_t s);
 // One pass of the column kernel (tmap: its 5-D view, group 16) that writes the

@@ -756,6 +756,143 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
 }
 
+// ===========================================================================
+// Column mode, 64-row bands (quantized axis a multiple of 64)
+// ===========================================================================
+// Tile: 256 x-rows (four bands of 64) x 64 columns. Thread (column c = 8 w +
+// l / 4 of warp w, band q = l % 4) takes the 64 consecutive x-rows of band q
+// of its column: 64 / G whole groups, four 16-element (or two 32-element)
+// scale blocks, i.e. one 4-byte (NVFP4) or 2-byte (MXFP4) scale word, 32
+// bytes of codes and, for Quartet II, one Philox quad per tile.
+// The 4-D tensor map (column, r % 2, r / 64, (r / 2) % 32) delivers x-row
+// r = k + 2 v + 64 q (k < 2, v < 32) to 128-byte shared-memory row
+// s = k + 2 q + 8 v. Lane l of ldmatrix.x4 number n (n < 8) supplies smem row
+// s = l + 32 n, i.e. matrix l / 8 row l % 8 = (q = (l % 8) / 2, k = l % 2) at
+// v = 4 n + l / 8; the 8 rows of a phase have s % 8 = l % 8 all distinct
+// (conflict-free with the 128-byte swizzle), and after the transposing load
+// lane (c, q) holds x-rows 64 q + 8 n + [0, 8) of column c in order.
+template <int FMT, int RND, int NH, int STAGES>
+__global__ void __launch_bounds__(kThreads, 2)
+    quant_col64_kernel(const __grid_constant__ CUtensorMap tmap, const QuantParams p) {
+    using Grp = Group<FMT, RND, NH>;
+    constexpr int NB = Grp::NB;
+    constexpr int G = Grp::G;
+    constexpr int TILE_ROWS = 256, TILE_COLS = 64;
+    constexpr int STAGE_BYTES = TILE_ROWS * TILE_COLS * 2;  // 32 KiB
+    static_assert(64 % G == 0, "groups tile a 64-row band");
+    extern __shared__ __align__(1024) uint8_t dyn_smem[];
+    uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
+    __shared__ Ring<STAGES> ring;
+    __shared__ float red[33];
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    // output rows = x columns, walked up to the 128-row padding of the scale
+    // atoms: the tiles past the last column read zeros and write zero scales
+    const int tiles_c = (int)((p.rows + 127) / 128 * 2);
+    const int tiles_r = (int)((p.k + TILE_ROWS - 1) / TILE_ROWS);
+
+    if (tid == 0) {
+        prefetch_tmap(&tmap);
+        ring_init(ring);
+    }
+    __syncthreads();
+    __shared__ float rtab[128];
+    float s_enc = 1.0f;
+    if constexpr (FMT == kNvfp4) {
+        s_enc = nvfp4_encode_scale(p, red, blockIdx.x == 0);
+        fill_rtab(rtab, s_enc);
+    }
+    if constexpr (FMT == kMxfp4) {
+        if (blockIdx.x == 0 && tid == 0) *p.tensor_scale = 1.0f;
+    }
+
+    if (warp == kComputeWarps) {
+        if (lane == 0) {
+            int i = 0;
+            for (TileWalk<STAGES> w(tiles_c); w.tr < tiles_r; w.next(), ++i) {
+                const int s = w.stage;
+                if (i >= STAGES && !mbar_wait(&ring.empty[s], w.phase ^ 1u)) break;
+                mbar_arrive_expect_tx(&ring.full[s], STAGE_BYTES);
+                tma_load_4d(tiles + s * STAGE_BYTES, &tmap, &ring.full[s], w.tc * TILE_COLS, 0, 4 * w.tr, 0);
+            }
+        }
+        return;
+    }
+
+    const int64_t rows_pad = (p.rows + 127) / 128 * 128;
+    const int q = lane & 3;
+    const int cc = warp * 8 + (lane >> 2);  // column within the tile
+    // ldmatrix address of instruction n: lm_base + 4096 n (smem row lane + 32 n)
+    const uint32_t lm_base = (uint32_t)lane * 128u + ((uint32_t)(warp ^ (lane & 7)) << 4);
+    const int64_t atom_row_bytes = (p.kb4 / 4) * 512;
+    uint32_t smask[G / 2];
+#pragma unroll
+    for (int i = 0; i < G / 2; ++i) smask[i] = Grp::sign_mask(p.signs, i);
+    ScaleRng srng;
+    for (TileWalk<STAGES> w(tiles_c); w.tr < tiles_r; w.next()) {
+        const int s = w.stage;
+        if (!mbar_wait(&ring.full[s], w.phase)) break;
+        const int64_t c = (int64_t)w.tc * TILE_COLS + cc;          // x column = output row
+        const int64_t rb = (int64_t)w.tr * TILE_ROWS + 64 * q;     // first k index of this thread's band
+        const uint32_t stage_base = smem_u32(tiles) + (uint32_t)(s * STAGE_BYTES) + lm_base;
+        uint32_t codes[8];
+        uint32_t scodes[64 / NB];
+#pragma unroll
+        for (int g = 0; g < 64 / G; ++g) {
+            float v[G];
+#pragma unroll
+            for (int u = 0; u < G / 8; ++u) {
+                const uint32_t addr = stage_base + (uint32_t)((g * (G / 8) + u) * 4096);
+                uint32_t a0, a1, a2, a3;
+                asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                             : "=r"(a0), "=r"(a1), "=r"(a2), "=r"(a3)
+                             : "r"(addr));
+                if (NH > 0 && p.signs != 0u) {
+                    a0 ^= smask[4 * u + 0];
+                    a1 ^= smask[4 * u + 1];
+                    a2 ^= smask[4 * u + 2];
+                    a3 ^= smask[4 * u + 3];
+                }
+                v[8 * u + 0] = bf16lo(a0); v[8 * u + 1] = bf16hi(a0);
+                v[8 * u + 2] = bf16lo(a1); v[8 * u + 3] = bf16hi(a1);
+                v[8 * u + 4] = bf16lo(a2); v[8 * u + 5] = bf16hi(a2);
+                v[8 * u + 6] = bf16lo(a3); v[8 * u + 7] = bf16hi(a3);
+            }
+            Grp::rotate(v);
+            const int64_t r_grp = rb + g * G;
+            Grp::quantize(v, s_enc, rtab, p, (uint64_t)c * (uint64_t)p.k + (uint64_t)r_grp,
+                          (uint64_t)c * (uint64_t)(p.k / NB) + (uint64_t)(r_grp / NB), srng, codes + g * (G / 8),
+                          scodes + g * (G / NB));
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ring.empty[s]);
+        if (rb < p.k) {  // k is a multiple of 64: a band is wholly inside or wholly outside
+            if (c < p.rows) {
+                uint4* dst = reinterpret_cast<uint4*>(p.codes + c * (p.k / 2) + rb / 2);
+                dst[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+                dst[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
+            }
+            if (c < rows_pad) {
+                const int64_t kb0 = rb / NB;
+                uint8_t* sc = p.scales + (c / 128) * atom_row_bytes + (kb0 / 4) * 512 + (c % 32) * 16 + ((c / 32) % 4) * 4;
+                if constexpr (NB == 16) {
+                    *reinterpret_cast<uint32_t*>(sc) =
+                        scodes[0] | (scodes[1] << 8) | (scodes[2] << 16) | (scodes[3] << 24);
+                } else {
+                    // two scale columns: half of an atom word; when this is the
+                    // word's first half and the band is the last, the other
+                    // half is padding and is written as zero
+                    const uint32_t half = scodes[0] | (scodes[1] << 8);
+                    if ((kb0 & 3) == 0 && rb + 64 >= p.k)
+                        *reinterpret_cast<uint32_t*>(sc) = half;
+                    else
+                        *reinterpret_cast<uint16_t*>(sc + (kb0 & 3)) = (uint16_t)half;
+                }
+            }
+        }
+    }
+}
+
 int g_sm_count = 0;
 
 int persistent_grid(int64_t tiles, int per_sm) {
@@ -800,8 +937,24 @@ cudaError_t launch_t(const QuantParams& p, int axis, const CUtensorMap* tmap, in
     }
 }
 
+// Column mode over 64-row bands (axis code 2; the quantized axis a multiple of 64).
+template <int FMT, int RND, int NH>
+cudaError_t launch_col64(const QuantParams& p, const CUtensorMap* tmap, cudaStream_t s) {
+    constexpr int S = 3;
+    const int64_t tiles = ((p.rows + 127) / 128 * 2) * ((p.k + 255) / 256);
+    const int smem = S * 256 * 64 * 2 + 1024;
+    return launch_persistent(quant_col64_kernel<FMT, RND, NH, S>, persistent_grid(tiles, 2), smem, *tmap, p, s);
+}
+
 template <int FMT, int RND>
 cudaError_t dispatch_nh(const QuantParams& p, int nh, int axis, const CUtensorMap* tmap, cudaStream_t s) {
+    if (axis == 2) {
+        switch (nh) {
+            case 0: return launch_col64<FMT, RND, 0>(p, tmap, s);
+            case 16: return launch_col64<FMT, RND, 16>(p, tmap, s);
+            default: return launch_col64<FMT, RND, 32>(p, tmap, s);
+        }
+    }
     switch (nh) {
         case 0: return launch_t<FMT, RND, 0, false>(p, axis, tmap, 0, s);
         case 16: return launch_t<FMT, RND, 16, false>(p, axis, tmap, 0, s);

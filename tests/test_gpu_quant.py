@@ -64,6 +64,22 @@ def test_quantize_matches_oracle_ragged(fmt, rnd, had, axis):
     assert_same(q, oracle_quant(x, fmt, rnd, had, axis), fmt)
 
 
+@pytest.mark.parametrize("shape", [(320, 424), (448, 136)], ids=["320x424", "448x136"])
+@pytest.mark.parametrize("had", HADS, ids=["none", "det16", "det32", "rand16", "rand32"])
+@pytest.mark.parametrize("rnd", [Q.RTN, Q.SR, Q.QUARTET2], ids=["rtn", "sr", "q2"])
+@pytest.mark.parametrize("fmt", [Q.NVFP4, Q.MXFP4, Q.MXFP4_RU], ids=["nvfp4", "mxfp4", "mxfp4ru"])
+def test_column_bands_match_oracle(fmt, rnd, had, shape, monkeypatch):
+    """The column quantizer over 64-row bands (quantized axis a multiple of
+    64): a partial last tile of 256 rows (320 = 5 bands; 448 = 7 bands, which
+    also leaves half of the last MXFP4 scale word as padding) and a partial
+    last tile of 64 columns; and the group-walking kernel on the same input."""
+    x = sweep_like(*shape)
+    ref = oracle_quant(x, fmt, rnd, had, Q.COL)
+    assert_same(gpu_quant(x.cuda(), fmt, rnd, had, Q.COL), ref, fmt)
+    monkeypatch.setenv("QFP4_COL_BANDS", "0")
+    assert_same(gpu_quant(x.cuda(), fmt, rnd, had, Q.COL), ref, fmt)
+
+
 @pytest.mark.parametrize("case", [
     (Q.NVFP4, Q.RTN, Q.HAD_RAND16, Q.ROW), (Q.NVFP4, Q.QUARTET2, Q.HAD_RAND16, Q.COL),
     (Q.MXFP4, Q.SR, Q.HAD_DET32, Q.COL), (Q.NVFP4, Q.SR, Q.HAD_NONE, Q.ROW),
