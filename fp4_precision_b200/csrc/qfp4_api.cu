@@ -395,6 +395,80 @@ int quantize_impl(const void* x, int64_t R, int64_t C, int64_t ld, int32_t fmt, 
     return e == cudaSuccess ? QFP4_OK : cuda_fail(e);
 }
 
+// Can one read of x (R x C) give both orientations' quantizations? Same
+// format and rounding (caller), R a multiple of 64, the row orientation's
+// Hadamard none or of the column one's size.
+bool dual_ok(int64_t R, int32_t had_row, int32_t had_col) {
+    return R % 64 == 0 && (had_n(had_row) == 0 || had_n(had_row) == had_n(had_col)) && col_bands_enabled();
+}
+
+void fill_out(qfp4_tensor* out, int64_t rows, int64_t k, int32_t fmt, int32_t had, const qfp4_seed* seed) {
+    out->rows = rows;
+    out->k = k;
+    out->fmt = (fmt == QFP4_MXFP4_RU) ? QFP4_MXFP4 : fmt;
+    out->had = had;
+    out->rot_seed = had_random(had) ? seed->rot : 0;
+    out->rot_stream = had_random(had) ? seed->rot_stream : 0;
+    out->reserved = 0;
+}
+
+int quantize_dual_impl(const void* x, int64_t R, int64_t C, int64_t ld, int32_t fmt, int32_t rounding, int32_t had_row,
+                       int32_t had_col, const qfp4_seed* seed_row, const qfp4_seed* seed_col, const float* amax_row,
+                       const float* amax_col, qfp4_tensor* out_row, qfp4_tensor* out_col, cudaStream_t s) {
+    int sms = 0;
+    int rc = bind_context(s);
+    if (rc) return rc;
+    rc = check_device(&sms);
+    if (rc) return rc;
+    if (!valid_fmt(fmt)) return QFP4_ERR_INVALID_ARG;
+    if (rounding < QFP4_RTN || rounding > QFP4_QUARTET2) return QFP4_ERR_INVALID_ARG;
+    if (!out_row || !out_col || !seed_row || !seed_col) return QFP4_ERR_INVALID_ARG;
+    for (const qfp4_seed* sd : {seed_row, seed_col})
+        if (sd->rot_stream >= (1u << 28) || sd->sr_stream >= (1u << 28)) return QFP4_ERR_INVALID_ARG;
+    Geometry gr, gc;
+    if ((rc = validate_input(x, R, C, ld, had_row, QFP4_AXIS_ROW, &gr))) return rc;
+    if ((rc = validate_input(x, R, C, ld, had_col, QFP4_AXIS_COL, &gc))) return rc;
+    const int NB = block_of(fmt);
+    if (C % NB != 0 || R % NB != 0) return QFP4_ERR_INVALID_ARG;
+    if (R == 0 || C == 0) return QFP4_ERR_INVALID_ARG;
+    if (!dual_ok(R, had_row, had_col)) return QFP4_ERR_INVALID_ARG;
+    if (fmt == QFP4_NVFP4 && (amax_row == nullptr || amax_col == nullptr)) return QFP4_ERR_INVALID_ARG;
+    for (const qfp4_tensor* o : {out_row, out_col}) {
+        if (!o->codes || !o->scales || !o->tensor_scale) return QFP4_ERR_INVALID_ARG;
+        if (!aligned16(o->codes) || !aligned16(o->scales)) return QFP4_ERR_MISALIGNED;
+    }
+    fill_out(out_row, R, C, fmt, had_row, seed_row);
+    fill_out(out_col, C, R, fmt, had_col, seed_col);
+    QuantParams p{};
+    p.x = static_cast<const uint16_t*>(x);
+    p.R = R; p.C = C; p.ld = ld;
+    p.rows = C; p.k = R;  // the column orientation
+    p.codes = out_col->codes;
+    p.scales = out_col->scales;
+    p.tensor_scale = out_col->tensor_scale;
+    p.kb4 = (R / NB + 3) / 4 * 4;
+    p.signs = had_random(had_col) ? host_sign_bits(seed_col->rot, seed_col->rot_stream) : 0u;
+    p.sr_seed = seed_col->sr;
+    p.sr_tag_elem = (uint32_t)kTagElement | (seed_col->sr_stream << 4);
+    p.sr_tag_scale = (uint32_t)kTagScale | (seed_col->sr_stream << 4);
+    p.amax_in = amax_col;
+    p.mx_round_up = (fmt == QFP4_MXFP4_RU) ? 1u : 0u;
+    p.codes_row = out_row->codes;
+    p.scales_row = out_row->scales;
+    p.tensor_scale_row = out_row->tensor_scale;
+    p.amax_in_row = amax_row;
+    p.kb4_row = (C / NB + 3) / 4 * 4;
+    p.signs_row = had_random(had_row) ? host_sign_bits(seed_row->rot, seed_row->rot_stream) : 0u;
+    p.sr_seed_row = seed_row->sr;
+    p.sr_tag_elem_row = (uint32_t)kTagElement | (seed_row->sr_stream << 4);
+    p.sr_tag_scale_row = (uint32_t)kTagScale | (seed_row->sr_stream << 4);
+    CUtensorMap tm;
+    if ((rc = make_col64_tmap(&tm, x, R, C, ld))) return rc;
+    const int sfmt = (fmt == QFP4_MXFP4_RU) ? QFP4_MXFP4 : fmt;
+    cudaError_t e = launch_quant_dual(p, sfmt, rounding, had_n(had_col), had_n(had_row), &tm, s);
+    return e == cudaSuccess ? QFP4_OK : cuda_fail(e);
+}
+
 int gemm_impl(const qfp4_tensor* A, const qfp4_tensor* B, void* D, int64_t ldd, int32_t out_dtype, bool accumulate,
               cudaStream_t s) {
     int rc = bind_context(s);
@@ -664,6 +738,14 @@ int qfp4_quantize(const void* x, int64_t R, int64_t C, int64_t ld, int32_t fmt, 
                          static_cast<cudaStream_t>(stream));
 }
 
+int qfp4_quantize_dual(const void* x, int64_t R, int64_t C, int64_t ld, int32_t fmt, int32_t rounding,
+                       int32_t had_row, int32_t had_col, const qfp4_seed* seed_row, const qfp4_seed* seed_col,
+                       const float* amax_row, const float* amax_col, qfp4_tensor* out_row, qfp4_tensor* out_col,
+                       void* stream) {
+    return quantize_dual_impl(x, R, C, ld, fmt, rounding, had_row, had_col, seed_row, seed_col, amax_row, amax_col,
+                              out_row, out_col, static_cast<cudaStream_t>(stream));
+}
+
 int qfp4_gemm(const qfp4_tensor* A, const qfp4_tensor* B, void* D, int64_t ldd, int32_t out_dtype, void* stream) {
     return gemm_impl(A, B, D, ldd, out_dtype, false, static_cast<cudaStream_t>(stream));
 }
@@ -752,22 +834,37 @@ int qfp4_linear_bwd(const void* dY, const void* X, const void* W, void* dX, void
     qfp4_seed s2 = op_seed(seed, 2, 4), s3 = op_seed(seed, 2, 5);
     // dY is quantized along both axes (Dgrad: along N; Wgrad: along M). When
     // both are NVFP4 with the same Hadamard (size <= 16; the sign vectors
-    // differ per GEMM), one read of dY gives both tensor amaxes.
+    // differ per GEMM), one read of dY gives both tensor amaxes; when both
+    // quantizations share format and rounding, one more read gives both
+    // quantized operands.
+    const bool dual = d.fmt == w.fmt && d.rnd_a == w.rnd_a && dual_ok(M, d.had, w.had);
     const float* am_row = nullptr;
     const float* am_col = nullptr;
     if (d.fmt == QFP4_NVFP4 && w.fmt == QFP4_NVFP4 && d.had == w.had && had_n(d.had) <= 16) {
         if ((rc = amax_rowcol_impl(dY, M, N, N, d.had, &s0, &s2, dy_amax, dy_amax + 1, partials, pws, s))) return rc;
         am_row = dy_amax;
         am_col = dy_amax + 1;
+    } else if (dual && d.fmt == QFP4_NVFP4) {
+        if ((rc = qfp4_amax(dY, M, N, N, d.had, QFP4_AXIS_ROW, &s0, dy_amax, partials, pws, s))) return rc;
+        if ((rc = qfp4_amax(dY, M, N, N, w.had, QFP4_AXIS_COL, &s2, dy_amax + 1, partials, pws, s))) return rc;
+        am_row = dy_amax;
+        am_col = dy_amax + 1;
     }
     // Dgrad dX[M,K] = dY[M,N] . W[N,K]: reduce over N.
-    if ((rc = quantize_impl(dY, M, N, N, d.fmt, d.rnd_a, d.had, QFP4_AXIS_ROW, &s0, am_row, &t[0], partials, pws, s)))
+    if (dual) {
+        if ((rc = quantize_dual_impl(dY, M, N, N, d.fmt, d.rnd_a, d.had, w.had, &s0, &s2, am_row, am_col, &t[0],
+                                     &t[2], s)))
+            return rc;
+    } else if ((rc = quantize_impl(dY, M, N, N, d.fmt, d.rnd_a, d.had, QFP4_AXIS_ROW, &s0, am_row, &t[0], partials,
+                                   pws, s))) {
         return rc;
+    }
     if ((rc = quantize_impl(W, N, K, K, d.fmt, d.rnd_b, d.had, QFP4_AXIS_COL, &s1, nullptr, &t[1], partials, pws, s)))
         return rc;
     if ((rc = gemm_impl(&t[0], &t[1], dX, K, recipe->dx_dtype, false, s))) return rc;
     // Wgrad dW[N,K] = dY^T[N,M] . X[M,K]: reduce over M (tokens).
-    if ((rc = quantize_impl(dY, M, N, N, w.fmt, w.rnd_a, w.had, QFP4_AXIS_COL, &s2, am_col, &t[2], partials, pws, s)))
+    if (!dual &&
+        (rc = quantize_impl(dY, M, N, N, w.fmt, w.rnd_a, w.had, QFP4_AXIS_COL, &s2, am_col, &t[2], partials, pws, s)))
         return rc;
     if ((rc = quantize_impl(X, M, K, K, w.fmt, w.rnd_b, w.had, QFP4_AXIS_COL, &s3, nullptr, &t[3], partials, pws, s)))
         return rc;

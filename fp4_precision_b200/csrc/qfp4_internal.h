@@ -37,6 +37,17 @@ struct QuantParams {
     uint32_t sr_tag_elem;         // kTagElement | stream << 4
     uint32_t sr_tag_scale;        // kTagScale | stream << 4
     uint32_t mx_round_up;         // MXFP4: 1 = the smallest E with amax_b <= 6 * 2^E (no clipping)
+    // Dual quantization (the column kernel over 64-row bands also quantizes
+    // x along its rows): the row orientation's outputs, tensor amax and
+    // randomness; its sign bits are signs_row.
+    uint8_t* codes_row;
+    uint8_t* scales_row;
+    float* tensor_scale_row;
+    const float* amax_in_row;
+    int64_t kb4_row;
+    uint64_t sr_seed_row;
+    uint32_t sr_tag_elem_row;
+    uint32_t sr_tag_scale_row;
 };
 
 // Launchers (quant.cu). Return cudaSuccess or the launch error.
@@ -47,6 +58,11 @@ cudaError_t launch_amax(const QuantParams& p, int axis, int nh, const CUtensorMa
 // 4-D band view; quantized axis a multiple of 64).
 cudaError_t launch_quant(const QuantParams& p, int fmt, int rnd, int nh, int axis, const CUtensorMap* tmap,
                          cudaStream_t s);
+// Dual quantization of x (R x C, R a multiple of 64; tmap: the 64-row band
+// view): p describes the column orientation, p.*_row the row orientation.
+// nh: the column orientation's Hadamard size; nh_row: 0 or nh.
+cudaError_t launch_quant_dual(const QuantParams& p, int fmt, int rnd, int nh, int nh_row, const CUtensorMap* tmap,
+                              cudaStream_t s);
 // One pass of the column kernel (tmap: its 5-D view, group 16) that writes the
 // column orientation's partial maxima to p.amax_out and the row orientation's
 // to p.amax_out_row (n_partials each). nh: 0 or 16.

@@ -131,6 +131,19 @@ __device__ __forceinline__ float2 e2m1x2_decode(uint32_t byte) {
     return __half22float2(*reinterpret_cast<__half2*>(&h2));
 }
 
+// s_enc = 2688 / amax (clamped to the largest finite fp32), g = amax / 2688
+// (both 1 when amax = 0); g written by thread 0 when write_g.
+__device__ __forceinline__ float nvfp4_scale_from_amax(float amax, float* tensor_scale, bool write_g) {
+    float s_enc = 1.0f, g = 1.0f;
+    if (amax > 0.0f) {
+        s_enc = __fdiv_rn(2688.0f, amax);
+        if (s_enc > 3.402823466e38f) s_enc = 3.402823466e38f;
+        g = __fdiv_rn(amax, 2688.0f);
+    }
+    if (write_g && threadIdx.x == 0) *tensor_scale = g;
+    return s_enc;
+}
+
 // Reduce the CTA's amax partials (NVFP4) to s_enc; CTA 0 writes g.
 __device__ float nvfp4_encode_scale(const QuantParams& p, float* red_smem, bool write_g) {
     float amax = 0.0f;
@@ -152,14 +165,7 @@ __device__ float nvfp4_encode_scale(const QuantParams& p, float* red_smem, bool 
         __syncthreads();
         amax = red_smem[32];
     }
-    float s_enc = 1.0f, g = 1.0f;
-    if (amax > 0.0f) {
-        s_enc = __fdiv_rn(2688.0f, amax);
-        if (s_enc > 3.402823466e38f) s_enc = 3.402823466e38f;
-        g = __fdiv_rn(amax, 2688.0f);
-    }
-    if (write_g && threadIdx.x == 0) *p.tensor_scale = g;
-    return s_enc;
+    return nvfp4_scale_from_amax(amax, p.tensor_scale, write_g);
 }
 
 // rtab[c] = s_enc / S(c) for every E4M3 code c the saturating conversion can
@@ -171,15 +177,30 @@ __device__ void fill_rtab(float* rtab, float s_enc) {
     __syncthreads();
 }
 
+// The random streams and MXFP4 exponent rule of one orientation (what the
+// per-group quantization reads besides the values).
+struct Stream {
+    uint64_t seed;
+    uint32_t tag_elem;   // element SR: kTagElement | stream << 4
+    uint32_t tag_scale;  // Quartet II scale SR: kTagScale | stream << 4
+    uint32_t mx_round_up;
+};
+__device__ __forceinline__ Stream col_stream(const QuantParams& p) {
+    return Stream{p.sr_seed, p.sr_tag_elem, p.sr_tag_scale, p.mx_round_up};
+}
+__device__ __forceinline__ Stream row_stream(const QuantParams& p) {
+    return Stream{p.sr_seed_row, p.sr_tag_elem_row, p.sr_tag_scale_row, p.mx_round_up};
+}
+
 // The four Quartet II scale uniforms of one Philox quad, computed once per quad.
 struct ScaleRng {
     uint64_t quad = ~0ull;
     uint4 w;
     // Philox word of the block (its uniform is (word >> 8) * 2^-24).
-    __device__ __forceinline__ uint32_t word(const QuantParams& p, uint64_t block_index) {
+    __device__ __forceinline__ uint32_t word(const Stream& p, uint64_t block_index) {
         const uint64_t q = block_index >> 2;
         if (q != quad) {
-            w = philox_quad(p.sr_seed, p.sr_tag_scale, q);
+            w = philox_quad(p.seed, p.tag_scale, q);
             quad = q;
         }
         const uint32_t i = (uint32_t)(block_index & 3);
@@ -228,7 +249,7 @@ struct Group {
     }
 
     // rtab[c] = s_enc / (E4M3 value of c) for codes 1-126, 0 for code 0.
-    __device__ __forceinline__ static void quantize(float* v, float s_enc, const float* rtab, const QuantParams& p,
+    __device__ __forceinline__ static void quantize(float* v, float s_enc, const float* rtab, const Stream& p,
                                                     uint64_t elem0, uint64_t block0, ScaleRng& srng,
                                                     uint32_t* codes, uint32_t* scodes) {
 #pragma unroll
@@ -276,7 +297,7 @@ struct Group {
                 const uint64_t i0 = elem0 + (uint64_t)(b * NB);
 #pragma unroll
                 for (int e4 = 0; e4 < NB; e4 += 4) {
-                    const uint4 w = philox_quad(p.sr_seed, p.sr_tag_elem, (i0 + e4) >> 2);
+                    const uint4 w = philox_quad(p.seed, p.tag_elem, (i0 + e4) >> 2);
                     vb[e4 + 0] = e2m1_sr_value(vb[e4 + 0], uniform24(w.x));
                     vb[e4 + 1] = e2m1_sr_value(vb[e4 + 1], uniform24(w.y));
                     vb[e4 + 2] = e2m1_sr_value(vb[e4 + 2], uniform24(w.z));
@@ -310,6 +331,19 @@ struct Group {
         }
     }
 };
+
+// 32 bytes of codes (64 elements of one row): two 16-byte stores, or four
+// 8-byte ones when the row length in bytes (k / 2) is not a multiple of 16
+// (k a multiple of 16 but not of 32: rows start 8-byte aligned).
+__device__ __forceinline__ void store_codes32(uint8_t* dst, const uint32_t* codes, bool aligned16) {
+    if (aligned16) {
+        reinterpret_cast<uint4*>(dst)[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+        reinterpret_cast<uint4*>(dst)[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
+    } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) reinterpret_cast<uint2*>(dst)[i] = make_uint2(codes[2 * i], codes[2 * i + 1]);
+    }
+}
 
 // This CTA's tiles of a tiles_r x tiles_c grid (blockIdx.x, + gridDim.x, ...)
 // as (tr, tc), advanced without divisions, with the TMA ring stage and phase
@@ -470,7 +504,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             } else {
                 Grp::rotate(v);
                 const int64_t j0 = col0 + g * G;
-                Grp::quantize(v, s_enc, rtab, p, (uint64_t)row * (uint64_t)p.k + (uint64_t)j0,
+                Grp::quantize(v, s_enc, rtab, col_stream(p), (uint64_t)row * (uint64_t)p.k + (uint64_t)j0,
                               (uint64_t)row * (uint64_t)(p.k / NB) + (uint64_t)(j0 / NB), srng,
                               codes + g * (G / 8), scodes + g * (G / NB));
             }
@@ -481,8 +515,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             if (row < p.rows) {
                 uint8_t* dst = p.codes + row * (p.k / 2) + col0 / 2;
                 if (col0 + kRowTileCols <= p.k) {
-                    reinterpret_cast<uint4*>(dst)[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
-                    reinterpret_cast<uint4*>(dst)[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
+                    store_codes32(dst, codes, ((p.k / 2) & 15) == 0);
                 } else {
 #pragma unroll
                     for (int w = 0; w < 8; ++w)
@@ -711,7 +744,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                         srng.quad = blk >> 2;
                     }
                 }
-                Grp::quantize(v, s_enc, rtab, p, (uint64_t)c * (uint64_t)p.k + (uint64_t)r_grp, blk, srng, codes,
+                Grp::quantize(v, s_enc, rtab, col_stream(p), (uint64_t)c * (uint64_t)p.k + (uint64_t)r_grp, blk, srng, codes,
                               scodes);
                 if (c < p.rows && r_grp < p.k) {
                     uint8_t* dst = p.codes + c0 * (p.k / 2) + code_off[ci] + r_grp / 2;
@@ -771,9 +804,86 @@ __global__ void __launch_bounds__(kThreads, 2)
 // v = 4 n + l / 8; the 8 rows of a phase have s % 8 = l % 8 all distinct
 // (conflict-free with the 128-byte swizzle), and after the transposing load
 // lane (c, q) holds x-rows 64 q + 8 n + [0, 8) of column c in order.
-template <int FMT, int RND, int NH, int STAGES>
+// Dual mode's row work on one band tile (see below): thread t quantizes
+// shared-memory row t of the stage at `stage`, x-row r = r0 + k + 2 v + 64 q
+// (t = k + 2 q + 8 v) over the tile's 64 columns, and stores its codes and
+// scale word(s) in the row orientation (rows = R, k = C).
+template <int FMT, int RND, int NH_ROW>
+__device__ __forceinline__ void dual_row_work(const QuantParams& p, float s_enc_row,
+                                              const float* rtab_row, ScaleRng& srng, uint32_t stage, int tr, int tc) {
+    using GrpR = Group<FMT, RND, NH_ROW>;
+    constexpr int NB = GrpR::NB;
+    constexpr int GR = GrpR::G;
+    const int t = threadIdx.x;
+    const int64_t r = (int64_t)tr * 256 + (t & 1) + 2 * (t >> 3) + 64 * ((t >> 1) & 3);
+    const int64_t c0 = (int64_t)tc * 64;
+    if (c0 >= p.C) return;  // the column tiles past C exist for the column orientation's padding only
+    const uint32_t rbase = stage + (uint32_t)t * 128u;
+    uint32_t codes[8];
+    uint32_t scodes[64 / NB];
+#pragma unroll
+    for (int g = 0; g < 64 / GR; ++g) {
+        float v[GR];
+#pragma unroll
+        for (int c8 = 0; c8 < GR / 8; ++c8) {
+            const int chunk = g * (GR / 8) + c8;
+            uint32_t w0, w1, w2, w3;
+            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(w0), "=r"(w1), "=r"(w2), "=r"(w3)
+                         : "r"(rbase + ((uint32_t)(chunk ^ (t & 7)) << 4)));
+            if (NH_ROW > 0 && p.signs_row != 0u) {
+                w0 ^= GrpR::sign_mask(p.signs_row, 4 * c8 + 0);
+                w1 ^= GrpR::sign_mask(p.signs_row, 4 * c8 + 1);
+                w2 ^= GrpR::sign_mask(p.signs_row, 4 * c8 + 2);
+                w3 ^= GrpR::sign_mask(p.signs_row, 4 * c8 + 3);
+            }
+            v[8 * c8 + 0] = bf16lo(w0); v[8 * c8 + 1] = bf16hi(w0);
+            v[8 * c8 + 2] = bf16lo(w1); v[8 * c8 + 3] = bf16hi(w1);
+            v[8 * c8 + 4] = bf16lo(w2); v[8 * c8 + 5] = bf16hi(w2);
+            v[8 * c8 + 6] = bf16lo(w3); v[8 * c8 + 7] = bf16hi(w3);
+        }
+        GrpR::rotate(v);
+        const int64_t j0 = c0 + g * GR;
+        GrpR::quantize(v, s_enc_row, rtab_row, row_stream(p), (uint64_t)r * (uint64_t)p.C + (uint64_t)j0,
+                       (uint64_t)r * (uint64_t)(p.C / NB) + (uint64_t)(j0 / NB), srng, codes + g * (GR / 8),
+                       scodes + g * (GR / NB));
+    }
+    if (r < p.R) {
+        uint8_t* dst = p.codes_row + r * (p.C / 2) + c0 / 2;
+        if (c0 + 64 <= p.C) {
+            store_codes32(dst, codes, ((p.C / 2) & 15) == 0);
+        } else {
+#pragma unroll
+            for (int w = 0; w < 8; ++w)
+                if (c0 + 8 * w < p.C) reinterpret_cast<uint32_t*>(dst)[w] = codes[w];
+        }
+    }
+    if (r < (p.R + 127) / 128 * 128) {
+        const int64_t kb0 = c0 / NB;
+        uint8_t* sc = p.scales_row + ((r / 128) * (p.kb4_row / 4) + kb0 / 4) * 512 + (r % 32) * 16 +
+                      ((r / 32) % 4) * 4;
+        if constexpr (NB == 16) {
+            *reinterpret_cast<uint32_t*>(sc) = scodes[0] | (scodes[1] << 8) | (scodes[2] << 16) | (scodes[3] << 24);
+        } else {
+            const uint32_t half = scodes[0] | (scodes[1] << 8);
+            if ((kb0 & 3) == 0 && c0 + 64 >= p.C)
+                *reinterpret_cast<uint32_t*>(sc) = half;
+            else
+                *reinterpret_cast<uint16_t*>(sc + (kb0 & 3)) = (uint16_t)half;
+        }
+    }
+}
+
+//
+// Dual mode (NH_ROW >= 0): after its column work on a tile, thread t also
+// quantizes shared-memory row t, i.e. x-row k + 2 v + 64 q of the tile over its
+// 64 columns, in the row orientation (rotation of size NH_ROW with the row
+// sign vector, the row tensor amax and random streams), as the row kernel
+// would: one read of x gives both orientations.
+template <int FMT, int RND, int NH, int STAGES, int NH_ROW = -1>
 __global__ void __launch_bounds__(kThreads, 2)
     quant_col64_kernel(const __grid_constant__ CUtensorMap tmap, const QuantParams p) {
+    constexpr bool kDual = NH_ROW >= 0;
     using Grp = Group<FMT, RND, NH>;
     constexpr int NB = Grp::NB;
     constexpr int G = Grp::G;
@@ -797,13 +907,21 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     __syncthreads();
     __shared__ float rtab[128];
-    float s_enc = 1.0f;
+    __shared__ float rtab_row[kDual ? 128 : 1];
+    float s_enc = 1.0f, s_enc_row = 1.0f;
     if constexpr (FMT == kNvfp4) {
         s_enc = nvfp4_encode_scale(p, red, blockIdx.x == 0);
         fill_rtab(rtab, s_enc);
+        if constexpr (kDual) {  // the row orientation's amax is always given
+            s_enc_row = nvfp4_scale_from_amax(__ldg(p.amax_in_row), p.tensor_scale_row, blockIdx.x == 0);
+            fill_rtab(rtab_row, s_enc_row);
+        }
     }
     if constexpr (FMT == kMxfp4) {
-        if (blockIdx.x == 0 && tid == 0) *p.tensor_scale = 1.0f;
+        if (blockIdx.x == 0 && tid == 0) {
+            *p.tensor_scale = 1.0f;
+            if constexpr (kDual) *p.tensor_scale_row = 1.0f;
+        }
     }
 
     if (warp == kComputeWarps) {
@@ -825,10 +943,13 @@ __global__ void __launch_bounds__(kThreads, 2)
     // ldmatrix address of instruction n: lm_base + 4096 n (smem row lane + 32 n)
     const uint32_t lm_base = (uint32_t)lane * 128u + ((uint32_t)(warp ^ (lane & 7)) << 4);
     const int64_t atom_row_bytes = (p.kb4 / 4) * 512;
-    uint32_t smask[G / 2];
+    // sign masks held in registers, except in dual mode (registers for the row work)
+    uint32_t smask[kDual ? 1 : G / 2];
+    if constexpr (!kDual) {
 #pragma unroll
-    for (int i = 0; i < G / 2; ++i) smask[i] = Grp::sign_mask(p.signs, i);
-    ScaleRng srng;
+        for (int i = 0; i < G / 2; ++i) smask[i] = Grp::sign_mask(p.signs, i);
+    }
+    ScaleRng srng, srng_row;
     for (TileWalk<STAGES> w(tiles_c); w.tr < tiles_r; w.next()) {
         const int s = w.stage;
         if (!mbar_wait(&ring.full[s], w.phase)) break;
@@ -848,10 +969,10 @@ __global__ void __launch_bounds__(kThreads, 2)
                              : "=r"(a0), "=r"(a1), "=r"(a2), "=r"(a3)
                              : "r"(addr));
                 if (NH > 0 && p.signs != 0u) {
-                    a0 ^= smask[4 * u + 0];
-                    a1 ^= smask[4 * u + 1];
-                    a2 ^= smask[4 * u + 2];
-                    a3 ^= smask[4 * u + 3];
+                    a0 ^= kDual ? Grp::sign_mask(p.signs, 4 * u + 0) : smask[kDual ? 0 : 4 * u + 0];
+                    a1 ^= kDual ? Grp::sign_mask(p.signs, 4 * u + 1) : smask[kDual ? 0 : 4 * u + 1];
+                    a2 ^= kDual ? Grp::sign_mask(p.signs, 4 * u + 2) : smask[kDual ? 0 : 4 * u + 2];
+                    a3 ^= kDual ? Grp::sign_mask(p.signs, 4 * u + 3) : smask[kDual ? 0 : 4 * u + 3];
                 }
                 v[8 * u + 0] = bf16lo(a0); v[8 * u + 1] = bf16hi(a0);
                 v[8 * u + 2] = bf16lo(a1); v[8 * u + 3] = bf16hi(a1);
@@ -860,10 +981,12 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
             Grp::rotate(v);
             const int64_t r_grp = rb + g * G;
-            Grp::quantize(v, s_enc, rtab, p, (uint64_t)c * (uint64_t)p.k + (uint64_t)r_grp,
+            Grp::quantize(v, s_enc, rtab, col_stream(p), (uint64_t)c * (uint64_t)p.k + (uint64_t)r_grp,
                           (uint64_t)c * (uint64_t)(p.k / NB) + (uint64_t)(r_grp / NB), srng, codes + g * (G / 8),
                           scodes + g * (G / NB));
         }
+        if constexpr (kDual) dual_row_work<FMT, RND, NH_ROW>(p, s_enc_row, rtab_row, srng_row,
+                                                          smem_u32(tiles) + (uint32_t)(s * STAGE_BYTES), w.tr, w.tc);
         __syncwarp();
         if (lane == 0) mbar_arrive(&ring.empty[s]);
         if (rb < p.k) {  // k is a multiple of 64: a band is wholly inside or wholly outside
@@ -1004,6 +1127,34 @@ cudaError_t launch_quant(const QuantParams& p, int fmt, int rnd, int nh, int axi
     if (rnd == kRtn) return dispatch_nh<kMxfp4, kRtn>(p, nh, axis, tmap, s);
     if (rnd == kSr) return dispatch_nh<kMxfp4, kSr>(p, nh, axis, tmap, s);
     return dispatch_nh<kMxfp4, kQuartet2>(p, nh, axis, tmap, s);
+}
+
+template <int FMT, int RND, int NH, int NH_ROW>
+cudaError_t launch_dual_t(const QuantParams& p, const CUtensorMap* tmap, cudaStream_t s) {
+    constexpr int S = 3;
+    const int64_t tiles = ((p.rows + 127) / 128 * 2) * ((p.k + 255) / 256);
+    const int smem = S * 256 * 64 * 2 + 1024;
+    return launch_persistent(quant_col64_kernel<FMT, RND, NH, S, NH_ROW>, persistent_grid(tiles, 2), smem, *tmap, p,
+                             s);
+}
+
+template <int FMT, int RND>
+cudaError_t dispatch_dual(const QuantParams& p, int nh, int nh_row, const CUtensorMap* tmap, cudaStream_t s) {
+    if (nh == 0) return launch_dual_t<FMT, RND, 0, 0>(p, tmap, s);
+    if (nh == 16) return nh_row == 0 ? launch_dual_t<FMT, RND, 16, 0>(p, tmap, s) : launch_dual_t<FMT, RND, 16, 16>(p, tmap, s);
+    return nh_row == 0 ? launch_dual_t<FMT, RND, 32, 0>(p, tmap, s) : launch_dual_t<FMT, RND, 32, 32>(p, tmap, s);
+}
+
+cudaError_t launch_quant_dual(const QuantParams& p, int fmt, int rnd, int nh, int nh_row, const CUtensorMap* tmap,
+                              cudaStream_t s) {
+    if (fmt == kNvfp4) {
+        if (rnd == kRtn) return dispatch_dual<kNvfp4, kRtn>(p, nh, nh_row, tmap, s);
+        if (rnd == kSr) return dispatch_dual<kNvfp4, kSr>(p, nh, nh_row, tmap, s);
+        return dispatch_dual<kNvfp4, kQuartet2>(p, nh, nh_row, tmap, s);
+    }
+    if (rnd == kRtn) return dispatch_dual<kMxfp4, kRtn>(p, nh, nh_row, tmap, s);
+    if (rnd == kSr) return dispatch_dual<kMxfp4, kSr>(p, nh, nh_row, tmap, s);
+    return dispatch_dual<kMxfp4, kQuartet2>(p, nh, nh_row, tmap, s);
 }
 
 cudaError_t launch_amax_rowcol(const QuantParams& p, int nh, const CUtensorMap* tmap, int n_partials,

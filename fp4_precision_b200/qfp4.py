@@ -73,6 +73,9 @@ _SIGNATURES = {
                                         _VOID, _VOID, _VOID, _SZ, _VOID]),
     "qfp4_quantize": (ctypes.c_int, [_VOID, _I64, _I64, _I64, _I32, _I32, _I32, _I32, ctypes.POINTER(Seed), _VOID,
                                      ctypes.POINTER(TensorDesc), _VOID, _SZ, _VOID]),
+    "qfp4_quantize_dual": (ctypes.c_int, [_VOID, _I64, _I64, _I64, _I32, _I32, _I32, _I32, ctypes.POINTER(Seed),
+                                          ctypes.POINTER(Seed), _VOID, _VOID, ctypes.POINTER(TensorDesc),
+                                          ctypes.POINTER(TensorDesc), _VOID]),
     "qfp4_gemm": (ctypes.c_int, [ctypes.POINTER(TensorDesc), ctypes.POINTER(TensorDesc), _VOID, _I64, _I32, _VOID]),
     "qfp4_gemm_accumulate": (ctypes.c_int, [ctypes.POINTER(TensorDesc), ctypes.POINTER(TensorDesc), _VOID, _I64,
                                             _VOID]),
@@ -221,6 +224,21 @@ def quantize(x: torch.Tensor, fmt: int, rounding: int, had: int, axis: int, seed
                                _ptr(amax_in), ctypes.byref(out.desc), _ptr(ws), ws.numel(), _stream(stream)),
            "qfp4_quantize")
     return out
+
+
+def quantize_dual(x: torch.Tensor, fmt: int, rounding: int, had_row: int, had_col: int, seed_row: Seed,
+                  seed_col: Seed, amax_row: torch.Tensor | None = None, amax_col: torch.Tensor | None = None,
+                  out_row: QTensor | None = None, out_col: QTensor | None = None, stream=None):
+    """Row and column quantization of a bf16 matrix from one read; see qfp4_quantize_dual."""
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
+    R, C = x.shape
+    out_row = empty_qtensor(fmt, R, C, x.device) if out_row is None else out_row
+    out_col = empty_qtensor(fmt, C, R, x.device) if out_col is None else out_col
+    _check(lib().qfp4_quantize_dual(_ptr(x), R, C, x.stride(0), fmt, rounding, had_row, had_col,
+                                    ctypes.byref(seed_row), ctypes.byref(seed_col), _ptr(amax_row), _ptr(amax_col),
+                                    ctypes.byref(out_row.desc), ctypes.byref(out_col.desc), _stream(stream)),
+           "qfp4_quantize_dual")
+    return out_row, out_col
 
 
 def gemm(A: QTensor, B: QTensor, out_dtype=torch.bfloat16, out: torch.Tensor | None = None,

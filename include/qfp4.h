@@ -203,6 +203,22 @@ int qfp4_amax_rowcol(const void* x, int64_t R, int64_t C, int64_t ld, int32_t ha
 int qfp4_quantize(const void* x, int64_t R, int64_t C, int64_t ld, int32_t fmt, int32_t rounding, int32_t had,
                   int32_t axis, const qfp4_seed* seed, const float* amax_in, qfp4_tensor* out, void* workspace,
                   size_t workspace_bytes, void* stream);
+/* qfp4_quantize_dual: both orientations of x from one read of it — exactly
+ * what qfp4_quantize gives with axis ROW (had_row, seed_row, *amax_row) into
+ * out_row and with axis COL (had_col, seed_col, *amax_col) into out_col, same
+ * format and rounding. It serves the backward linear layer, where dY is
+ * quantized along N for Dgrad and along the tokens for Wgrad (pages: "New AMD
+ * paper overturns conventional wisdom: FP4 training...", section
+ * "Poiskovaya eksperimental'naya rabota", the three GEMMs of the layer).
+ * Requirements: those of qfp4_quantize for both axes; R a multiple of 64,
+ * R and C > 0; had_row none or of had_col's size (16 or 32); for NVFP4,
+ * amax_row and amax_col are the two tensor amaxes (device fp32, e.g. from
+ * qfp4_amax_rowcol or qfp4_amax), required; ignored for MXFP4. No workspace.
+ * Unsupported combinations return QFP4_ERR_INVALID_ARG. */
+int qfp4_quantize_dual(const void* x, int64_t R, int64_t C, int64_t ld, int32_t fmt, int32_t rounding,
+                       int32_t had_row, int32_t had_col, const qfp4_seed* seed_row, const qfp4_seed* seed_col,
+                       const float* amax_row, const float* amax_col, qfp4_tensor* out_row, qfp4_tensor* out_col,
+                       void* stream);
 
 /* ---- GEMM -------------------------------------------------------------------
  * D[i][j] = gA * gB * sum_k A(i,k) B(j,k) over the decoded FP4 operands, fp32

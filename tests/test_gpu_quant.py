@@ -80,6 +80,59 @@ def test_column_bands_match_oracle(fmt, rnd, had, shape, monkeypatch):
     assert_same(gpu_quant(x.cuda(), fmt, rnd, had, Q.COL), ref, fmt)
 
 
+DUAL_HADS = [(Q.HAD_NONE, Q.HAD_NONE), (Q.HAD_NONE, Q.HAD_RAND16), (Q.HAD_RAND16, Q.HAD_RAND16),
+             (Q.HAD_DET16, Q.HAD_RAND16), (Q.HAD_NONE, Q.HAD_DET32), (Q.HAD_RAND32, Q.HAD_RAND32)]
+
+
+@pytest.mark.parametrize("shape", [(320, 416), (448, 160)], ids=["320x416", "448x160"])
+@pytest.mark.parametrize("hads", DUAL_HADS, ids=lambda h: f"row{h[0]}-col{h[1]}")
+@pytest.mark.parametrize("rnd", [Q.RTN, Q.SR, Q.QUARTET2], ids=["rtn", "sr", "q2"])
+@pytest.mark.parametrize("fmt", [Q.NVFP4, Q.MXFP4, Q.MXFP4_RU], ids=["nvfp4", "mxfp4", "mxfp4ru"])
+def test_quantize_dual_matches_oracle(fmt, rnd, hads, shape):
+    """Both orientations from one read (qfp4_quantize_dual) equal the oracle's
+    row and column quantizations: partial last tiles in rows (5 or 7 bands of
+    64) and columns, MXFP4 scale words half padding, different sign vectors
+    and Hadamard sizes for the two orientations."""
+    had_row, had_col = hads
+    x = sweep_like(*shape)
+    xd = x.cuda()
+    s_row = Q.make_seed(SEED["rot"], SEED["sr"], 1, 2)
+    s_col = Q.make_seed(SEED["rot"], SEED["sr"], 2, 4)
+    am_row = am_col = None
+    if fmt == Q.NVFP4:
+        am_row = Q.amax(xd, had_row, Q.ROW, s_row)
+        am_col = Q.amax(xd, had_col, Q.COL, s_col)
+    qr, qc = Q.quantize_dual(xd, fmt, rnd, had_row, had_col, s_row, s_col, am_row, am_col)
+    torch.cuda.synchronize()
+    Q.status()
+    assert qr.fmt == qc.fmt == (Q.MXFP4 if fmt == Q.MXFP4_RU else fmt)
+    assert_same(qr, O.quantize(x, fmt, rnd, had_row, Q.ROW, SEED["rot"], 1, SEED["sr"], 2), fmt)
+    assert_same(qc, O.quantize(x, fmt, rnd, had_col, Q.COL, SEED["rot"], 2, SEED["sr"], 4), fmt)
+
+
+def test_quantize_dual_rejects_unsupported():
+    x = sweep_like(128, 128).cuda()
+    s = Q.make_seed(1, 2)
+    with pytest.raises(Q.QFP4Error):  # rows not a multiple of 64
+        Q.quantize_dual(x[:96], Q.MXFP4, Q.RTN, Q.HAD_NONE, Q.HAD_NONE, s, s)
+    with pytest.raises(Q.QFP4Error):  # row Hadamard neither none nor the column one's size
+        Q.quantize_dual(x, Q.MXFP4, Q.RTN, Q.HAD_DET16, Q.HAD_DET32, s, s)
+    with pytest.raises(Q.QFP4Error):  # NVFP4 needs both tensor amaxes
+        Q.quantize_dual(x, Q.NVFP4, Q.RTN, Q.HAD_NONE, Q.HAD_NONE, s, s)
+    torch.cuda.synchronize()
+
+
+@pytest.mark.parametrize("axis", [Q.ROW, Q.COL], ids=["row", "col"])
+@pytest.mark.parametrize("rnd", [Q.RTN, Q.SR, Q.QUARTET2], ids=["rtn", "sr", "q2"])
+def test_nvfp4_axis_not_a_multiple_of_32(rnd, axis):
+    """NVFP4 needs only k % 16 == 0: with k = 208 the codes of a row start
+    8-byte aligned (the 32-byte code stores split into 8-byte ones)."""
+    x = sweep_like(208, 208)
+    for had in (Q.HAD_NONE, Q.HAD_DET16, Q.HAD_RAND16):
+        q = gpu_quant(x.cuda(), Q.NVFP4, rnd, had, axis)
+        assert_same(q, oracle_quant(x, Q.NVFP4, rnd, had, axis), Q.NVFP4)
+
+
 @pytest.mark.parametrize("case", [
     (Q.NVFP4, Q.RTN, Q.HAD_RAND16, Q.ROW), (Q.NVFP4, Q.QUARTET2, Q.HAD_RAND16, Q.COL),
     (Q.MXFP4, Q.SR, Q.HAD_DET32, Q.COL), (Q.NVFP4, Q.SR, Q.HAD_NONE, Q.ROW),
