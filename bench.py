@@ -181,10 +181,10 @@ def run_ours(args, rank, world, local_rank):
     gemm_flops = [2.0 * M * N * K] * 3
     quant_elems = [t.numel() for (t, *_rest) in ops]
 
-    # dY is quantized along both axes; with NVFP4 and the same Hadamard for Dgrad
-    # and Wgrad one pass gives both tensor amaxes (as qfp4_linear_bwd does)
-    fused_dy_amax = (c[1].fmt == Q.NVFP4 and c[2].fmt == Q.NVFP4 and c[1].had == c[2].had
-                     and c[1].had in (Q.HAD_NONE, Q.HAD_DET16, Q.HAD_RAND16))
+    # dY is quantized along both axes, as qfp4_linear_bwd does it: with NVFP4 and
+    # the same Hadamard for Dgrad and Wgrad one pass gives both tensor amaxes;
+    # with round-to-nearest one pass gives both quantizations
+    fused_dy_amax, dual_dy = dy_plan(Q, c, M)
     dy_amax = torch.empty((2,), dtype=torch.float32, device=dev)
 
     def step(ev=None):
@@ -192,12 +192,10 @@ def run_ours(args, rank, world, local_rank):
         for i, (t, fmt, rnd, had, axis, sd) in enumerate(ops):
             if ev is not None:
                 ev[i][0].record(stream)
-            am = None
-            if fused_dy_amax and i == 2:
-                Q.amax_rowcol(dY, had, ops[2][5], ops[4][5], out=dy_amax, workspace=ws, stream=stream)
-            if fused_dy_amax and i in (2, 4):
-                am = dy_amax[0:1] if i == 2 else dy_amax[1:2]
-            Q.quantize(t, fmt, rnd, had, axis, sd, amax_in=am, out=qs[i], workspace=ws, stream=stream)
+            if i in (2, 4):
+                quantize_dy(Q, dY, c, ops, qs, i, fused_dy_amax, dual_dy, dy_amax, ws, stream)
+            else:
+                Q.quantize(t, fmt, rnd, had, axis, sd, out=qs[i], workspace=ws, stream=stream)
             if ev is not None:
                 ev[i][1].record(stream)
             if i == 1:
@@ -330,6 +328,38 @@ def run_ours(args, rank, world, local_rank):
     return out
 
 
+def dy_plan(Q, c, M):
+    """How the layer quantizes dY, as qfp4_linear_bwd does: (fused row-and-column
+    amax, dual row-and-column quantization from one read). The dual pass is
+    taken for round-to-nearest only (memory-bound); stochastic and Quartet II
+    rounding keep two passes."""
+    had_n = {Q.HAD_NONE: 0, Q.HAD_DET16: 16, Q.HAD_DET32: 32, Q.HAD_RAND16: 16, Q.HAD_RAND32: 32}
+    fused = (c[1].fmt == Q.NVFP4 and c[2].fmt == Q.NVFP4 and c[1].had == c[2].had
+             and c[1].had in (Q.HAD_NONE, Q.HAD_DET16, Q.HAD_RAND16))
+    dual = (c[1].fmt == c[2].fmt and c[1].rnd_a == Q.RTN and c[2].rnd_a == Q.RTN and M % 64 == 0
+            and had_n[c[1].had] in (0, had_n[c[2].had]))
+    return fused, dual
+
+
+def quantize_dy(Q, dY, c, ops, qs, i, fused, dual, dy_amax, ws, stream):
+    """Operand i (2: dY along N, 4: dY along the tokens) of the step."""
+    t, fmt, rnd, had, axis, sd = ops[i]
+    nv = c[1].fmt == Q.NVFP4
+    if i == 2:
+        if fused:
+            Q.amax_rowcol(dY, had, ops[2][5], ops[4][5], out=dy_amax, workspace=ws, stream=stream)
+        elif dual and nv:
+            Q.amax(dY, c[1].had, Q.ROW, ops[2][5], out=dy_amax[0:1], workspace=ws, stream=stream)
+            Q.amax(dY, c[2].had, Q.COL, ops[4][5], out=dy_amax[1:2], workspace=ws, stream=stream)
+    am = dy_amax[0:1] if i == 2 else dy_amax[1:2]
+    if dual:
+        if i == 2:
+            Q.quantize_dual(dY, fmt, rnd, c[1].had, c[2].had, ops[2][5], ops[4][5], dy_amax[0:1] if nv else None,
+                            dy_amax[1:2] if nv else None, out_row=qs[2], out_col=qs[4], stream=stream)
+        return
+    Q.quantize(t, fmt, rnd, had, axis, sd, amax_in=am if fused else None, out=qs[i], workspace=ws, stream=stream)
+
+
 def layer_step(Q, X, W, dY, rec, seed, steps, stream, dev):
     """One linear layer's fwd+bwd through the six quantize and three GEMM calls
     (the same sequence as the headline step), timed with CUDA events on the
@@ -355,18 +385,15 @@ def layer_step(Q, X, W, dY, rec, seed, steps, stream, dev):
     dW = torch.empty((N, K), dtype=dw_dtype, device=dev)
     outs = [(0, 1, Y, torch.bfloat16), (2, 3, dX, torch.bfloat16), (4, 5, dW, dw_dtype)]
 
-    fused_dy_amax = (c[1].fmt == Q.NVFP4 and c[2].fmt == Q.NVFP4 and c[1].had == c[2].had
-                     and c[1].had in (Q.HAD_NONE, Q.HAD_DET16, Q.HAD_RAND16))
+    fused_dy_amax, dual_dy = dy_plan(Q, c, M)
     dy_amax = torch.empty((2,), dtype=torch.float32, device=dev)
 
     def step(ev):
         for i, (t, fmt, rnd, had, axis, sd) in enumerate(ops):
-            am = None
-            if fused_dy_amax and i == 2:
-                Q.amax_rowcol(dY, had, ops[2][5], ops[4][5], out=dy_amax, workspace=ws, stream=stream)
-            if fused_dy_amax and i in (2, 4):
-                am = dy_amax[0:1] if i == 2 else dy_amax[1:2]
-            Q.quantize(t, fmt, rnd, had, axis, sd, amax_in=am, out=qs[i], workspace=ws, stream=stream)
+            if i in (2, 4):
+                quantize_dy(Q, dY, c, ops, qs, i, fused_dy_amax, dual_dy, dy_amax, ws, stream)
+            else:
+                Q.quantize(t, fmt, rnd, had, axis, sd, out=qs[i], workspace=ws, stream=stream)
             if i % 2 == 1:
                 a, b, D, odt = outs[i // 2]
                 if ev is not None:

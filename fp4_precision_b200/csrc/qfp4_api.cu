@@ -834,10 +834,12 @@ int qfp4_linear_bwd(const void* dY, const void* X, const void* W, void* dX, void
     qfp4_seed s2 = op_seed(seed, 2, 4), s3 = op_seed(seed, 2, 5);
     // dY is quantized along both axes (Dgrad: along N; Wgrad: along M). When
     // both are NVFP4 with the same Hadamard (size <= 16; the sign vectors
-    // differ per GEMM), one read of dY gives both tensor amaxes; when both
-    // quantizations share format and rounding, one more read gives both
-    // quantized operands.
-    const bool dual = d.fmt == w.fmt && d.rnd_a == w.rnd_a && dual_ok(M, d.had, w.had);
+    // differ per GEMM), one read of dY gives both tensor amaxes. When both
+    // quantizations round to nearest with the same format, one more read gives
+    // both quantized operands (memory-bound, so one read instead of two is a
+    // quarter faster); stochastic and Quartet II rounding are bound by
+    // instruction issue, and there the two separate passes are faster.
+    const bool dual = d.fmt == w.fmt && d.rnd_a == QFP4_RTN && w.rnd_a == QFP4_RTN && dual_ok(M, d.had, w.had);
     const float* am_row = nullptr;
     const float* am_col = nullptr;
     if (d.fmt == QFP4_NVFP4 && w.fmt == QFP4_NVFP4 && d.had == w.had && had_n(d.had) <= 16) {

@@ -1,6 +1,7 @@
 """The benchmark's layers at their full sizes, in the launch configuration
 bench.py times: the six quantizations of one linear fwd+bwd (with the fused
-row-and-column amax of dY where the recipe allows it) and the three GEMMs.
+row-and-column amax of dY, and its row and column quantizations from one read,
+where the recipe allows them) and the three GEMMs.
 
 Checked on samples the oracle computes one by one: 64 rows of every quantized
 operand (first and last rows, the rows around a 128-row tile edge, random
@@ -59,18 +60,32 @@ def test_layer_full_size_sampled(workload, preset, M):
            (dY, c[1], c[1].rnd_a, Q.ROW, 1, 2), (W, c[1], c[1].rnd_b, Q.COL, 1, 3),
            (dY, c[2], c[2].rnd_a, Q.COL, 2, 4), (X, c[2], c[2].rnd_b, Q.COL, 2, 5)]
     ws = torch.empty((Q.quantize_workspace_bytes(),), dtype=torch.uint8, device=dev)
+    # dY as the layer quantizes it: both tensor amaxes from one pass (NVFP4, same
+    # Hadamard), both quantizations from one read (round-to-nearest)
+    had_n = {Q.HAD_NONE: 0, Q.HAD_DET16: 16, Q.HAD_DET32: 32, Q.HAD_RAND16: 16, Q.HAD_RAND32: 32}
     fused = (c[1].fmt == Q.NVFP4 and c[2].fmt == Q.NVFP4 and c[1].had == c[2].had
              and c[1].had in (Q.HAD_NONE, Q.HAD_DET16, Q.HAD_RAND16))
+    dual = (c[1].fmt == c[2].fmt and c[1].rnd_a == Q.RTN and c[2].rnd_a == Q.RTN
+            and had_n[c[1].had] in (0, had_n[c[2].had]))
+    s_row, s_col = Q.make_seed(ROT, SR, 1, 2), Q.make_seed(ROT, SR, 2, 4)
     dy_amax = torch.empty((2,), dtype=torch.float32, device=dev)
     if fused:
-        Q.amax_rowcol(dY, c[1].had, Q.make_seed(ROT, SR, 1, 2), Q.make_seed(ROT, SR, 2, 4), out=dy_amax,
-                      workspace=ws)
-    qs = []
+        Q.amax_rowcol(dY, c[1].had, s_row, s_col, out=dy_amax, workspace=ws)
+    elif dual and c[1].fmt == Q.NVFP4:
+        Q.amax(dY, c[1].had, Q.ROW, s_row, out=dy_amax[0:1], workspace=ws)
+        Q.amax(dY, c[2].had, Q.COL, s_col, out=dy_amax[1:2], workspace=ws)
+    qs = [None] * 6
+    if dual:
+        nv = c[1].fmt == Q.NVFP4
+        qs[2], qs[4] = Q.quantize_dual(dY, c[1].fmt, Q.RTN, c[1].had, c[2].had, s_row, s_col,
+                                       dy_amax[0:1] if nv else None, dy_amax[1:2] if nv else None)
     for i, (t, cfg, rnd, axis, g, o) in enumerate(ops):
+        if qs[i] is not None:
+            continue
         am = None
         if fused and i in (2, 4):
             am = dy_amax[0:1] if i == 2 else dy_amax[1:2]
-        qs.append(Q.quantize(t, cfg.fmt, rnd, cfg.had, axis, Q.make_seed(ROT, SR, g, o), amax_in=am, workspace=ws))
+        qs[i] = Q.quantize(t, cfg.fmt, rnd, cfg.had, axis, Q.make_seed(ROT, SR, g, o), amax_in=am, workspace=ws)
     Y = Q.gemm(qs[0], qs[1], torch.bfloat16)
     dX = Q.gemm(qs[2], qs[3], torch.bfloat16)
     dW = Q.gemm(qs[4], qs[5], torch.float32)
