@@ -969,10 +969,17 @@ __global__ void __launch_bounds__(kThreads, 2)
                              : "=r"(a0), "=r"(a1), "=r"(a2), "=r"(a3)
                              : "r"(addr));
                 if (NH > 0 && p.signs != 0u) {
-                    a0 ^= kDual ? Grp::sign_mask(p.signs, 4 * u + 0) : smask[kDual ? 0 : 4 * u + 0];
-                    a1 ^= kDual ? Grp::sign_mask(p.signs, 4 * u + 1) : smask[kDual ? 0 : 4 * u + 1];
-                    a2 ^= kDual ? Grp::sign_mask(p.signs, 4 * u + 2) : smask[kDual ? 0 : 4 * u + 2];
-                    a3 ^= kDual ? Grp::sign_mask(p.signs, 4 * u + 3) : smask[kDual ? 0 : 4 * u + 3];
+                    if constexpr (kDual) {
+                        a0 ^= Grp::sign_mask(p.signs, 4 * u + 0);
+                        a1 ^= Grp::sign_mask(p.signs, 4 * u + 1);
+                        a2 ^= Grp::sign_mask(p.signs, 4 * u + 2);
+                        a3 ^= Grp::sign_mask(p.signs, 4 * u + 3);
+                    } else {
+                        a0 ^= smask[4 * u + 0];
+                        a1 ^= smask[4 * u + 1];
+                        a2 ^= smask[4 * u + 2];
+                        a3 ^= smask[4 * u + 3];
+                    }
                 }
                 v[8 * u + 0] = bf16lo(a0); v[8 * u + 1] = bf16hi(a0);
                 v[8 * u + 2] = bf16lo(a1); v[8 * u + 3] = bf16hi(a1);
