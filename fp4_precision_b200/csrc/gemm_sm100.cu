@@ -357,6 +357,45 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tadd
     }
 }
 
+// The next layer's operand from the epilogue: row r's 128 output columns from
+// n0, as packed bf16 words w (the values just stored as D), quantized to MXFP4
+// along N exactly as the row quantizer does it (round to nearest, a Hadamard of
+// size NHQ with sign bits p.q_signs applied to the bf16 words, the floor
+// exponent): four 32-element blocks, 16 bytes of codes each, one scale word.
+template <int NHQ>
+__device__ __forceinline__ void quantize_out_row128(const GemmParams& p, const uint32_t* w, int r, int n0) {
+    using Grp = Group<kMxfp4, kRtn, NHQ>;
+    static_assert(Grp::G == 32, "32-element MXFP4 blocks");
+    const Stream st{0, 0, 0, 0};
+    ScaleRng srng;
+    uint32_t scodes[4];
+#pragma unroll
+    for (int blk = 0; blk < 4; ++blk) {
+        float v[32];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            uint32_t x = w[16 * blk + i];
+            if (NHQ > 0 && p.q_signs != 0u) x ^= Grp::sign_mask(p.q_signs, i);
+            v[2 * i] = bf16lo(x);
+            v[2 * i + 1] = bf16hi(x);
+        }
+        Grp::rotate(v);
+        uint32_t codes[4];
+        Grp::quantize(v, 1.0f, nullptr, st, 0, 0, srng, codes, scodes + blk);
+        if (r < p.M && n0 + 32 * blk < p.N)
+            *reinterpret_cast<uint4*>(p.q_codes + (int64_t)r * (p.N / 2) + (n0 + 32 * blk) / 2) =
+                make_uint4(codes[0], codes[1], codes[2], codes[3]);
+    }
+    // rows up to the 128-row padding of the atoms; past M the accumulator is
+    // zero (zero-filled A rows), so those scales are the zero padding
+    if (r < (p.M + 127) / 128 * 128) {
+        const int64_t kb0 = n0 / 32;
+        *reinterpret_cast<uint32_t*>(p.q_scales + ((int64_t)(r / 128) * (p.q_kb4 / 4) + kb0 / 4) * 512 +
+                                     (r % 32) * 16 + ((r / 32) % 4) * 4) =
+            scodes[0] | (scodes[1] << 8) | (scodes[2] << 16) | (scodes[3] << 24);
+    }
+}
+
 // Epilogue of one tile for one warp with TMA stores (bf16 output): its 32
 // rows x 128 columns of the accumulator go to registers (packed bf16), the
 // accumulator is released, then each 64-column half is written row by row into
@@ -364,7 +403,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tadd
 // of row r at chunk j ^ (r % 8): conflict-free) and stored by one TMA bulk
 // store, which writes whole lines and clips rows >= M and columns >= N. The
 // box is rewritten only after the previous store has read it.
-template <typename Release>
+template <int NHQ, typename Release>
 __device__ __forceinline__ void epilogue_tile_tma(const GemmParams& p, const CUtensorMap* tmD, uint32_t taddr, int row0,
                                                   int n0, float scale, uint32_t obox, int lane, Release release) {
     uint32_t w[64];
@@ -395,6 +434,9 @@ __device__ __forceinline__ void epilogue_tile_tma(const GemmParams& p, const CUt
             tma_store_2d(tmD, obox, n0 + 64 * h, row0);
             bulk_commit_group();
         }
+    }
+    if constexpr (NHQ >= 0) {
+        if (n0 < p.N) quantize_out_row128<NHQ>(p, w, row0 + lane, n0);
     }
 }
 
@@ -650,7 +692,7 @@ constexpr int P_OUT_BOX = 4096;      // one epilogue warp's TMA-store box (32 ro
 constexpr int P_SMEM = P_STAGES * P_STAGE + kEpiWarps * P_OUT_BOX + 1024 + 512;
 constexpr int P_GROUP_M = 4;  // 256-row tiles per group of the tile order
 
-template <int FMT>
+template <int FMT, int NHQ = -1>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     gemm_bs_fp4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                             const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
@@ -812,7 +854,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             if (p.out_f32)
                 epilogue_tile_tma_f32(p, &tmD, taddr, row0, nb * BN + chalf * 128, scale, obox, lane, release);
             else
-                epilogue_tile_tma(p, &tmD, taddr, row0, nb * BN + chalf * 128, scale, obox, lane, release);
+                epilogue_tile_tma<NHQ>(p, &tmD, taddr, row0, nb * BN + chalf * 128, scale, obox, lane, release);
         }
         if (lane == 0) bulk_wait_group0();  // this warp's stores are complete
     }
@@ -846,25 +888,42 @@ cudaError_t launch_gemm(const GemmParams& p, int fmt, const CUtensorMap* tmapA, 
     return cudaGetLastError();
 }
 
+template <int FMT, int NHQ>
+cudaError_t run_pair(const GemmParams& p, const CUtensorMap* tmapA, const CUtensorMap* tmapB,
+                     const CUtensorMap* tmapSFA, const CUtensorMap* tmapSFB, const CUtensorMap* tmapD, cudaStream_t s,
+                     int clusters) {
+    cudaError_t e =
+        cudaFuncSetAttribute(gemm_bs_fp4_pair_kernel<FMT, NHQ>, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM);
+    if (e != cudaSuccess) return e;
+    gemm_bs_fp4_pair_kernel<FMT, NHQ><<<2 * clusters, kGemmThreads, P_SMEM, s>>>(*tmapA, *tmapB, *tmapSFA, *tmapSFB,
+                                                                                *tmapD, p);
+    return cudaSuccess;
+}
+
 cudaError_t launch_gemm_pair(const GemmParams& p, int fmt, const CUtensorMap* tmapA, const CUtensorMap* tmapB,
                              const CUtensorMap* tmapSFA, const CUtensorMap* tmapSFB, const CUtensorMap* tmapD,
-                             cudaStream_t s, int sms) {
+                             cudaStream_t s, int sms, int nhq) {
     const int tiles = ((p.M + 2 * BM - 1) / (2 * BM)) * ((p.N + BN - 1) / BN);
     int clusters = sms / 2;
     if (clusters > tiles) clusters = tiles;
     if (clusters < 1) clusters = 1;
     cudaError_t e;
     if (fmt == kNvfp4) {
-        e = cudaFuncSetAttribute(gemm_bs_fp4_pair_kernel<kNvfp4>, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM);
-        if (e != cudaSuccess) return e;
-        gemm_bs_fp4_pair_kernel<kNvfp4><<<2 * clusters, kGemmThreads, P_SMEM, s>>>(*tmapA, *tmapB, *tmapSFA,
-                                                                                   *tmapSFB, *tmapD, p);
+        switch (nhq) {
+            case -1: e = run_pair<kNvfp4, -1>(p, tmapA, tmapB, tmapSFA, tmapSFB, tmapD, s, clusters); break;
+            case 0: e = run_pair<kNvfp4, 0>(p, tmapA, tmapB, tmapSFA, tmapSFB, tmapD, s, clusters); break;
+            case 16: e = run_pair<kNvfp4, 16>(p, tmapA, tmapB, tmapSFA, tmapSFB, tmapD, s, clusters); break;
+            default: e = run_pair<kNvfp4, 32>(p, tmapA, tmapB, tmapSFA, tmapSFB, tmapD, s, clusters); break;
+        }
     } else {
-        e = cudaFuncSetAttribute(gemm_bs_fp4_pair_kernel<kMxfp4>, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM);
-        if (e != cudaSuccess) return e;
-        gemm_bs_fp4_pair_kernel<kMxfp4><<<2 * clusters, kGemmThreads, P_SMEM, s>>>(*tmapA, *tmapB, *tmapSFA,
-                                                                                   *tmapSFB, *tmapD, p);
+        switch (nhq) {
+            case -1: e = run_pair<kMxfp4, -1>(p, tmapA, tmapB, tmapSFA, tmapSFB, tmapD, s, clusters); break;
+            case 0: e = run_pair<kMxfp4, 0>(p, tmapA, tmapB, tmapSFA, tmapSFB, tmapD, s, clusters); break;
+            case 16: e = run_pair<kMxfp4, 16>(p, tmapA, tmapB, tmapSFA, tmapSFB, tmapD, s, clusters); break;
+            default: e = run_pair<kMxfp4, 32>(p, tmapA, tmapB, tmapSFA, tmapSFB, tmapD, s, clusters); break;
+        }
     }
+    if (e != cudaSuccess) return e;
     count_launch();
     return cudaGetLastError();
 }

@@ -469,8 +469,15 @@ int quantize_dual_impl(const void* x, int64_t R, int64_t C, int64_t ld, int32_t 
     return e == cudaSuccess ? QFP4_OK : cuda_fail(e);
 }
 
+// The optional MXFP4 copy of a bf16 GEMM output (qfp4_gemm_quantize).
+struct QuantOut {
+    int32_t had;
+    const qfp4_seed* seed;
+    qfp4_tensor* out;
+};
+
 int gemm_impl(const qfp4_tensor* A, const qfp4_tensor* B, void* D, int64_t ldd, int32_t out_dtype, bool accumulate,
-              cudaStream_t s) {
+              cudaStream_t s, const QuantOut* qo = nullptr) {
     int rc = bind_context(s);
     if (rc) return rc;
     int sms = 0;
@@ -479,6 +486,13 @@ int gemm_impl(const qfp4_tensor* A, const qfp4_tensor* B, void* D, int64_t ldd, 
     if (A == nullptr || B == nullptr) return QFP4_ERR_INVALID_ARG;
     if (out_dtype != QFP4_OUT_BF16 && out_dtype != QFP4_OUT_F32) return QFP4_ERR_INVALID_ARG;
     if (accumulate && out_dtype != QFP4_OUT_F32) return QFP4_ERR_INVALID_ARG;
+    if (qo != nullptr) {
+        if (out_dtype != QFP4_OUT_BF16 || qo->out == nullptr || qo->seed == nullptr) return QFP4_ERR_INVALID_ARG;
+        if (qo->had < QFP4_HAD_NONE || qo->had > QFP4_HAD_RAND32) return QFP4_ERR_INVALID_ARG;
+        if (B->rows % 32 != 0 || A->rows <= 0 || B->rows <= 0 || A->k <= 0) return QFP4_ERR_INVALID_ARG;
+        if (!qo->out->codes || !qo->out->scales || !qo->out->tensor_scale) return QFP4_ERR_INVALID_ARG;
+        if (!aligned16(qo->out->codes) || !aligned16(qo->out->scales)) return QFP4_ERR_MISALIGNED;
+    }
     if (A->fmt != B->fmt || (A->fmt != QFP4_NVFP4 && A->fmt != QFP4_MXFP4)) return QFP4_ERR_INVALID_ARG;
     if (A->k != B->k || A->k < 0 || A->rows < 0 || B->rows < 0) return QFP4_ERR_INVALID_ARG;
     if (A->had != B->had) return QFP4_ERR_INVALID_ARG;
@@ -513,6 +527,14 @@ int gemm_impl(const qfp4_tensor* A, const qfp4_tensor* B, void* D, int64_t ldd, 
     p.ldd = ldd;
     p.out_f32 = out_dtype == QFP4_OUT_F32;
     p.accumulate = accumulate ? 1 : 0;
+    int nhq = -1;
+    if (qo != nullptr && pair) {
+        nhq = had_n(qo->had);
+        p.q_codes = qo->out->codes;
+        p.q_scales = qo->out->scales;
+        p.q_kb4 = (N / 32 + 3) / 4 * 4;
+        p.q_signs = had_random(qo->had) ? host_sign_bits(qo->seed->rot, qo->seed->rot_stream) : 0u;
+    }
     p.M = (int)M; p.N = (int)N; p.K = (int)K;
     const int NB = block_of(A->fmt);
     p.atoms_k = (int)((K / NB + 3) / 4);
@@ -523,11 +545,19 @@ int gemm_impl(const qfp4_tensor* A, const qfp4_tensor* B, void* D, int64_t ldd, 
         if ((rc = make_scale_tmap(&tSFA, A->scales, M, p.atoms_k, atoms_per_kt, 1))) return rc;
         if ((rc = make_scale_tmap(&tSFB, B->scales, N, p.atoms_k, atoms_per_kt, 2))) return rc;
         if ((rc = make_out_tmap(&tD, D, M, N, ldd, p.out_f32))) return rc;
-        e = launch_gemm_pair(p, A->fmt, &tA, &tB, &tSFA, &tSFB, &tD, s, sms);
+        e = launch_gemm_pair(p, A->fmt, &tA, &tB, &tSFA, &tSFB, &tD, s, sms, nhq);
     } else {
         e = launch_gemm(p, A->fmt, &tA, &tB, s, sms);
     }
-    return e == cudaSuccess ? QFP4_OK : cuda_fail(e);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (qo != nullptr) {
+        if (!pair)  // the single-CTA kernel has no quantizing epilogue: quantize D afterwards
+            return quantize_impl(D, M, N, ldd, QFP4_MXFP4, QFP4_RTN, qo->had, QFP4_AXIS_ROW, qo->seed, nullptr,
+                                 qo->out, nullptr, 0, s);
+        fill_out(qo->out, M, N, QFP4_MXFP4, qo->had, qo->seed);
+        if ((rc = write_one(qo->out->tensor_scale, s))) return rc;
+    }
+    return QFP4_OK;
 }
 
 // ---- linear layer -------------------------------------------------------------
@@ -748,6 +778,12 @@ int qfp4_quantize_dual(const void* x, int64_t R, int64_t C, int64_t ld, int32_t 
 
 int qfp4_gemm(const qfp4_tensor* A, const qfp4_tensor* B, void* D, int64_t ldd, int32_t out_dtype, void* stream) {
     return gemm_impl(A, B, D, ldd, out_dtype, false, static_cast<cudaStream_t>(stream));
+}
+
+int qfp4_gemm_quantize(const qfp4_tensor* A, const qfp4_tensor* B, void* D, int64_t ldd, int32_t had,
+                       const qfp4_seed* seed, qfp4_tensor* out, void* stream) {
+    const QuantOut qo{had, seed, out};
+    return gemm_impl(A, B, D, ldd, QFP4_OUT_BF16, false, static_cast<cudaStream_t>(stream), &qo);
 }
 
 int qfp4_gemm_accumulate(const qfp4_tensor* A, const qfp4_tensor* B, float* D, int64_t ldd, void* stream) {

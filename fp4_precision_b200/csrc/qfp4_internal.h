@@ -84,6 +84,13 @@ struct GemmParams {
     int64_t ldd;
     int out_f32;
     int accumulate;  // fp32 output only: D += result (one fp32 add per element)
+    // bf16 output only, pair kernel: the output also quantized to MXFP4 along
+    // N (round to nearest, Hadamard of the kernel's NHQ with these sign bits),
+    // codes [M][N/2] and scales in the atom layout (q_kb4 scale columns)
+    uint8_t* q_codes;
+    uint8_t* q_scales;
+    int64_t q_kb4;
+    uint32_t q_signs;
     int M, N, K;
     int atoms_k;  // scale atoms per 128-row block along k: ceil(K / block / 4)
 };
@@ -94,9 +101,11 @@ cudaError_t launch_gemm(const GemmParams& p, int fmt, const CUtensorMap* tmapA, 
 // 2-SM (CTA pair) variant; tmapSFA / tmapSFB are 3-D views of the scale
 // buffers, tmapD a 2-D view of D for TMA stores (see make_scale_tmap and
 // make_out_tmap in qfp4_api.cu).
+// nhq: -1 (no quantized output) or the Hadamard size (0, 16, 32) of the
+// MXFP4 output quantization (p.q_codes etc.).
 cudaError_t launch_gemm_pair(const GemmParams& p, int fmt, const CUtensorMap* tmapA, const CUtensorMap* tmapB,
                              const CUtensorMap* tmapSFA, const CUtensorMap* tmapSFB, const CUtensorMap* tmapD,
-                             cudaStream_t s, int sms);
+                             cudaStream_t s, int sms, int nhq = -1);
 constexpr int kGemmBM = 128, kGemmBN = 256, kGemmBK = 256;
 
 void count_launch();

@@ -77,6 +77,8 @@ _SIGNATURES = {
                                           ctypes.POINTER(Seed), _VOID, _VOID, ctypes.POINTER(TensorDesc),
                                           ctypes.POINTER(TensorDesc), _VOID]),
     "qfp4_gemm": (ctypes.c_int, [ctypes.POINTER(TensorDesc), ctypes.POINTER(TensorDesc), _VOID, _I64, _I32, _VOID]),
+    "qfp4_gemm_quantize": (ctypes.c_int, [ctypes.POINTER(TensorDesc), ctypes.POINTER(TensorDesc), _VOID, _I64, _I32,
+                                          ctypes.POINTER(Seed), ctypes.POINTER(TensorDesc), _VOID]),
     "qfp4_gemm_accumulate": (ctypes.c_int, [ctypes.POINTER(TensorDesc), ctypes.POINTER(TensorDesc), _VOID, _I64,
                                             _VOID]),
     "qfp4_recipe_preset": (ctypes.c_int, [_I32, ctypes.POINTER(Recipe)]),
@@ -250,6 +252,18 @@ def gemm(A: QTensor, B: QTensor, out_dtype=torch.bfloat16, out: torch.Tensor | N
     _check(lib().qfp4_gemm(ctypes.byref(A.desc), ctypes.byref(B.desc), _ptr(out), out.stride(0), dt,
                            _stream(stream)), "qfp4_gemm")
     return out
+
+
+def gemm_quantize(A: QTensor, B: QTensor, had: int, seed: Seed, out: torch.Tensor | None = None,
+                  qout: QTensor | None = None, stream=None):
+    """bf16 D = gA gB A . B^T and its MXFP4 quantization along N; see qfp4_gemm_quantize."""
+    if out is None:
+        out = torch.empty((A.rows, B.rows), dtype=torch.bfloat16, device=A.codes.device)
+    qout = empty_qtensor(MXFP4, A.rows, B.rows, A.codes.device) if qout is None else qout
+    _check(lib().qfp4_gemm_quantize(ctypes.byref(A.desc), ctypes.byref(B.desc), _ptr(out), out.stride(0), had,
+                                    ctypes.byref(seed), ctypes.byref(qout.desc), _stream(stream)),
+           "qfp4_gemm_quantize")
+    return out, qout
 
 
 def gemm_accumulate(A: QTensor, B: QTensor, out: torch.Tensor, stream=None) -> torch.Tensor:

@@ -240,6 +240,18 @@ int qfp4_gemm(const qfp4_tensor* A, const qfp4_tensor* B, void* D, int64_t ldd, 
  * by a read-modify-write of the element it owns. D must not be written by
  * anything else until the call completes. Requirements as qfp4_gemm. */
 int qfp4_gemm_accumulate(const qfp4_tensor* A, const qfp4_tensor* B, float* D, int64_t ldd, void* stream);
+/* qfp4_gemm_quantize: D = A . B^T as qfp4_gemm with a bf16 output, and *out =
+ * that bf16 D quantized to MXFP4 along its rows (k = B.rows), round to
+ * nearest, with Hadamard `had` and seed->rot / rot_stream for a random one —
+ * exactly what qfp4_quantize(D, MXFP4, RTN, had, ROW, seed) gives — so a
+ * layer's output is also the next layer's forward operand. With the CTA-pair
+ * kernel (A.rows > 128) the quantization happens in the GEMM's epilogue from
+ * the values it stores; otherwise D is quantized by a second launch.
+ * Requirements: those of qfp4_gemm; B.rows a multiple of 32; out's codes
+ * (A.rows x B.rows/2 bytes) and scales (qfp4_scales_bytes(MXFP4, A.rows,
+ * B.rows)) 16-byte aligned, and its tensor_scale (set to 1). No workspace. */
+int qfp4_gemm_quantize(const qfp4_tensor* A, const qfp4_tensor* B, void* D, int64_t ldd, int32_t had,
+                       const qfp4_seed* seed, qfp4_tensor* out, void* stream);
 
 /* ---- linear layer -------------------------------------------------------------
  * X [M x K], W [N x K], dY [M x N] bf16 row-major (contiguous); Y [M x N],

@@ -98,6 +98,64 @@ def test_gemm_accumulate_matches_oracle(fmt, shape, kernel_variant):
     assert np.all(err2 <= 2 * tol + 2.0 ** -23 * np.abs(d0 + 2 * ref))
 
 
+def grid_operand(rows, k, seed):
+    """bf16 [rows, k] of E2M1 grid values with a +-6 in every 32-element block
+    along k: its MXFP4 RTN quantization is exact with every scale 2^0."""
+    g = np.random.default_rng(seed)
+    vals = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6], dtype=np.float32)
+    x = vals[g.integers(0, 8, size=(rows, k))] * np.where(g.random((rows, k)) < 0.5, -1.0, 1.0)
+    x[:, ::32] = 6.0 * np.where(g.random((rows, k // 32)) < 0.5, -1.0, 1.0)
+    return torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("had", [O.HAD_NONE, O.HAD_DET16, O.HAD_DET32, O.HAD_RAND16, O.HAD_RAND32],
+                         ids=["none", "det16", "det32", "rand16", "rand32"])
+@pytest.mark.parametrize("shape", [(300, 288, 256), (128, 256, 128), (512, 1024, 512)],
+                         ids=lambda s: "x".join(map(str, s)))
+def test_gemm_quantize_matches_oracle(shape, had, kernel_variant):
+    """qfp4_gemm_quantize: the bf16 output and its MXFP4 quantization along N.
+    The operands are exactly representable and every partial sum is exact in
+    fp32, so D is known exactly: the bf16 D must equal bf16(D) and the
+    quantized output the oracle's quantization of it, bit for bit (rows and
+    scale columns past the tensor included as zero padding)."""
+    M, N, K = shape
+    X, W = grid_operand(M, K, 1), grid_operand(N, K, 2)
+    A_o = O.quantize(X, O.MXFP4, O.RTN, O.HAD_NONE, O.ROW)
+    B_o = O.quantize(W, O.MXFP4, O.RTN, O.HAD_NONE, O.ROW)
+    assert np.all(A_o.scales == 127) and np.all(B_o.scales == 127)
+    d_exact = X.double().numpy() @ W.double().numpy().T
+    d_bf16 = torch.from_numpy(d_exact.astype(np.float32)).to(torch.bfloat16)
+    ref = O.quantize(d_bf16, O.MXFP4, O.RTN, had, O.ROW, 0x77, 5)
+    D, q = Q.gemm_quantize(upload(A_o), upload(B_o), had, Q.make_seed(rot=0x77, rot_stream=5))
+    torch.cuda.synchronize()
+    Q.status()
+    assert torch.equal(D.cpu(), d_bf16)
+    assert q.fmt == Q.MXFP4 and q.rows == M and q.k == N
+    codes = helpers.to_numpy_u8(q.codes)
+    assert np.array_equal(codes, ref.codes), f"{np.sum(codes != ref.codes)} code bytes differ"
+    flat = helpers.to_numpy_u8(q.scales)
+    assert np.array_equal(helpers.unswizzle_scales(flat, M, N, 32), ref.scales)
+    assert helpers.padding_is_zero(flat, M, N, 32)
+    assert float(q.tensor_scale.cpu()[0]) == 1.0
+
+
+@pytest.mark.parametrize("had", [O.HAD_NONE, O.HAD_RAND32], ids=["none", "rand32"])
+def test_gemm_quantize_equals_quantizing_the_output(had):
+    """With NVFP4 operands and a general K the fused quantization equals the
+    row quantizer run on the GEMM's own bf16 output (same stream of values)."""
+    M, N, K = 640, 544, 1024
+    X = inputs.normal_with_outliers((M, K), 31, "qa")
+    W = inputs.normal((N, K), 0.02, 31, "qb")
+    A = upload(O.quantize(X, O.NVFP4, O.RTN, O.HAD_NONE, O.ROW))
+    B = upload(O.quantize(W, O.NVFP4, O.RTN, O.HAD_NONE, O.ROW))
+    seed = Q.make_seed(rot=0x55, rot_stream=2)
+    D, q = Q.gemm_quantize(A, B, had, seed)
+    q2 = Q.quantize(D, Q.MXFP4, Q.RTN, had, Q.ROW, seed)
+    torch.cuda.synchronize()
+    Q.status()
+    assert torch.equal(q.codes, q2.codes) and torch.equal(q.scales, q2.scales)
+
+
 def test_linear_dw_accumulate_needs_fp32_dw():
     """A recipe that accumulates into dW must have an fp32 dW: the call is
     rejected on the host, before anything is launched."""
