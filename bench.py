@@ -271,6 +271,33 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize()
         wg[acc] = e0.elapsed_time(e1) / 10
     Q.status()
+    # Fprop whose epilogue also writes the MXFP4 operand of a next layer (Y along N)
+    qy = Q.empty_qtensor(Q.MXFP4, M, N, dev)
+    qseed = Q.make_seed(seed.rot, seed.sr, 3, 6)
+    fq = {}
+    for kind in ("gemm", "fused", "separate", "gemm", "fused", "separate"):
+        def fprop_q():
+            if kind == "gemm":
+                Q.gemm(qs[0], qs[1], torch.bfloat16, out=Y, stream=stream)
+            elif kind == "fused":
+                Q.gemm_quantize(qs[0], qs[1], Q.HAD_NONE, qseed, out=Y, qout=qy, stream=stream)
+            else:
+                Q.gemm(qs[0], qs[1], torch.bfloat16, out=Y, stream=stream)
+                Q.quantize(Y, Q.MXFP4, Q.RTN, Q.HAD_NONE, Q.ROW, qseed, out=qy, stream=stream)
+        for _ in range(2):
+            fprop_q()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(10):
+            fprop_q()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        fq[kind] = min(fq.get(kind, 1e9), e0.elapsed_time(e1) / 10)
+    Q.status()
+    fprop_quant = {"gemm_ms": round(fq["gemm"], 4), "fused_ms": round(fq["fused"], 4),
+                   "gemm_then_quantize_ms": round(fq["separate"], 4),
+                   "what": f"Fprop Y[{M}x{N}] bf16 alone, with its MXFP4 copy along N from the epilogue "
+                           "(qfp4_gemm_quantize), and followed by a separate row quantization of Y; 10 launches each"}
     wgrad_acc = {"store_ms": round(wg[False], 4), "accumulate_ms": round(wg[True], 4),
                  "accumulate_TFLOP/s": round(gemm_flops[2] / (wg[True] * 1e-3) / 1e12, 1),
                  "what": "Wgrad of the step, dW = dY^T X vs dW += dY^T X (TMA reduce-add epilogue), fp32 dW "
@@ -320,6 +347,7 @@ def run_ours(args, rank, world, local_rank):
         "layers": layers,
         "study": study,
         "wgrad_accumulate": wgrad_acc,
+        "fprop_quantized_output": fprop_quant,
         "linear_api_ms_per_step": round(api_ms, 4),
         "e2e": e2e,
         "gpu_launches": launches,
