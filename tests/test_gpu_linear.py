@@ -60,6 +60,29 @@ def test_tiny_linear_mxfp4_round_up():
     within(dW, dw_ref, dw_b, False)
 
 
+@pytest.mark.parametrize("hads", [(Q.HAD_NONE, Q.HAD_RAND16), (Q.HAD_RAND16, Q.HAD_RAND16)],
+                         ids=["none-rand16", "rand16-rand16"])
+def test_tiny_linear_nvfp4_rtn_backward(hads):
+    """NVFP4 round-to-nearest on both backward GEMMs: dY's two quantizations
+    come from one read (qfp4_quantize_dual), its tensor amaxes from two passes
+    (different Hadamards) or one (the same)."""
+    import dataclasses
+    wl = inputs.workload("tiny")
+    X, W, dY = wl["X"], wl["W"], wl["dY"]
+    rec = Q.recipe("QUARTET2_NVFP4")
+    for c, had in ((rec.dgrad, hads[0]), (rec.wgrad, hads[1])):
+        c.rnd_a, c.rnd_b, c.had = Q.RTN, Q.RTN, had
+    seed = Q.make_seed(ROT, SRS)
+    dX, dW = Q.linear_bwd(dY.cuda(), X.cuda(), W.cuda(), rec, seed)
+    Q.status()
+    r0 = O.preset("QUARTET2_NVFP4")
+    r = O.Recipe(r0.fprop, dataclasses.replace(r0.dgrad, rnd_a=O.RTN, rnd_b=O.RTN, had=hads[0]),
+                 dataclasses.replace(r0.wgrad, rnd_a=O.RTN, rnd_b=O.RTN, had=hads[1]))
+    (dx_ref, dx_b), (dw_ref, dw_b) = O.linear_bwd(dY, X, W, r, ROT, SRS)
+    within(dX, dx_ref, dx_b, True)
+    within(dW, dw_ref, dw_b, False)
+
+
 def test_tiny_linear_dw_accumulate():
     """dw_accumulate = 1: dW += dY^T X into the caller's fp32 buffer (a main
     gradient across micro-batches); dX as without it."""
