@@ -182,6 +182,10 @@ size_t qfp4_quantize_workspace_bytes(void);
  *   for NVFP4 without amax_in, workspace >= qfp4_quantize_workspace_bytes(),
  *   16-byte aligned (its contents on entry do not matter). The result depends
  *   only on the inputs and seeds, never on the launch configuration.
+ * Kernels: persistent, TMA-fed; along COL with k a multiple of 64 a thread
+ *   takes 64 consecutive rows of one column (64-row bands), otherwise one
+ *   group of rows; QFP4_COL_BANDS=0 in the environment selects the latter
+ *   (same results; read on every call).
  * out: caller sets codes, scales and tensor_scale; the call sets the rest. */
 int qfp4_amax(const void* x, int64_t R, int64_t C, int64_t ld, int32_t had, int32_t axis, const qfp4_seed* seed,
               float* amax, void* workspace, size_t workspace_bytes, void* stream);
