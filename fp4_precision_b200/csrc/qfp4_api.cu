@@ -399,7 +399,7 @@ int quantize_impl(const void* x, int64_t R, int64_t C, int64_t ld, int32_t fmt, 
 // format and rounding (caller), R a multiple of 64, the row orientation's
 // Hadamard none or of the column one's size.
 bool dual_ok(int64_t R, int32_t had_row, int32_t had_col) {
-    return R % 64 == 0 && (had_n(had_row) == 0 || had_n(had_row) == had_n(had_col)) && col_bands_enabled();
+    return R % 64 == 0 && (had_n(had_row) == 0 || had_n(had_row) == had_n(had_col));
 }
 
 void fill_out(qfp4_tensor* out, int64_t rows, int64_t k, int32_t fmt, int32_t had, const qfp4_seed* seed) {
@@ -875,7 +875,8 @@ int qfp4_linear_bwd(const void* dY, const void* X, const void* W, void* dX, void
     // both quantized operands (memory-bound, so one read instead of two is a
     // quarter faster); stochastic and Quartet II rounding are bound by
     // instruction issue, and there the two separate passes are faster.
-    const bool dual = d.fmt == w.fmt && d.rnd_a == QFP4_RTN && w.rnd_a == QFP4_RTN && dual_ok(M, d.had, w.had);
+    const bool dual = d.fmt == w.fmt && d.rnd_a == QFP4_RTN && w.rnd_a == QFP4_RTN && dual_ok(M, d.had, w.had) &&
+                      col_bands_enabled();
     const float* am_row = nullptr;
     const float* am_col = nullptr;
     if (d.fmt == QFP4_NVFP4 && w.fmt == QFP4_NVFP4 && d.had == w.had && had_n(d.had) <= 16) {
