@@ -342,6 +342,25 @@ def check_quartet2_projection_unbiased():
         assert np.mean(np.abs(proj_rtn - 1.0) / se < 4.0) < 0.5, fmt
 
 
+def check_quartet2_error_half_of_sr():
+    """[Quartet II]: rounding only the renormalised scales stochastically (the
+    element codes stay RTN) leaves about half the total error of per-element
+    stochastic rounding. On N(0,1) data with and without a random 16x16
+    rotation the mean squared error of the NVFP4 reconstruction (rotated
+    domain, 4 rounding seeds) is within 0.4-0.6 of SR's; the part added by the
+    scale rounding (over RTN) is at least 10x smaller than SR's."""
+    ratio = golden("pages.json")["quartet2_error_vs_plain_sr"]
+    x = inputs.normal((256, 1024), 1.0, 9, "mse")
+    for had in (O.HAD_RAND16, O.HAD_NONE):
+        v = O.rotate(x, had, O.ROW, 5, 0).astype(np.float64)
+        mse = {}
+        for rnd in (O.RTN, O.SR, O.QUARTET2):
+            mse[rnd] = np.mean([np.mean((O.dequantize(O.quantize(x, O.NVFP4, rnd, had, O.ROW, 5, 0, 100 + s, 0))
+                                         - v) ** 2) for s in range(4)])
+        assert abs(mse[O.QUARTET2] / mse[O.SR] - ratio) < 0.1, mse
+        assert (mse[O.SR] - mse[O.RTN]) > 10 * (mse[O.QUARTET2] - mse[O.RTN]) > 0, mse
+
+
 def check_quartet2_alpha_range():
     """[Quartet II]: the renormalisation is of order 0.94-1.06. On N(0,1) data
     with a random 16x16 rotation at least 90% of the NVFP4 blocks' alpha fall in
@@ -539,7 +558,8 @@ ALL_CHECKS = [
     check_e2m1_value_set, check_e2m1_rtn_exhaustive_bf16, check_e4m3_matches_torch, check_e8m0_matches_torch,
     check_philox_matches_torch_engine, check_sylvester_matches_scipy, check_fwht_is_matrix_product,
     check_rotation_orthonormal, check_sr_threshold_exact, check_e4m3_sr_threshold_exact,
-    check_sr_unbiased_rtn_biased, check_quartet2_projection_unbiased, check_quartet2_alpha_range,
+    check_sr_unbiased_rtn_biased, check_quartet2_projection_unbiased, check_quartet2_error_half_of_sr,
+    check_quartet2_alpha_range,
     check_nvfp4_scales, check_mxfp4_scales, check_mxfp4_round_up, check_zero_and_degenerate, check_col_is_row_of_transpose,
     check_seed_determinism, check_gemm_brute_force, check_hadamard_cancels_in_gemm,
 ]
