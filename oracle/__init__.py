@@ -103,6 +103,8 @@ def load(path: str) -> ctypes.CDLL:
     L.oracle_e4m3_sr.restype = u8
     L.oracle_e8m0_value.argtypes = [u8]
     L.oracle_e8m0_value.restype = ctypes.c_double
+    L.oracle_e8m0_sr.argtypes = [ctypes.c_float, ctypes.c_float]
+    L.oracle_e8m0_sr.restype = u8
     L.oracle_hadamard_matrix.argtypes = [ctypes.c_int, ctypes.c_void_p]
     L.oracle_fwht.argtypes = [ctypes.c_void_p, ctypes.c_int]
     L.oracle_sign_bits.argtypes = [u64, u32]
@@ -166,6 +168,11 @@ def e4m3_sr(t: float, rho: float) -> int:
 
 def e8m0_value(code: int) -> float:
     return lib().oracle_e8m0_value(code)
+
+
+def e8m0_sr(t: float, rho: float) -> int:
+    """Stochastic rounding of t > 0 onto powers of two: the E8M0 code."""
+    return lib().oracle_e8m0_sr(t, rho)
 
 
 def hadamard_matrix(n: int) -> np.ndarray:

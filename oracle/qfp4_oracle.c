@@ -204,7 +204,7 @@ static int floor_log2f(float a) {
 /* Stochastic rounding of a positive fp32 onto powers of two (E8M0 grid). The
  * Quartet II step applied to an E8M0 scale (an extension: the pages define it
  * for FP8 scales only). Returns the E8M0 code, clamped to [0, 254]. */
-static uint8_t e8m0_sr(float t, float rho) {
+uint8_t oracle_e8m0_sr(float t, float rho) {
     int e = floor_log2f(t);
     float lo = ldexpf(1.0f, e);
     float p = (t - lo) / lo; /* exact: t in [lo, 2 lo) */
@@ -431,7 +431,7 @@ int oracle_quantize_rows(const uint16_t* x, int64_t R, int64_t C, int64_t ld, in
                     alpha = (den == 0.0f) ? 1.0f : num / den;
                     float t = s_val * alpha;
                     float rho = uniform24(random_word(sr_seed, TAG_SCALE, sr_stream, (uint64_t)blk_index));
-                    s_code = (fmt == FMT_NVFP4) ? oracle_e4m3_sr(t, rho) : e8m0_sr(t, rho);
+                    s_code = (fmt == FMT_NVFP4) ? oracle_e4m3_sr(t, rho) : oracle_e8m0_sr(t, rho);
                 }
                 if (alpha_out) alpha_out[blk_out] = alpha;
                 scales[blk_out] = s_code;

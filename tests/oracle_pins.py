@@ -258,6 +258,34 @@ def check_e4m3_sr_threshold_exact():
             assert O.e4m3_sr(t, n * 2.0**-24) == i, t
 
 
+def check_e8m0_sr_threshold_exact():
+    """Stochastic rounding onto powers of two (the Quartet II scale step of
+    MXFP4): for t in [2^e, 2^(e+1)) the round-up probability is p = (t - 2^e) /
+    2^e, exact as a Fraction; the code is e + 127, plus one for exactly the
+    ceil(p 2^24) uniforms below p. Exponents are clamped to [-127, 127], and a
+    power of two never rounds up."""
+    rng = np.random.default_rng(6)
+    ts = [float(np.float32(v)) for v in rng.uniform(0.5, 2.0, 20) * np.exp2(rng.integers(-130, 120, 20))]
+    ts += [1.0, 1.5, 3.0, 1.9999999, 0.75, 2.0**-127 * 1.25, 2.0**127 * 1.5, 2.0**-130 * 1.7]
+    for t in ts:
+        t = float(np.float32(t))
+        a = Fraction(t)
+        e = a.numerator.bit_length() - a.denominator.bit_length()
+        if Fraction(2) ** e > a:
+            e -= 1
+        lo = Fraction(2) ** e
+        p = (a - lo) / lo
+        n = -((-p * 2**24).numerator // (p * 2**24).denominator)  # ceil
+        clamp = lambda k: min(max(k, -127), 127) + 127  # noqa: E731
+        if n > 0:
+            assert O.e8m0_sr(t, (n - 1) * 2.0**-24) == clamp(e + 1), (t, n)
+        if n < 2**24:
+            assert O.e8m0_sr(t, n * 2.0**-24) == clamp(e), (t, n)
+    for e in (-20, 0, 5, 100):
+        assert O.e8m0_sr(2.0**e, 0.0) == e + 127
+        assert O.e8m0_sr(2.0**e, 1.0 - 2.0**-24) == e + 127
+
+
 def _stats_over_seeds(x, fmt, rnd, had, n_seeds, rot_varies):
     """Mean and variance of the de-rotated estimate over seeds, and the mean
     product of the errors of neighbouring elements (j, j+1)."""
@@ -558,6 +586,7 @@ ALL_CHECKS = [
     check_e2m1_value_set, check_e2m1_rtn_exhaustive_bf16, check_e4m3_matches_torch, check_e8m0_matches_torch,
     check_philox_matches_torch_engine, check_sylvester_matches_scipy, check_fwht_is_matrix_product,
     check_rotation_orthonormal, check_sr_threshold_exact, check_e4m3_sr_threshold_exact,
+    check_e8m0_sr_threshold_exact,
     check_sr_unbiased_rtn_biased, check_quartet2_projection_unbiased, check_quartet2_error_half_of_sr,
     check_quartet2_alpha_range,
     check_nvfp4_scales, check_mxfp4_scales, check_mxfp4_round_up, check_zero_and_degenerate, check_col_is_row_of_transpose,

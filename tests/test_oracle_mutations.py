@@ -35,6 +35,9 @@ MUTATIONS = [
      "for (int64_t j = 0; j < k; ++j) seg[j] = bf16_to_f32(x[(j ^ 1) * ld + row]);"),
     ("scale_sr_always_down", "return (uint8_t)((rho < p) ? lo + 1 : lo);", "return (uint8_t)lo;"),
     ("element_sr_index", "const uint64_t i = (uint64_t)(r * k + b * nb + j);", "const uint64_t i = (uint64_t)(r * k + b * nb);"),
+    ("e8m0_sr_compare_flipped", "    if (rho < p) e += 1;\n", "    if (rho > p) e += 1;\n"),
+    ("e8m0_sr_probability", "float p = (t - lo) / lo; /* exact: t in [lo, 2 lo) */",
+     "float p = (t - lo) / (2.0f * lo); /* exact: t in [lo, 2 lo) */"),
 ]
 
 
