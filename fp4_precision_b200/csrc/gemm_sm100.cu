@@ -198,12 +198,6 @@ __device__ __forceinline__ void tmem_st_x32(uint32_t taddr, const uint32_t* r) {
 }
 __device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
-__device__ __forceinline__ uint4 lds128(uint32_t saddr) {
-    uint4 v;
-    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(saddr));
-    return v;
-}
-
 // Scale writer for TMEM lane quarter q (lanes 32q..32q+31): lane i copies
 // line i of the k-tile's scale atoms from shared memory into TMEM lane 32q + i.
 // Line i of an atom holds four words, word w the four scales of row i + 32w;
@@ -396,6 +390,34 @@ __device__ __forceinline__ void quantize_out_row128(const GemmParams& p, const u
     }
 }
 
+// The NVFP4 tensor amax of the output along its rows, as the next layer's
+// quantizer takes it: max |v| over one row's 128 columns (the packed bf16
+// words w, exactly the values stored in D) after the rotation of size AMX
+// (none, 16 or 32; the sign flips as XORs on the bf16 words, then the
+// butterflies) without its 1/sqrt(n_h) factor, which is applied once to the
+// CTA's maximum (rounding c * y is monotone in y). Output columns past N are
+// zero (zero-filled B rows) and groups never straddle N (a multiple of the
+// group), so padding adds nothing.
+template <int AMX>
+__device__ __forceinline__ float row128_rot_amax(const uint32_t* w, uint32_t signs, float m) {
+    using Grp = Group<kNvfp4, kRtn, AMX>;
+    constexpr int G = Grp::G;
+#pragma unroll
+    for (int g = 0; g < 128 / G; ++g) {
+        float v[G];
+#pragma unroll
+        for (int i = 0; i < G / 2; ++i) {
+            uint32_t x = w[g * (G / 2) + i];
+            if (AMX > 0 && signs != 0u) x ^= Grp::sign_mask(signs, i);
+            v[2 * i] = bf16lo(x);
+            v[2 * i + 1] = bf16hi(x);
+        }
+        Grp::template rotate<false>(v);
+        m = abs_max<G>(m, v);
+    }
+    return m;
+}
+
 // Epilogue of one tile for one warp with TMA stores (bf16 output): its 32
 // rows x 128 columns of the accumulator go to registers (packed bf16), the
 // accumulator is released, then each 64-column half is written row by row into
@@ -403,9 +425,10 @@ __device__ __forceinline__ void quantize_out_row128(const GemmParams& p, const u
 // of row r at chunk j ^ (r % 8): conflict-free) and stored by one TMA bulk
 // store, which writes whole lines and clips rows >= M and columns >= N. The
 // box is rewritten only after the previous store has read it.
-template <int NHQ, typename Release>
+template <int NHQ, int AMX, typename Release>
 __device__ __forceinline__ void epilogue_tile_tma(const GemmParams& p, const CUtensorMap* tmD, uint32_t taddr, int row0,
-                                                  int n0, float scale, uint32_t obox, int lane, Release release) {
+                                                  int n0, float scale, uint32_t obox, int lane, float& amax_acc,
+                                                  Release release) {
     uint32_t w[64];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
@@ -438,6 +461,7 @@ __device__ __forceinline__ void epilogue_tile_tma(const GemmParams& p, const CUt
     if constexpr (NHQ >= 0) {
         if (n0 < p.N) quantize_out_row128<NHQ>(p, w, row0 + lane, n0);
     }
+    if constexpr (AMX >= 0) amax_acc = row128_rot_amax<AMX>(w, p.amax_signs, amax_acc);
 }
 
 // fp32 output: the same with boxes of 32 rows x 32 columns (128-byte rows),
@@ -526,7 +550,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint64_t* sf_full = sf_load + STAGES; // scale slot s written
     uint64_t* acc_full = sf_full + STAGES;
     uint64_t* acc_empty = acc_full + 1;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
+    uint64_t* drain = acc_empty + 1;      // every MMA this CTA issued has completed
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int KT = (p.K + BK - 1) / BK;
@@ -544,6 +569,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         mbar_init(acc_full, 1);
         mbar_init(acc_empty, kEpiWarps);
+        mbar_init(drain, 1);
         fence_mbarrier_init();
     }
     if (warp == 0) tmem_alloc(tmem_slot, TMEM_COLS);
@@ -585,6 +611,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     tma_load_2d(sB + s * B_STAGE, &tmB, &full[s], kt * (BK / 2), n0);
                 }
             }
+            drain_loads(full, sf_load, STAGES, it);
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
@@ -615,6 +642,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 }
                 tc_commit(acc_full);
             }
+            // no MMA may still write tensor memory or read shared memory when
+            // the CTA frees them (after a timed-out wait too)
+            tc_commit(drain);
+            (void)mbar_wait(drain, 0);
         }
     } else if (warp < kFirstEpiWarp) {
         // ---------------- scale writers ----------------
@@ -692,7 +723,7 @@ constexpr int P_OUT_BOX = 4096;      // one epilogue warp's TMA-store box (32 ro
 constexpr int P_SMEM = P_STAGES * P_STAGE + kEpiWarps * P_OUT_BOX + 1024 + 512;
 constexpr int P_GROUP_M = 4;  // 256-row tiles per group of the tile order
 
-template <int FMT, int NHQ = -1>
+template <int FMT, int NHQ = -1, int AMX = -1>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     gemm_bs_fp4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                             const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
@@ -714,7 +745,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     uint64_t* sf_full = sf_load + P_STAGES;  // scale slot s written in both CTAs (leader's)
     uint64_t* acc_full = sf_full + P_STAGES;
     uint64_t* acc_empty = acc_full + 1;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
+    uint64_t* drain = acc_empty + 1;  // every MMA the leader issued has completed (both CTAs)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();
@@ -737,6 +769,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         }
         mbar_init(acc_full, 1);
         mbar_init(acc_empty, 2 * kEpiWarps);
+        mbar_init(drain, 1);
         fence_mbarrier_init();
     }
     if (warp == 0) tmem_alloc_pair(tmem_slot, TMEM_COLS);
@@ -770,6 +803,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                     tma_load_2d_pair(sB + s * P_B, &tmB, bar_leader, kt * (BK / 2), nb * BN + (int)rank * 128);
                 }
             }
+            // both CTAs' operand tiles complete on the leader's full barriers,
+            // each CTA's scale atoms on its own sf_load barriers
+            drain_loads(rank == 0 ? full : nullptr, sf_load, P_STAGES, it);
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer (leader CTA only) ----------------
@@ -800,6 +836,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                 }
                 tc_commit_pair(acc_full);  // both CTAs' accumulators are complete
             }
+            // no MMA may still write either CTA's tensor memory or read shared
+            // memory when the pair frees them (after a timed-out wait too); the
+            // peer is held at the final cluster barrier until then
+            tc_commit_pair(drain);
+            (void)mbar_wait(drain, 0);
         }
     } else if (warp < kFirstEpiWarp) {
         // ---------------- scale writers (both CTAs) ----------------
@@ -840,6 +881,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         const float scale = __fmul_rn(__ldg(p.ga), __ldg(p.gb));
         const uint32_t acc_empty_leader = mapa_shared(smem_u32(acc_empty), 0);
         const uint32_t obox = smem_u32(sOut) + (uint32_t)(warp - kFirstEpiWarp) * P_OUT_BOX;
+        float amax_acc = 0.0f;
         int lt = 0;
         for (int t = cid; t < tiles; t += nclusters, ++lt) {
             int mb, nb;
@@ -854,9 +896,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             if (p.out_f32)
                 epilogue_tile_tma_f32(p, &tmD, taddr, row0, nb * BN + chalf * 128, scale, obox, lane, release);
             else
-                epilogue_tile_tma<NHQ>(p, &tmD, taddr, row0, nb * BN + chalf * 128, scale, obox, lane, release);
+                epilogue_tile_tma<NHQ, AMX>(p, &tmD, taddr, row0, nb * BN + chalf * 128, scale, obox, lane, amax_acc,
+                                            release);
         }
         if (lane == 0) bulk_wait_group0();  // this warp's stores are complete
+        if constexpr (AMX >= 0) {
+            // the CTA's partial maximum: warp maxima in shared memory, one
+            // barrier of the eight epilogue warps, written by the first
+            __shared__ float warp_max[kEpiWarps];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) amax_acc = fmaxf(amax_acc, __shfl_xor_sync(0xffffffffu, amax_acc, o));
+            if (lane == 0) warp_max[warp - kFirstEpiWarp] = amax_acc;
+            asm volatile("bar.sync 1, %0;" ::"r"(kEpiWarps * 32) : "memory");
+            if (warp == kFirstEpiWarp && lane == 0) {
+                float m = 0.0f;
+#pragma unroll
+                for (int i = 0; i < kEpiWarps; ++i) m = fmaxf(m, warp_max[i]);
+                if constexpr (AMX > 0) m = __fmul_rn(m, AMX == 16 ? 0.25f : 0x1.6a09e6p-3f);  // fp32(1/sqrt(n_h))
+                p.amax_partials[blockIdx.x] = m;
+            }
+        }
     }
 
     tc_fence_before();
@@ -888,26 +947,41 @@ cudaError_t launch_gemm(const GemmParams& p, int fmt, const CUtensorMap* tmapA, 
     return cudaGetLastError();
 }
 
-template <int FMT, int NHQ>
+template <int FMT, int NHQ, int AMX = -1>
 cudaError_t run_pair(const GemmParams& p, const CUtensorMap* tmapA, const CUtensorMap* tmapB,
                      const CUtensorMap* tmapSFA, const CUtensorMap* tmapSFB, const CUtensorMap* tmapD, cudaStream_t s,
                      int clusters) {
-    cudaError_t e =
-        cudaFuncSetAttribute(gemm_bs_fp4_pair_kernel<FMT, NHQ>, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM);
+    cudaError_t e = cudaFuncSetAttribute(gemm_bs_fp4_pair_kernel<FMT, NHQ, AMX>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM);
     if (e != cudaSuccess) return e;
-    gemm_bs_fp4_pair_kernel<FMT, NHQ><<<2 * clusters, kGemmThreads, P_SMEM, s>>>(*tmapA, *tmapB, *tmapSFA, *tmapSFB,
-                                                                                *tmapD, p);
+    gemm_bs_fp4_pair_kernel<FMT, NHQ, AMX><<<2 * clusters, kGemmThreads, P_SMEM, s>>>(*tmapA, *tmapB, *tmapSFA,
+                                                                                     *tmapSFB, *tmapD, p);
     return cudaSuccess;
 }
 
 cudaError_t launch_gemm_pair(const GemmParams& p, int fmt, const CUtensorMap* tmapA, const CUtensorMap* tmapB,
                              const CUtensorMap* tmapSFA, const CUtensorMap* tmapSFB, const CUtensorMap* tmapD,
-                             cudaStream_t s, int sms, int nhq) {
+                             cudaStream_t s, int sms, int nhq, int amx, int* n_partials) {
     const int tiles = ((p.M + 2 * BM - 1) / (2 * BM)) * ((p.N + BN - 1) / BN);
     int clusters = sms / 2;
     if (clusters > tiles) clusters = tiles;
     if (clusters < 1) clusters = 1;
+    if (n_partials != nullptr) *n_partials = 2 * clusters;
     cudaError_t e;
+    if (amx >= 0) {  // bf16 output with the NVFP4 tensor amax of the output
+        const bool nv = fmt == kNvfp4;
+        switch (amx) {
+            case 0: e = nv ? run_pair<kNvfp4, -1, 0>(p, tmapA, tmapB, tmapSFA, tmapSFB, tmapD, s, clusters)
+                           : run_pair<kMxfp4, -1, 0>(p, tmapA, tmapB, tmapSFA, tmapSFB, tmapD, s, clusters); break;
+            case 16: e = nv ? run_pair<kNvfp4, -1, 16>(p, tmapA, tmapB, tmapSFA, tmapSFB, tmapD, s, clusters)
+                            : run_pair<kMxfp4, -1, 16>(p, tmapA, tmapB, tmapSFA, tmapSFB, tmapD, s, clusters); break;
+            default: e = nv ? run_pair<kNvfp4, -1, 32>(p, tmapA, tmapB, tmapSFA, tmapSFB, tmapD, s, clusters)
+                            : run_pair<kMxfp4, -1, 32>(p, tmapA, tmapB, tmapSFA, tmapSFB, tmapD, s, clusters); break;
+        }
+        if (e != cudaSuccess) return e;
+        count_launch();
+        return cudaGetLastError();
+    }
     if (fmt == kNvfp4) {
         switch (nhq) {
             case -1: e = run_pair<kNvfp4, -1>(p, tmapA, tmapB, tmapSFA, tmapSFB, tmapD, s, clusters); break;

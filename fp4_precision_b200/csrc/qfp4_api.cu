@@ -476,8 +476,18 @@ struct QuantOut {
     qfp4_tensor* out;
 };
 
+// The optional NVFP4 tensor amax of a bf16 GEMM output along its rows
+// (qfp4_gemm_amax).
+struct AmaxOut {
+    int32_t had;
+    const qfp4_seed* seed;
+    float* amax;
+    void* workspace;
+    size_t workspace_bytes;
+};
+
 int gemm_impl(const qfp4_tensor* A, const qfp4_tensor* B, void* D, int64_t ldd, int32_t out_dtype, bool accumulate,
-              cudaStream_t s, const QuantOut* qo = nullptr) {
+              cudaStream_t s, const QuantOut* qo = nullptr, const AmaxOut* ao = nullptr) {
     int rc = bind_context(s);
     if (rc) return rc;
     int sms = 0;
@@ -493,6 +503,16 @@ int gemm_impl(const qfp4_tensor* A, const qfp4_tensor* B, void* D, int64_t ldd, 
         if (!qo->out->codes || !qo->out->scales || !qo->out->tensor_scale) return QFP4_ERR_INVALID_ARG;
         if (!aligned16(qo->out->codes) || !aligned16(qo->out->scales)) return QFP4_ERR_MISALIGNED;
     }
+    if (ao != nullptr) {
+        if (out_dtype != QFP4_OUT_BF16 || ao->amax == nullptr) return QFP4_ERR_INVALID_ARG;
+        if (ao->had < QFP4_HAD_NONE || ao->had > QFP4_HAD_RAND32) return QFP4_ERR_INVALID_ARG;
+        if (had_random(ao->had) && ao->seed == nullptr) return QFP4_ERR_INVALID_ARG;
+        const int nh = had_n(ao->had);
+        if (B->rows % 16 != 0 || (nh && B->rows % nh != 0)) return QFP4_ERR_INVALID_ARG;
+        if (ao->workspace == nullptr || ao->workspace_bytes < qfp4_quantize_workspace_bytes())
+            return QFP4_ERR_WORKSPACE;
+        if (!aligned16(ao->workspace)) return QFP4_ERR_MISALIGNED;
+    }
     if (A->fmt != B->fmt || (A->fmt != QFP4_NVFP4 && A->fmt != QFP4_MXFP4)) return QFP4_ERR_INVALID_ARG;
     if (A->k != B->k || A->k < 0 || A->rows < 0 || B->rows < 0) return QFP4_ERR_INVALID_ARG;
     if (A->had != B->had) return QFP4_ERR_INVALID_ARG;
@@ -501,13 +521,18 @@ int gemm_impl(const qfp4_tensor* A, const qfp4_tensor* B, void* D, int64_t ldd, 
     if (A->k % 64 != 0) return QFP4_ERR_INVALID_ARG;
     if (A->rows > 0x7fffffffLL || B->rows > 0x7fffffffLL || A->k > 0x7fffffffLL) return QFP4_ERR_INVALID_ARG;
     const int64_t M = A->rows, N = B->rows, K = A->k;
-    if (M == 0 || N == 0) return QFP4_OK;
+    if (M == 0 || N == 0) {
+        if (ao == nullptr) return QFP4_OK;
+        const cudaError_t e = cudaMemsetAsync(ao->amax, 0, sizeof(float), s);  // the amax of an empty tensor
+        return e == cudaSuccess ? QFP4_OK : cuda_fail(e);
+    }
     const size_t esz = out_dtype == QFP4_OUT_F32 ? 4 : 2;
     if (D == nullptr || ldd < N) return QFP4_ERR_INVALID_ARG;
     if (!aligned16(D) || (ldd * (int64_t)esz) % 16 != 0) return QFP4_ERR_MISALIGNED;
     if (K == 0) {
         if (accumulate) return QFP4_OK;  // D += 0
         cudaError_t e = cudaMemset2DAsync(D, (size_t)ldd * esz, 0, (size_t)N * esz, (size_t)M, s);
+        if (e == cudaSuccess && ao != nullptr) e = cudaMemsetAsync(ao->amax, 0, sizeof(float), s);
         return e == cudaSuccess ? QFP4_OK : cuda_fail(e);
     }
     if (!A->codes || !B->codes || !A->scales || !B->scales || !A->tensor_scale || !B->tensor_scale)
@@ -535,21 +560,46 @@ int gemm_impl(const qfp4_tensor* A, const qfp4_tensor* B, void* D, int64_t ldd, 
         p.q_kb4 = (N / 32 + 3) / 4 * 4;
         p.q_signs = had_random(qo->had) ? host_sign_bits(qo->seed->rot, qo->seed->rot_stream) : 0u;
     }
+    int amx = -1;
+    uint32_t amax_signs = 0;
+    if (ao != nullptr) {
+        amax_signs = had_random(ao->had) ? host_sign_bits(ao->seed->rot, ao->seed->rot_stream) : 0u;
+        if (pair) {
+            amx = had_n(ao->had);
+            p.amax_partials = static_cast<float*>(ao->workspace);
+            p.amax_signs = amax_signs;
+        }
+    }
     p.M = (int)M; p.N = (int)N; p.K = (int)K;
     const int NB = block_of(A->fmt);
     p.atoms_k = (int)((K / NB + 3) / 4);
     cudaError_t e;
+    int n_partials = 0;
     if (pair) {
         const int atoms_per_kt = kGemmBK / (4 * NB);
         CUtensorMap tSFA, tSFB, tD;
         if ((rc = make_scale_tmap(&tSFA, A->scales, M, p.atoms_k, atoms_per_kt, 1))) return rc;
         if ((rc = make_scale_tmap(&tSFB, B->scales, N, p.atoms_k, atoms_per_kt, 2))) return rc;
         if ((rc = make_out_tmap(&tD, D, M, N, ldd, p.out_f32))) return rc;
-        e = launch_gemm_pair(p, A->fmt, &tA, &tB, &tSFA, &tSFB, &tD, s, sms, nhq);
+        e = launch_gemm_pair(p, A->fmt, &tA, &tB, &tSFA, &tSFB, &tD, s, sms, nhq, amx, &n_partials);
     } else {
         e = launch_gemm(p, A->fmt, &tA, &tB, s, sms);
     }
     if (e != cudaSuccess) return cuda_fail(e);
+    if (ao != nullptr) {
+        if (pair) {  // one maximum over the CTAs' partials
+            e = launch_reduce_max(p.amax_partials, n_partials, ao->amax, s);
+            return e == cudaSuccess ? QFP4_OK : cuda_fail(e);
+        }
+        // the single-CTA kernel has no amax epilogue: a pass over D afterwards
+        Geometry g{M, N};
+        int n = 0;
+        if ((rc = run_amax(D, M, N, ldd, ao->had, QFP4_AXIS_ROW, amax_signs, g, static_cast<float*>(ao->workspace), &n,
+                           sms, s)))
+            return rc;
+        e = launch_reduce_max(static_cast<const float*>(ao->workspace), n, ao->amax, s);
+        return e == cudaSuccess ? QFP4_OK : cuda_fail(e);
+    }
     if (qo != nullptr) {
         if (!pair)  // the single-CTA kernel has no quantizing epilogue: quantize D afterwards
             return quantize_impl(D, M, N, ldd, QFP4_MXFP4, QFP4_RTN, qo->had, QFP4_AXIS_ROW, qo->seed, nullptr,
@@ -786,6 +836,12 @@ int qfp4_gemm_quantize(const qfp4_tensor* A, const qfp4_tensor* B, void* D, int6
     return gemm_impl(A, B, D, ldd, QFP4_OUT_BF16, false, static_cast<cudaStream_t>(stream), &qo);
 }
 
+int qfp4_gemm_amax(const qfp4_tensor* A, const qfp4_tensor* B, void* D, int64_t ldd, int32_t had,
+                   const qfp4_seed* seed, float* amax, void* workspace, size_t workspace_bytes, void* stream) {
+    const AmaxOut ao{had, seed, amax, workspace, workspace_bytes};
+    return gemm_impl(A, B, D, ldd, QFP4_OUT_BF16, false, static_cast<cudaStream_t>(stream), nullptr, &ao);
+}
+
 int qfp4_gemm_accumulate(const qfp4_tensor* A, const qfp4_tensor* B, float* D, int64_t ldd, void* stream) {
     return gemm_impl(A, B, D, ldd, QFP4_OUT_F32, true, static_cast<cudaStream_t>(stream));
 }
@@ -825,15 +881,28 @@ size_t qfp4_linear_workspace_bytes(int32_t backward, int64_t M, int64_t N, int64
     return total;
 }
 
-int qfp4_linear_fwd(const void* X, const void* W, void* Y, int64_t M, int64_t N, int64_t K, const qfp4_recipe* recipe,
-                    const qfp4_seed* seed, void* workspace, size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace qfp4 {
+namespace {
+// The forward pass (qfp4_linear_fwd, qfp4_linear_fwd_chain): X and W quantized
+// along K, then Fprop. x_amax (nullable): X's NVFP4 tensor amax for this
+// Fprop's rotation, given by the caller; amax_out (nullable): Y's NVFP4 tensor
+// amax along its rows for the rotation (next_had, next_seed), from the GEMM.
+int linear_fwd_impl(const void* X, const void* W, void* Y, int64_t M, int64_t N, int64_t K, const qfp4_recipe* recipe,
+                    const qfp4_seed* seed, const float* x_amax, int32_t next_had, const qfp4_seed* next_seed,
+                    float* y_amax, void* workspace, size_t workspace_bytes, cudaStream_t s) {
     int rc = check_linear_args(M, N, K, recipe, seed);
     if (rc) return rc;
     if (!X || !W || !Y) return QFP4_ERR_INVALID_ARG;
+    if (y_amax != nullptr) {
+        if (recipe->y_dtype != QFP4_OUT_BF16) return QFP4_ERR_INVALID_ARG;
+        if (next_had < QFP4_HAD_NONE || next_had > QFP4_HAD_RAND32) return QFP4_ERR_INVALID_ARG;
+        if (had_random(next_had) && next_seed == nullptr) return QFP4_ERR_INVALID_ARG;
+    }
     if (workspace == nullptr || workspace_bytes < qfp4_linear_workspace_bytes(0, M, N, K, recipe))
         return QFP4_ERR_WORKSPACE;
     if (!aligned16(workspace)) return QFP4_ERR_MISALIGNED;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
     qfp4_tensor t[4];
     float* partials;
     size_t total;
@@ -841,11 +910,36 @@ int qfp4_linear_fwd(const void* X, const void* W, void* Y, int64_t M, int64_t N,
     const qfp4_gemm_cfg& c = recipe->fprop;
     const size_t pws = qfp4_quantize_workspace_bytes();
     qfp4_seed sx = op_seed(seed, 0, 0), sw = op_seed(seed, 0, 1);
-    if ((rc = quantize_impl(X, M, K, K, c.fmt, c.rnd_a, c.had, QFP4_AXIS_ROW, &sx, nullptr, &t[0], partials, pws, s)))
+    const float* ax = c.fmt == QFP4_NVFP4 ? x_amax : nullptr;
+    if ((rc = quantize_impl(X, M, K, K, c.fmt, c.rnd_a, c.had, QFP4_AXIS_ROW, &sx, ax, &t[0], partials, pws, s)))
         return rc;
     if ((rc = quantize_impl(W, N, K, K, c.fmt, c.rnd_b, c.had, QFP4_AXIS_ROW, &sw, nullptr, &t[1], partials, pws, s)))
         return rc;
-    return gemm_impl(&t[0], &t[1], Y, N, recipe->y_dtype, false, s);
+    if (y_amax == nullptr) return gemm_impl(&t[0], &t[1], Y, N, recipe->y_dtype, false, s);
+    // the next layer rotates its input with the sign vector of its own Fprop:
+    // key next_seed->rot, stream 0 (the linear layer's seed rule)
+    qfp4_seed ns{};
+    if (next_seed != nullptr) ns = op_seed(next_seed, 0, 0);
+    const AmaxOut ao{next_had, &ns, y_amax, partials, pws};
+    return gemm_impl(&t[0], &t[1], Y, N, QFP4_OUT_BF16, false, s, nullptr, &ao);
+}
+}  // namespace
+}  // namespace qfp4
+
+extern "C" {
+
+int qfp4_linear_fwd(const void* X, const void* W, void* Y, int64_t M, int64_t N, int64_t K, const qfp4_recipe* recipe,
+                    const qfp4_seed* seed, void* workspace, size_t workspace_bytes, void* stream) {
+    return linear_fwd_impl(X, W, Y, M, N, K, recipe, seed, nullptr, QFP4_HAD_NONE, nullptr, nullptr, workspace,
+                           workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+int qfp4_linear_fwd_chain(const void* X, const void* W, void* Y, int64_t M, int64_t N, int64_t K,
+                          const qfp4_recipe* recipe, const qfp4_seed* seed, const float* x_amax, int32_t next_had,
+                          const qfp4_seed* next_seed, float* y_amax, void* workspace, size_t workspace_bytes,
+                          void* stream) {
+    return linear_fwd_impl(X, W, Y, M, N, K, recipe, seed, x_amax, next_had, next_seed, y_amax, workspace,
+                           workspace_bytes, static_cast<cudaStream_t>(stream));
 }
 
 int qfp4_linear_bwd(const void* dY, const void* X, const void* W, void* dX, void* dW, int64_t M, int64_t N, int64_t K,
@@ -956,23 +1050,42 @@ int qfp4_selftest_wait_timeout(int64_t limit_ns, void* stream) {
 // ---- forward pass without allocation ------------------------------------------
 // The scratch of qfp4_linear_fwd_noalloc: a fixed device array (every GPU that
 // loads the library holds it until the process exits). Host code cannot use
-// the array's name as a device address; its address is looked up once per
-// device with cudaGetSymbolAddress, with that device current.
+// the array's name as a device address; its address is looked up with
+// cudaGetSymbolAddress, with the caller's device current. The lookup is done
+// once per CUDA context: the cache is keyed by the context's unique ID
+// (cuCtxGetId, never reused within a process), so a device that was reset
+// (cudaDeviceReset gives it a new primary context) or a stream of another
+// context on the same device gets a fresh lookup instead of a stale address.
 static __device__ __align__(256) uint8_t g_noalloc_scratch[QFP4_NOALLOC_SCRATCH_BYTES];
 
 static int noalloc_scratch(void** out) {
+    using CtxIdFn = CUresult (*)(CUcontext, unsigned long long*);
+    using CurCtxFn = CUresult (*)(CUcontext*);
+    static CtxIdFn ctx_id = nullptr;
+    static CurCtxFn cur_ctx = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        ctx_id = driver_fn<CtxIdFn>("cuCtxGetId");
+        cur_ctx = driver_fn<CurCtxFn>("cuCtxGetCurrent");
+    });
     static std::mutex mu;
+    static unsigned long long key[64] = {0};  // context ID of addr[dev]; 0: none
     static void* addr[64] = {nullptr};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_fail(e);
     if (dev < 0 || dev >= 64) return QFP4_ERR_UNSUPPORTED_ARCH;
+    unsigned long long id = 0;
+    CUcontext ctx = nullptr;
+    const bool have_id = ctx_id != nullptr && cur_ctx != nullptr && cur_ctx(&ctx) == CUDA_SUCCESS && ctx != nullptr &&
+                         ctx_id(ctx, &id) == CUDA_SUCCESS && id != 0;
     std::lock_guard<std::mutex> lock(mu);
-    if (addr[dev] == nullptr) {
+    if (!have_id || addr[dev] == nullptr || key[dev] != id) {
         void* p = nullptr;
         e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
         if (e != cudaSuccess) return cuda_fail(e);
         addr[dev] = p;
+        key[dev] = have_id ? id : 0;
     }
     *out = addr[dev];
     return QFP4_OK;

@@ -220,6 +220,21 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
     return mbar_wait_for(bar, parity, kWaitLimitNs);
 }
 
+// Before a TMA producer thread leaves: wait (bounded) until the loads of its
+// last min(issued, stages) ring iterations have landed, so that no TMA write
+// into this CTA's shared memory is outstanding when the CTA exits, also after a
+// timed-out wait cut the loop short. full and sf_load (either may be null:
+// none, or waited elsewhere) are the ring's completion barriers; iteration i
+// used stage i % stages with phase parity (i / stages) & 1, which is each
+// barrier's latest armed phase.
+__device__ __forceinline__ void drain_loads(uint64_t* full, uint64_t* sf_load, int stages, int issued) {
+    for (int i = issued > stages ? issued - stages : 0; i < issued; ++i) {
+        const uint32_t par = (uint32_t)((i / stages) & 1);
+        if (full != nullptr && !mbar_wait(&full[i % stages], par)) return;
+        if (sf_load != nullptr && !mbar_wait(&sf_load[i % stages], par)) return;
+    }
+}
+
 // The same wait with cluster-scope acquire: for barriers the peer CTA of a
 // pair arrives on.
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
@@ -278,6 +293,11 @@ __device__ __forceinline__ void bulk_wait_group_read0() {
 __device__ __forceinline__ void bulk_wait_group0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ void sts128(uint32_t saddr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(saddr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+__device__ __forceinline__ uint4 lds128(uint32_t saddr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(saddr));
+    return v;
 }
 __device__ __forceinline__ void tma_load_3d(void* dst, const void* tmap, uint64_t* bar, int32_t x, int32_t y,
                                             int32_t z) {

@@ -91,6 +91,11 @@ struct GemmParams {
     uint8_t* q_scales;
     int64_t q_kb4;
     uint32_t q_signs;
+    // bf16 output only, pair kernel: the NVFP4 tensor amax of the output along
+    // its rows after the next layer's rotation (the kernel's AMX size, these
+    // sign bits): one partial maximum per CTA into amax_partials[blockIdx.x]
+    float* amax_partials;
+    uint32_t amax_signs;
     int M, N, K;
     int atoms_k;  // scale atoms per 128-row block along k: ceil(K / block / 4)
 };
@@ -103,9 +108,11 @@ cudaError_t launch_gemm(const GemmParams& p, int fmt, const CUtensorMap* tmapA, 
 // make_out_tmap in qfp4_api.cu).
 // nhq: -1 (no quantized output) or the Hadamard size (0, 16, 32) of the
 // MXFP4 output quantization (p.q_codes etc.).
+// amx: -1 (no amax of the output) or the Hadamard size (0, 16, 32) of the
+// output's tensor amax (p.amax_partials; *n_partials receives their count).
 cudaError_t launch_gemm_pair(const GemmParams& p, int fmt, const CUtensorMap* tmapA, const CUtensorMap* tmapB,
                              const CUtensorMap* tmapSFA, const CUtensorMap* tmapSFB, const CUtensorMap* tmapD,
-                             cudaStream_t s, int sms, int nhq = -1);
+                             cudaStream_t s, int sms, int nhq = -1, int amx = -1, int* n_partials = nullptr);
 constexpr int kGemmBM = 128, kGemmBN = 256, kGemmBK = 256;
 
 void count_launch();

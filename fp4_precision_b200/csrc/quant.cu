@@ -59,17 +59,26 @@ __device__ __forceinline__ float abs_max(float m, const float* v) {
     return m;
 }
 
-// x / 6 correctly rounded. For finite x >= 2^-125: one product with RN(1/6)
-// and one fused correction (the division-by-a-known-divisor method of
-// Brisebarre, Muller and Raina, IEEE Trans. Computers 53(8), 2004), checked
-// against the division for every such fp32 x; below 2^-125 (subnormal
-// quotients), and for inf or NaN, the division itself.
+// x / 6 correctly rounded, for x >= 0 (a block amax), with no division
+// subroutine. For finite x >= 2^-125: one product with RN(1/6) and one fused
+// correction (the division-by-a-known-divisor method of Brisebarre, Muller and
+// Raina, IEEE Trans. Computers 53(8), 2004). Below 2^-125 the quotient is
+// subnormal: x = N * 2^-149 with N = the bits of x (exponent field 0 or 1),
+// and x / 6 rounds to round-half-even(N / 6) * 2^-149, whose bits are that
+// integer. Both are checked against the division for every such fp32 x.
+// inf and NaN give x * (1/6) (inf, NaN).
 __device__ __forceinline__ float div6(float x) {
-    if (!(x >= 0x1p-125f && x <= 0x1.fffffep127f)) return __fdiv_rn(x, 6.0f);
-    constexpr float C = 1.0f / 6.0f;
-    const float q = __fmul_rn(x, C);
-    const float r = __fmaf_rn(-q, 6.0f, x);
-    return __fmaf_rn(r, C, q);
+    if (x >= 0x1p-125f && x <= 0x1.fffffep127f) {
+        constexpr float C = 1.0f / 6.0f;
+        const float q = __fmul_rn(x, C);
+        const float r = __fmaf_rn(-q, 6.0f, x);
+        return __fmaf_rn(r, C, q);
+    }
+    if (x >= 0.0f && x < 0x1p-125f) {
+        const uint32_t n = __float_as_uint(x), q = n / 6u, r = n - 6u * q;
+        return __uint_as_float(q + ((2u * r > 6u || (2u * r == 6u && (q & 1u) != 0u)) ? 1u : 0u));
+    }
+    return __fmul_rn(x, 1.0f / 6.0f);
 }
 __device__ __forceinline__ float2 neg2(float2 a) { return make_float2(-a.x, -a.y); }
 
@@ -345,6 +354,267 @@ __device__ __forceinline__ void store_codes32(uint8_t* dst, const uint32_t* code
     }
 }
 
+// ===========================================================================
+// NVFP4 unit of 64 elements with two blocks per packed lane pair
+// ===========================================================================
+// The row and band-column kernels give each thread 64 consecutive elements of
+// the quantized axis: four NVFP4 blocks. For NVFP4 with no Hadamard or a
+// 16-point one, they are processed as two pairs (blocks 0 and 1, then 2 and 3)
+// whose blocks sit in the .x and .y lanes of every packed f32x2 value:
+// P[j] = (v_{2bp}[j], v_{2bp+1}[j]). All four Hadamard stages, the
+// normalisation, the scale product and the Quartet II sums are then one packed
+// instruction per pair of lanes, without data movement between lanes, and each
+// lane performs exactly its own block's fp32 operations in the stated order.
+
+// bf16 -> fp32 of the low / high element of a packed word, with its sign flip
+// m (0 or 0x80000000): low = w * 2^16 + m (adding 2^31 modulo 2^32 flips bit
+// 31), high = (w & 0xFFFF0000) ^ m.
+__device__ __forceinline__ float bf16lo_flip(uint32_t w, uint32_t m) { return __uint_as_float(w * 65536u + m); }
+__device__ __forceinline__ float bf16hi_flip(uint32_t w, uint32_t m) { return __uint_as_float((w & 0xFFFF0000u) ^ m); }
+
+// A zero magnitude keeps code 0 whatever its sign (no -0 codes): per nibble,
+// mag + 7 has bit 3 set iff mag >= 1 (no carry leaves a nibble).
+__device__ __forceinline__ uint32_t e2m1_clear_neg_zero(uint32_t out) {
+    const uint32_t mag = out & 0x77777777u;
+    return out & ((mag + 0x77777777u) | 0x77777777u);
+}
+
+// Round-to-nearest-even E2M1 codes of eight values (element 0 in the low
+// nibble), saturating at +-6.
+__device__ __forceinline__ uint32_t e2m1x8_words(float a0, float a1, float a2, float a3, float a4, float a5, float a6,
+                                                 float a7) {
+    uint32_t out;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(out)
+        : "f"(a0), "f"(a1), "f"(a2), "f"(a3), "f"(a4), "f"(a5), "f"(a6), "f"(a7));
+    return e2m1_clear_neg_zero(out);
+}
+
+// The same, also returning the eight code values as f16 pairs (h[i]: elements
+// 2i, 2i + 1), decoded from the code bytes before the zero-sign clean-up: a -0
+// code decodes to -0, which changes no sum it enters.
+__device__ __forceinline__ uint32_t e2m1x8_words_dec(float a0, float a1, float a2, float a3, float a4, float a5,
+                                                     float a6, float a7, uint32_t* h) {
+    uint32_t out;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %8, %7;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %10, %9;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %12, %11;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %1, b0;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %2, b1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %3, b2;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %4, b3;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(out), "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
+        : "f"(a0), "f"(a1), "f"(a2), "f"(a3), "f"(a4), "f"(a5), "f"(a6), "f"(a7));
+    return e2m1_clear_neg_zero(out);
+}
+
+// E4M3 codes (round to nearest even, saturating at 448) of both lanes: the low
+// byte is lane .x's, the next byte lane .y's.
+__device__ __forceinline__ uint32_t e4m3x2_rn(float2 t) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(t.y), "f"(t.x));
+    return r;
+}
+
+// x / 6 correctly rounded in both lanes: the packed form of div6 (one product
+// with RN(1/6), one fused correction) when both lanes are in [2^-125,
+// FLT_MAX], else div6 per lane.
+__device__ __forceinline__ float2 div6x2(float2 x) {
+    if (fminf(x.x, x.y) >= 0x1p-125f && fmaxf(x.x, x.y) <= 0x1.fffffep127f) {
+        constexpr float C = 1.0f / 6.0f;
+        const float2 q = __fmul2_rn(x, f2(C, C));
+        const float2 r = __ffma2_rn(q, f2(-6.0f, -6.0f), x);
+        return __ffma2_rn(r, f2(C, C), q);
+    }
+    return f2(div6(x.x), div6(x.y));
+}
+
+// Largest magnitude of each lane over the 16 packed elements of a pair: a tree
+// of three-input maxima (depth 3; the maximum does not depend on the order).
+__device__ __forceinline__ float2 abs_max_pair(const float2* P) {
+    float x[5], y[5];
+#pragma unroll
+    for (int i = 0; i < 5; ++i) {
+        x[i] = max3(fabsf(P[3 * i].x), fabsf(P[3 * i + 1].x), fabsf(P[3 * i + 2].x));
+        y[i] = max3(fabsf(P[3 * i].y), fabsf(P[3 * i + 1].y), fabsf(P[3 * i + 2].y));
+    }
+    return f2(fmaxf(max3(x[0], x[1], x[2]), max3(x[3], x[4], fabsf(P[15].x))),
+              fmaxf(max3(y[0], y[1], y[2]), max3(y[3], y[4], fabsf(P[15].y))));
+}
+
+// One butterfly stage of half-width H over the 16 packed elements of a pair.
+template <int H>
+__device__ __forceinline__ void fwht_pair_stage(float2* P) {
+#pragma unroll
+    for (int j0 = 0; j0 < 16; j0 += 2 * H)
+#pragma unroll
+        for (int j = j0; j < j0 + H; ++j) {
+            const float2 a = P[j], b = P[j + H];
+            P[j] = __fadd2_rn(a, b);
+            P[j + H] = __fadd2_rn(a, neg2(b));
+        }
+}
+
+// Halving-stride tree sum of the 16 packed terms of a pair (both lanes).
+__device__ __forceinline__ float2 tree_sum_pair(float2* s) {
+#pragma unroll
+    for (int st = 8; st >= 1; st >>= 1)
+#pragma unroll
+        for (int j = 0; j < st; ++j) s[j] = __fadd2_rn(s[j], s[j + st]);
+    return s[0];
+}
+
+// Per-CTA table of (s_enc / S, S) for every E4M3 code S can take (1-126; code
+// 0 gives (0, 0)), the same divisions as per block. Ends with a CTA barrier.
+__device__ void fill_tab2(float2* tab, float s_enc) {
+    for (int c = threadIdx.x; c < 128; c += blockDim.x) {
+        const float S = e4m3_decode((uint32_t)c);
+        tab[c] = (c == 0 || c == 127) ? f2(0.0f, 0.0f) : f2(__fdiv_rn(s_enc, S), S);
+    }
+    __syncthreads();
+}
+
+// Hadamard sign flips of the 8 words of a block, at bit 31 of each element:
+// lo[i] for element 2i, hi[i] for element 2i + 1.
+struct SignFlips {
+    uint32_t lo[8], hi[8];
+    __device__ __forceinline__ explicit SignFlips(uint32_t signs) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            lo[i] = ((signs >> (2 * i)) & 1u) << 31;
+            hi[i] = ((signs >> (2 * i + 1)) & 1u) << 31;
+        }
+    }
+};
+
+// Word i (0-3) of a Philox quad.
+__device__ __forceinline__ uint32_t quad_word(uint4 q, uint32_t i) {
+    return i == 0 ? q.x : i == 1 ? q.y : i == 2 ? q.z : q.w;
+}
+
+// Quantize one 64-element NVFP4 unit. load(c) returns chunk c (elements 8c ..
+// 8c + 7 as four packed bf16 words, element 2i of the chunk in the low half
+// of word i). elem0: index of element 0 in the quantized orientation (a
+// multiple of 16); block0: its block index. Writes the 8 code words and
+// returns the scale word (block b's E4M3 code in byte b).
+template <int RND, int NH, typename Load>
+__device__ __forceinline__ uint32_t nv64_quantize(Load load, const SignFlips& sf, float s_enc, const float2* tab,
+                                                  const Stream& st, uint64_t elem0, uint64_t block0, uint32_t* codes) {
+    static_assert(NH == 0 || NH == 16, "the packed unit takes no Hadamard or a 16-point one");
+    uint32_t scw = 0;
+    uint4 rq = make_uint4(0u, 0u, 0u, 0u);
+    if constexpr (RND == kQuartet2) {
+        // the scale words of the four blocks: one Philox quad when block0 is a
+        // multiple of 4, else one per block below
+        if ((block0 & 3u) == 0) rq = philox_quad(st.seed, st.tag_scale, block0 >> 2);
+    }
+#pragma unroll
+    for (int bp = 0; bp < 2; ++bp) {
+        float2 P[16];
+        // blocks 2bp (chunks 4bp, 4bp + 1) and 2bp + 1 (chunks 4bp + 2, 4bp + 3)
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+            const uint4 a = load(4 * bp + c), b = load(4 * bp + 2 + c);
+            const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int wi = 4 * c + i;  // word of the block
+                if constexpr (NH > 0) {
+                    P[2 * wi] = f2(bf16lo_flip(wa[i], sf.lo[wi]), bf16lo_flip(wb[i], sf.lo[wi]));
+                    P[2 * wi + 1] = f2(bf16hi_flip(wa[i], sf.hi[wi]), bf16hi_flip(wb[i], sf.hi[wi]));
+                } else {
+                    P[2 * wi] = f2(bf16lo(wa[i]), bf16lo(wb[i]));
+                    P[2 * wi + 1] = f2(bf16hi(wa[i]), bf16hi(wb[i]));
+                }
+            }
+        }
+        if constexpr (NH == 16) {
+            fwht_pair_stage<1>(P);
+            fwht_pair_stage<2>(P);
+            fwht_pair_stage<4>(P);
+            fwht_pair_stage<8>(P);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) P[j] = __fmul2_rn(P[j], f2(0.25f, 0.25f));  // fp32(1/sqrt(16))
+        }
+        // block scales from the block amaxes
+        const float2 t = __fmul2_rn(div6x2(abs_max_pair(P)), f2(s_enc, s_enc));
+        const uint32_t sc2 = e4m3x2_rn(t);  // block 2bp in the low byte
+        // t >= 0 gives codes 0-126 (0x7F only for a NaN amax): the mask only
+        // keeps the table index in range
+        const float2 e0 = tab[sc2 & 0x7Fu], e1 = tab[(sc2 >> 8) & 0x7Fu];
+        const float2 rr = f2(e0.x, e1.x);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) P[j] = __fmul2_rn(P[j], rr);
+        uint32_t* cw = codes + 4 * bp;  // block 2bp: cw[0..1], block 2bp + 1: cw[2..3]
+        if constexpr (RND == kSr) {
+#pragma unroll
+            for (int lane = 0; lane < 2; ++lane) {
+                const uint64_t i0 = elem0 + (uint64_t)(16 * (2 * bp + lane));
+#pragma unroll
+                for (int e4 = 0; e4 < 16; e4 += 4) {
+                    const uint4 w = philox_quad(st.seed, st.tag_elem, (i0 >> 2) + (uint64_t)(e4 >> 2));
+                    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        float& u = lane ? P[e4 + e].y : P[e4 + e].x;
+                        u = e2m1_sr_value(u, uniform24(ws[e]));
+                    }
+                }
+            }
+        }
+        if constexpr (RND != kQuartet2) {
+            cw[0] = e2m1x8_words(P[0].x, P[1].x, P[2].x, P[3].x, P[4].x, P[5].x, P[6].x, P[7].x);
+            cw[1] = e2m1x8_words(P[8].x, P[9].x, P[10].x, P[11].x, P[12].x, P[13].x, P[14].x, P[15].x);
+            cw[2] = e2m1x8_words(P[0].y, P[1].y, P[2].y, P[3].y, P[4].y, P[5].y, P[6].y, P[7].y);
+            cw[3] = e2m1x8_words(P[8].y, P[9].y, P[10].y, P[11].y, P[12].y, P[13].y, P[14].y, P[15].y);
+            scw |= sc2 << (16 * bp);
+        } else {
+            // RTN codes and their values q; alpha = T(u u) / T(u q) per lane
+            uint32_t h[4][4];
+            cw[0] = e2m1x8_words_dec(P[0].x, P[1].x, P[2].x, P[3].x, P[4].x, P[5].x, P[6].x, P[7].x, h[0]);
+            cw[1] = e2m1x8_words_dec(P[8].x, P[9].x, P[10].x, P[11].x, P[12].x, P[13].x, P[14].x, P[15].x, h[1]);
+            cw[2] = e2m1x8_words_dec(P[0].y, P[1].y, P[2].y, P[3].y, P[4].y, P[5].y, P[6].y, P[7].y, h[2]);
+            cw[3] = e2m1x8_words_dec(P[8].y, P[9].y, P[10].y, P[11].y, P[12].y, P[13].y, P[14].y, P[15].y, h[3]);
+            float2 uu[16], uq[16];
+#pragma unroll
+            for (int j = 0; j < 16; j += 2) {
+                const float2 qx = __half22float2(*reinterpret_cast<const __half2*>(&h[j / 8][(j % 8) / 2]));
+                const float2 qy = __half22float2(*reinterpret_cast<const __half2*>(&h[2 + j / 8][(j % 8) / 2]));
+                uu[j] = __fmul2_rn(P[j], P[j]);
+                uu[j + 1] = __fmul2_rn(P[j + 1], P[j + 1]);
+                uq[j] = __fmul2_rn(P[j], f2(qx.x, qy.x));
+                uq[j + 1] = __fmul2_rn(P[j + 1], f2(qx.y, qy.y));
+            }
+            const float2 num = tree_sum_pair(uu), den = tree_sum_pair(uq);
+            const float a0 = (den.x == 0.0f) ? 1.0f : __fdiv_rn(num.x, den.x);
+            const float a1 = (den.y == 0.0f) ? 1.0f : __fdiv_rn(num.y, den.y);
+            const float2 ts = __fmul2_rn(f2(e0.y, e1.y), f2(a0, a1));
+            uint32_t w0, w1;
+            if ((block0 & 3u) == 0) {
+                w0 = bp ? rq.z : rq.x;
+                w1 = bp ? rq.w : rq.y;
+            } else {
+                const uint64_t b0 = block0 + (uint64_t)(2 * bp), b1 = b0 + 1;
+                w0 = quad_word(philox_quad(st.seed, st.tag_scale, b0 >> 2), (uint32_t)b0 & 3u);
+                w1 = quad_word(philox_quad(st.seed, st.tag_scale, b1 >> 2), (uint32_t)b1 & 3u);
+            }
+            scw |= (e4m3_sr(ts.x, w0) | (e4m3_sr(ts.y, w1) << 8)) << (16 * bp);
+        }
+        // The next pair's loads (volatile) stay after this pair's codes: it
+        // bounds the live values to one pair (no spills at 96 registers).
+        asm volatile("" ::"r"(cw[0]), "r"(cw[1]), "r"(cw[2]), "r"(cw[3]));
+    }
+    return scw;
+}
+
 // This CTA's tiles of a tiles_r x tiles_c grid (blockIdx.x, + gridDim.x, ...)
 // as (tr, tc), advanced without divisions, with the TMA ring stage and phase
 // of each.
@@ -412,6 +682,9 @@ __global__ void __launch_bounds__(kThreads, 2)
     constexpr int NB = Grp::NB;
     constexpr int G = AMAX_ONLY ? ((NH > 16) ? NH : 16) : Grp::G;
     constexpr int STAGE_BYTES = kRowTileRows * kRowTileCols * 2;  // 32 KiB
+    // NVFP4 with no Hadamard or a 16-point one, round-to-nearest or Quartet
+    // II: the packed 64-element unit
+    constexpr bool kPacked = FMT == kNvfp4 && (NH == 0 || NH == 16) && RND != kSr && !AMAX_ONLY;
     extern __shared__ __align__(1024) uint8_t dyn_smem[];
     uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
     __shared__ Ring<STAGES> ring;
@@ -426,11 +699,15 @@ __global__ void __launch_bounds__(kThreads, 2)
         ring_init(ring);
     }
     __syncthreads();
-    __shared__ float rtab[128];
+    __shared__ float rtab[kPacked ? 1 : 128];
+    __shared__ float2 tab2[kPacked ? 128 : 1];
     float s_enc = 1.0f;
     if constexpr (!AMAX_ONLY && FMT == kNvfp4) {
         s_enc = nvfp4_encode_scale(p, red, blockIdx.x == 0);
-        fill_rtab(rtab, s_enc);
+        if constexpr (kPacked)
+            fill_tab2(tab2, s_enc);
+        else
+            fill_rtab(rtab, s_enc);
     }
     if constexpr (!AMAX_ONLY && FMT == kMxfp4) {
         if (blockIdx.x == 0 && tid == 0) *p.tensor_scale = 1.0f;
@@ -446,6 +723,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 mbar_arrive_expect_tx(&ring.full[s], STAGE_BYTES);
                 tma_load_2d(tiles + s * STAGE_BYTES, &tmap, &ring.full[s], w.tc * kRowTileCols, w.tr * kRowTileRows);
             }
+            drain_loads(ring.full, nullptr, STAGES, i);  // no load lands after this CTA exits
         }
         return;
     }
@@ -460,15 +738,20 @@ __global__ void __launch_bounds__(kThreads, 2)
     // masks (the per-element SR kernels too: timed 7-9 % faster with them
     // hoisted than recomputing them, with fewer spills).
     constexpr bool kHoist = true;
-    uint32_t chunk_off[kRowTileCols / 8];
+    uint32_t chunk_off[kPacked ? 1 : kRowTileCols / 8];
+    if constexpr (!kPacked) {
 #pragma unroll
-    for (int c = 0; c < kRowTileCols / 8; ++c) chunk_off[c] = (uint32_t)(tid * 128 + ((c ^ (tid & 7)) << 4));
+        for (int c = 0; c < kRowTileCols / 8; ++c) chunk_off[c] = (uint32_t)(tid * 128 + ((c ^ (tid & 7)) << 4));
+    }
     const int64_t atom_row_bytes = (p.kb4 / 4) * 512;  // one 128-row block of scale atoms
     const int64_t sc_row_off = (tid / 128) * atom_row_bytes + (tid % 32) * 16 + ((tid / 32) % 4) * 4;
     // the random Hadamard's sign-flip masks of the packed bf16 words of a group
-    uint32_t smask[G / 2];
+    uint32_t smask[kPacked ? 1 : G / 2];
+    if constexpr (!kPacked) {
 #pragma unroll
-    for (int i = 0; i < G / 2; ++i) smask[i] = Grp::sign_mask(p.signs, i);
+        for (int i = 0; i < G / 2; ++i) smask[i] = Grp::sign_mask(p.signs, i);
+    }
+    const SignFlips sf(kPacked && NH > 0 ? p.signs : 0u);
     for (TileWalk<STAGES> w(tiles_c); w.tr < tiles_r; w.next()) {
         const int s = w.stage;
         if (!mbar_wait(&ring.full[s], w.phase)) break;
@@ -477,6 +760,15 @@ __global__ void __launch_bounds__(kThreads, 2)
         const uint32_t sbase = smem_u32(tiles) + (uint32_t)(s * STAGE_BYTES) + (kHoist ? 0u : (uint32_t)tid * 128u);
         uint32_t codes[kRowTileCols / 8];
         uint32_t scodes[kRowTileCols / 16];
+        uint32_t scw = 0;
+        if constexpr (kPacked) {
+            // chunk c of this thread's row: 16-byte chunk c ^ (tid % 8) of its 128-byte line
+            const uint32_t rb = smem_u32(tiles) + (uint32_t)(s * STAGE_BYTES) + (uint32_t)tid * 128u +
+                                ((uint32_t)(tid & 7) << 4);
+            auto load = [&](int c) { return lds128(rb ^ ((uint32_t)c << 4)); };
+            scw = nv64_quantize<RND, NH>(load, sf, s_enc, tab2, col_stream(p), (uint64_t)row * (uint64_t)p.k + (uint64_t)col0,
+                                         (uint64_t)row * (uint64_t)(p.k / 16) + (uint64_t)(col0 / 16), codes);
+        } else {
 #pragma unroll
         for (int g = 0; g < kRowTileCols / G; ++g) {
             float v[G];
@@ -510,6 +802,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                               codes + g * (G / 8), scodes + g * (G / NB));
             }
         }
+        }
         __syncwarp();
         if (lane == 0) mbar_arrive(&ring.empty[s]);
         if constexpr (!AMAX_ONLY) {
@@ -532,8 +825,11 @@ __global__ void __launch_bounds__(kThreads, 2)
                     kHoist ? (2 * (int64_t)w.tr) * atom_row_bytes + (kb0 / 4) * 512 + sc_row_off
                            : ((row / 128) * (p.kb4 / 4) + kb0 / 4) * 512 + (row % 32) * 16 + ((row / 32) % 4) * 4;
                 if constexpr (NB == 16) {
-                    *reinterpret_cast<uint32_t*>(p.scales + off) =
-                        scodes[0] | (scodes[1] << 8) | (scodes[2] << 16) | (scodes[3] << 24);
+                    if constexpr (kPacked)
+                        *reinterpret_cast<uint32_t*>(p.scales + off) = scw;
+                    else
+                        *reinterpret_cast<uint32_t*>(p.scales + off) =
+                            scodes[0] | (scodes[1] << 8) | (scodes[2] << 16) | (scodes[3] << 24);
                 } else {
                     const uint32_t half = scodes[0] | (scodes[1] << 8);
                     if ((kb0 & 3) == 0 && col0 + kRowTileCols >= p.k)
@@ -607,6 +903,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 tma_load_5d(tiles + s * STAGE_BYTES + BOX_BYTES, &tmap, &ring.full[s], (int32_t)(c0 + 64), 0, tr4, 0,
                             0);
             }
+            drain_loads(ring.full, nullptr, STAGES, i);  // no load lands after this CTA exits
         }
         return;
     }
@@ -810,11 +1107,12 @@ __global__ void __launch_bounds__(kThreads, 2)
 // (t = k + 2 q + 8 v) over the tile's 64 columns, and stores its codes and
 // scale word(s) in the row orientation (rows = R, k = C).
 template <int FMT, int RND, int NH_ROW>
-__device__ __forceinline__ void dual_row_work(const QuantParams& p, float s_enc_row,
-                                              const float* rtab_row, ScaleRng& srng, uint32_t stage, int tr, int tc) {
+__device__ __forceinline__ void dual_row_work(const QuantParams& p, float s_enc_row, const float* rtab_row,
+                                              const float2* tab2_row, ScaleRng& srng, uint32_t stage, int tr, int tc) {
     using GrpR = Group<FMT, RND, NH_ROW>;
     constexpr int NB = GrpR::NB;
     constexpr int GR = GrpR::G;
+    constexpr bool kPackedRow = FMT == kNvfp4 && (NH_ROW == 0 || NH_ROW == 16) && RND != kSr;
     const int t = threadIdx.x;
     const int64_t r = (int64_t)tr * 256 + (t & 1) + 2 * (t >> 3) + 64 * ((t >> 1) & 3);
     const int64_t c0 = (int64_t)tc * 64;
@@ -822,6 +1120,15 @@ __device__ __forceinline__ void dual_row_work(const QuantParams& p, float s_enc_
     const uint32_t rbase = stage + (uint32_t)t * 128u;
     uint32_t codes[8];
     uint32_t scodes[64 / NB];
+    uint32_t scw = 0;
+    if constexpr (kPackedRow) {
+        const SignFlips sf(NH_ROW > 0 ? p.signs_row : 0u);
+        const uint32_t rb = rbase + ((uint32_t)(t & 7) << 4);
+        auto load = [&](int c) { return lds128(rb ^ ((uint32_t)c << 4)); };
+        scw = nv64_quantize<RND, NH_ROW>(load, sf, s_enc_row, tab2_row, row_stream(p),
+                                         (uint64_t)r * (uint64_t)p.C + (uint64_t)c0,
+                                         (uint64_t)r * (uint64_t)(p.C / 16) + (uint64_t)(c0 / 16), codes);
+    } else {
 #pragma unroll
     for (int g = 0; g < 64 / GR; ++g) {
         float v[GR];
@@ -849,6 +1156,7 @@ __device__ __forceinline__ void dual_row_work(const QuantParams& p, float s_enc_
                        (uint64_t)r * (uint64_t)(p.C / NB) + (uint64_t)(j0 / NB), srng, codes + g * (GR / 8),
                        scodes + g * (GR / NB));
     }
+    }
     if (r < p.R) {
         uint8_t* dst = p.codes_row + r * (p.C / 2) + c0 / 2;
         if (c0 + 64 <= p.C) {
@@ -864,7 +1172,10 @@ __device__ __forceinline__ void dual_row_work(const QuantParams& p, float s_enc_
         uint8_t* sc = p.scales_row + ((r / 128) * (p.kb4_row / 4) + kb0 / 4) * 512 + (r % 32) * 16 +
                       ((r / 32) % 4) * 4;
         if constexpr (NB == 16) {
-            *reinterpret_cast<uint32_t*>(sc) = scodes[0] | (scodes[1] << 8) | (scodes[2] << 16) | (scodes[3] << 24);
+            if constexpr (kPackedRow)
+                *reinterpret_cast<uint32_t*>(sc) = scw;
+            else
+                *reinterpret_cast<uint32_t*>(sc) = scodes[0] | (scodes[1] << 8) | (scodes[2] << 16) | (scodes[3] << 24);
         } else {
             const uint32_t half = scodes[0] | (scodes[1] << 8);
             if ((kb0 & 3) == 0 && c0 + 64 >= p.C)
@@ -891,6 +1202,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     constexpr int TILE_ROWS = 256, TILE_COLS = 64;
     constexpr int STAGE_BYTES = TILE_ROWS * TILE_COLS * 2;  // 32 KiB
     static_assert(64 % G == 0, "groups tile a 64-row band");
+    // NVFP4 with no Hadamard or a 16-point one, round-to-nearest or Quartet
+    // II: the packed 64-element unit
+    constexpr bool kPacked = FMT == kNvfp4 && (NH == 0 || NH == 16) && RND != kSr;
+    constexpr bool kPackedRow = kDual && FMT == kNvfp4 && (NH_ROW == 0 || NH_ROW == 16) && RND != kSr;
     extern __shared__ __align__(1024) uint8_t dyn_smem[];
     uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
     __shared__ Ring<STAGES> ring;
@@ -907,15 +1222,23 @@ __global__ void __launch_bounds__(kThreads, 2)
         ring_init(ring);
     }
     __syncthreads();
-    __shared__ float rtab[128];
-    __shared__ float rtab_row[kDual ? 128 : 1];
+    __shared__ float rtab[kPacked ? 1 : 128];
+    __shared__ float2 tab2[kPacked ? 128 : 1];
+    __shared__ float rtab_row[kDual && !kPackedRow ? 128 : 1];
+    __shared__ float2 tab2_row[kPackedRow ? 128 : 1];
     float s_enc = 1.0f, s_enc_row = 1.0f;
     if constexpr (FMT == kNvfp4) {
         s_enc = nvfp4_encode_scale(p, red, blockIdx.x == 0);
-        fill_rtab(rtab, s_enc);
+        if constexpr (kPacked)
+            fill_tab2(tab2, s_enc);
+        else
+            fill_rtab(rtab, s_enc);
         if constexpr (kDual) {  // the row orientation's amax is always given
             s_enc_row = nvfp4_scale_from_amax(__ldg(p.amax_in_row), p.tensor_scale_row, blockIdx.x == 0);
-            fill_rtab(rtab_row, s_enc_row);
+            if constexpr (kPackedRow)
+                fill_tab2(tab2_row, s_enc_row);
+            else
+                fill_rtab(rtab_row, s_enc_row);
         }
     }
     if constexpr (FMT == kMxfp4) {
@@ -934,6 +1257,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 mbar_arrive_expect_tx(&ring.full[s], STAGE_BYTES);
                 tma_load_4d(tiles + s * STAGE_BYTES, &tmap, &ring.full[s], w.tc * TILE_COLS, 0, 4 * w.tr, 0);
             }
+            drain_loads(ring.full, nullptr, STAGES, i);  // no load lands after this CTA exits
         }
         return;
     }
@@ -945,11 +1269,12 @@ __global__ void __launch_bounds__(kThreads, 2)
     const uint32_t lm_base = (uint32_t)lane * 128u + ((uint32_t)(warp ^ (lane & 7)) << 4);
     const int64_t atom_row_bytes = (p.kb4 / 4) * 512;
     // sign masks held in registers, except in dual mode (registers for the row work)
-    uint32_t smask[kDual ? 1 : G / 2];
-    if constexpr (!kDual) {
+    uint32_t smask[kDual || kPacked ? 1 : G / 2];
+    if constexpr (!kDual && !kPacked) {
 #pragma unroll
         for (int i = 0; i < G / 2; ++i) smask[i] = Grp::sign_mask(p.signs, i);
     }
+    const SignFlips sf(kPacked && NH > 0 ? p.signs : 0u);
     ScaleRng srng, srng_row;
     for (TileWalk<STAGES> w(tiles_c); w.tr < tiles_r; w.next()) {
         const int s = w.stage;
@@ -959,6 +1284,19 @@ __global__ void __launch_bounds__(kThreads, 2)
         const uint32_t stage_base = smem_u32(tiles) + (uint32_t)(s * STAGE_BYTES) + lm_base;
         uint32_t codes[8];
         uint32_t scodes[64 / NB];
+        uint32_t scw = 0;
+        if constexpr (kPacked) {
+            // chunk n = rows 8n .. 8n + 7 of the band: ldmatrix number n
+            auto load = [&](int n) {
+                uint4 v;
+                asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                             : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                             : "r"(stage_base + (uint32_t)(n * 4096)));
+                return v;
+            };
+            scw = nv64_quantize<RND, NH>(load, sf, s_enc, tab2, col_stream(p), (uint64_t)c * (uint64_t)p.k + (uint64_t)rb,
+                                         (uint64_t)c * (uint64_t)(p.k / 16) + (uint64_t)(rb / 16), codes);
+        } else {
 #pragma unroll
         for (int g = 0; g < 64 / G; ++g) {
             float v[G];
@@ -993,7 +1331,8 @@ __global__ void __launch_bounds__(kThreads, 2)
                           (uint64_t)c * (uint64_t)(p.k / NB) + (uint64_t)(r_grp / NB), srng, codes + g * (G / 8),
                           scodes + g * (G / NB));
         }
-        if constexpr (kDual) dual_row_work<FMT, RND, NH_ROW>(p, s_enc_row, rtab_row, srng_row,
+        }
+        if constexpr (kDual) dual_row_work<FMT, RND, NH_ROW>(p, s_enc_row, rtab_row, tab2_row, srng_row,
                                                           smem_u32(tiles) + (uint32_t)(s * STAGE_BYTES), w.tr, w.tc);
         __syncwarp();
         if (lane == 0) mbar_arrive(&ring.empty[s]);
@@ -1007,8 +1346,11 @@ __global__ void __launch_bounds__(kThreads, 2)
                 const int64_t kb0 = rb / NB;
                 uint8_t* sc = p.scales + (c / 128) * atom_row_bytes + (kb0 / 4) * 512 + (c % 32) * 16 + ((c / 32) % 4) * 4;
                 if constexpr (NB == 16) {
-                    *reinterpret_cast<uint32_t*>(sc) =
-                        scodes[0] | (scodes[1] << 8) | (scodes[2] << 16) | (scodes[3] << 24);
+                    if constexpr (kPacked)
+                        *reinterpret_cast<uint32_t*>(sc) = scw;
+                    else
+                        *reinterpret_cast<uint32_t*>(sc) =
+                            scodes[0] | (scodes[1] << 8) | (scodes[2] << 16) | (scodes[3] << 24);
                 } else {
                     // two scale columns: half of an atom word; when this is the
                     // word's first half and the band is the last, the other

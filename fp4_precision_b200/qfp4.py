@@ -81,12 +81,17 @@ _SIGNATURES = {
                                           ctypes.POINTER(Seed), ctypes.POINTER(TensorDesc), _VOID]),
     "qfp4_gemm_accumulate": (ctypes.c_int, [ctypes.POINTER(TensorDesc), ctypes.POINTER(TensorDesc), _VOID, _I64,
                                             _VOID]),
+    "qfp4_gemm_amax": (ctypes.c_int, [ctypes.POINTER(TensorDesc), ctypes.POINTER(TensorDesc), _VOID, _I64, _I32,
+                                      ctypes.POINTER(Seed), _VOID, _VOID, _SZ, _VOID]),
     "qfp4_recipe_preset": (ctypes.c_int, [_I32, ctypes.POINTER(Recipe)]),
     "qfp4_linear_workspace_bytes": (_SZ, [_I32, _I64, _I64, _I64, ctypes.POINTER(Recipe)]),
     "qfp4_linear_fwd": (ctypes.c_int, [_VOID, _VOID, _VOID, _I64, _I64, _I64, ctypes.POINTER(Recipe),
                                        ctypes.POINTER(Seed), _VOID, _SZ, _VOID]),
     "qfp4_linear_bwd": (ctypes.c_int, [_VOID, _VOID, _VOID, _VOID, _VOID, _I64, _I64, _I64, ctypes.POINTER(Recipe),
                                        ctypes.POINTER(Seed), _VOID, _SZ, _VOID]),
+    "qfp4_linear_fwd_chain": (ctypes.c_int, [_VOID, _VOID, _VOID, _I64, _I64, _I64, ctypes.POINTER(Recipe),
+                                             ctypes.POINTER(Seed), _VOID, _I32, ctypes.POINTER(Seed), _VOID, _VOID,
+                                             _SZ, _VOID]),
     "qfp4_linear_fwd_noalloc": (ctypes.c_int, [_VOID, _VOID, _VOID, _I64, _I64, _I64, ctypes.POINTER(Recipe),
                                                ctypes.POINTER(Seed), _VOID]),
     "qfp4_status": (ctypes.c_int, [_VOID]),
@@ -266,6 +271,23 @@ def gemm_quantize(A: QTensor, B: QTensor, had: int, seed: Seed, out: torch.Tenso
     return out, qout
 
 
+def gemm_amax(A: QTensor, B: QTensor, had: int, seed: Seed | None = None, out: torch.Tensor | None = None,
+              amax: torch.Tensor | None = None, workspace=None, stream=None):
+    """bf16 D = gA gB A . B^T and the NVFP4 tensor amax of D along its rows
+    after the rotation `had`; see qfp4_gemm_amax. Returns (D, amax)."""
+    if out is None:
+        out = torch.empty((A.rows, B.rows), dtype=torch.bfloat16, device=A.codes.device)
+    amax = torch.empty((1,), dtype=torch.float32, device=A.codes.device) if amax is None else amax
+    ws = workspace
+    if ws is None:
+        ws = torch.empty((quantize_workspace_bytes(),), dtype=torch.uint8, device=A.codes.device)
+    seed = seed or make_seed()
+    _check(lib().qfp4_gemm_amax(ctypes.byref(A.desc), ctypes.byref(B.desc), _ptr(out), out.stride(0), had,
+                                ctypes.byref(seed), _ptr(amax), _ptr(ws), ws.numel(), _stream(stream)),
+           "qfp4_gemm_amax")
+    return out, amax
+
+
 def gemm_accumulate(A: QTensor, B: QTensor, out: torch.Tensor, stream=None) -> torch.Tensor:
     """out += gA gB A . B^T in fp32 (A.rows x B.rows); see qfp4_gemm_accumulate."""
     assert out.dtype == torch.float32 and out.dim() == 2 and out.stride(1) == 1
@@ -298,6 +320,24 @@ def linear_fwd(X, W, rec: Recipe, seed: Seed, Y=None, workspace=None, stream=Non
     _check(lib().qfp4_linear_fwd(_ptr(X), _ptr(W), _ptr(Y), M, N, K, ctypes.byref(rec), ctypes.byref(seed),
                                  _ptr(workspace), workspace.numel(), _stream(stream)), "qfp4_linear_fwd")
     return Y
+
+
+def linear_fwd_chain(X, W, rec: Recipe, seed: Seed, x_amax=None, next_had: int = HAD_NONE,
+                     next_seed: Seed | None = None, want_y_amax: bool = True, Y=None, workspace=None, stream=None):
+    """qfp4_linear_fwd_chain: the forward pass taking X's NVFP4 tensor amax
+    (x_amax, from the previous layer) and returning Y's for the next layer's
+    Fprop rotation (next_had, next_seed). Returns (Y, y_amax or None)."""
+    M, K = X.shape
+    N = W.shape[0]
+    Y = torch.empty((M, N), dtype=_dtype(rec.y_dtype), device=X.device) if Y is None else Y
+    if workspace is None:
+        workspace = torch.empty((linear_workspace_bytes(False, M, N, K, rec),), dtype=torch.uint8, device=X.device)
+    y_amax = torch.empty((1,), dtype=torch.float32, device=X.device) if want_y_amax else None
+    ns = ctypes.byref(next_seed) if next_seed is not None else None
+    _check(lib().qfp4_linear_fwd_chain(_ptr(X), _ptr(W), _ptr(Y), M, N, K, ctypes.byref(rec), ctypes.byref(seed),
+                                       _ptr(x_amax), next_had, ns, _ptr(y_amax), _ptr(workspace), workspace.numel(),
+                                       _stream(stream)), "qfp4_linear_fwd_chain")
+    return Y, y_amax
 
 
 def linear_fwd_noalloc(X, W, rec: Recipe, seed: Seed, Y=None, stream=None) -> torch.Tensor:

@@ -225,6 +225,11 @@ int qfp4_quantize_dual(const void* x, int64_t R, int64_t C, int64_t ld, int32_t 
                        void* stream);
 
 /* ---- GEMM -------------------------------------------------------------------
+ * The three products of a linear layer trained in FP4 (page "New AMD paper
+ * overturns conventional wisdom: FP4 training...", section "Poiskovaya
+ * eksperimental'naya rabota": Fprop Y = X W^T, Dgrad dX = dY W, Wgrad
+ * dW = dY^T X, each with both operands quantized) are all of this form, with
+ * the operands quantized along their reduction axis by qfp4_quantize:
  * D[i][j] = gA * gB * sum_k A(i,k) B(j,k) over the decoded FP4 operands, fp32
  * accumulation on the tcgen05 tensor cores, D = A . B^T of shape
  * A.rows x B.rows, written as bf16 or fp32 with row stride ldd elements.
@@ -256,8 +261,36 @@ int qfp4_gemm_accumulate(const qfp4_tensor* A, const qfp4_tensor* B, float* D, i
  * B.rows)) 16-byte aligned, and its tensor_scale (set to 1). No workspace. */
 int qfp4_gemm_quantize(const qfp4_tensor* A, const qfp4_tensor* B, void* D, int64_t ldd, int32_t had,
                        const qfp4_seed* seed, qfp4_tensor* out, void* stream);
+/* qfp4_gemm_amax: D = A . B^T as qfp4_gemm with a bf16 output, and *amax (a
+ * device fp32) = the NVFP4 tensor amax of that bf16 D along its rows after
+ * the rotation `had` (seed->rot / rot_stream for a random one) — exactly what
+ * qfp4_amax(D, A.rows, B.rows, ldd, had, ROW, seed, ...) gives. Passing it as
+ * amax_in to qfp4_quantize(D, NVFP4, ..., had, ROW, seed) quantizes a layer's
+ * output for the next layer without the separate read of D that the tensor
+ * scale otherwise needs (NVFP4's FP32 tensor scale must be known before any
+ * block scale; page "Quartet II - obuchenie v NVFP4 s tochnymi
+ * nesmeshchyonnymi gradientami" on NVFP4 with FP8 block scales). With the
+ * CTA-pair kernel (A.rows > 128) each CTA's epilogue takes the rotated
+ * maximum of the rows it stores and a one-CTA reduction combines them;
+ * otherwise D is read once more by an amax pass.
+ * Requirements: those of qfp4_gemm; B.rows a multiple of 16 and of the
+ * Hadamard size; workspace >= qfp4_quantize_workspace_bytes(), 16-byte
+ * aligned (its contents on entry do not matter). */
+int qfp4_gemm_amax(const qfp4_tensor* A, const qfp4_tensor* B, void* D, int64_t ldd, int32_t had,
+                   const qfp4_seed* seed, float* amax, void* workspace, size_t workspace_bytes, void* stream);
 
 /* ---- linear layer -------------------------------------------------------------
+ * One linear layer's FP4 forward (Fprop) and backward (Dgrad and Wgrad) pass:
+ * six quantizations and three GEMMs (page "New AMD paper overturns
+ * conventional wisdom: FP4 training...", section "Poiskovaya
+ * eksperimental'naya rabota"; the recipes: QFP4_PRESET_NVIDIA_NVFP4 follows
+ * "NVIDIA sozdala metod obucheniya neyrosetey v 4-bit tochnosti", section
+ * "Kak eto rabotaet" (16x16 random Hadamard on the Wgrad inputs, stochastic
+ * rounding of the gradient); QFP4_PRESET_QUARTET2_NVFP4 follows "Quartet II -
+ * obuchenie v NVFP4 s tochnymi nesmeshchyonnymi gradientami" (random rotation
+ * and the stochastically rounded scale renormalisation on the backward pass);
+ * QFP4_PRESET_AMD_MXFP4_H the AMD page's MXFP4 with a deterministic Hadamard
+ * on Wgrad).
  * X [M x K], W [N x K], dY [M x N] bf16 row-major (contiguous); Y [M x N],
  * dX [M x K], dW [N x K] in the recipe's output types (contiguous).
  * Seeds: the sign vector of GEMM g (0 Fprop, 1 Dgrad, 2 Wgrad) uses key
@@ -273,6 +306,27 @@ int qfp4_linear_fwd(const void* X, const void* W, void* Y, int64_t M, int64_t N,
 int qfp4_linear_bwd(const void* dY, const void* X, const void* W, void* dX, void* dW, int64_t M, int64_t N, int64_t K,
                     const qfp4_recipe* recipe, const qfp4_seed* seed, void* workspace, size_t workspace_bytes,
                     void* stream);
+/* qfp4_linear_fwd_chain: qfp4_linear_fwd for a layer between two FP4 layers,
+ * where one layer's output Y is the next layer's input X, so that NVFP4's
+ * tensor scale (needed before any block scale) costs no extra read of it:
+ *   x_amax (device fp32, or NULL): X's NVFP4 tensor amax for this layer's
+ *     Fprop rotation, as the previous layer's call returned it in its y_amax;
+ *     X's quantization then skips its amax pass (ignored unless the Fprop
+ *     format is NVFP4; NULL: the pass runs as in qfp4_linear_fwd);
+ *   y_amax (device fp32, or NULL): receives Y's NVFP4 tensor amax along its
+ *     rows for the next layer's Fprop rotation next_had, whose sign vector
+ *     is the next layer's (key next_seed->rot, stream 0, by the seed rule
+ *     above), taken in the GEMM's epilogue as qfp4_gemm_amax does; needs a
+ *     bf16 y_dtype and N a multiple of 16 and of the Hadamard size.
+ * The result is bit for bit what qfp4_linear_fwd gives (and y_amax what
+ * qfp4_amax(Y, ..., next_had, ROW, ...) gives). Workspace as qfp4_linear_fwd.
+ * The pages have no such interface; it applies the tensor scale of NVFP4
+ * ("Quartet II - obuchenie v NVFP4 s tochnymi nesmeshchyonnymi gradientami")
+ * to a stack of linear layers. */
+int qfp4_linear_fwd_chain(const void* X, const void* W, void* Y, int64_t M, int64_t N, int64_t K,
+                          const qfp4_recipe* recipe, const qfp4_seed* seed, const float* x_amax, int32_t next_had,
+                          const qfp4_seed* next_seed, float* y_amax, void* workspace, size_t workspace_bytes,
+                          void* stream);
 
 /* ---- forward pass without any allocation ----------------------------------
  * qfp4_linear_fwd_noalloc: the same computation as qfp4_linear_fwd, for
@@ -288,9 +342,11 @@ int qfp4_linear_bwd(const void* dY, const void* X, const void* W, void* dX, void
  * qfp4_linear_workspace_bytes(0, ...) exceeds it is rejected with
  * QFP4_ERR_TOO_LARGE before anything is launched. The call makes no
  * cudaMalloc / cudaFree or other allocation.
- * Set-up: the first call on a device looks up the array's device address (once
- * per device, with the stream's device current); make that first call before
- * any stream capture. All calls share the one array and it keeps the last
+ * Set-up: the first call in a CUDA context (a device's primary context, and
+ * again after cudaDeviceReset replaces it) looks up the array's device address
+ * with the stream's device current, and later calls in that context reuse it;
+ * make that first call before any stream capture. All calls share the one
+ * array and it keeps the last
  * call's contents; every byte a call reads there it has written first, so
  * nothing needs clearing, but calls that overlap on the GPU (on different
  * streams, or from different threads) race on it: serialise them.

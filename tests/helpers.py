@@ -50,3 +50,56 @@ def padding_is_zero(flat: np.ndarray, rows: int, k: int, block: int) -> bool:
 
 def to_numpy_u8(t: torch.Tensor) -> np.ndarray:
     return t.detach().cpu().numpy().astype(np.uint8)
+
+
+# ---------------------------------------------------------------------------
+# Canary guard bytes around GPU output buffers (out-of-bounds write evidence)
+
+GUARD_BYTES = 4096    # a multiple of 16 and of 128: the view keeps the alignment TMA stores need
+GUARD_PATTERN = 0xA5
+
+
+class Guarded:
+    """A device buffer of `nbytes` between two guard regions of GUARD_BYTES
+    filled with GUARD_PATTERN; `view(dtype, shape)` is the usable middle."""
+
+    def __init__(self, nbytes: int, device):
+        self.nbytes = int(nbytes)
+        self.base = torch.full((self.nbytes + 2 * GUARD_BYTES,), GUARD_PATTERN, dtype=torch.uint8, device=device)
+
+    def view(self, dtype, shape):
+        mid = self.base[GUARD_BYTES:GUARD_BYTES + self.nbytes]
+        return mid.view(dtype).view(shape)
+
+    def intact(self) -> bool:
+        g = self.base.cpu().numpy()
+        return bool(np.all(g[:GUARD_BYTES] == GUARD_PATTERN) and np.all(g[GUARD_BYTES + self.nbytes:] == GUARD_PATTERN))
+
+
+def guarded_qtensor(Q, fmt: int, rows: int, k: int, device):
+    """A quantized-operand buffer (codes, scales, tensor scale) whose three
+    parts each sit between guard bytes; returns (qtensor, guards)."""
+    gc = Guarded(max(rows * k // 2, 16), device)
+    gs = Guarded(max(Q.scales_bytes(fmt, rows, k), 16), device)
+    gt = Guarded(16, device)
+    codes = gc.view(torch.uint8, (max(rows * k // 2, 16),))[: rows * k // 2].view(rows, k // 2)
+    scales = gs.view(torch.uint8, (gs.nbytes,))
+    ts = gt.view(torch.float32, (4,))[:1]
+    desc = Q.TensorDesc(codes.data_ptr(), scales.data_ptr(), ts.data_ptr(), 0, 0, 0, 0, 0, 0, 0)
+    return Q.QTensor(codes, scales, ts, desc), (gc, gs, gt)
+
+
+def guarded_matrix(rows: int, cols: int, dtype, device):
+    """A [rows, cols] output matrix between guard bytes; returns (tensor, guard)."""
+    esz = torch.tensor([], dtype=dtype).element_size()
+    g = Guarded(max(rows * cols * esz, 16), device)
+    return g.view(torch.uint8, (g.nbytes,))[: rows * cols * esz].view(dtype).view(rows, cols), g
+
+
+def assert_guards_intact(*guards):
+    torch.cuda.synchronize()
+    for g in guards:
+        if isinstance(g, (tuple, list)):
+            assert_guards_intact(*g)
+        else:
+            assert g.intact(), "a kernel wrote outside its output buffer (canary bytes changed)"

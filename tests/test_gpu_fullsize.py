@@ -1,5 +1,6 @@
-"""The benchmark's layers at their full sizes, in the launch configuration
-bench.py times: the six quantizations of one linear fwd+bwd (with the fused
+"""The benchmark's layers at their full sizes (the MLP up/gate layer, the
+attention QKV projection, the MLP down layer at 2048, 16384 and 32768 tokens),
+in the launch configuration bench.py times: the six quantizations of one linear fwd+bwd (with the fused
 row-and-column amax of dY, and its row and column quantizations from one read,
 where the recipe allows them) and the three GEMMs.
 
@@ -23,7 +24,9 @@ import helpers
 pytestmark = pytest.mark.gpu
 
 ROT, SR = 0x0123_4567, 0x89AB_CDEF
-LAYERS = [("mlp_up", "QUARTET2_NVFP4", None), ("mlp_up", "AMD_MXFP4_H", None), ("mlp_down", "NVIDIA_NVFP4", 16384)]
+LAYERS = [("mlp_up", "QUARTET2_NVFP4", None), ("mlp_up", "AMD_MXFP4_H", None), ("mlp_down", "NVIDIA_NVFP4", 16384),
+          ("qkv", "QUARTET2_NVFP4", None), ("mlp_down", "QUARTET2_NVFP4", 2048), ("mlp_down", "NVIDIA_NVFP4", 32768),
+          ("mlp_down", "QUARTET2_NVFP4", 32768)]
 
 
 def sample_rows(n, rng, count=64):
@@ -48,7 +51,7 @@ def assert_rows_same(q_gpu, q_ref, rows, fmt):
     assert np.float32(g).tobytes() == np.float32(q_ref.g).tobytes(), (g, q_ref.g)
 
 
-@pytest.mark.parametrize("workload,preset,M", LAYERS, ids=[f"{w}-{p}" for w, p, _ in LAYERS])
+@pytest.mark.parametrize("workload,preset,M", LAYERS, ids=[f"{w}-{p}" + (f"-M{m}" if m else "") for w, p, m in LAYERS])
 def test_layer_full_size_sampled(workload, preset, M):
     dev = torch.device("cuda", 0)
     wl = inputs.workload(workload, device=dev, M=M)

@@ -35,9 +35,11 @@ def upload(qo: O.QTensor, rot_seed=0, rot_stream=0) -> Q.QTensor:
 
 def check_gemm(A_o, B_o, out_dtype, rows=None, cols=None, rot=(0, 0)):
     A, B = upload(A_o, *rot), upload(B_o, *rot)
-    D = Q.gemm(A, B, out_dtype)
+    D, guard = helpers.guarded_matrix(A.rows, B.rows, out_dtype, "cuda")
+    Q.gemm(A, B, out_dtype, out=D)
     torch.cuda.synchronize()
     Q.status()
+    helpers.assert_guards_intact(guard)
     Dg = D.float().cpu().numpy().astype(np.float64)
     if rows is None:
         ref, bound = O.gemm(A_o, B_o), O.gemm_bound(A_o, B_o)
@@ -126,9 +128,12 @@ def test_gemm_quantize_matches_oracle(shape, had, kernel_variant):
     d_exact = X.double().numpy() @ W.double().numpy().T
     d_bf16 = torch.from_numpy(d_exact.astype(np.float32)).to(torch.bfloat16)
     ref = O.quantize(d_bf16, O.MXFP4, O.RTN, had, O.ROW, 0x77, 5)
-    D, q = Q.gemm_quantize(upload(A_o), upload(B_o), had, Q.make_seed(rot=0x77, rot_stream=5))
+    Dg, g_d = helpers.guarded_matrix(M, N, torch.bfloat16, "cuda")
+    qg, g_q = helpers.guarded_qtensor(Q, Q.MXFP4, M, N, "cuda")
+    D, q = Q.gemm_quantize(upload(A_o), upload(B_o), had, Q.make_seed(rot=0x77, rot_stream=5), out=Dg, qout=qg)
     torch.cuda.synchronize()
     Q.status()
+    helpers.assert_guards_intact(g_d, g_q)
     assert torch.equal(D.cpu(), d_bf16)
     assert q.fmt == Q.MXFP4 and q.rows == M and q.k == N
     codes = helpers.to_numpy_u8(q.codes)
@@ -222,3 +227,48 @@ def test_gemm_rejects_mismatched_operands():
     C = upload(O.quantize(X, O.MXFP4, O.RTN, O.HAD_RAND16, O.ROW, 1, 0), 1, 0)
     with pytest.raises(Q.QFP4Error):
         Q.gemm(A, C)
+
+
+@pytest.mark.parametrize("had", [O.HAD_NONE, O.HAD_DET16, O.HAD_RAND16, O.HAD_RAND32],
+                         ids=["none", "det16", "rand16", "rand32"])
+@pytest.mark.parametrize("shape", [(300, 288, 256), (128, 256, 128), (640, 544, 1024), (1024, 2080, 512)],
+                         ids=lambda s: "x".join(map(str, s)))
+def test_gemm_amax_matches_oracle(shape, had, kernel_variant):
+    """qfp4_gemm_amax: the bf16 D is exactly qfp4_gemm's, and the amax is the
+    NVFP4 tensor amax of that D along its rows after the rotation (the
+    oracle's max |rotated D|, bit for bit); quantizing D with it gives the
+    same operand as quantizing D with its own amax pass. Ragged tiles in both
+    directions, outputs between guard bytes."""
+    M, N, K = shape
+    X = inputs.normal_with_outliers((M, K), 41, "ga")
+    W = inputs.normal((N, K), 0.02, 41, "gb")
+    A = upload(O.quantize(X, O.NVFP4, O.RTN, O.HAD_NONE, O.ROW))
+    B = upload(O.quantize(W, O.NVFP4, O.RTN, O.HAD_NONE, O.ROW))
+    seed = Q.make_seed(rot=0x99, rot_stream=4)
+    Dg, g_d = helpers.guarded_matrix(M, N, torch.bfloat16, "cuda")
+    am = torch.full((1,), -1.0, device="cuda")
+    D, am = Q.gemm_amax(A, B, had, seed, out=Dg, amax=am)
+    D_ref = Q.gemm(A, B, torch.bfloat16)
+    torch.cuda.synchronize()
+    Q.status()
+    helpers.assert_guards_intact(g_d)
+    assert torch.equal(D, D_ref)
+    v = O.rotate(D.cpu(), had, O.ROW, 0x99, 4)
+    assert np.float32(am.cpu()[0]).tobytes() == np.float32(np.abs(v).max()).tobytes()
+    assert float(Q.amax(D, had, Q.ROW, seed).cpu()[0]) == float(am.cpu()[0])
+    q1 = Q.quantize(D, Q.NVFP4, Q.RTN, had, Q.ROW, seed, amax_in=am)
+    q2 = Q.quantize(D, Q.NVFP4, Q.RTN, had, Q.ROW, seed)
+    torch.cuda.synchronize()
+    assert torch.equal(q1.codes, q2.codes) and torch.equal(q1.scales, q2.scales)
+    assert torch.equal(q1.tensor_scale, q2.tensor_scale)
+
+
+def test_gemm_amax_rejects_bad_arguments():
+    A = upload(O.quantize(inputs.normal((256, 128), 1.0, 3, "ra"), O.NVFP4, O.RTN, O.HAD_NONE, O.ROW))
+    B = upload(O.quantize(inputs.normal((200, 128), 1.0, 3, "rb"), O.NVFP4, O.RTN, O.HAD_NONE, O.ROW))
+    with pytest.raises(Q.QFP4Error):  # B.rows (the next layer's k) not a multiple of 16
+        Q.gemm_amax(A, B, Q.HAD_NONE)
+    B2 = upload(O.quantize(inputs.normal((208, 128), 1.0, 3, "rb"), O.NVFP4, O.RTN, O.HAD_NONE, O.ROW))
+    with pytest.raises(Q.QFP4Error):  # ... nor of the Hadamard size
+        Q.gemm_amax(A, B2, Q.HAD_RAND32, Q.make_seed(1))
+    torch.cuda.synchronize()

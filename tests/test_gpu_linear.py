@@ -168,3 +168,31 @@ def test_calls_from_a_worker_thread():
         assert torch.equal(out[k], ref_dX)
     for k in ("dW", "dW0"):
         assert torch.equal(out[k], ref_dW)
+
+
+@pytest.mark.parametrize("M", [512, 128], ids=["pair", "single"])
+@pytest.mark.parametrize("had", [Q.HAD_NONE, Q.HAD_DET16, Q.HAD_RAND16], ids=["none", "det16", "rand16"])
+def test_linear_fwd_chain(had, M):
+    """Two stacked layers through qfp4_linear_fwd_chain: layer 1's output Y1
+    comes with its NVFP4 tensor amax for layer 2's Fprop rotation (from the
+    GEMM epilogue with the CTA-pair kernel, M = 512; by an amax pass with the
+    single-CTA one, M = 128), and layer 2 takes it for its input. Both outputs
+    equal qfp4_linear_fwd's bit for bit, and the amax equals qfp4_amax of Y1
+    with layer 2's sign vector (its seed's rot key, stream 0)."""
+    K, N1, N2 = 256, 384, 256
+    X = inputs.normal_with_outliers((M, K), 51, "cx").cuda()
+    W1 = inputs.normal((N1, K), 0.05, 51, "cw1").cuda()
+    W2 = inputs.normal((N2, N1), 0.05, 51, "cw2").cuda()
+    rec = Q.recipe("QUARTET2_NVFP4")
+    rec.fprop.had = had
+    s1, s2 = Q.make_seed(11, 12), Q.make_seed(21, 22)
+    Y1, a1 = Q.linear_fwd_chain(X, W1, rec, s1, next_had=had, next_seed=s2)
+    Y2, none = Q.linear_fwd_chain(Y1, W2, rec, s2, x_amax=a1, want_y_amax=False)
+    R1 = Q.linear_fwd(X, W1, rec, s1)
+    R2 = Q.linear_fwd(Y1, W2, rec, s2)
+    ref = Q.amax(Y1, had, Q.ROW, Q.make_seed(21, 0, 0, 0))
+    torch.cuda.synchronize()
+    Q.status()
+    assert none is None
+    assert torch.equal(Y1, R1) and torch.equal(Y2, R2)
+    assert float(a1.cpu()[0]) == float(ref.cpu()[0]) > 0.0

@@ -19,10 +19,16 @@ SEED = dict(rot=0x5EED_0001_2345_6789, sr=0xABCD_EF01_2345_6789, rot_stream=3, s
 
 
 def gpu_quant(x_dev, fmt, rnd, had, axis, **kw):
+    """Quantize on the GPU into guarded output buffers and check that no byte
+    outside codes, scales and tensor scale changed."""
     seed = Q.make_seed(**SEED)
-    q = Q.quantize(x_dev, fmt, rnd, had, axis, seed, **kw)
+    R, C = x_dev.shape
+    rows, k = (R, C) if axis == Q.ROW else (C, R)
+    out, guards = helpers.guarded_qtensor(Q, fmt, rows, k, x_dev.device)
+    q = Q.quantize(x_dev, fmt, rnd, had, axis, seed, out=out, **kw)
     torch.cuda.synchronize()
     Q.status()
+    helpers.assert_guards_intact(guards)
     return q
 
 
@@ -102,9 +108,14 @@ def test_quantize_dual_matches_oracle(fmt, rnd, hads, shape):
     if fmt == Q.NVFP4:
         am_row = Q.amax(xd, had_row, Q.ROW, s_row)
         am_col = Q.amax(xd, had_col, Q.COL, s_col)
-    qr, qc = Q.quantize_dual(xd, fmt, rnd, had_row, had_col, s_row, s_col, am_row, am_col)
+    R, C = shape
+    out_row, g_row = helpers.guarded_qtensor(Q, fmt, R, C, xd.device)
+    out_col, g_col = helpers.guarded_qtensor(Q, fmt, C, R, xd.device)
+    qr, qc = Q.quantize_dual(xd, fmt, rnd, had_row, had_col, s_row, s_col, am_row, am_col, out_row=out_row,
+                             out_col=out_col)
     torch.cuda.synchronize()
     Q.status()
+    helpers.assert_guards_intact(g_row, g_col)
     assert qr.fmt == qc.fmt == (Q.MXFP4 if fmt == Q.MXFP4_RU else fmt)
     assert_same(qr, O.quantize(x, fmt, rnd, had_row, Q.ROW, SEED["rot"], 1, SEED["sr"], 2), fmt)
     assert_same(qc, O.quantize(x, fmt, rnd, had_col, Q.COL, SEED["rot"], 2, SEED["sr"], 4), fmt)
