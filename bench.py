@@ -41,6 +41,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-sustained", action="store_true",
+                    help="leave out the two-second sustained run of the step (its own key, not the headline)")
     ap.add_argument("--profile", choices=["gemm_fprop", "gemm_dgrad", "gemm_wgrad", "quant_row", "quant_col",
                                           "quant_sr_row", "quant_sr_col", "amax_row", "amax_col"],
                     help="run only one kernel 3 times on a bounded case (for ncu captures), print nothing else")
@@ -70,25 +72,59 @@ def max_over_ranks(x: float, world: int, device) -> float:
 
 def measured_gemm_traffic():
     """DRAM bytes per GEMM launch (dram__bytes_read.sum + dram__bytes_write.sum)
-    from the committed ncu summary of this workload, or None when the GEMM
-    kernel's source has changed since those counters were taken."""
+    from the committed ncu record of this workload (profiles/gemm_traffic.json),
+    or None when the GEMM kernel's sources have changed since those counters
+    were taken (their SHA-256 is recorded beside the figures)."""
     import hashlib
-    import re
     try:
-        with open(os.path.join(ROOT, "profiles", "gemm_bs_fp4_mlp_up.md")) as f:
-            text = f.read()
-    except OSError:
+        with open(os.path.join(ROOT, "profiles", "gemm_traffic.json")) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
         return None
     csrc = os.path.join(ROOT, "fp4_precision_b200", "csrc")
-    for key, fname in (("gemm_source_sha256", "gemm_sm100.cu"), ("device_header_sha256", "qfp4_device.cuh")):
-        m = re.search(key + r"\s+([0-9a-f]{64})", text)
-        with open(os.path.join(csrc, fname), "rb") as f:
-            if m is None or hashlib.sha256(f.read()).hexdigest() != m.group(1):
-                return None
-    m = re.search(r"traffic_bytes_per_launch fprop=(\d+) dgrad=(\d+) wgrad=(\d+)", text)
-    if m is None:
+    for fname, digest in rec.get("source_sha256", {}).items():
+        try:
+            with open(os.path.join(csrc, fname), "rb") as f:
+                if hashlib.sha256(f.read()).hexdigest() != digest:
+                    return None
+        except OSError:
+            return None
+    t = rec.get("traffic_bytes_per_launch")
+    if not rec.get("source_sha256") or not isinstance(t, dict):
         return None
-    return dict(zip(("fprop", "dgrad", "wgrad"), (int(v) for v in m.groups())))
+    return {k: int(t[k]) for k in ("fprop", "dgrad", "wgrad")}
+
+
+# FP4 tensor-core work per SM and clock: one M128 x N256 x K64 block-scaled
+# MMA (2 * 128 * 256 * 64 flops) per 128 cycles (9 PFLOP/s dense over 148 SMs
+# at 1.855 GHz is the same figure).
+FP4_FLOP_PER_SM_CYCLE = 2 * 128 * 256 * 64 / 128
+
+
+def gemm_roofline(gemm_flops, gemm_ms, peaks, src, clocks, sms, timed_ms):
+    """The dominant kernel's roofline object: the three GEMMs' algorithmic
+    flops over their CUDA-event time against the dense FP4 peak derived from
+    the measured bf16 cuBLAS peak (x 4, the nominal FP4/BF16 ratio): the burst
+    figure when the timed region is short (under one second), else the
+    sustained one; plus the clock-normalised fraction (flops per SM and cycle
+    at the sampled median SM clock over the FP4 MMA's per-cycle work)."""
+    achieved = sum(gemm_flops) / (sum(gemm_ms) * 1e-3) / 1e12
+    sustained = timed_ms >= 1000.0
+    key = "bf16_tflops_sustained" if sustained else "bf16_tflops"
+    peak = peaks[key] * NOMINAL_FP4_OVER_BF16
+    out = {"bound": "tensor", "kernel": "gemm_bs_fp4 (tcgen05 kind::mxf4nvf4)", "achieved": round(achieved, 1),
+           "peak": round(peak, 1), "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+           "peak_source": f"{src}: {key} {peaks[key]} x nominal FP4/BF16 ratio {NOMINAL_FP4_OVER_BF16} "
+                          f"({'sustained: timed region >= 1 s' if sustained else 'burst: timed region < 1 s'})",
+           "frac_of_nominal_9pf": round(achieved / 9000.0, 4)}
+    mhz = clocks.get("sm_mhz")
+    if mhz:
+        per_cycle = achieved * 1e12 / (sms * mhz * 1e6)
+        out["clock_normalised"] = {
+            "sm_mhz_median": mhz, "flop_per_sm_cycle": round(per_cycle, 1),
+            "fp4_mma_flop_per_sm_cycle": FP4_FLOP_PER_SM_CYCLE, "frac": round(per_cycle / FP4_FLOP_PER_SM_CYCLE, 4),
+            "gemm_ms_x_mhz": round(sum(gemm_ms) * mhz, 1)}
+    return out
 
 
 # ---------------------------------------------------------------------------
@@ -188,33 +224,29 @@ def run_ours(args, rank, world, local_rank):
     dy_amax = torch.empty((2,), dtype=torch.float32, device=dev)
 
     def step(ev=None):
-        # ev: list of (start, end) event pairs per kernel group, or None
+        # ev: per kernel group (6 quantize calls, 3 GEMMs) a (start, end)
+        # event pair or None; ev itself may be None
+        def mark(j, k):
+            if ev is not None and ev[j] is not None:
+                ev[j][k].record(stream)
         for i, (t, fmt, rnd, had, axis, sd) in enumerate(ops):
-            if ev is not None:
-                ev[i][0].record(stream)
+            mark(i, 0)
             if i in (2, 4):
                 quantize_dy(Q, dY, c, ops, qs, i, fused_dy_amax, dual_dy, dy_amax, ws, stream)
             else:
                 Q.quantize(t, fmt, rnd, had, axis, sd, out=qs[i], workspace=ws, stream=stream)
-            if ev is not None:
-                ev[i][1].record(stream)
+            mark(i, 1)
             if i == 1:
-                if ev is not None:
-                    ev[6][0].record(stream)
+                mark(6, 0)
                 Q.gemm(qs[0], qs[1], torch.bfloat16, out=Y, stream=stream)
-                if ev is not None:
-                    ev[6][1].record(stream)
+                mark(6, 1)
             if i == 3:
-                if ev is not None:
-                    ev[7][0].record(stream)
+                mark(7, 0)
                 Q.gemm(qs[2], qs[3], torch.bfloat16, out=dX, stream=stream)
-                if ev is not None:
-                    ev[7][1].record(stream)
-        if ev is not None:
-            ev[8][0].record(stream)
+                mark(7, 1)
+        mark(8, 0)
         Q.gemm(qs[4], qs[5], torch.float32, out=dW, stream=stream)
-        if ev is not None:
-            ev[8][1].record(stream)
+        mark(8, 1)
 
     def barrier():
         if world > 1:
@@ -249,9 +281,46 @@ def run_ours(args, rank, world, local_rank):
     value = world * flops_step / (ms_step * 1e-3) / 1e12
 
     peaks, src = measured_peaks()
-    fp4_peak = peaks["bf16_tflops_sustained"] * NOMINAL_FP4_OVER_BF16
-    gemm_achieved = sum(gemm_flops) / (sum(gemm_ms) * 1e-3) / 1e12
+    clocks = clk.summary()
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    roofline = gemm_roofline(gemm_flops, gemm_ms, peaks, src, clocks, sms, ms)
     traffic = measured_gemm_traffic()
+    roofline.update({
+        "traffic": None if traffic is None else int(statistics.mean(traffic.values())),
+        "traffic_unit": "DRAM bytes per GEMM launch (mean of Fprop, Dgrad, Wgrad; ncu dram__bytes_read.sum + "
+                        "dram__bytes_write.sum, profiles/gemm_traffic.json; null when the GEMM sources changed since)",
+        "traffic_per_gemm": traffic,
+        "algorithmic_bytes_per_gemm": {
+            "fprop": (M + N) * (K // 2 + K // 16) + M * N * 2,
+            "dgrad": (M + K) * (N // 2 + N // 16) + M * K * 2,
+            "wgrad": (N + K) * (M // 2 + M // 16) + N * K * 4},
+        "per_gemm_ms": {"fprop": round(gemm_ms[0], 4), "dgrad": round(gemm_ms[1], 4), "wgrad": round(gemm_ms[2], 4)}})
+
+    # the same step run for about two seconds (the GPU settles at its power cap):
+    # step time and GEMM roofline against the sustained peak, with its clocks
+    n_sus = 0 if args.no_sustained else max(20, int(2000.0 / max(ms_step, 0.05)))
+    sevs = [[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)] for _ in range(3 * n_sus)]
+    with ClockSampler(local_rank) as sclk:
+        barrier()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        for i in range(n_sus):
+            step([None] * 6 + [sevs[3 * i], sevs[3 * i + 1], sevs[3 * i + 2]])
+        s1.record(stream)
+        barrier()
+    Q.status()
+    sus_ms = max_over_ranks(s0.elapsed_time(s1), world, dev)
+    sustained = None
+    if n_sus:
+        sus_gemm = [statistics.mean(sevs[3 * i + g][0].elapsed_time(sevs[3 * i + g][1]) for i in range(n_sus))
+                    for g in range(3)]
+        sus_clocks = sclk.summary()
+        sus_roof = gemm_roofline(gemm_flops, sus_gemm, peaks, src, sus_clocks, sms, sus_ms)
+        sustained = {"steps": n_sus, "seconds": round(sus_ms / 1e3, 3), "ms_per_step": round(sus_ms / n_sus, 4),
+                     "TFLOP/s": round(world * flops_step / (sus_ms / n_sus * 1e-3) / 1e12, 2),
+                     "gemm_ms": {"fprop": round(sus_gemm[0], 4), "dgrad": round(sus_gemm[1], 4),
+                                 "wgrad": round(sus_gemm[2], 4)},
+                     "roofline": sus_roof, "clocks": sus_clocks}
 
     # Wgrad accumulating into an fp32 main gradient (dW += dY^T X) on the step's operands
     def wgrad(acc):
@@ -271,19 +340,30 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize()
         wg[acc] = e0.elapsed_time(e1) / 10
     Q.status()
-    # Fprop whose epilogue also writes the MXFP4 operand of a next layer (Y along N)
+    # Fprop whose epilogue also writes the MXFP4 operand of a next layer (Y along
+    # N), or the NVFP4 tensor amax of Y that the next layer's quantization needs
     qy = Q.empty_qtensor(Q.MXFP4, M, N, dev)
+    qyn = Q.empty_qtensor(Q.NVFP4, M, N, dev)
+    y_amax = torch.empty((1,), dtype=torch.float32, device=dev)
     qseed = Q.make_seed(seed.rot, seed.sr, 3, 6)
+    nh_next = rec.fprop.had  # the next layer's Fprop rotation of its input (Y)
     fq = {}
-    for kind in ("gemm", "fused", "separate", "gemm", "fused", "separate"):
+    for kind in ("gemm", "fused", "separate", "nv_fused", "nv_separate") * 2:
         def fprop_q():
             if kind == "gemm":
                 Q.gemm(qs[0], qs[1], torch.bfloat16, out=Y, stream=stream)
             elif kind == "fused":
                 Q.gemm_quantize(qs[0], qs[1], Q.HAD_NONE, qseed, out=Y, qout=qy, stream=stream)
-            else:
+            elif kind == "separate":
                 Q.gemm(qs[0], qs[1], torch.bfloat16, out=Y, stream=stream)
                 Q.quantize(Y, Q.MXFP4, Q.RTN, Q.HAD_NONE, Q.ROW, qseed, out=qy, stream=stream)
+            elif kind == "nv_fused":
+                Q.gemm_amax(qs[0], qs[1], nh_next, qseed, out=Y, amax=y_amax, workspace=ws, stream=stream)
+                Q.quantize(Y, Q.NVFP4, Q.RTN, nh_next, Q.ROW, qseed, amax_in=y_amax, out=qyn, workspace=ws,
+                           stream=stream)
+            else:
+                Q.gemm(qs[0], qs[1], torch.bfloat16, out=Y, stream=stream)
+                Q.quantize(Y, Q.NVFP4, Q.RTN, nh_next, Q.ROW, qseed, out=qyn, workspace=ws, stream=stream)
         for _ in range(2):
             fprop_q()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -296,8 +376,13 @@ def run_ours(args, rank, world, local_rank):
     Q.status()
     fprop_quant = {"gemm_ms": round(fq["gemm"], 4), "fused_ms": round(fq["fused"], 4),
                    "gemm_then_quantize_ms": round(fq["separate"], 4),
-                   "what": f"Fprop Y[{M}x{N}] bf16 alone, with its MXFP4 copy along N from the epilogue "
-                           "(qfp4_gemm_quantize), and followed by a separate row quantization of Y; 10 launches each"}
+                   "nvfp4_gemm_amax_then_quantize_ms": round(fq["nv_fused"], 4),
+                   "nvfp4_gemm_then_quantize_ms": round(fq["nv_separate"], 4),
+                   "what": f"Fprop Y[{M}x{N}] bf16 alone; with its MXFP4 copy along N from the epilogue "
+                           "(qfp4_gemm_quantize) vs followed by a separate row quantization of Y; and the next "
+                           "layer's NVFP4 quantization of Y (round to nearest, its Fprop Hadamard) with the tensor "
+                           "amax from the GEMM's epilogue (qfp4_gemm_amax, quantize with amax_in) vs quantize with "
+                           "its own amax pass over Y; 10 launches each"}
     wgrad_acc = {"store_ms": round(wg[False], 4), "accumulate_ms": round(wg[True], 4),
                  "accumulate_TFLOP/s": round(gemm_flops[2] / (wg[True] * 1e-3) / 1e12, 1),
                  "what": "Wgrad of the step, dW = dY^T X vs dW += dY^T X (TMA reduce-add epilogue), fp32 dW "
@@ -309,7 +394,7 @@ def run_ours(args, rank, world, local_rank):
     quant["large"] = quant_large(Q, dY, stream, peaks)
 
     # the other configurations of the MLP shapes (not part of the headline value)
-    layers = more_layers(Q, inputs, X, W, dY, seed, stream, dev)
+    layers = more_layers(Q, inputs, X, W, dY, seed, stream, dev, roofline["peak"])
 
     # MXFP4 variants on the Wgrad product of this layer (quality, not speed)
     study = mxfp4_wgrad_study(Q, X, dY, stream)
@@ -327,21 +412,8 @@ def run_ours(args, rank, world, local_rank):
                    "M": M, "N": N, "K": K, "recipe": RECIPE,
                    "l2": "inputs larger than L2 (dY 940 MB, W 235 MB, X 134 MB); no flush between steps",
                    "parallelism": f"replicas x{world}"},
-        "roofline": {"bound": "tensor", "kernel": "gemm_bs_fp4 (tcgen05 kind::mxf4nvf4)",
-                     "achieved": round(gemm_achieved, 1),
-                     "peak": round(fp4_peak, 1), "unit": "TFLOP/s", "frac": round(gemm_achieved / fp4_peak, 4),
-                     "traffic": None if traffic is None else int(statistics.mean(traffic.values())),
-                     "traffic_unit": "DRAM bytes per GEMM launch (mean of Fprop, Dgrad, Wgrad; ncu, "
-                                     "profiles/gemm_bs_fp4_mlp_up.md)",
-                     "traffic_per_gemm": traffic,
-                     "algorithmic_bytes_per_gemm": {
-                         "fprop": (M + N) * (K // 2 + K // 16) + M * N * 2,
-                         "dgrad": (M + K) * (N // 2 + N // 16) + M * K * 2,
-                         "wgrad": (N + K) * (M // 2 + M // 16) + N * K * 4},
-                     "peak_source": f"{src}: bf16_tflops_sustained {peaks['bf16_tflops_sustained']} x nominal FP4/BF16 "
-                                    f"ratio {NOMINAL_FP4_OVER_BF16}",
-                     "per_gemm_ms": {"fprop": round(gemm_ms[0], 4), "dgrad": round(gemm_ms[1], 4),
-                                     "wgrad": round(gemm_ms[2], 4)}},
+        "roofline": roofline,
+        "sustained": sustained,
         "step_breakdown_ms": {"quantize": [round(v, 4) for v in quant_ms], "gemm": [round(v, 4) for v in gemm_ms]},
         "quantize": quant,
         "layers": layers,
@@ -351,7 +423,7 @@ def run_ours(args, rank, world, local_rank):
         "linear_api_ms_per_step": round(api_ms, 4),
         "e2e": e2e,
         "gpu_launches": launches,
-        "clocks": clk.summary(),
+        "clocks": clocks,
     }
     return out
 
@@ -449,80 +521,105 @@ def layer_step(Q, X, W, dY, rec, seed, steps, stream, dev):
             "gemm_TFLOP/s": round(3 * flops / (sum(gemm_ms) * 1e-3) / 1e12, 1)}
 
 
-def more_layers(Q, inputs, X, W, dY, seed, stream, dev):
-    """The other arm of the MLP up/gate configuration (MXFP4, deterministic
-    32x32 Hadamard on Wgrad) and the MLP down layer at 16384 tokens with the
-    Quartet II and the per-element SR NVFP4 recipes."""
+def more_layers(Q, inputs, X, W, dY, seed, stream, dev, fp4_peak):
+    """The other configurations of the Llama-3.1-8B layer shapes (not part of
+    the headline value): the MLP up/gate layer with the AMD MXFP4 recipe
+    (deterministic 32x32 Hadamard on Wgrad), the attention QKV projection with
+    the Quartet II NVFP4 recipe, and the MLP down layer with the Quartet II and
+    the per-element SR NVFP4 recipes at 2048 ... 32768 tokens. Each entry: ms
+    per fwd+bwd, TFLOP/s, per-GEMM ms and the GEMMs' fraction of the FP4 peak."""
     import torch
-    out = {"mlp_up_AMD_MXFP4_H": layer_step(Q, X, W, dY, Q.recipe("AMD_MXFP4_H"), seed, 10, stream, dev)}
-    wl = inputs.workload("mlp_down", device=dev, M=16384)
-    for rec in ("QUARTET2_NVFP4", "NVIDIA_NVFP4"):
-        out["mlp_down_" + rec] = layer_step(Q, wl["X"], wl["W"], wl["dY"], Q.recipe(rec), seed, 10, stream, dev)
-    out["workloads"] = {"mlp_up": "X[16384x4096] W[28672x4096] dY[16384x28672]",
-                        "mlp_down": "X[16384x14336] = SiLU(N(0,1))*N(0,1), W[4096x14336] N(0,0.02), "
-                                    "dY[16384x4096] N(0,1e-3)"}
+
+    def entry(r):
+        r["gemm_frac_of_peak"] = round(r["gemm_TFLOP/s"] / fp4_peak, 4)
+        return r
+    out = {"mlp_up_AMD_MXFP4_H": entry(layer_step(Q, X, W, dY, Q.recipe("AMD_MXFP4_H"), seed, 10, stream, dev))}
+    wl = inputs.workload("qkv", device=dev)
+    out["qkv_QUARTET2_NVFP4"] = entry(layer_step(Q, wl["X"], wl["W"], wl["dY"], Q.recipe("QUARTET2_NVFP4"), seed, 10,
+                                                 stream, dev))
     del wl
-    torch.cuda.empty_cache()
+    for M in (2048, 4096, 8192, 16384, 32768):
+        wl = inputs.workload("mlp_down", device=dev, M=M)
+        for rec in ("QUARTET2_NVFP4", "NVIDIA_NVFP4"):
+            out[f"mlp_down_M{M}_{rec}"] = entry(layer_step(Q, wl["X"], wl["W"], wl["dY"], Q.recipe(rec), seed, 10,
+                                                           stream, dev))
+        del wl
+        torch.cuda.empty_cache()
+    out["workloads"] = {"mlp_up": "X[16384x4096] W[28672x4096] dY[16384x28672]",
+                        "qkv": "X[8192x4096] N(0,1)+0.1% x50 outliers, W[6144x4096] N(0,0.02), dY[8192x6144] N(0,1e-3)",
+                        "mlp_down": "X[Mx14336] = SiLU(N(0,1))*N(0,1), W[4096x14336] N(0,0.02), dY[Mx4096] N(0,1e-3)"}
+    out["peak_TFLOP/s"] = round(fp4_peak, 1)
     return out
 
 
+SWEEP_FMTS = (("nvfp4", 0), ("mxfp4", 1), ("mxfp4ru", 2))          # Q.NVFP4, Q.MXFP4, Q.MXFP4_RU
+SWEEP_HADS = (("none", 0), ("det16", 1), ("det32", 2), ("rand16", 3), ("rand32", 4))
+SWEEP_RNDS = (("rtn", 0), ("sr", 1), ("q2", 2))
+SWEEP_AXES = (("row", 0), ("col", 1))
+
+
+def sweep_cases():
+    """Every (format, Hadamard, rounding, axis) case of the quantizer sweep:
+    NVFP4 and MXFP4 (60 cases) and the round-up MXFP4 variant (30 more)."""
+    return [(f"{fn}_{rn}_{hn}_{an}", f, r, h, a) for fn, f in SWEEP_FMTS for hn, h in SWEEP_HADS
+            for rn, r in SWEEP_RNDS for an, a in SWEEP_AXES]
+
+
 def quant_sweep(Q, inputs, dev, stream, peaks):
-    """The quantizer-sweep tensor [8192x4096]: GB/s of algorithmic bytes
-    (2 B read + 0.5 B codes + scale bytes per element; the NVFP4 amax pass
-    counted separately at 2 B/elem), L2 flushed before every launch."""
+    """The quantizer-sweep tensor [8192x4096] (67 MB, fits in L2): GB/s of
+    algorithmic bytes (2 B read + 0.5 B codes + 1/16 (NVFP4) or 1/32 (MXFP4)
+    B scales per element; the NVFP4 amax pass, counted separately at 2 B per
+    element, is taken before the timed launch) for every case. Before every
+    launch L2 is evicted by reading a 256 MiB buffer (a reduction that writes
+    nothing back to it), so the launch reads its input from DRAM and finds no
+    dirty lines left for it to write back."""
     import torch
     T = inputs.workload("sweep", device=dev)["T"]
     R, C = T.shape
-    flush = torch.empty((256 << 20,), dtype=torch.uint8, device=dev)
+    flush = torch.ones((64 << 20,), dtype=torch.float32, device=dev)  # 256 MiB
     ws = torch.empty((Q.quantize_workspace_bytes(),), dtype=torch.uint8, device=dev)
-    amax = Q.amax(T, Q.HAD_NONE, Q.ROW, workspace=ws, stream=stream)
+    seed = Q.make_seed(5, 6, 1, 2)
     res = {}
-    cases = [("nvfp4_rtn_none_row", Q.NVFP4, Q.RTN, Q.HAD_NONE, Q.ROW),
-             ("nvfp4_q2_rand16_row", Q.NVFP4, Q.QUARTET2, Q.HAD_RAND16, Q.ROW),
-             ("nvfp4_sr_rand16_row", Q.NVFP4, Q.SR, Q.HAD_RAND16, Q.ROW),
-             ("nvfp4_q2_rand16_col", Q.NVFP4, Q.QUARTET2, Q.HAD_RAND16, Q.COL),
-             ("mxfp4_rtn_det32_col", Q.MXFP4, Q.RTN, Q.HAD_DET32, Q.COL),
-             ("mxfp4_rtn_none_row", Q.MXFP4, Q.RTN, Q.HAD_NONE, Q.ROW),
-             ("mxfp4ru_rtn_det32_col", Q.MXFP4_RU, Q.RTN, Q.HAD_DET32, Q.COL)]
-    seed = Q.make_seed(5, 6)
-    for name, fmt, rnd, had, axis in cases:
+
+    def timed(fn, n=6):
+        times = []
+        for it in range(n + 2):
+            flush.sum()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            if it >= 2:
+                times.append(e0.elapsed_time(e1))
+        return statistics.median(times)
+
+    for name, fmt, rnd, had, axis in sweep_cases():
         rows, k = (R, C) if axis == Q.ROW else (C, R)
         q = Q.empty_qtensor(fmt, rows, k, dev)
         # a pre-computed amax isolates the one-pass quantizer kernel
         am = Q.amax(T, had, axis, seed, workspace=ws, stream=stream) if fmt == Q.NVFP4 else None
-        times = []
-        for it in range(8):
-            flush.zero_()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            Q.quantize(T, fmt, rnd, had, axis, seed, amax_in=am, out=q, workspace=ws, stream=stream)
-            e1.record(stream)
-            torch.cuda.synchronize()
-            if it >= 3:
-                times.append(e0.elapsed_time(e1))
-        ms = statistics.median(times)
+        ms = timed(lambda: Q.quantize(T, fmt, rnd, had, axis, seed, amax_in=am, out=q, workspace=ws, stream=stream))
         byts = R * C * (2 + 0.5 + (1 / 16 if fmt == Q.NVFP4 else 1 / 32))
         gbs = byts / (ms * 1e-3) / 1e9
         res[name] = {"ms": round(ms, 4), "GB/s": round(gbs, 1), "frac_of_measured_hbm": round(gbs / peaks["hbm_gbs"], 3)}
-    # the amax pass alone
-    times = []
-    for it in range(8):
-        flush.zero_()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        Q.amax(T, Q.HAD_RAND16, Q.ROW, seed, out=amax, workspace=ws, stream=stream)
-        e1.record(stream)
-        torch.cuda.synchronize()
-        if it >= 3:
-            times.append(e0.elapsed_time(e1))
-    ms = statistics.median(times)
-    gbs = R * C * 2 / (ms * 1e-3) / 1e9
-    res["amax_rand16_row"] = {"ms": round(ms, 4), "GB/s": round(gbs, 1),
-                              "frac_of_measured_hbm": round(gbs / peaks["hbm_gbs"], 3)}
+        del q
+    am = torch.empty((1,), dtype=torch.float32, device=dev)
+    for hn, had in (("none", Q.HAD_NONE), ("rand16", Q.HAD_RAND16), ("rand32", Q.HAD_RAND32)):
+        for an, axis in SWEEP_AXES:
+            ms = timed(lambda: Q.amax(T, had, axis, seed, out=am, workspace=ws, stream=stream))
+            gbs = R * C * 2 / (ms * 1e-3) / 1e9
+            res[f"amax_{hn}_{an}"] = {"ms": round(ms, 4), "GB/s": round(gbs, 1),
+                                      "frac_of_measured_hbm": round(gbs / peaks["hbm_gbs"], 3)}
     Q.status()
+    summary = {}
+    for rn, _ in SWEEP_RNDS:
+        fr = [v["frac_of_measured_hbm"] for k, v in res.items() if f"_{rn}_" in k]
+        summary[rn] = {"min": min(fr), "median": statistics.median(fr), "max": max(fr), "cases": len(fr)}
     return {"workload": "quantizer sweep tensor [8192x4096] bf16, Student-t(3)*0.02*LogNormal(0,1) column gains",
             "bytes_per_elem": "2 read + 0.5 codes + 1/16 (NVFP4) or 1/32 (MXFP4) scales; amax pass 2 read",
-            "l2": "256 MiB buffer written before every launch", "unit": "GB/s", "cases": res}
+            "l2": "a 256 MiB buffer read (summed) before every launch: L2 evicted, no dirty lines left",
+            "unit": "GB/s", "frac_summary_by_rounding": summary, "cases": res}
 
 
 def quant_large(Q, T, stream, peaks):
@@ -724,6 +821,30 @@ def cpu_baseline_obj(m_rows=256, n_rows=16384):
                       f"the MLP up/gate workload: six quantizations (fp32 decisions) + three fp64 GEMMs; {dt:.1f} s"}
 
 
+def cpu_quantize_modes():
+    """The oracle's quantizer (plain C, OpenMP over rows) on the whole quantizer
+    sweep tensor [8192 x 4096], once per mode: NVFP4 and MXFP4 x Hadamard
+    none / det16 / det32 / rand16 / rand32 x RTN / SR / Quartet II x row /
+    column (60 modes; the NVFP4 amax pass included). GB/s of the same
+    algorithmic bytes as the GPU sweep."""
+    import oracle as O
+    from fp4_precision_b200 import inputs
+    T = inputs.workload("sweep", device="cpu")["T"]
+    R, C = T.shape
+    res = {}
+    t_all = time.perf_counter()
+    for name, fmt, rnd, had, axis in sweep_cases():
+        if fmt == 2:  # the round-up variant costs what MXFP4 does
+            continue
+        t0 = time.perf_counter()
+        O.quantize(T, fmt, rnd, had, axis, 1, 0, 2, 0)
+        dt = time.perf_counter() - t0
+        byts = R * C * (2 + 0.5 + (1 / 16 if fmt == 0 else 1 / 32))
+        res[name] = {"s": round(dt, 3), "GB/s": round(byts / dt / 1e9, 4)}
+    return {"kind": "oracle", "cores": os.cpu_count(), "unit": "GB/s", "seconds": round(time.perf_counter() - t_all, 1),
+            "sample": "the whole quantizer sweep tensor [8192x4096] per mode (60 modes)", "cases": res}
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return None
@@ -820,6 +941,7 @@ def main():
     out = run_ours(args, rank, world, local_rank)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline_obj()
+        out["cpu_baseline_quantize"] = cpu_quantize_modes()
     if world > 1:
         import torch.distributed as dist
         dist.barrier()

@@ -1,7 +1,9 @@
 """Host-side logic of bench.py, without a GPU: how the timed step quantizes dY
-for each recipe (the policy qfp4_linear_bwd follows), and when the committed
-DRAM-traffic figure of the GEMM may be reported."""
+for each recipe (the policy qfp4_linear_bwd follows), when the committed
+DRAM-traffic figure of the GEMM may be reported, the roofline arithmetic and
+the quantizer sweep's case list."""
 import hashlib
+import json
 import os
 import shutil
 
@@ -40,11 +42,6 @@ def test_dy_plan_of_custom_recipes():
     assert bench.dy_plan(Q, c, 16384 + 32) == (True, False)  # tokens not a multiple of 64
 
 
-def _profile_text(gemm_hash, header_hash):
-    return ("traffic_bytes_per_launch fprop=100 dgrad=200 wgrad=300\n"
-            f"gemm_source_sha256 {gemm_hash}\ndevice_header_sha256 {header_hash}\n")
-
-
 def test_traffic_is_reported_only_for_the_profiled_sources(monkeypatch):
     root = helpers.scratch_dir("bench_root_")
     try:
@@ -56,15 +53,41 @@ def test_traffic_is_reported_only_for_the_profiled_sources(monkeypatch):
                 fh.write(text)
         h = {f: hashlib.sha256(open(os.path.join(csrc, f), "rb").read()).hexdigest()
              for f in ("gemm_sm100.cu", "qfp4_device.cuh")}
-        prof = os.path.join(root, "profiles", "gemm_bs_fp4_mlp_up.md")
-        with open(prof, "w") as fh:
-            fh.write(_profile_text(h["gemm_sm100.cu"], h["qfp4_device.cuh"]))
+        rec = os.path.join(root, "profiles", "gemm_traffic.json")
+        with open(rec, "w") as fh:
+            json.dump({"traffic_bytes_per_launch": {"fprop": 100, "dgrad": 200, "wgrad": 300},
+                       "source_sha256": h}, fh)
         monkeypatch.setattr(bench, "ROOT", root)
         assert bench.measured_gemm_traffic() == {"fprop": 100, "dgrad": 200, "wgrad": 300}
         with open(os.path.join(csrc, "qfp4_device.cuh"), "a") as fh:
             fh.write("// changed\n")
         assert bench.measured_gemm_traffic() is None
-        os.remove(prof)
+        os.remove(rec)
         assert bench.measured_gemm_traffic() is None
     finally:
         shutil.rmtree(root, ignore_errors=True)
+
+
+def test_roofline_follows_the_timed_region_and_the_clock():
+    """The GEMM roofline uses the burst bf16 peak (x 4) for a short timed
+    region and the sustained one for a region of a second or more; the
+    clock-normalised fraction is the flops per SM and sampled cycle over the
+    FP4 MMA's per-cycle work."""
+    peaks = {"hbm_gbs": 6000.0, "bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0}
+    flops = [1e12, 1e12, 1e12]
+    ms = [0.5, 0.5, 0.5]  # 2000 TFLOP/s
+    clocks = {"sm_mhz": 1500.0}
+    short = bench.gemm_roofline(flops, ms, peaks, "measured", clocks, 148, 100.0)
+    assert short["achieved"] == 2000.0 and short["peak"] == 6400.0 and short["frac"] == 0.3125
+    long = bench.gemm_roofline(flops, ms, peaks, "measured", clocks, 148, 2500.0)
+    assert long["peak"] == 5600.0
+    per_cycle = 2000e12 / (148 * 1500e6)
+    assert abs(long["clock_normalised"]["frac"] - per_cycle / bench.FP4_FLOP_PER_SM_CYCLE) < 1e-4
+    assert bench.FP4_FLOP_PER_SM_CYCLE == 32768
+    assert "clock_normalised" not in bench.gemm_roofline(flops, ms, peaks, "measured", {"sm_mhz": None}, 148, 1.0)
+
+
+def test_sweep_covers_every_case():
+    cases = bench.sweep_cases()
+    assert len(cases) == 90 and len({c[0] for c in cases}) == 90
+    assert sum(1 for c in cases if c[1] != 2) == 60  # NVFP4 and MXFP4; the rest are the round-up variant
