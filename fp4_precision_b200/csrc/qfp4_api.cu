@@ -709,13 +709,22 @@ int amax_rowcol_impl(const void* x, int64_t R, int64_t C, int64_t ld, int32_t ha
         p.rows = gc.rows; p.k = gc.k;
         p.signs = signs_col;
         p.signs_row = signs_row;
-        const int n = amax_partial_count(sms, quant_tiles(QFP4_AXIS_COL, gc.rows, gc.k, 16));
+        // over 64-row bands when R allows it (both orientations packed), else
+        // the group-walking column kernel
+        const bool bands = R % 64 == 0 && col_bands_enabled();
+        const int n = amax_partial_count(
+            sms, bands ? amax_rowcol64_tiles(gc.rows, gc.k) : quant_tiles(QFP4_AXIS_COL, gc.rows, gc.k, 16));
         if (2 * n > kMaxAmaxPartials) return QFP4_ERR_WORKSPACE;
         p.amax_out = partials;
         p.amax_out_row = partials + n;
         CUtensorMap tm;
-        if ((rc = make_input_tmap(&tm, x, R, C, ld, QFP4_AXIS_COL, 16))) return rc;
-        e = launch_amax_rowcol(p, nh, &tm, n, s);
+        if (bands) {
+            if ((rc = make_col64_tmap(&tm, x, R, C, ld))) return rc;
+            e = launch_amax_rowcol64(p, nh, &tm, n, s);
+        } else {
+            if ((rc = make_input_tmap(&tm, x, R, C, ld, QFP4_AXIS_COL, 16))) return rc;
+            e = launch_amax_rowcol(p, nh, &tm, n, s);
+        }
         if (e == cudaSuccess) e = launch_reduce_max(partials, n, amax_col, s);
         if (e == cudaSuccess) e = launch_reduce_max(partials + n, n, amax_row, s);
     } else {

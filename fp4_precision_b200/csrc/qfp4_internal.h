@@ -67,6 +67,12 @@ cudaError_t launch_quant_dual(const QuantParams& p, int fmt, int rnd, int nh, in
 // column orientation's partial maxima to p.amax_out and the row orientation's
 // to p.amax_out_row (n_partials each). nh: 0 or 16.
 cudaError_t launch_amax_rowcol(const QuantParams& p, int nh, const CUtensorMap* tmap, int n_partials, cudaStream_t s);
+// The same over 64-row bands (R a multiple of 64; tmap: the 4-D band view),
+// both orientations as two packed pairs of 16-element groups per thread.
+cudaError_t launch_amax_rowcol64(const QuantParams& p, int nh, const CUtensorMap* tmap, int n_partials,
+                                 cudaStream_t s);
+// Tiles the band amax pass walks (rows, k of the column orientation).
+int64_t amax_rowcol64_tiles(int64_t rows, int64_t k);
 cudaError_t launch_reduce_max(const float* in, int n, float* out, cudaStream_t s);
 // Column-mode geometry: group G = max(block, n_h), tile = 4G rows x 128 columns.
 int col_group(int fmt_or_amax_block, int nh);

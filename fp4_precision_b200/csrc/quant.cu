@@ -153,25 +153,32 @@ __device__ __forceinline__ float nvfp4_scale_from_amax(float amax, float* tensor
     return s_enc;
 }
 
-// Reduce the CTA's amax partials (NVFP4) to s_enc; CTA 0 writes g.
+// Barrier of the compute warps only (named barrier 1): the producer warp has
+// gone ahead to issue the first loads while they set up the scales.
+__device__ __forceinline__ void bar_compute() {
+    asm volatile("bar.sync 1, %0;" ::"r"(kComputeWarps * 32) : "memory");
+}
+
+// Reduce the CTA's amax partials (NVFP4) to s_enc; CTA 0 writes g. Run by the
+// compute warps (threads 0 .. 255).
 __device__ float nvfp4_encode_scale(const QuantParams& p, float* red_smem, bool write_g) {
     float amax = 0.0f;
     if (p.amax_in != nullptr) {
         amax = __ldg(p.amax_in);
     } else {
         float m = 0.0f;
-        for (int i = threadIdx.x; i < p.n_partials; i += blockDim.x) m = fmaxf(m, __ldg(p.amax_partials + i));
+        for (int i = threadIdx.x; i < p.n_partials; i += kComputeWarps * 32) m = fmaxf(m, __ldg(p.amax_partials + i));
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
         if ((threadIdx.x & 31) == 0) red_smem[threadIdx.x >> 5] = m;
-        __syncthreads();
+        bar_compute();
         if (threadIdx.x < 32) {
-            m = threadIdx.x < (blockDim.x >> 5) ? red_smem[threadIdx.x] : 0.0f;
+            m = threadIdx.x < kComputeWarps ? red_smem[threadIdx.x] : 0.0f;
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
             if (threadIdx.x == 0) red_smem[32] = m;
         }
-        __syncthreads();
+        bar_compute();
         amax = red_smem[32];
     }
     return nvfp4_scale_from_amax(amax, p.tensor_scale, write_g);
@@ -179,11 +186,11 @@ __device__ float nvfp4_encode_scale(const QuantParams& p, float* red_smem, bool 
 
 // rtab[c] = s_enc / S(c) for every E4M3 code c the saturating conversion can
 // produce (1-126; S(0) = 0 gives 0), the same divisions as per block, once per
-// CTA. Ends with a CTA barrier.
+// CTA, by the compute warps. Ends with their barrier.
 __device__ void fill_rtab(float* rtab, float s_enc) {
-    for (int c = threadIdx.x; c < 128; c += blockDim.x)
+    for (int c = threadIdx.x; c < 128; c += kComputeWarps * 32)
         rtab[c] = (c == 0 || c == 127) ? 0.0f : __fdiv_rn(s_enc, e4m3_decode((uint32_t)c));
-    __syncthreads();
+    bar_compute();
 }
 
 // The random streams and MXFP4 exponent rule of one orientation (what the
@@ -473,13 +480,14 @@ __device__ __forceinline__ float2 tree_sum_pair(float2* s) {
 }
 
 // Per-CTA table of (s_enc / S, S) for every E4M3 code S can take (1-126; code
-// 0 gives (0, 0)), the same divisions as per block. Ends with a CTA barrier.
+// 0 gives (0, 0)), the same divisions as per block, by the compute warps. Ends
+// with their barrier.
 __device__ void fill_tab2(float2* tab, float s_enc) {
-    for (int c = threadIdx.x; c < 128; c += blockDim.x) {
+    for (int c = threadIdx.x; c < 128; c += kComputeWarps * 32) {
         const float S = e4m3_decode((uint32_t)c);
         tab[c] = (c == 0 || c == 127) ? f2(0.0f, 0.0f) : f2(__fdiv_rn(s_enc, S), S);
     }
-    __syncthreads();
+    bar_compute();
 }
 
 // Hadamard sign flips of the 8 words of a block, at bit 31 of each element:
@@ -699,19 +707,6 @@ __global__ void __launch_bounds__(kThreads, 2)
         ring_init(ring);
     }
     __syncthreads();
-    __shared__ float rtab[kPacked ? 1 : 128];
-    __shared__ float2 tab2[kPacked ? 128 : 1];
-    float s_enc = 1.0f;
-    if constexpr (!AMAX_ONLY && FMT == kNvfp4) {
-        s_enc = nvfp4_encode_scale(p, red, blockIdx.x == 0);
-        if constexpr (kPacked)
-            fill_tab2(tab2, s_enc);
-        else
-            fill_rtab(rtab, s_enc);
-    }
-    if constexpr (!AMAX_ONLY && FMT == kMxfp4) {
-        if (blockIdx.x == 0 && tid == 0) *p.tensor_scale = 1.0f;
-    }
 
     if (warp == kComputeWarps) {
         // ---------------- producer ----------------
@@ -726,6 +721,19 @@ __global__ void __launch_bounds__(kThreads, 2)
             drain_loads(ring.full, nullptr, STAGES, i);  // no load lands after this CTA exits
         }
         return;
+    }
+    __shared__ float rtab[kPacked ? 1 : 128];
+    __shared__ float2 tab2[kPacked ? 128 : 1];
+    float s_enc = 1.0f;
+    if constexpr (!AMAX_ONLY && FMT == kNvfp4) {
+        s_enc = nvfp4_encode_scale(p, red, blockIdx.x == 0);
+        if constexpr (kPacked)
+            fill_tab2(tab2, s_enc);
+        else
+            fill_rtab(rtab, s_enc);
+    }
+    if constexpr (!AMAX_ONLY && FMT == kMxfp4) {
+        if (blockIdx.x == 0 && tid == 0) *p.tensor_scale = 1.0f;
     }
 
     // ---------------- compute: thread = one row of the tile ----------------
@@ -880,15 +888,6 @@ __global__ void __launch_bounds__(kThreads, 2)
         ring_init(ring);
     }
     __syncthreads();
-    __shared__ float rtab[128];
-    float s_enc = 1.0f;
-    if constexpr (!AMAX_ONLY && FMT == kNvfp4) {
-        s_enc = nvfp4_encode_scale(p, red, blockIdx.x == 0);
-        fill_rtab(rtab, s_enc);
-    }
-    if constexpr (!AMAX_ONLY && FMT == kMxfp4) {
-        if (blockIdx.x == 0 && tid == 0) *p.tensor_scale = 1.0f;
-    }
 
     if (warp == kComputeWarps) {
         if (lane == 0) {
@@ -906,6 +905,15 @@ __global__ void __launch_bounds__(kThreads, 2)
             drain_loads(ring.full, nullptr, STAGES, i);  // no load lands after this CTA exits
         }
         return;
+    }
+    __shared__ float rtab[128];
+    float s_enc = 1.0f;
+    if constexpr (!AMAX_ONLY && FMT == kNvfp4) {
+        s_enc = nvfp4_encode_scale(p, red, blockIdx.x == 0);
+        fill_rtab(rtab, s_enc);
+    }
+    if constexpr (!AMAX_ONLY && FMT == kMxfp4) {
+        if (blockIdx.x == 0 && tid == 0) *p.tensor_scale = 1.0f;
     }
 
     const int64_t rows_pad = (p.rows + 127) / 128 * 128;
@@ -1222,6 +1230,20 @@ __global__ void __launch_bounds__(kThreads, 2)
         ring_init(ring);
     }
     __syncthreads();
+
+    if (warp == kComputeWarps) {
+        if (lane == 0) {
+            int i = 0;
+            for (TileWalk<STAGES> w(tiles_c); w.tr < tiles_r; w.next(), ++i) {
+                const int s = w.stage;
+                if (i >= STAGES && !mbar_wait(&ring.empty[s], w.phase ^ 1u)) break;
+                mbar_arrive_expect_tx(&ring.full[s], STAGE_BYTES);
+                tma_load_4d(tiles + s * STAGE_BYTES, &tmap, &ring.full[s], w.tc * TILE_COLS, 0, 4 * w.tr, 0);
+            }
+            drain_loads(ring.full, nullptr, STAGES, i);  // no load lands after this CTA exits
+        }
+        return;
+    }
     __shared__ float rtab[kPacked ? 1 : 128];
     __shared__ float2 tab2[kPacked ? 128 : 1];
     __shared__ float rtab_row[kDual && !kPackedRow ? 128 : 1];
@@ -1246,20 +1268,6 @@ __global__ void __launch_bounds__(kThreads, 2)
             *p.tensor_scale = 1.0f;
             if constexpr (kDual) *p.tensor_scale_row = 1.0f;
         }
-    }
-
-    if (warp == kComputeWarps) {
-        if (lane == 0) {
-            int i = 0;
-            for (TileWalk<STAGES> w(tiles_c); w.tr < tiles_r; w.next(), ++i) {
-                const int s = w.stage;
-                if (i >= STAGES && !mbar_wait(&ring.empty[s], w.phase ^ 1u)) break;
-                mbar_arrive_expect_tx(&ring.full[s], STAGE_BYTES);
-                tma_load_4d(tiles + s * STAGE_BYTES, &tmap, &ring.full[s], w.tc * TILE_COLS, 0, 4 * w.tr, 0);
-            }
-            drain_loads(ring.full, nullptr, STAGES, i);  // no load lands after this CTA exits
-        }
-        return;
     }
 
     const int64_t rows_pad = (p.rows + 127) / 128 * 128;
@@ -1364,6 +1372,114 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
         }
     }
+}
+
+// ===========================================================================
+// Both orientations' rotated amax over 64-row bands
+// ===========================================================================
+// The band kernel's tile (256 x-rows x 64 columns through the 4-D view) read
+// once for both tensor amaxes (the R a multiple of 64 case of
+// qfp4_amax_rowcol): thread (column c, band q) takes 64 consecutive rows of
+// column c (eight ldmatrix.trans, as the column quantizer) and shared-memory
+// row t's 64 columns (as the dual row work), each as two pairs of 16-element
+// groups with the butterflies packed across the pair. The rotation's
+// 1/sqrt(n_h) is applied once to each CTA's maxima (rounding c * y is
+// monotone in y). Zero-filled columns and rows past the tensor add nothing.
+
+// max |H D x| (no 1/sqrt(n_h)) of a 64-element unit loaded by chunks.
+template <int NH, typename Load>
+__device__ __forceinline__ float rot_amax64(Load load, const SignFlips& sf, float m) {
+#pragma unroll
+    for (int bp = 0; bp < 2; ++bp) {
+        float2 P[16];
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+            const uint4 a = load(4 * bp + c), b = load(4 * bp + 2 + c);
+            const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int wi = 4 * c + i;
+                if constexpr (NH > 0) {
+                    P[2 * wi] = f2(bf16lo_flip(wa[i], sf.lo[wi]), bf16lo_flip(wb[i], sf.lo[wi]));
+                    P[2 * wi + 1] = f2(bf16hi_flip(wa[i], sf.hi[wi]), bf16hi_flip(wb[i], sf.hi[wi]));
+                } else {
+                    P[2 * wi] = f2(bf16lo(wa[i]), bf16lo(wb[i]));
+                    P[2 * wi + 1] = f2(bf16hi(wa[i]), bf16hi(wb[i]));
+                }
+            }
+        }
+        if constexpr (NH == 16) {
+            fwht_pair_stage<1>(P);
+            fwht_pair_stage<2>(P);
+            fwht_pair_stage<4>(P);
+            fwht_pair_stage<8>(P);
+        }
+        const float2 am = abs_max_pair(P);
+        m = max3(m, am.x, am.y);
+    }
+    return m;
+}
+
+template <int NH, int STAGES>
+__global__ void __launch_bounds__(kThreads, 2)
+    amax_rowcol64_kernel(const __grid_constant__ CUtensorMap tmap, const QuantParams p) {
+    static_assert(NH == 0 || NH == 16, "16-element groups");
+    constexpr int TILE_ROWS = 256, TILE_COLS = 64;
+    constexpr int STAGE_BYTES = TILE_ROWS * TILE_COLS * 2;  // 32 KiB
+    extern __shared__ __align__(1024) uint8_t dyn_smem[];
+    uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
+    __shared__ Ring<STAGES> ring;
+    __shared__ float red[33];
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int tiles_c = (int)((p.rows + TILE_COLS - 1) / TILE_COLS);  // x columns
+    const int tiles_r = (int)((p.k + TILE_ROWS - 1) / TILE_ROWS);     // x rows
+    if (tid == 0) {
+        prefetch_tmap(&tmap);
+        ring_init(ring);
+    }
+    __syncthreads();
+    if (warp == kComputeWarps) {
+        if (lane == 0) {
+            int i = 0;
+            for (TileWalk<STAGES> w(tiles_c); w.tr < tiles_r; w.next(), ++i) {
+                const int s = w.stage;
+                if (i >= STAGES && !mbar_wait(&ring.empty[s], w.phase ^ 1u)) break;
+                mbar_arrive_expect_tx(&ring.full[s], STAGE_BYTES);
+                tma_load_4d(tiles + s * STAGE_BYTES, &tmap, &ring.full[s], w.tc * TILE_COLS, 0, 4 * w.tr, 0);
+            }
+            drain_loads(ring.full, nullptr, STAGES, i);  // no load lands after this CTA exits
+        }
+        return;
+    }
+    const SignFlips sf_col(NH > 0 ? p.signs : 0u), sf_row(NH > 0 ? p.signs_row : 0u);
+    // ldmatrix address of instruction n: lm_base + 4096 n (smem row lane + 32 n)
+    const uint32_t lm_base = (uint32_t)lane * 128u + ((uint32_t)(warp ^ (lane & 7)) << 4);
+    const uint32_t row_off = (uint32_t)tid * 128u + ((uint32_t)(tid & 7) << 4);
+    float m_col = 0.0f, m_row = 0.0f;
+    for (TileWalk<STAGES> w(tiles_c); w.tr < tiles_r; w.next()) {
+        const int s = w.stage;
+        if (!mbar_wait(&ring.full[s], w.phase)) break;
+        const uint32_t stage = smem_u32(tiles) + (uint32_t)(s * STAGE_BYTES);
+        auto load_col = [&](int n) {
+            uint4 v;
+            asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                         : "r"(stage + lm_base + (uint32_t)(n * 4096)));
+            return v;
+        };
+        m_col = rot_amax64<NH>(load_col, sf_col, m_col);
+        auto load_row = [&](int c) { return lds128((stage + row_off) ^ ((uint32_t)c << 4)); };
+        m_row = rot_amax64<NH>(load_row, sf_row, m_row);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ring.empty[s]);
+    }
+    if constexpr (NH > 0) {
+        m_col = __fmul_rn(m_col, had_norm<NH>());  // c * max |y| = max |c * y|
+        m_row = __fmul_rn(m_row, had_norm<NH>());
+    }
+    write_partial(m_col, red, p.amax_out);
+    write_partial(m_row, red + 16, p.amax_out_row);
 }
 
 int g_sm_count = 0;
@@ -1506,6 +1622,16 @@ cudaError_t launch_quant_dual(const QuantParams& p, int fmt, int rnd, int nh, in
     if (rnd == kSr) return dispatch_dual<kMxfp4, kSr>(p, nh, nh_row, tmap, s);
     return dispatch_dual<kMxfp4, kQuartet2>(p, nh, nh_row, tmap, s);
 }
+
+cudaError_t launch_amax_rowcol64(const QuantParams& p, int nh, const CUtensorMap* tmap, int n_partials,
+                                 cudaStream_t s) {
+    constexpr int S = 3;
+    const int smem = S * 256 * 64 * 2 + 1024;
+    if (nh == 16) return launch_persistent(amax_rowcol64_kernel<16, S>, n_partials, smem, *tmap, p, s);
+    return launch_persistent(amax_rowcol64_kernel<0, S>, n_partials, smem, *tmap, p, s);
+}
+
+int64_t amax_rowcol64_tiles(int64_t rows, int64_t k) { return ((rows + 63) / 64) * ((k + 255) / 256); }
 
 cudaError_t launch_amax_rowcol(const QuantParams& p, int nh, const CUtensorMap* tmap, int n_partials,
                                cudaStream_t s) {
