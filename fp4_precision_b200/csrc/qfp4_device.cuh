@@ -135,17 +135,17 @@ __device__ __forceinline__ float e4m3_decode(uint32_t code) {
 // mantissa bits rebased (bias 127 -> 7), and (t - lo) / gap is exactly the
 // cut-off 20 mantissa bits over 2^20, so the comparison is an integer one:
 // (w >> 8) < (those 20 bits) * 16. Below 2^-6 (subnormal E4M3, gap 2^-9):
-// t * 2^9 split into integer code and fraction.
+// t * 2^9 split into integer code and fraction. Both candidates are formed
+// and the right one selected (no branches: both are cheap and a branch costs
+// more in the issue-bound quantizers).
 __device__ __forceinline__ uint32_t e4m3_sr(float t, uint32_t w) {
-    if (!(t < 448.0f)) return 0x7Eu;
-    if (t >= 0x1p-6f) {
-        const uint32_t b = __float_as_uint(t);
-        const uint32_t lo = (b >> 20) - (120u << 3);
-        return lo + ((w >> 8) < ((b & 0xFFFFFu) << 4) ? 1u : 0u);
-    }
+    const uint32_t b = __float_as_uint(t);
+    const uint32_t normal = ((b >> 20) - (120u << 3)) + ((w >> 8) < ((b & 0xFFFFFu) << 4) ? 1u : 0u);
     const float x = t * 512.0f;  // exact
     const float fl = floorf(x);
-    return (uint32_t)fl + (uniform24(w) < x - fl ? 1u : 0u);
+    const uint32_t sub = (uint32_t)fl + (uniform24(w) < x - fl ? 1u : 0u);
+    const uint32_t c = t >= 0x1p-6f ? normal : sub;
+    return t < 448.0f ? c : 0x7Eu;
 }
 
 // floor(log2(a)) of a positive finite fp32, exact (subnormals included).
