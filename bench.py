@@ -223,29 +223,30 @@ def run_ours(args, rank, world, local_rank):
     fused_dy_amax, dual_dy = dy_plan(Q, c, M)
     dy_amax = torch.empty((2,), dtype=torch.float32, device=dev)
 
-    def step(ev=None):
+    def step(ev=None, st=None):
+        st = stream if st is None else st
         # ev: per kernel group (6 quantize calls, 3 GEMMs) a (start, end)
         # event pair or None; ev itself may be None
         def mark(j, k):
             if ev is not None and ev[j] is not None:
-                ev[j][k].record(stream)
+                ev[j][k].record(st)
         for i, (t, fmt, rnd, had, axis, sd) in enumerate(ops):
             mark(i, 0)
             if i in (2, 4):
-                quantize_dy(Q, dY, c, ops, qs, i, fused_dy_amax, dual_dy, dy_amax, ws, stream)
+                quantize_dy(Q, dY, c, ops, qs, i, fused_dy_amax, dual_dy, dy_amax, ws, st)
             else:
-                Q.quantize(t, fmt, rnd, had, axis, sd, out=qs[i], workspace=ws, stream=stream)
+                Q.quantize(t, fmt, rnd, had, axis, sd, out=qs[i], workspace=ws, stream=st)
             mark(i, 1)
             if i == 1:
                 mark(6, 0)
-                Q.gemm(qs[0], qs[1], torch.bfloat16, out=Y, stream=stream)
+                Q.gemm(qs[0], qs[1], torch.bfloat16, out=Y, stream=st)
                 mark(6, 1)
             if i == 3:
                 mark(7, 0)
-                Q.gemm(qs[2], qs[3], torch.bfloat16, out=dX, stream=stream)
+                Q.gemm(qs[2], qs[3], torch.bfloat16, out=dX, stream=st)
                 mark(7, 1)
         mark(8, 0)
-        Q.gemm(qs[4], qs[5], torch.float32, out=dW, stream=stream)
+        Q.gemm(qs[4], qs[5], torch.float32, out=dW, stream=st)
         mark(8, 1)
 
     def barrier():
@@ -388,10 +389,15 @@ def run_ours(args, rank, world, local_rank):
                  "what": "Wgrad of the step, dW = dY^T X vs dW += dY^T X (TMA reduce-add epilogue), fp32 dW "
                          f"[{N}x{K}]; 10 back-to-back launches each"}
 
+    # the step captured once in a CUDA graph and replayed (the same launches, no
+    # host-side launch work between them)
+    graph = graph_time(step, args, stream, flops_step, world, dev)
+
     # quantizer sweep workload (GB/s of algorithmic bytes), L2 flushed between launches,
     # and the same kernels on dY [16384 x 28672] (940 MB, steady state)
     quant = quant_sweep(Q, inputs, dev, stream, peaks)
     quant["large"] = quant_large(Q, dY, stream, peaks)
+    quant["startup_fit"] = quant_startup_fit(Q, dY, stream, peaks)
 
     # the other configurations of the MLP shapes (not part of the headline value)
     layers = more_layers(Q, inputs, X, W, dY, seed, stream, dev, roofline["peak"])
@@ -414,6 +420,7 @@ def run_ours(args, rank, world, local_rank):
                    "parallelism": f"replicas x{world}"},
         "roofline": roofline,
         "sustained": sustained,
+        "graph": graph,
         "step_breakdown_ms": {"quantize": [round(v, 4) for v in quant_ms], "gemm": [round(v, 4) for v in gemm_ms]},
         "quantize": quant,
         "layers": layers,
@@ -426,6 +433,81 @@ def run_ours(args, rank, world, local_rank):
         "clocks": clocks,
     }
     return out
+
+
+def graph_time(step, args, stream, flops_step, world, dev):
+    """The step captured into one CUDA graph (on a side stream, as capture
+    requires) and replayed K times, timed with CUDA events on that stream."""
+    import torch
+    s = torch.cuda.Stream(device=dev)
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    try:
+        with torch.cuda.stream(s):
+            step(None, s)  # outside the capture: lazy set-up, tensor maps, attributes
+            torch.cuda.synchronize()
+            with torch.cuda.graph(g, stream=s):
+                step(None, s)
+    except RuntimeError as e:  # capture refused: report why instead of a number
+        return {"error": str(e).splitlines()[0][:200]}
+    torch.cuda.synchronize()
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n = max(3, args.steps)
+    with torch.cuda.stream(s):
+        e0.record(s)
+        for _ in range(n):
+            g.replay()
+        e1.record(s)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1) / n, world, dev)
+    del g
+    return {"ms_per_step": round(ms, 4), "TFLOP/s": round(world * flops_step / (ms * 1e-3) / 1e12, 2), "steps": n,
+            "what": "the headline step captured once in a CUDA graph and replayed"}
+
+
+def quant_startup_fit(Q, dY, stream, peaks):
+    """Why short quantizer launches read below the large-tensor figure: the
+    NVFP4 RTN row quantizer (amax given) on the first 1024, 4096, 16384 (all)
+    rows of dY — 58, 235, 940 MB — and on 256 rows (15 MB), L2 evicted before
+    each launch by a 256 MiB read; a least-squares fit time = t0 + bytes / BW
+    gives the fixed cost per launch t0 and the steady-state bandwidth BW."""
+    import torch
+    flush = torch.ones((64 << 20,), dtype=torch.float32, device=dY.device)
+    ws = torch.empty((Q.quantize_workspace_bytes(),), dtype=torch.uint8, device=dY.device)
+    seed = Q.make_seed(1, 2)
+    pts = []
+    for rows in (256, 1024, 4096, dY.shape[0]):
+        x = dY[:rows]
+        q = Q.empty_qtensor(Q.NVFP4, rows, x.shape[1], dY.device)
+        am = Q.amax(x, Q.HAD_NONE, Q.ROW, seed, workspace=ws, stream=stream)
+        times = []
+        for it in range(7):
+            flush.sum()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            Q.quantize(x, Q.NVFP4, Q.RTN, Q.HAD_NONE, Q.ROW, seed, amax_in=am, out=q, workspace=ws, stream=stream)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            if it >= 2:
+                times.append(e0.elapsed_time(e1))
+        pts.append((x.numel() * (2 + 0.5 + 1 / 16), statistics.median(times)))
+        del q
+    Q.status()
+    n = len(pts)
+    mx = sum(b for b, _ in pts) / n
+    my = sum(t for _, t in pts) / n
+    slope = sum((b - mx) * (t - my) for b, t in pts) / sum((b - mx) ** 2 for b, _ in pts)
+    t0 = my - slope * mx
+    bw = 1.0 / slope / 1e6  # bytes per ms -> GB/s
+    return {"points": [{"MB": round(b / 1e6, 1), "ms": round(t, 4), "GB/s": round(b / (t * 1e-3) / 1e9, 1)}
+                       for b, t in pts],
+            "fixed_cost_us": round(t0 * 1e3, 2), "steady_GB/s": round(bw, 1),
+            "steady_frac_of_measured_hbm": round(bw / peaks["hbm_gbs"], 3),
+            "what": "NVFP4 RTN row quantizer on row slices of dY, L2 evicted before each launch; "
+                    "time = fixed_cost + bytes / steady_GB/s"}
 
 
 def dy_plan(Q, c, M):

@@ -242,6 +242,16 @@ bool col_bands_enabled() {
     return !(e != nullptr && e[0] == '0');
 }
 
+// NVFP4 tensors up to this size (bf16 bytes) are quantized by the fused
+// one-launch kernel, whose second pass then reads them from L2 (126 MB, split
+// between the two dies); QFP4_FUSED_AMAX=0 selects the separate amax pass
+// (same results; read on every call).
+constexpr int64_t kFusedAmaxMaxBytes = (int64_t)96 << 20;
+bool fused_amax_enabled() {
+    const char* e = std::getenv("QFP4_FUSED_AMAX");
+    return !(e != nullptr && e[0] == '0');
+}
+
 // CTA-pair kernel unless A has at most 128 rows (one pair tile would be half
 // empty); QFP4_GEMM_PAIR=1 / =0 forces one kernel (read on every call).
 bool use_pair_gemm(int64_t M) {
@@ -376,7 +386,22 @@ int quantize_impl(const void* x, int64_t R, int64_t C, int64_t ld, int32_t fmt, 
     p.sr_tag_scale = (uint32_t)kTagScale | (seed->sr_stream << 4);
     p.amax_in = amax_in;
     p.mx_round_up = (fmt == QFP4_MXFP4_RU) ? 1u : 0u;
-    if (need_ws) {
+    // the column quantizer walks 64-row bands when the quantized axis allows it
+    const bool bands = axis == QFP4_AXIS_COL && g.k % 64 == 0 && col_bands_enabled();
+    // An NVFP4 tensor that fits in L2, in the packed unit's cases, is quantized
+    // by one cooperative launch that takes its own amax first (the second pass
+    // reads from L2) instead of an amax pass, a reduction and the quantizer.
+    const bool fused = need_ws && (rounding == QFP4_RTN || rounding == QFP4_QUARTET2) && (nh == 0 || nh == 16) &&
+                       (axis == QFP4_AXIS_ROW || bands) && R * C * 2 <= kFusedAmaxMaxBytes && fused_amax_enabled();
+    if (fused) {
+        float* partials = static_cast<float*>(workspace);
+        uint32_t* counter = static_cast<uint32_t*>(workspace) + (kMaxAmaxPartials - 1);
+        const cudaError_t e = cudaMemsetAsync(counter, 0, sizeof(uint32_t), s);
+        if (e != cudaSuccess) return cuda_fail(e);
+        p.amax_out = partials;
+        p.amax_partials = partials;
+        p.grid_counter = counter;
+    } else if (need_ws) {
         int n = 0;
         float* partials = static_cast<float*>(workspace);
         if ((rc = run_amax(x, R, C, ld, had, axis, signs, g, partials, &n, sms, s))) return rc;
@@ -384,14 +409,13 @@ int quantize_impl(const void* x, int64_t R, int64_t C, int64_t ld, int32_t fmt, 
         p.n_partials = n;
     }
     CUtensorMap tm;
-    // the column quantizer walks 64-row bands when the quantized axis allows it
-    const bool bands = axis == QFP4_AXIS_COL && g.k % 64 == 0 && col_bands_enabled();
     if (bands)
         rc = make_col64_tmap(&tm, x, R, C, ld);
     else
         rc = make_input_tmap(&tm, x, R, C, ld, axis, col_group(NB, nh));
     if (rc) return rc;
-    cudaError_t e = launch_quant(p, sfmt, rounding, nh, bands ? 2 : axis, &tm, s);
+    cudaError_t e = fused ? launch_quant_fused(p, rounding, nh, bands ? 2 : axis, &tm, s)
+                          : launch_quant(p, sfmt, rounding, nh, bands ? 2 : axis, &tm, s);
     return e == cudaSuccess ? QFP4_OK : cuda_fail(e);
 }
 

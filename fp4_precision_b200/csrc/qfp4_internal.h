@@ -48,6 +48,10 @@ struct QuantParams {
     uint64_t sr_seed_row;
     uint32_t sr_tag_elem_row;
     uint32_t sr_tag_scale_row;
+    // Fused amax and quantization (one cooperative launch): the grid barrier's
+    // arrival counter, zeroed before the launch; the partials go to amax_out
+    // and are read back through amax_partials.
+    uint32_t* grid_counter;
 };
 
 // Launchers (quant.cu). Return cudaSuccess or the launch error.
@@ -58,6 +62,13 @@ cudaError_t launch_amax(const QuantParams& p, int axis, int nh, const CUtensorMa
 // 4-D band view; quantized axis a multiple of 64).
 cudaError_t launch_quant(const QuantParams& p, int fmt, int rnd, int nh, int axis, const CUtensorMap* tmap,
                          cudaStream_t s);
+// NVFP4 amax and quantization in one cooperative launch (a first pass takes the
+// rotated amax, a grid barrier, then the quantizing pass re-reads the tiles,
+// from L2 for a tensor that fits there): rnd RTN or Quartet II, nh 0 or 16,
+// axis 0 (row) or 2 (64-row bands). p.amax_out == p.amax_partials (room for
+// 2 x SM count partials) and p.grid_counter (zeroed) are set by the caller.
+cudaError_t launch_quant_fused(const QuantParams& p, int rnd, int nh, int axis, const CUtensorMap* tmap,
+                               cudaStream_t s);
 // Dual quantization of x (R x C, R a multiple of 64; tmap: the 64-row band
 // view): p describes the column orientation, p.*_row the row orientation.
 // nh: the column orientation's Hadamard size; nh_row: 0 or nh.

@@ -167,7 +167,9 @@ __device__ float nvfp4_encode_scale(const QuantParams& p, float* red_smem, bool 
         amax = __ldg(p.amax_in);
     } else {
         float m = 0.0f;
-        for (int i = threadIdx.x; i < p.n_partials; i += kComputeWarps * 32) m = fmaxf(m, __ldg(p.amax_partials + i));
+        // coherent loads: in the fused pass the partials were written by the
+        // other CTAs of this launch
+        for (int i = threadIdx.x; i < p.n_partials; i += kComputeWarps * 32) m = fmaxf(m, __ldcg(p.amax_partials + i));
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
         if ((threadIdx.x & 31) == 0) red_smem[threadIdx.x >> 5] = m;
@@ -623,6 +625,40 @@ __device__ __forceinline__ uint32_t nv64_quantize(Load load, const SignFlips& sf
     return scw;
 }
 
+// max |H D x| (no 1/sqrt(n_h)) of a 64-element unit loaded by chunks.
+template <int NH, typename Load>
+__device__ __forceinline__ float rot_amax64(Load load, const SignFlips& sf, float m) {
+#pragma unroll
+    for (int bp = 0; bp < 2; ++bp) {
+        float2 P[16];
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+            const uint4 a = load(4 * bp + c), b = load(4 * bp + 2 + c);
+            const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int wi = 4 * c + i;
+                if constexpr (NH > 0) {
+                    P[2 * wi] = f2(bf16lo_flip(wa[i], sf.lo[wi]), bf16lo_flip(wb[i], sf.lo[wi]));
+                    P[2 * wi + 1] = f2(bf16hi_flip(wa[i], sf.hi[wi]), bf16hi_flip(wb[i], sf.hi[wi]));
+                } else {
+                    P[2 * wi] = f2(bf16lo(wa[i]), bf16lo(wb[i]));
+                    P[2 * wi + 1] = f2(bf16hi(wa[i]), bf16hi(wb[i]));
+                }
+            }
+        }
+        if constexpr (NH == 16) {
+            fwht_pair_stage<1>(P);
+            fwht_pair_stage<2>(P);
+            fwht_pair_stage<4>(P);
+            fwht_pair_stage<8>(P);
+        }
+        const float2 am = abs_max_pair(P);
+        m = max3(m, am.x, am.y);
+    }
+    return m;
+}
+
 // This CTA's tiles of a tiles_r x tiles_c grid (blockIdx.x, + gridDim.x, ...)
 // as (tr, tc), advanced without divisions, with the TMA ring stage and phase
 // of each.
@@ -630,11 +666,15 @@ template <int STAGES>
 struct TileWalk {
     int tr, tc, tiles_c, step_r, step_c, stage = 0;
     uint32_t phase = 0;
-    __device__ __forceinline__ explicit TileWalk(int tiles_c_) : tiles_c(tiles_c_) {
+    // issued: ring iterations this CTA has already used (a second pass over
+    // the same tiles continues the ring where the first one left it)
+    __device__ __forceinline__ explicit TileWalk(int tiles_c_, int issued = 0) : tiles_c(tiles_c_) {
         tr = (int)blockIdx.x / tiles_c;
         tc = (int)blockIdx.x % tiles_c;
         step_r = (int)gridDim.x / tiles_c;
         step_c = (int)gridDim.x % tiles_c;
+        stage = issued % STAGES;
+        phase = (uint32_t)((issued / STAGES) & 1);
     }
     __device__ __forceinline__ void next() {
         tc += step_c;
@@ -680,10 +720,64 @@ __device__ __forceinline__ void write_partial(float m, float* red, float* out) {
     }
 }
 
+// Grid-wide barrier of a cooperative launch, by one thread of each CTA: the
+// CTA's earlier global writes are published (fence, then one arrival on the
+// counter, which the caller zeroed before the launch) and the thread waits,
+// bounded, until every CTA has arrived. False (and the device error word set)
+// if the wait gave up.
+__device__ __forceinline__ bool grid_arrive_and_wait(uint32_t* counter) {
+    __threadfence();
+    atomicAdd(counter, 1u);
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        uint32_t v;
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(counter) : "memory");
+        if (v >= gridDim.x) break;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            raise_device_error(DEV_ERR_TIMEOUT);
+            return false;
+        }
+        __nanosleep(64);
+    }
+    __threadfence();
+    return true;
+}
+
+// Fused NVFP4 amax (first pass of a two-pass kernel, packed unit): every tile
+// of this CTA rotated and its maximum taken; the CTA's partial (times
+// 1/sqrt(n_h)) written to p.amax_out[blockIdx.x]; after the grid barrier the
+// tensor scale is set up from all partials exactly as the separate amax pass
+// and quantizer would (max over the partials, s_enc, g). Returns the ring
+// iterations used.
+template <int NH, int STAGES, typename LoadAt>
+__device__ int fused_amax_pass(const QuantParams& p, Ring<STAGES>& ring, int tiles_c, int tiles_r, float* red,
+                               LoadAt load_at) {
+    const SignFlips sf(NH > 0 ? p.signs : 0u);
+    float m = 0.0f;
+    for (TileWalk<STAGES> w(tiles_c); w.tr < tiles_r; w.next()) {
+        const int s = w.stage;
+        if (!mbar_wait(&ring.full[s], w.phase)) break;
+        m = rot_amax64<NH>([&](int c) { return load_at(s, c); }, sf, m);
+        __syncwarp();
+        if ((threadIdx.x & 31) == 0) mbar_arrive(&ring.empty[s]);
+    }
+    if constexpr (NH > 0) m = __fmul_rn(m, had_norm<NH>());  // c * max |y| = max |c * y|
+    write_partial(m, red, p.amax_out);
+    if (threadIdx.x == 0) (void)grid_arrive_and_wait(p.grid_counter);
+    bar_compute();
+    // this CTA's tiles (blockIdx.x, + gridDim.x, ...): the second pass starts
+    // the ring there even if a wait above gave up early
+    const int64_t total = (int64_t)tiles_c * tiles_r;
+    return total > (int64_t)blockIdx.x ? (int)((total - blockIdx.x + gridDim.x - 1) / gridDim.x) : 0;
+}
+
 // ===========================================================================
 // Row mode
 // ===========================================================================
-template <int FMT, int RND, int NH, bool AMAX_ONLY, int STAGES>
+// FUSED: an NVFP4 tensor that fits in L2 in one cooperative launch — a first
+// pass over the tiles takes the rotated amax, a grid barrier, then the
+// quantizing pass re-reads the tiles (from L2).
+template <int FMT, int RND, int NH, bool AMAX_ONLY, int STAGES, bool FUSED = false>
 __global__ void __launch_bounds__(kThreads, 2)
     quant_row_kernel(const __grid_constant__ CUtensorMap tmap, const QuantParams p) {
     using Grp = Group<FMT, RND, NH>;
@@ -693,6 +787,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     // NVFP4 with no Hadamard or a 16-point one, round-to-nearest or Quartet
     // II: the packed 64-element unit
     constexpr bool kPacked = FMT == kNvfp4 && (NH == 0 || NH == 16) && RND != kSr && !AMAX_ONLY;
+    static_assert(!FUSED || kPacked, "the fused amax pass serves the packed NVFP4 unit");
     extern __shared__ __align__(1024) uint8_t dyn_smem[];
     uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
     __shared__ Ring<STAGES> ring;
@@ -712,12 +807,18 @@ __global__ void __launch_bounds__(kThreads, 2)
         // ---------------- producer ----------------
         if (lane == 0) {
             int i = 0;
-            for (TileWalk<STAGES> w(tiles_c); w.tr < tiles_r; w.next(), ++i) {
-                const int s = w.stage;
-                if (i >= STAGES && !mbar_wait(&ring.empty[s], w.phase ^ 1u)) break;
-                mbar_arrive_expect_tx(&ring.full[s], STAGE_BYTES);
-                tma_load_2d(tiles + s * STAGE_BYTES, &tmap, &ring.full[s], w.tc * kRowTileCols, w.tr * kRowTileRows);
-            }
+            bool ok = true;
+            for (int pass = 0; pass < (FUSED ? 2 : 1) && ok; ++pass)
+                for (TileWalk<STAGES> w(tiles_c, i); w.tr < tiles_r; w.next(), ++i) {
+                    const int s = w.stage;
+                    if (i >= STAGES && !mbar_wait(&ring.empty[s], w.phase ^ 1u)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&ring.full[s], STAGE_BYTES);
+                    tma_load_2d(tiles + s * STAGE_BYTES, &tmap, &ring.full[s], w.tc * kRowTileCols,
+                                w.tr * kRowTileRows);
+                }
             drain_loads(ring.full, nullptr, STAGES, i);  // no load lands after this CTA exits
         }
         return;
@@ -725,6 +826,13 @@ __global__ void __launch_bounds__(kThreads, 2)
     __shared__ float rtab[kPacked ? 1 : 128];
     __shared__ float2 tab2[kPacked ? 128 : 1];
     float s_enc = 1.0f;
+    int issued = 0;  // ring iterations of the fused amax pass
+    if constexpr (FUSED) {
+        issued = fused_amax_pass<NH>(p, ring, tiles_c, tiles_r, red, [&](int st, int c) {
+            return lds128((smem_u32(tiles) + (uint32_t)(st * STAGE_BYTES) + (uint32_t)tid * 128u +
+                           ((uint32_t)(tid & 7) << 4)) ^ ((uint32_t)c << 4));
+        });
+    }
     if constexpr (!AMAX_ONLY && FMT == kNvfp4) {
         s_enc = nvfp4_encode_scale(p, red, blockIdx.x == 0);
         if constexpr (kPacked)
@@ -760,7 +868,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         for (int i = 0; i < G / 2; ++i) smask[i] = Grp::sign_mask(p.signs, i);
     }
     const SignFlips sf(kPacked && NH > 0 ? p.signs : 0u);
-    for (TileWalk<STAGES> w(tiles_c); w.tr < tiles_r; w.next()) {
+    for (TileWalk<STAGES> w(tiles_c, issued); w.tr < tiles_r; w.next()) {
         const int s = w.stage;
         if (!mbar_wait(&ring.full[s], w.phase)) break;
         const int64_t row = (int64_t)w.tr * kRowTileRows + tid;
@@ -1200,7 +1308,7 @@ __device__ __forceinline__ void dual_row_work(const QuantParams& p, float s_enc_
 // 64 columns, in the row orientation (rotation of size NH_ROW with the row
 // sign vector, the row tensor amax and random streams), as the row kernel
 // would: one read of x gives both orientations.
-template <int FMT, int RND, int NH, int STAGES, int NH_ROW = -1>
+template <int FMT, int RND, int NH, int STAGES, int NH_ROW = -1, bool FUSED = false>
 __global__ void __launch_bounds__(kThreads, 2)
     quant_col64_kernel(const __grid_constant__ CUtensorMap tmap, const QuantParams p) {
     constexpr bool kDual = NH_ROW >= 0;
@@ -1214,6 +1322,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     // II: the packed 64-element unit
     constexpr bool kPacked = FMT == kNvfp4 && (NH == 0 || NH == 16) && RND != kSr;
     constexpr bool kPackedRow = kDual && FMT == kNvfp4 && (NH_ROW == 0 || NH_ROW == 16) && RND != kSr;
+    static_assert(!FUSED || (kPacked && !kDual), "the fused amax pass serves the packed NVFP4 unit");
     extern __shared__ __align__(1024) uint8_t dyn_smem[];
     uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
     __shared__ Ring<STAGES> ring;
@@ -1234,12 +1343,17 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (warp == kComputeWarps) {
         if (lane == 0) {
             int i = 0;
-            for (TileWalk<STAGES> w(tiles_c); w.tr < tiles_r; w.next(), ++i) {
-                const int s = w.stage;
-                if (i >= STAGES && !mbar_wait(&ring.empty[s], w.phase ^ 1u)) break;
-                mbar_arrive_expect_tx(&ring.full[s], STAGE_BYTES);
-                tma_load_4d(tiles + s * STAGE_BYTES, &tmap, &ring.full[s], w.tc * TILE_COLS, 0, 4 * w.tr, 0);
-            }
+            bool ok = true;
+            for (int pass = 0; pass < (FUSED ? 2 : 1) && ok; ++pass)
+                for (TileWalk<STAGES> w(tiles_c, i); w.tr < tiles_r; w.next(), ++i) {
+                    const int s = w.stage;
+                    if (i >= STAGES && !mbar_wait(&ring.empty[s], w.phase ^ 1u)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&ring.full[s], STAGE_BYTES);
+                    tma_load_4d(tiles + s * STAGE_BYTES, &tmap, &ring.full[s], w.tc * TILE_COLS, 0, 4 * w.tr, 0);
+                }
             drain_loads(ring.full, nullptr, STAGES, i);  // no load lands after this CTA exits
         }
         return;
@@ -1249,6 +1363,17 @@ __global__ void __launch_bounds__(kThreads, 2)
     __shared__ float rtab_row[kDual && !kPackedRow ? 128 : 1];
     __shared__ float2 tab2_row[kPackedRow ? 128 : 1];
     float s_enc = 1.0f, s_enc_row = 1.0f;
+    int issued = 0;  // ring iterations of the fused amax pass
+    if constexpr (FUSED) {
+        const uint32_t lm = (uint32_t)lane * 128u + ((uint32_t)(warp ^ (lane & 7)) << 4);
+        issued = fused_amax_pass<NH>(p, ring, tiles_c, tiles_r, red, [&](int st, int n) {
+            uint4 v;
+            asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                         : "r"(smem_u32(tiles) + (uint32_t)(st * STAGE_BYTES) + lm + (uint32_t)(n * 4096)));
+            return v;
+        });
+    }
     if constexpr (FMT == kNvfp4) {
         s_enc = nvfp4_encode_scale(p, red, blockIdx.x == 0);
         if constexpr (kPacked)
@@ -1284,7 +1409,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     const SignFlips sf(kPacked && NH > 0 ? p.signs : 0u);
     ScaleRng srng, srng_row;
-    for (TileWalk<STAGES> w(tiles_c); w.tr < tiles_r; w.next()) {
+    for (TileWalk<STAGES> w(tiles_c, issued); w.tr < tiles_r; w.next()) {
         const int s = w.stage;
         if (!mbar_wait(&ring.full[s], w.phase)) break;
         const int64_t c = (int64_t)w.tc * TILE_COLS + cc;          // x column = output row
@@ -1386,40 +1511,6 @@ __global__ void __launch_bounds__(kThreads, 2)
 // 1/sqrt(n_h) is applied once to each CTA's maxima (rounding c * y is
 // monotone in y). Zero-filled columns and rows past the tensor add nothing.
 
-// max |H D x| (no 1/sqrt(n_h)) of a 64-element unit loaded by chunks.
-template <int NH, typename Load>
-__device__ __forceinline__ float rot_amax64(Load load, const SignFlips& sf, float m) {
-#pragma unroll
-    for (int bp = 0; bp < 2; ++bp) {
-        float2 P[16];
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-            const uint4 a = load(4 * bp + c), b = load(4 * bp + 2 + c);
-            const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int wi = 4 * c + i;
-                if constexpr (NH > 0) {
-                    P[2 * wi] = f2(bf16lo_flip(wa[i], sf.lo[wi]), bf16lo_flip(wb[i], sf.lo[wi]));
-                    P[2 * wi + 1] = f2(bf16hi_flip(wa[i], sf.hi[wi]), bf16hi_flip(wb[i], sf.hi[wi]));
-                } else {
-                    P[2 * wi] = f2(bf16lo(wa[i]), bf16lo(wb[i]));
-                    P[2 * wi + 1] = f2(bf16hi(wa[i]), bf16hi(wb[i]));
-                }
-            }
-        }
-        if constexpr (NH == 16) {
-            fwht_pair_stage<1>(P);
-            fwht_pair_stage<2>(P);
-            fwht_pair_stage<4>(P);
-            fwht_pair_stage<8>(P);
-        }
-        const float2 am = abs_max_pair(P);
-        m = max3(m, am.x, am.y);
-    }
-    return m;
-}
-
 template <int NH, int STAGES>
 __global__ void __launch_bounds__(kThreads, 2)
     amax_rowcol64_kernel(const __grid_constant__ CUtensorMap tmap, const QuantParams p) {
@@ -1501,6 +1592,28 @@ cudaError_t launch_persistent(Kern kern, int grid, int smem, const CUtensorMap& 
     return cudaGetLastError();
 }
 
+// A cooperative launch (all CTAs co-resident, as the fused kernels' grid
+// barrier needs) of a persistent quantizer: at most as many CTAs per SM as
+// fit, and no more than two; p.n_partials is set to the grid size (the fused
+// amax pass writes one partial per CTA).
+template <typename Kern>
+cudaError_t launch_cooperative(Kern kern, int64_t tiles, int smem, const CUtensorMap& tmap, const QuantParams& p,
+                               cudaStream_t s) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    int per_sm = 0;
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem)) != cudaSuccess) return e;
+    if (per_sm < 1) return cudaErrorCooperativeLaunchTooLarge;
+    const int grid = persistent_grid(tiles, per_sm < 2 ? per_sm : 2);
+    QuantParams q = p;
+    q.n_partials = grid;
+    void* args[] = {const_cast<CUtensorMap*>(&tmap), &q};
+    e = cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kern), dim3(grid), dim3(kThreads), args,
+                                    (size_t)smem, s);
+    count_launch();
+    return e;
+}
+
 constexpr int kRowStages = 3;
 template <int G>
 constexpr int col_stages() {
@@ -1533,6 +1646,23 @@ cudaError_t launch_col64(const QuantParams& p, const CUtensorMap* tmap, cudaStre
     const int64_t tiles = ((p.rows + 127) / 128 * 2) * ((p.k + 255) / 256);
     const int smem = S * 256 * 64 * 2 + 1024;
     return launch_persistent(quant_col64_kernel<FMT, RND, NH, S>, persistent_grid(tiles, 2), smem, *tmap, p, s);
+}
+
+// The fused (one-launch) NVFP4 quantization: packed unit, RTN or Quartet II,
+// no Hadamard or a 16-point one, along rows (axis 0) or 64-row bands (2).
+template <int RND, int NH>
+cudaError_t launch_fused_t(const QuantParams& p, int axis, const CUtensorMap* tmap, cudaStream_t s) {
+    if (axis == 0) {
+        const int64_t tiles =
+            ((p.rows + kRowTileRows - 1) / kRowTileRows) * ((p.k + kRowTileCols - 1) / kRowTileCols);
+        const int smem = kRowStages * kRowTileRows * kRowTileCols * 2 + 1024;
+        return launch_cooperative(quant_row_kernel<kNvfp4, RND, NH, false, kRowStages, true>, tiles, smem, *tmap, p,
+                                  s);
+    }
+    constexpr int S = 3;
+    const int64_t tiles = ((p.rows + 127) / 128 * 2) * ((p.k + 255) / 256);
+    const int smem = S * 256 * 64 * 2 + 1024;
+    return launch_cooperative(quant_col64_kernel<kNvfp4, RND, NH, S, -1, true>, tiles, smem, *tmap, p, s);
 }
 
 template <int FMT, int RND>
@@ -1582,6 +1712,12 @@ cudaError_t launch_reduce_max(const float* in, int n, float* out, cudaStream_t s
 }
 
 int col_group(int block, int nh) { return nh > block ? nh : block; }
+
+cudaError_t launch_quant_fused(const QuantParams& p, int rnd, int nh, int axis, const CUtensorMap* tmap,
+                               cudaStream_t s) {
+    if (rnd == kRtn) return nh == 16 ? launch_fused_t<kRtn, 16>(p, axis, tmap, s) : launch_fused_t<kRtn, 0>(p, axis, tmap, s);
+    return nh == 16 ? launch_fused_t<kQuartet2, 16>(p, axis, tmap, s) : launch_fused_t<kQuartet2, 0>(p, axis, tmap, s);
+}
 
 cudaError_t launch_quant(const QuantParams& p, int fmt, int rnd, int nh, int axis, const CUtensorMap* tmap,
                          cudaStream_t s) {
