@@ -112,14 +112,15 @@ __device__ __forceinline__ void fwht(float* v) {
     if constexpr (N == 32) fwht_stage<N, 16>(v);
 }
 
-// One stride of the halving tree: s[j] += s[j + ST] for j < ST, packed x2.
+// One stride of the halving tree: s[j] += s[j + ST] for j < ST. Scalar
+// __fadd_rn, like the products that feed the tree (__fmul_rn): those are never
+// merged into a fused multiply-add, whereas a packed f32x2 product feeding a
+// packed sum was (by the assembler, even as explicit mul.rn.f32x2 /
+// add.rn.f32x2), which moved alpha by an ulp in about 15 % of blocks.
 template <int ST>
 __device__ __forceinline__ void tree_stage(float* s) {
 #pragma unroll
-    for (int j = 0; j < ST; j += 2) {
-        const float2 r = __fadd2_rn(f2(s[j], s[j + 1]), f2(s[j + ST], s[j + ST + 1]));
-        s[j] = r.x; s[j + 1] = r.y;
-    }
+    for (int j = 0; j < ST; ++j) s[j] = __fadd_rn(s[j], s[j + ST]);
 }
 
 // Halving-stride tree sum of n fp32 terms (s[j] += s[j + stride], stride n/2 .. 1).
@@ -329,11 +330,11 @@ struct Group {
                 float sa[NB], sb[NB];
 #pragma unroll
                 for (int e = 0; e < NB; e += 2) {
-                    const float2 u = f2(vb[e], vb[e + 1]);
                     const float2 q = e2m1x2_decode((cb[e / 8] >> (4 * (e & 7))) & 0xFFu);
-                    const float2 uu = __fmul2_rn(u, u), uq = __fmul2_rn(u, q);
-                    sa[e] = uu.x; sa[e + 1] = uu.y;
-                    sb[e] = uq.x; sb[e + 1] = uq.y;
+                    sa[e] = __fmul_rn(vb[e], vb[e]);
+                    sa[e + 1] = __fmul_rn(vb[e + 1], vb[e + 1]);
+                    sb[e] = __fmul_rn(vb[e], q.x);
+                    sb[e + 1] = __fmul_rn(vb[e + 1], q.y);
                 }
                 const float num = tree_sum<NB>(sa);
                 const float den = tree_sum<NB>(sb);
@@ -472,12 +473,14 @@ __device__ __forceinline__ void fwht_pair_stage(float2* P) {
         }
 }
 
-// Halving-stride tree sum of the 16 packed terms of a pair (both lanes).
+// Halving-stride tree sum of the 16 terms of each lane of a pair, in scalar
+// __fadd_rn (see tree_stage: the terms are products, and a packed sum of
+// packed products was fused into multiply-adds).
 __device__ __forceinline__ float2 tree_sum_pair(float2* s) {
 #pragma unroll
     for (int st = 8; st >= 1; st >>= 1)
 #pragma unroll
-        for (int j = 0; j < st; ++j) s[j] = __fadd2_rn(s[j], s[j + st]);
+        for (int j = 0; j < st; ++j) s[j] = f2(__fadd_rn(s[j].x, s[j + st].x), __fadd_rn(s[j].y, s[j + st].y));
     return s[0];
 }
 
@@ -598,10 +601,11 @@ __device__ __forceinline__ uint32_t nv64_quantize(Load load, const SignFlips& sf
             for (int j = 0; j < 16; j += 2) {
                 const float2 qx = __half22float2(*reinterpret_cast<const __half2*>(&h[j / 8][(j % 8) / 2]));
                 const float2 qy = __half22float2(*reinterpret_cast<const __half2*>(&h[2 + j / 8][(j % 8) / 2]));
-                uu[j] = __fmul2_rn(P[j], P[j]);
-                uu[j + 1] = __fmul2_rn(P[j + 1], P[j + 1]);
-                uq[j] = __fmul2_rn(P[j], f2(qx.x, qy.x));
-                uq[j + 1] = __fmul2_rn(P[j + 1], f2(qx.y, qy.y));
+                // scalar products (never fused with the tree's sums)
+                uu[j] = f2(__fmul_rn(P[j].x, P[j].x), __fmul_rn(P[j].y, P[j].y));
+                uu[j + 1] = f2(__fmul_rn(P[j + 1].x, P[j + 1].x), __fmul_rn(P[j + 1].y, P[j + 1].y));
+                uq[j] = f2(__fmul_rn(P[j].x, qx.x), __fmul_rn(P[j].y, qy.x));
+                uq[j + 1] = f2(__fmul_rn(P[j + 1].x, qx.y), __fmul_rn(P[j + 1].y, qy.y));
             }
             const float2 num = tree_sum_pair(uu), den = tree_sum_pair(uq);
             const float a0 = (den.x == 0.0f) ? 1.0f : __fdiv_rn(num.x, den.x);
