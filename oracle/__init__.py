@@ -89,6 +89,8 @@ def load(path: str) -> ctypes.CDLL:
     L.oracle_philox4x32_10.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
     L.oracle_random_word.argtypes = [u64, u32, u32, u64]
     L.oracle_random_word.restype = u32
+    L.oracle_element_uniform.argtypes = [u64, u32, u64]
+    L.oracle_element_uniform.restype = ctypes.c_float
     L.oracle_e2m1_value.argtypes = [u8]
     L.oracle_e2m1_value.restype = ctypes.c_double
     L.oracle_e2m1_rtn.argtypes = [ctypes.c_float]
@@ -140,6 +142,11 @@ def philox4x32_10(ctr, key) -> np.ndarray:
 
 def random_word(seed: int, tag: int, stream: int, i: int) -> int:
     return int(lib().oracle_random_word(seed, tag, stream, i))
+
+
+def element_uniform(seed: int, stream: int, i: int) -> float:
+    """The uniform of element i's stochastic rounding (16 bits, two per word)."""
+    return float(lib().oracle_element_uniform(seed, stream, i))
 
 
 def e2m1_value(code: int) -> float:

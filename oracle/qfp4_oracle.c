@@ -88,6 +88,22 @@ uint32_t oracle_random_word(uint64_t seed, uint32_t tag, uint32_t stream, uint64
     return random_word(seed, tag, stream, i);
 }
 
+/* The uniform of element i's stochastic rounding. The pages ([AMD MXFP4]
+ * glossary: rounding whose error has zero expectation; [NVIDIA NVFP4] "Kak
+ * eto rabotaet"; [Quartet II]) fix no width for the random draw. Reading: 16
+ * bits per element, half (i mod 2) of word floor(i/2) of the element stream
+ * (the low half for even i), rho = half * 2^-16, so one Philox call serves
+ * eight elements. Rounding up iff rho < p (p the exact fraction) then has
+ * probability ceil(p 2^16) / 2^16: a bias below 2^-16 of the grid gap. */
+static float element_uniform(uint64_t seed, uint32_t stream, uint64_t i) {
+    const uint32_t w = random_word(seed, TAG_ELEMENT, stream, i >> 1);
+    return (float)((w >> (16u * (uint32_t)(i & 1u))) & 0xFFFFu) * 0x1p-16f;
+}
+
+float oracle_element_uniform(uint64_t seed, uint32_t stream, uint64_t i) {
+    return element_uniform(seed, stream, i);
+}
+
 /* ------------------------------------------------------------------------ */
 /* E2M1: the 4-bit float element of both formats ([AMD MXFP4] "Chto takoe
  * MXFP4": each element is a 4-bit floating-point number). Code = sign << 3 |
@@ -412,7 +428,7 @@ int oracle_quantize_rows(const uint16_t* x, int64_t R, int64_t C, int64_t ld, in
                 if (rnd == RND_SR) {
                     for (int j = 0; j < nb; ++j) {
                         const uint64_t i = (uint64_t)(r * k + b * nb + j);
-                        q[j] = oracle_e2m1_sr(u[j], uniform24(random_word(sr_seed, TAG_ELEMENT, sr_stream, i)));
+                        q[j] = oracle_e2m1_sr(u[j], element_uniform(sr_seed, sr_stream, i));
                     }
                 } else {
                     for (int j = 0; j < nb; ++j) q[j] = oracle_e2m1_rtn(u[j]);

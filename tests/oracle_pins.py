@@ -169,6 +169,19 @@ def check_philox_matches_torch_engine():
         assert O.random_word(seed, tag, stream, i) == ref[i // 4][i % 4]
 
 
+def check_element_uniform_layout():
+    """Element SR uniforms (16 bits each): element i takes half (i mod 2), low
+    half first, of word floor(i/2) of its stream, i.e. of word (i/2) mod 4 of
+    the Philox block with counter (i/8, TAG_ELEMENT | stream << 4, 0), scaled
+    by 2^-16 — checked against torch's Philox engine for 128 elements."""
+    seed, stream = 0x0F1E_2D3C_4B5A_6978, 9
+    ref = _torch_philox([(seed, O.TAG_ELEMENT | (stream << 4), i // 8) for i in range(0, 128, 8)])
+    for i in range(128):
+        w = ref[i // 8][(i // 2) % 4]
+        half = (w >> (16 * (i % 2))) & 0xFFFF
+        assert O.element_uniform(seed, stream, i) == half * 2.0**-16, i
+
+
 # ---------------------------------------------------------------------------
 # Hadamard
 
@@ -241,6 +254,26 @@ def check_sr_threshold_exact():
                 assert down == (sgn * lo if lo != 0 else 0.0), (u, n, down)
     for u in (6.0, 7.5, 1e9):
         assert O.e2m1_value(O.e2m1_sr(u, 0.999)) == 6.0
+
+
+def check_sr_threshold_exact_16bit():
+    """With the 16-bit element uniforms rho = m 2^-16, SR rounds up for exactly
+    ceil(p * 2^16) of the 2^16 values: up at m = n - 1, down at m = n (p the
+    exact fraction between the grid neighbours)."""
+    rng = np.random.default_rng(14)
+    grid = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    probe = [0.1, 0.3, 0.74, 1.1, 1.9, 2.2, 3.3, 3.99, 4.5, 5.9, 5.99999, 0.25 + 2.0**-20, 1.0 + 2.0**-17]
+    for u in probe + rng.uniform(0, 6, 40).tolist():
+        u = float(np.float32(u))
+        a = Fraction(u)
+        lo = max(g for g in grid if g <= a)
+        hi = min(g for g in grid if g > a)
+        p = (a - Fraction(lo)) / (Fraction(hi) - Fraction(lo))
+        n = -((-p * 2**16).numerator // (p * 2**16).denominator)  # ceil
+        if n > 0:
+            assert O.e2m1_value(O.e2m1_sr(u, (n - 1) * 2.0**-16)) == hi, (u, n)
+        if n < 2**16:
+            assert O.e2m1_value(O.e2m1_sr(u, n * 2.0**-16)) == lo, (u, n)
 
 
 def check_e4m3_sr_threshold_exact():
@@ -585,7 +618,8 @@ def check_hadamard_cancels_in_gemm():
 ALL_CHECKS = [
     check_e2m1_value_set, check_e2m1_rtn_exhaustive_bf16, check_e4m3_matches_torch, check_e8m0_matches_torch,
     check_philox_matches_torch_engine, check_sylvester_matches_scipy, check_fwht_is_matrix_product,
-    check_rotation_orthonormal, check_sr_threshold_exact, check_e4m3_sr_threshold_exact,
+    check_element_uniform_layout, check_rotation_orthonormal, check_sr_threshold_exact,
+    check_sr_threshold_exact_16bit, check_e4m3_sr_threshold_exact,
     check_e8m0_sr_threshold_exact,
     check_sr_unbiased_rtn_biased, check_quartet2_projection_unbiased, check_quartet2_error_half_of_sr,
     check_quartet2_alpha_range,

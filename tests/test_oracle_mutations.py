@@ -34,6 +34,10 @@ MUTATIONS = [
     ("col_orientation", "for (int64_t j = 0; j < k; ++j) seg[j] = bf16_to_f32(x[j * ld + row]);",
      "for (int64_t j = 0; j < k; ++j) seg[j] = bf16_to_f32(x[(j ^ 1) * ld + row]);"),
     ("scale_sr_always_down", "return (uint8_t)((rho < p) ? lo + 1 : lo);", "return (uint8_t)lo;"),
+    ("element_uniform_half", "return (float)((w >> (16u * (uint32_t)(i & 1u))) & 0xFFFFu) * 0x1p-16f;",
+     "return (float)(w & 0xFFFFu) * 0x1p-16f;"),
+    ("element_uniform_word", "const uint32_t w = random_word(seed, TAG_ELEMENT, stream, i >> 1);",
+     "const uint32_t w = random_word(seed, TAG_ELEMENT, stream, i >> 2);"),
     ("element_sr_index", "const uint64_t i = (uint64_t)(r * k + b * nb + j);", "const uint64_t i = (uint64_t)(r * k + b * nb);"),
     ("e8m0_sr_compare_flipped", "    if (rho < p) e += 1;\n", "    if (rho > p) e += 1;\n"),
     ("e8m0_sr_probability", "float p = (t - lo) / lo; /* exact: t in [lo, 2 lo) */",
