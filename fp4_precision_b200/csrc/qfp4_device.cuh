@@ -55,6 +55,8 @@ __device__ __forceinline__ uint4 philox_quad(uint64_t seed, uint32_t tag_stream,
 
 // Uniform in [0, 1) on the 2^-24 grid.
 __device__ __forceinline__ float uniform24(uint32_t w) { return __uint2float_rn(w >> 8) * 0x1p-24f; }
+// Uniform in [0, 1) on the 2^-16 grid from a 16-bit value (element SR).
+__device__ __forceinline__ float uniform16(uint32_t h) { return __uint2float_rn(h) * 0x1p-16f; }
 
 // ---------------------------------------------------------------------------
 // bf16 pairs -> fp32 (exact)

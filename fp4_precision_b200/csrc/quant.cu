@@ -313,14 +313,20 @@ struct Group {
             // element rounding
             uint32_t* cb = codes + b * (NB / 8);
             if constexpr (RND == kSr) {
+                // 16-bit uniforms, two per word: element j = i0 + e takes half
+                // j % 2 of word j / 2 of the element stream, i.e. of word
+                // (e / 2) % 4 of the Philox quad (i0 + e) / 8 (i0 is a
+                // multiple of 16)
                 const uint64_t i0 = elem0 + (uint64_t)(b * NB);
 #pragma unroll
-                for (int e4 = 0; e4 < NB; e4 += 4) {
-                    const uint4 w = philox_quad(p.seed, p.tag_elem, (i0 + e4) >> 2);
-                    vb[e4 + 0] = e2m1_sr_value(vb[e4 + 0], uniform24(w.x));
-                    vb[e4 + 1] = e2m1_sr_value(vb[e4 + 1], uniform24(w.y));
-                    vb[e4 + 2] = e2m1_sr_value(vb[e4 + 2], uniform24(w.z));
-                    vb[e4 + 3] = e2m1_sr_value(vb[e4 + 3], uniform24(w.w));
+                for (int e8 = 0; e8 < NB; e8 += 8) {
+                    const uint4 w = philox_quad(p.seed, p.tag_elem, (i0 + e8) >> 3);
+                    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                    for (int h = 0; h < 4; ++h) {
+                        vb[e8 + 2 * h] = e2m1_sr_value(vb[e8 + 2 * h], uniform16(ws[h] & 0xFFFFu));
+                        vb[e8 + 2 * h + 1] = e2m1_sr_value(vb[e8 + 2 * h + 1], uniform16(ws[h] >> 16));
+                    }
                 }
             }
 #pragma unroll
@@ -522,6 +528,7 @@ template <int RND, int NH, typename Load>
 __device__ __forceinline__ uint32_t nv64_quantize(Load load, const SignFlips& sf, float s_enc, const float2* tab,
                                                   const Stream& st, uint64_t elem0, uint64_t block0, uint32_t* codes) {
     static_assert(NH == 0 || NH == 16, "the packed unit takes no Hadamard or a 16-point one");
+    static_assert(RND != kSr, "per-element SR stays on the group path");
     uint32_t scw = 0;
     uint4 rq = make_uint4(0u, 0u, 0u, 0u);
     if constexpr (RND == kQuartet2) {
@@ -567,22 +574,6 @@ __device__ __forceinline__ uint32_t nv64_quantize(Load load, const SignFlips& sf
 #pragma unroll
         for (int j = 0; j < 16; ++j) P[j] = __fmul2_rn(P[j], rr);
         uint32_t* cw = codes + 4 * bp;  // block 2bp: cw[0..1], block 2bp + 1: cw[2..3]
-        if constexpr (RND == kSr) {
-#pragma unroll
-            for (int lane = 0; lane < 2; ++lane) {
-                const uint64_t i0 = elem0 + (uint64_t)(16 * (2 * bp + lane));
-#pragma unroll
-                for (int e4 = 0; e4 < 16; e4 += 4) {
-                    const uint4 w = philox_quad(st.seed, st.tag_elem, (i0 >> 2) + (uint64_t)(e4 >> 2));
-                    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        float& u = lane ? P[e4 + e].y : P[e4 + e].x;
-                        u = e2m1_sr_value(u, uniform24(ws[e]));
-                    }
-                }
-            }
-        }
         if constexpr (RND != kQuartet2) {
             cw[0] = e2m1x8_words(P[0].x, P[1].x, P[2].x, P[3].x, P[4].x, P[5].x, P[6].x, P[7].x);
             cw[1] = e2m1x8_words(P[8].x, P[9].x, P[10].x, P[11].x, P[12].x, P[13].x, P[14].x, P[15].x);
