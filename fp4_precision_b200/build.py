@@ -10,6 +10,9 @@ import subprocess
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libqfp4.so")
+# the same library with every kernel store address checked (QFP4_BOUNDS_CHECK):
+# a store outside its buffer is dropped and reported by qfp4_status
+LIB_BOUNDS_CHECK = os.path.join(HERE, "libqfp4_bc.so")
 SOURCES = sorted(glob.glob(os.path.join(HERE, "csrc", "*.cu")) + glob.glob(os.path.join(HERE, "csrc", "*.cuh"))
                  + glob.glob(os.path.join(HERE, "csrc", "*.h")) + [os.path.join(ROOT, "include", "qfp4.h")])
 
@@ -29,27 +32,29 @@ def nvcc() -> str:
     return "nvcc"
 
 
-def stale() -> bool:
-    if not os.path.exists(LIB):
+def stale(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return any(os.path.getmtime(s) > t for s in SOURCES)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and not stale():
-        return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
+def build(force: bool = False, verbose: bool = False, bounds_check: bool = False) -> str:
+    lib = LIB_BOUNDS_CHECK if bounds_check else LIB
+    if not force and not stale(lib):
+        return lib
+    tmp = lib + f".tmp{os.getpid()}"
     cmd = [nvcc(), *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"), os.path.join(HERE, "csrc", "qfp4_lib.cu"),
            "-o", tmp]
+    if bounds_check:
+        cmd[1:1] = ["-DQFP4_BOUNDS_CHECK"]
     if verbose:
         cmd[1:1] = ["-Xptxas", "-v"]
     subprocess.check_call(cmd)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
     import sys
-    build(force=True, verbose="-v" in sys.argv)
-    print(LIB)
+    print(build(force=True, verbose="-v" in sys.argv, bounds_check="--bounds-check" in sys.argv))

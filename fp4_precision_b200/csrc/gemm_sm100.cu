@@ -239,6 +239,16 @@ __device__ __forceinline__ uint32_t pack_bf16(uint32_t a, uint32_t b, float scal
     return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// Extents (bytes) of D and of the MXFP4 copy of the output, for the
+// bounds-checked build.
+__device__ __forceinline__ int64_t d_extent(const GemmParams& p) {
+    return p.M <= 0 ? 0 : ((int64_t)(p.M - 1) * p.ldd + p.N) * (p.out_f32 ? 4 : 2);
+}
+__device__ __forceinline__ int64_t q_codes_extent(const GemmParams& p) { return (int64_t)p.M * (p.N / 2); }
+__device__ __forceinline__ int64_t q_scales_extent(const GemmParams& p) {
+    return (int64_t)((p.M + 127) / 128) * (p.q_kb4 / 4) * 512;
+}
+
 // Epilogue stores of one row's NC columns from column n0, with evict-first
 // stores so the output stream does not push the operand tiles out of L2.
 // bf16: NC / 2 packed words; fp32: NC accumulator words times gA * gB.
@@ -248,7 +258,8 @@ __device__ __forceinline__ void store_bf16(const GemmParams& p, const uint32_t* 
     __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.D) + (int64_t)row * p.ldd + n0;
 #pragma unroll
     for (int c = 0; c < NC; c += 8)
-        __stcs(reinterpret_cast<uint4*>(dst + c), make_uint4(w[c / 2], w[c / 2 + 1], w[c / 2 + 2], w[c / 2 + 3]));
+        __stcs(chk(reinterpret_cast<uint4*>(dst + c), p.D, d_extent(p)),
+               make_uint4(w[c / 2], w[c / 2 + 1], w[c / 2 + 2], w[c / 2 + 3]));
 }
 // Ragged right edge: the first nv (< NC) of NC bf16 columns, element by element.
 template <int NC>
@@ -258,7 +269,7 @@ __device__ __forceinline__ void store_bf16_edge(const GemmParams& p, const uint3
     const int nv = p.N - n0;
 #pragma unroll
     for (int c = 0; c < NC; ++c)
-        if (c < nv) d16[c] = (uint16_t)(w[c >> 1] >> (16 * (c & 1)));
+        if (c < nv) *chk(d16 + c, p.D, d_extent(p)) = (uint16_t)(w[c >> 1] >> (16 * (c & 1)));
 }
 template <int NC>
 __device__ __forceinline__ void store_f32(const GemmParams& p, uint32_t* acc, int row, int n0, float scale) {
@@ -275,22 +286,27 @@ __device__ __forceinline__ void store_f32(const GemmParams& p, uint32_t* acc, in
         const int nv = p.N - n0;
 #pragma unroll
         for (int c = 0; c < NC; ++c)
-            if (c < nv) dst[c] = __fadd_rn(dst[c], __uint_as_float(acc[c]));
+            if (c < nv) {
+                float* d = chk(dst + c, p.D, d_extent(p));
+                *d = __fadd_rn(*d, __uint_as_float(acc[c]));
+            }
     } else if (n0 + NC <= p.N) {
 #pragma unroll
         for (int c = 0; c < NC; c += 4)
-            __stcs(reinterpret_cast<uint4*>(dst + c), make_uint4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]));
+            __stcs(chk(reinterpret_cast<uint4*>(dst + c), p.D, d_extent(p)),
+                   make_uint4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]));
     } else {  // ragged right edge: nv < NC valid columns, whole 4-column chunks first
         const int nv = p.N - n0, nfull = nv >> 2, rem = nv & 3;
         uint32_t* d32 = reinterpret_cast<uint32_t*>(dst);
 #pragma unroll
         for (int c = 0; c < NC; c += 4) {
             if ((c >> 2) < nfull) {
-                __stcs(reinterpret_cast<uint4*>(dst + c), make_uint4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]));
+                __stcs(chk(reinterpret_cast<uint4*>(dst + c), p.D, d_extent(p)),
+                       make_uint4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]));
             } else if ((c >> 2) == nfull && rem != 0) {
 #pragma unroll
                 for (int h = 0; h < 3; ++h)
-                    if (h < rem) d32[c + h] = acc[c + h];
+                    if (h < rem) *chk(d32 + c + h, p.D, d_extent(p)) = acc[c + h];
             }
         }
     }
@@ -377,16 +393,16 @@ __device__ __forceinline__ void quantize_out_row128(const GemmParams& p, const u
         uint32_t codes[4];
         Grp::quantize(v, 1.0f, nullptr, st, 0, 0, srng, codes, scodes + blk);
         if (r < p.M && n0 + 32 * blk < p.N)
-            *reinterpret_cast<uint4*>(p.q_codes + (int64_t)r * (p.N / 2) + (n0 + 32 * blk) / 2) =
-                make_uint4(codes[0], codes[1], codes[2], codes[3]);
+            *chk(reinterpret_cast<uint4*>(p.q_codes + (int64_t)r * (p.N / 2) + (n0 + 32 * blk) / 2), p.q_codes,
+                 q_codes_extent(p)) = make_uint4(codes[0], codes[1], codes[2], codes[3]);
     }
     // rows up to the 128-row padding of the atoms; past M the accumulator is
     // zero (zero-filled A rows), so those scales are the zero padding
     if (r < (p.M + 127) / 128 * 128) {
         const int64_t kb0 = n0 / 32;
-        *reinterpret_cast<uint32_t*>(p.q_scales + ((int64_t)(r / 128) * (p.q_kb4 / 4) + kb0 / 4) * 512 +
-                                     (r % 32) * 16 + ((r / 32) % 4) * 4) =
-            scodes[0] | (scodes[1] << 8) | (scodes[2] << 16) | (scodes[3] << 24);
+        *chk(reinterpret_cast<uint32_t*>(p.q_scales + ((int64_t)(r / 128) * (p.q_kb4 / 4) + kb0 / 4) * 512 +
+                                         (r % 32) * 16 + ((r / 32) % 4) * 4),
+             p.q_scales, q_scales_extent(p)) = scodes[0] | (scodes[1] << 8) | (scodes[2] << 16) | (scodes[3] << 24);
     }
 }
 
@@ -913,7 +929,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
                 for (int i = 0; i < kEpiWarps; ++i) m = fmaxf(m, warp_max[i]);
                 if constexpr (AMX > 0) m = __fmul_rn(m, AMX == 16 ? 0.25f : 0x1.6a09e6p-3f);  // fp32(1/sqrt(n_h))
-                p.amax_partials[blockIdx.x] = m;
+                *chk(p.amax_partials + blockIdx.x, p.amax_partials, (int64_t)gridDim.x * 4) = m;
             }
         }
     }

@@ -6,6 +6,7 @@
 // dX = dY W, Wgrad dW = dY^T X).
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <cstdlib>
 #include <cstring>
@@ -18,6 +19,17 @@ namespace qfp4 {
 namespace {
 
 thread_local int t_last_cuda_error = 0;
+
+// An NVTX range named after the entry point around every call that touches
+// the device, so that a profiler's timeline shows which library call issued
+// which launches (header-only NVTX: without an attached tool a push or pop is
+// one test of a null function pointer).
+struct ApiRange {
+    explicit ApiRange(const char* name) { nvtxRangePushA(name); }
+    ~ApiRange() { nvtxRangePop(); }
+    ApiRange(const ApiRange&) = delete;
+    ApiRange& operator=(const ApiRange&) = delete;
+};
 thread_local int64_t t_launches = 0;
 
 int cuda_fail(cudaError_t e) {
@@ -781,6 +793,7 @@ const char* qfp4_strerror(int status) {
         case QFP4_ERR_WORKSPACE: return "workspace missing or too small";
         case QFP4_ERR_CUDA: return "CUDA error";
         case QFP4_ERR_TIMEOUT: return "device-side bounded wait expired";
+        case QFP4_ERR_BOUNDS: return "bounds-checked build: a kernel store fell outside its buffer";
         case QFP4_ERR_TOO_LARGE: return "problem exceeds the fixed scratch of qfp4_linear_fwd_noalloc (32 MiB)";
         default: return "unknown status";
     }
@@ -814,6 +827,7 @@ size_t qfp4_quantize_workspace_bytes(void) { return (size_t)kMaxAmaxPartials * s
 
 int qfp4_amax(const void* x, int64_t R, int64_t C, int64_t ld, int32_t had, int32_t axis, const qfp4_seed* seed,
               float* amax, void* workspace, size_t workspace_bytes, void* stream) {
+    const ApiRange range("qfp4_amax");
     int sms = 0;
     int rc = bind_context(static_cast<cudaStream_t>(stream));
     if (rc) return rc;
@@ -840,6 +854,7 @@ int qfp4_amax(const void* x, int64_t R, int64_t C, int64_t ld, int32_t had, int3
 int qfp4_amax_rowcol(const void* x, int64_t R, int64_t C, int64_t ld, int32_t had, const qfp4_seed* seed_row,
                      const qfp4_seed* seed_col, float* amax_row, float* amax_col, void* workspace,
                      size_t workspace_bytes, void* stream) {
+    const ApiRange range("qfp4_amax_rowcol");
     return amax_rowcol_impl(x, R, C, ld, had, seed_row, seed_col, amax_row, amax_col, workspace, workspace_bytes,
                             static_cast<cudaStream_t>(stream));
 }
@@ -847,6 +862,7 @@ int qfp4_amax_rowcol(const void* x, int64_t R, int64_t C, int64_t ld, int32_t ha
 int qfp4_quantize(const void* x, int64_t R, int64_t C, int64_t ld, int32_t fmt, int32_t rounding, int32_t had,
                   int32_t axis, const qfp4_seed* seed, const float* amax_in, qfp4_tensor* out, void* workspace,
                   size_t workspace_bytes, void* stream) {
+    const ApiRange range("qfp4_quantize");
     return quantize_impl(x, R, C, ld, fmt, rounding, had, axis, seed, amax_in, out, workspace, workspace_bytes,
                          static_cast<cudaStream_t>(stream));
 }
@@ -855,27 +871,32 @@ int qfp4_quantize_dual(const void* x, int64_t R, int64_t C, int64_t ld, int32_t 
                        int32_t had_row, int32_t had_col, const qfp4_seed* seed_row, const qfp4_seed* seed_col,
                        const float* amax_row, const float* amax_col, qfp4_tensor* out_row, qfp4_tensor* out_col,
                        void* stream) {
+    const ApiRange range("qfp4_quantize_dual");
     return quantize_dual_impl(x, R, C, ld, fmt, rounding, had_row, had_col, seed_row, seed_col, amax_row, amax_col,
                               out_row, out_col, static_cast<cudaStream_t>(stream));
 }
 
 int qfp4_gemm(const qfp4_tensor* A, const qfp4_tensor* B, void* D, int64_t ldd, int32_t out_dtype, void* stream) {
+    const ApiRange range("qfp4_gemm");
     return gemm_impl(A, B, D, ldd, out_dtype, false, static_cast<cudaStream_t>(stream));
 }
 
 int qfp4_gemm_quantize(const qfp4_tensor* A, const qfp4_tensor* B, void* D, int64_t ldd, int32_t had,
                        const qfp4_seed* seed, qfp4_tensor* out, void* stream) {
+    const ApiRange range("qfp4_gemm_quantize");
     const QuantOut qo{had, seed, out};
     return gemm_impl(A, B, D, ldd, QFP4_OUT_BF16, false, static_cast<cudaStream_t>(stream), &qo);
 }
 
 int qfp4_gemm_amax(const qfp4_tensor* A, const qfp4_tensor* B, void* D, int64_t ldd, int32_t had,
                    const qfp4_seed* seed, float* amax, void* workspace, size_t workspace_bytes, void* stream) {
+    const ApiRange range("qfp4_gemm_amax");
     const AmaxOut ao{had, seed, amax, workspace, workspace_bytes};
     return gemm_impl(A, B, D, ldd, QFP4_OUT_BF16, false, static_cast<cudaStream_t>(stream), nullptr, &ao);
 }
 
 int qfp4_gemm_accumulate(const qfp4_tensor* A, const qfp4_tensor* B, float* D, int64_t ldd, void* stream) {
+    const ApiRange range("qfp4_gemm_accumulate");
     return gemm_impl(A, B, D, ldd, QFP4_OUT_F32, true, static_cast<cudaStream_t>(stream));
 }
 
@@ -963,6 +984,7 @@ extern "C" {
 
 int qfp4_linear_fwd(const void* X, const void* W, void* Y, int64_t M, int64_t N, int64_t K, const qfp4_recipe* recipe,
                     const qfp4_seed* seed, void* workspace, size_t workspace_bytes, void* stream) {
+    const ApiRange range("qfp4_linear_fwd");
     return linear_fwd_impl(X, W, Y, M, N, K, recipe, seed, nullptr, QFP4_HAD_NONE, nullptr, nullptr, workspace,
                            workspace_bytes, static_cast<cudaStream_t>(stream));
 }
@@ -971,6 +993,7 @@ int qfp4_linear_fwd_chain(const void* X, const void* W, void* Y, int64_t M, int6
                           const qfp4_recipe* recipe, const qfp4_seed* seed, const float* x_amax, int32_t next_had,
                           const qfp4_seed* next_seed, float* y_amax, void* workspace, size_t workspace_bytes,
                           void* stream) {
+    const ApiRange range("qfp4_linear_fwd_chain");
     return linear_fwd_impl(X, W, Y, M, N, K, recipe, seed, x_amax, next_had, next_seed, y_amax, workspace,
                            workspace_bytes, static_cast<cudaStream_t>(stream));
 }
@@ -978,6 +1001,7 @@ int qfp4_linear_fwd_chain(const void* X, const void* W, void* Y, int64_t M, int6
 int qfp4_linear_bwd(const void* dY, const void* X, const void* W, void* dX, void* dW, int64_t M, int64_t N, int64_t K,
                     const qfp4_recipe* recipe, const qfp4_seed* seed, void* workspace, size_t workspace_bytes,
                     void* stream) {
+    const ApiRange range("qfp4_linear_bwd");
     int rc = check_linear_args(M, N, K, recipe, seed);
     if (rc) return rc;
     if (!dY || !X || !W || !dX || !dW) return QFP4_ERR_INVALID_ARG;
@@ -1038,6 +1062,7 @@ int qfp4_linear_bwd(const void* dY, const void* X, const void* W, void* dX, void
 }
 
 int qfp4_status(void* stream) {
+    const ApiRange range("qfp4_status");
     const int rc = bind_context(static_cast<cudaStream_t>(stream));
     if (rc) return rc;
     cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
@@ -1047,7 +1072,7 @@ int qfp4_status(void* stream) {
     if (v != 0) {
         const uint32_t zero = 0;
         if ((e = cudaMemcpyToSymbol(g_dev_error, &zero, sizeof zero)) != cudaSuccess) return cuda_fail(e);
-        return QFP4_ERR_TIMEOUT;
+        return (v & DEV_ERR_BOUNDS) ? QFP4_ERR_BOUNDS : QFP4_ERR_TIMEOUT;
     }
     return QFP4_OK;
 }
@@ -1071,6 +1096,7 @@ __global__ void wait_timeout_kernel(uint64_t limit_ns) {
 }  // namespace qfp4
 
 int qfp4_selftest_wait_timeout(int64_t limit_ns, void* stream) {
+    const ApiRange range("qfp4_selftest_wait_timeout");
     const int rc = bind_context(static_cast<cudaStream_t>(stream));
     if (rc) return rc;
     if (limit_ns <= 0 || limit_ns > (int64_t)kWaitLimitNs) return QFP4_ERR_INVALID_ARG;
@@ -1126,6 +1152,7 @@ static int noalloc_scratch(void** out) {
 
 int qfp4_linear_fwd_noalloc(const void* X, const void* W, void* Y, int64_t M, int64_t N, int64_t K,
                             const qfp4_recipe* recipe, const qfp4_seed* seed, void* stream) {
+    const ApiRange range("qfp4_linear_fwd_noalloc");
     int rc = check_linear_args(M, N, K, recipe, seed);
     if (rc) return rc;
     if (qfp4_linear_workspace_bytes(0, M, N, K, recipe) > QFP4_NOALLOC_SCRATCH_BYTES) return QFP4_ERR_TOO_LARGE;

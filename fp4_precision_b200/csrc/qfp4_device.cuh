@@ -12,11 +12,35 @@ namespace qfp4 {
 
 // ---------------------------------------------------------------------------
 // error word: set by a kernel whose bounded wait expired; read by qfp4_status()
-enum : uint32_t { DEV_ERR_NONE = 0, DEV_ERR_TIMEOUT = 1 };
+// DEV_ERR_BOUNDS: a bounds-checked build caught a store outside its buffer
+enum : uint32_t { DEV_ERR_NONE = 0, DEV_ERR_TIMEOUT = 1, DEV_ERR_BOUNDS = 2 };
 // (the library is one translation unit, see qfp4_lib.cu, so this is its only definition)
 __device__ uint32_t g_dev_error = 0;
 
 __device__ __forceinline__ void raise_device_error(uint32_t code) { atomicOr(&g_dev_error, code); }
+
+// Store-address check. In a bounds-checked build (-DQFP4_BOUNDS_CHECK, see
+// fp4_precision_b200/build.py) every global store of the kernels goes through
+// chk(): if the n bytes at p do not lie inside [base, base + size), it raises
+// DEV_ERR_BOUNDS and returns a scratch sink instead, so nothing outside the
+// buffer is written and nothing traps (qfp4_status then returns
+// QFP4_ERR_BOUNDS). In the normal build chk() returns p.
+__device__ __align__(16) uint8_t g_bounds_sink[64];
+template <typename T>
+__device__ __forceinline__ T* chk(T* p, const void* base, int64_t size, int64_t n = (int64_t)sizeof(T)) {
+#ifdef QFP4_BOUNDS_CHECK
+    const int64_t off = reinterpret_cast<const uint8_t*>(p) - reinterpret_cast<const uint8_t*>(base);
+    if (base == nullptr || off < 0 || off + n > size || n > (int64_t)sizeof(g_bounds_sink)) {
+        raise_device_error(DEV_ERR_BOUNDS);
+        return reinterpret_cast<T*>(g_bounds_sink);
+    }
+#else
+    (void)base;
+    (void)size;
+    (void)n;
+#endif
+    return p;
+}
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {
     uint64_t t;

@@ -357,16 +357,28 @@ struct Group {
     }
 };
 
+// Extents of the output buffers (bytes), for the bounds-checked build.
+__device__ __forceinline__ int64_t codes_extent(const QuantParams& p) { return p.rows * (p.k / 2); }
+__device__ __forceinline__ int64_t scales_extent(const QuantParams& p) {
+    return (p.rows + 127) / 128 * (p.kb4 / 4) * 512;
+}
+__device__ __forceinline__ int64_t codes_row_extent(const QuantParams& p) { return p.R * (p.C / 2); }
+__device__ __forceinline__ int64_t scales_row_extent(const QuantParams& p) {
+    return (p.R + 127) / 128 * (p.kb4_row / 4) * 512;
+}
+
 // 32 bytes of codes (64 elements of one row): two 16-byte stores, or four
 // 8-byte ones when the row length in bytes (k / 2) is not a multiple of 16
 // (k a multiple of 16 but not of 32: rows start 8-byte aligned).
-__device__ __forceinline__ void store_codes32(uint8_t* dst, const uint32_t* codes, bool aligned16) {
+__device__ __forceinline__ void store_codes32(uint8_t* dst, const uint32_t* codes, bool aligned16, const void* base,
+                                              int64_t extent) {
     if (aligned16) {
-        reinterpret_cast<uint4*>(dst)[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
-        reinterpret_cast<uint4*>(dst)[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
+        *chk(reinterpret_cast<uint4*>(dst), base, extent) = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+        *chk(reinterpret_cast<uint4*>(dst) + 1, base, extent) = make_uint4(codes[4], codes[5], codes[6], codes[7]);
     } else {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) reinterpret_cast<uint2*>(dst)[i] = make_uint2(codes[2 * i], codes[2 * i + 1]);
+        for (int i = 0; i < 4; ++i)
+            *chk(reinterpret_cast<uint2*>(dst) + i, base, extent) = make_uint2(codes[2 * i], codes[2 * i + 1]);
     }
 }
 
@@ -711,7 +723,7 @@ __device__ __forceinline__ void write_partial(float m, float* red, float* out) {
     if (threadIdx.x == 0) {
         float r = 0.0f;
         for (int w = 0; w < kComputeWarps; ++w) r = fmaxf(r, red[w]);
-        out[blockIdx.x] = r;
+        *chk(out + blockIdx.x, out, (int64_t)kMaxAmaxPartials * 4) = r;
     }
 }
 
@@ -920,11 +932,11 @@ __global__ void __launch_bounds__(kThreads, 2)
             if (row < p.rows) {
                 uint8_t* dst = p.codes + row * (p.k / 2) + col0 / 2;
                 if (col0 + kRowTileCols <= p.k) {
-                    store_codes32(dst, codes, ((p.k / 2) & 15) == 0);
+                    store_codes32(dst, codes, ((p.k / 2) & 15) == 0, p.codes, codes_extent(p));
                 } else {
 #pragma unroll
                     for (int w = 0; w < 8; ++w)
-                        if (col0 + 8 * w < p.k) reinterpret_cast<uint32_t*>(dst)[w] = codes[w];
+                        if (col0 + 8 * w < p.k) *chk(reinterpret_cast<uint32_t*>(dst) + w, p.codes, codes_extent(p)) = codes[w];
                 }
             }
             if (row < rows_pad) {
@@ -937,16 +949,17 @@ __global__ void __launch_bounds__(kThreads, 2)
                            : ((row / 128) * (p.kb4 / 4) + kb0 / 4) * 512 + (row % 32) * 16 + ((row / 32) % 4) * 4;
                 if constexpr (NB == 16) {
                     if constexpr (kPacked)
-                        *reinterpret_cast<uint32_t*>(p.scales + off) = scw;
+                        *chk(reinterpret_cast<uint32_t*>(p.scales + off), p.scales, scales_extent(p)) = scw;
                     else
-                        *reinterpret_cast<uint32_t*>(p.scales + off) =
+                        *chk(reinterpret_cast<uint32_t*>(p.scales + off), p.scales, scales_extent(p)) =
                             scodes[0] | (scodes[1] << 8) | (scodes[2] << 16) | (scodes[3] << 24);
                 } else {
                     const uint32_t half = scodes[0] | (scodes[1] << 8);
                     if ((kb0 & 3) == 0 && col0 + kRowTileCols >= p.k)
-                        *reinterpret_cast<uint32_t*>(p.scales + off) = half;
+                        *chk(reinterpret_cast<uint32_t*>(p.scales + off), p.scales, scales_extent(p)) = half;
                     else
-                        *reinterpret_cast<uint16_t*>(p.scales + off + (kb0 & 3)) = (uint16_t)half;
+                        *chk(reinterpret_cast<uint16_t*>(p.scales + off + (kb0 & 3)), p.scales, scales_extent(p)) =
+                            (uint16_t)half;
                 }
             }
         }
@@ -1158,9 +1171,10 @@ __global__ void __launch_bounds__(kThreads, 2)
                 if (c < p.rows && r_grp < p.k) {
                     uint8_t* dst = p.codes + c0 * (p.k / 2) + code_off[ci] + r_grp / 2;
                     if constexpr (G == 16)
-                        *reinterpret_cast<uint2*>(dst) = make_uint2(codes[0], codes[1]);
+                        *chk(reinterpret_cast<uint2*>(dst), p.codes, codes_extent(p)) = make_uint2(codes[0], codes[1]);
                     else
-                        *reinterpret_cast<uint4*>(dst) = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+                        *chk(reinterpret_cast<uint4*>(dst), p.codes, codes_extent(p)) =
+                            make_uint4(codes[0], codes[1], codes[2], codes[3]);
                 }
                 // Scales: the 4 lanes of column c (q = 0..3, consecutive lanes) hold
                 // scale columns kb0 + (G/NB) q + b; gather them into 4-byte atom words.
@@ -1174,12 +1188,12 @@ __global__ void __launch_bounds__(kThreads, 2)
                     const int64_t rowoff = (c0 / 128) * atom_row_bytes + sc_off[ci];
                     if constexpr (G / NB == 1) {
                         if (q == 0 && kb0 / 4 < p.kb4 / 4)
-                            *reinterpret_cast<uint32_t*>(p.scales + rowoff + (kb0 / 4) * 512) =
-                                mine | (n1 << 8) | (n2 << 16) | (n3 << 24);
+                            *chk(reinterpret_cast<uint32_t*>(p.scales + rowoff + (kb0 / 4) * 512), p.scales,
+                                 scales_extent(p)) = mine | (n1 << 8) | (n2 << 16) | (n3 << 24);
                     } else {
                         if ((q == 0 || q == 2) && kb0 / 4 + q / 2 < p.kb4 / 4)
-                            *reinterpret_cast<uint32_t*>(p.scales + rowoff + (kb0 / 4 + q / 2) * 512) =
-                                mine | (n1 << 16);
+                            *chk(reinterpret_cast<uint32_t*>(p.scales + rowoff + (kb0 / 4 + q / 2) * 512), p.scales,
+                                 scales_extent(p)) = mine | (n1 << 16);
                     }
                 }
             }
@@ -1271,11 +1285,12 @@ __device__ __forceinline__ void dual_row_work(const QuantParams& p, float s_enc_
     if (r < p.R) {
         uint8_t* dst = p.codes_row + r * (p.C / 2) + c0 / 2;
         if (c0 + 64 <= p.C) {
-            store_codes32(dst, codes, ((p.C / 2) & 15) == 0);
+            store_codes32(dst, codes, ((p.C / 2) & 15) == 0, p.codes_row, codes_row_extent(p));
         } else {
 #pragma unroll
             for (int w = 0; w < 8; ++w)
-                if (c0 + 8 * w < p.C) reinterpret_cast<uint32_t*>(dst)[w] = codes[w];
+                if (c0 + 8 * w < p.C)
+                    *chk(reinterpret_cast<uint32_t*>(dst) + w, p.codes_row, codes_row_extent(p)) = codes[w];
         }
     }
     if (r < (p.R + 127) / 128 * 128) {
@@ -1284,15 +1299,16 @@ __device__ __forceinline__ void dual_row_work(const QuantParams& p, float s_enc_
                       ((r / 32) % 4) * 4;
         if constexpr (NB == 16) {
             if constexpr (kPackedRow)
-                *reinterpret_cast<uint32_t*>(sc) = scw;
+                *chk(reinterpret_cast<uint32_t*>(sc), p.scales_row, scales_row_extent(p)) = scw;
             else
-                *reinterpret_cast<uint32_t*>(sc) = scodes[0] | (scodes[1] << 8) | (scodes[2] << 16) | (scodes[3] << 24);
+                *chk(reinterpret_cast<uint32_t*>(sc), p.scales_row, scales_row_extent(p)) =
+                    scodes[0] | (scodes[1] << 8) | (scodes[2] << 16) | (scodes[3] << 24);
         } else {
             const uint32_t half = scodes[0] | (scodes[1] << 8);
             if ((kb0 & 3) == 0 && c0 + 64 >= p.C)
-                *reinterpret_cast<uint32_t*>(sc) = half;
+                *chk(reinterpret_cast<uint32_t*>(sc), p.scales_row, scales_row_extent(p)) = half;
             else
-                *reinterpret_cast<uint16_t*>(sc + (kb0 & 3)) = (uint16_t)half;
+                *chk(reinterpret_cast<uint16_t*>(sc + (kb0 & 3)), p.scales_row, scales_row_extent(p)) = (uint16_t)half;
         }
     }
 }
@@ -1467,17 +1483,17 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (rb < p.k) {  // k is a multiple of 64: a band is wholly inside or wholly outside
             if (c < p.rows) {
                 uint4* dst = reinterpret_cast<uint4*>(p.codes + c * (p.k / 2) + rb / 2);
-                dst[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
-                dst[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
+                *chk(dst, p.codes, codes_extent(p)) = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+                *chk(dst + 1, p.codes, codes_extent(p)) = make_uint4(codes[4], codes[5], codes[6], codes[7]);
             }
             if (c < rows_pad) {
                 const int64_t kb0 = rb / NB;
                 uint8_t* sc = p.scales + (c / 128) * atom_row_bytes + (kb0 / 4) * 512 + (c % 32) * 16 + ((c / 32) % 4) * 4;
                 if constexpr (NB == 16) {
                     if constexpr (kPacked)
-                        *reinterpret_cast<uint32_t*>(sc) = scw;
+                        *chk(reinterpret_cast<uint32_t*>(sc), p.scales, scales_extent(p)) = scw;
                     else
-                        *reinterpret_cast<uint32_t*>(sc) =
+                        *chk(reinterpret_cast<uint32_t*>(sc), p.scales, scales_extent(p)) =
                             scodes[0] | (scodes[1] << 8) | (scodes[2] << 16) | (scodes[3] << 24);
                 } else {
                     // two scale columns: half of an atom word; when this is the
@@ -1485,9 +1501,9 @@ __global__ void __launch_bounds__(kThreads, 2)
                     // half is padding and is written as zero
                     const uint32_t half = scodes[0] | (scodes[1] << 8);
                     if ((kb0 & 3) == 0 && rb + 64 >= p.k)
-                        *reinterpret_cast<uint32_t*>(sc) = half;
+                        *chk(reinterpret_cast<uint32_t*>(sc), p.scales, scales_extent(p)) = half;
                     else
-                        *reinterpret_cast<uint16_t*>(sc + (kb0 & 3)) = (uint16_t)half;
+                        *chk(reinterpret_cast<uint16_t*>(sc + (kb0 & 3)), p.scales, scales_extent(p)) = (uint16_t)half;
                 }
             }
         }

@@ -14,7 +14,9 @@ from dataclasses import dataclass
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libqfp4.so")
+# QFP4_BOUNDS_CHECK=1 selects the bounds-checked build (libqfp4_bc.so): the
+# same kernels with every store address checked, reported by qfp4_status
+LIB_PATH = os.path.join(_HERE, "libqfp4_bc.so" if os.environ.get("QFP4_BOUNDS_CHECK") == "1" else "libqfp4.so")
 
 NVFP4, MXFP4, MXFP4_RU = 0, 1, 2
 RTN, SR, QUARTET2 = 0, 1, 2
@@ -26,6 +28,7 @@ BLOCK = {NVFP4: 16, MXFP4: 32, MXFP4_RU: 32}
 
 OK, ERR_INVALID_ARG, ERR_MISALIGNED, ERR_UNSUPPORTED_ARCH, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT = 0, -1, -2, -3, -4, -5, -6
 ERR_TOO_LARGE = -7
+ERR_BOUNDS = -8
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
 

@@ -53,6 +53,8 @@ extern "C" {
 #define QFP4_ERR_CUDA (-5)             /* a CUDA runtime/driver call failed; see qfp4_last_cuda_error */
 #define QFP4_ERR_TIMEOUT (-6)          /* a device-side bounded wait expired (from qfp4_status) */
 #define QFP4_ERR_TOO_LARGE (-7)        /* the problem needs more than qfp4_linear_fwd_noalloc's fixed scratch */
+#define QFP4_ERR_BOUNDS (-8)           /* bounds-checked build only: a kernel store fell outside its buffer and was
+                                          dropped (from qfp4_status) */
 
 /* ---- enums ---------------------------------------------------------------- */
 /* QFP4_MXFP4_RU: MXFP4 whose shared exponent is rounded up instead of down,
@@ -359,7 +361,10 @@ int qfp4_linear_fwd_noalloc(const void* X, const void* W, void* Y, int64_t M, in
 /* ---- status ---------------------------------------------------------------
  * Synchronizes `stream`, then reads and clears the library's device error word
  * on the current device. Returns QFP4_OK, QFP4_ERR_TIMEOUT (a bounded wait in
- * a kernel expired; that kernel skipped the rest of its work), or
+ * a kernel expired; that kernel skipped the rest of its work), QFP4_ERR_BOUNDS
+ * (only from the bounds-checked build, libqfp4_bc.so, compiled with
+ * QFP4_BOUNDS_CHECK: a kernel computed a store address outside the output
+ * buffer the arguments describe; the store went to a scratch sink instead), or
  * QFP4_ERR_CUDA. */
 int qfp4_status(void* stream);
 
