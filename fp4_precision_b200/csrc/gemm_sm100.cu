@@ -593,6 +593,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    pdl_wait();  // the operands' quantizers have completed (and the previous readers of D)
+    pdl_launch_dependents();
 
     if (warp == 0) {
         // ---------------- TMA producer ----------------
@@ -793,6 +795,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     cluster_sync();  // barriers of both CTAs initialised, tensor memory allocated
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    pdl_wait();  // the operands' quantizers have completed (and the previous readers of D)
+    pdl_launch_dependents();
 
     if (warp == 0) {
         // ---------------- TMA producer (both CTAs) ----------------
@@ -953,14 +957,14 @@ cudaError_t launch_gemm(const GemmParams& p, int fmt, const CUtensorMap* tmapA, 
     if (fmt == kNvfp4) {
         e = cudaFuncSetAttribute(gemm_bs_fp4_kernel<kNvfp4>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
         if (e != cudaSuccess) return e;
-        gemm_bs_fp4_kernel<kNvfp4><<<grid, kGemmThreads, SMEM_BYTES, s>>>(*tmapA, *tmapB, p);
+        e = launch_pdl(gemm_bs_fp4_kernel<kNvfp4>, dim3(grid), dim3(kGemmThreads), SMEM_BYTES, s, *tmapA, *tmapB, p);
     } else {
         e = cudaFuncSetAttribute(gemm_bs_fp4_kernel<kMxfp4>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
         if (e != cudaSuccess) return e;
-        gemm_bs_fp4_kernel<kMxfp4><<<grid, kGemmThreads, SMEM_BYTES, s>>>(*tmapA, *tmapB, p);
+        e = launch_pdl(gemm_bs_fp4_kernel<kMxfp4>, dim3(grid), dim3(kGemmThreads), SMEM_BYTES, s, *tmapA, *tmapB, p);
     }
     count_launch();
-    return cudaGetLastError();
+    return e;
 }
 
 template <int FMT, int NHQ, int AMX = -1>
@@ -970,9 +974,8 @@ cudaError_t run_pair(const GemmParams& p, const CUtensorMap* tmapA, const CUtens
     cudaError_t e = cudaFuncSetAttribute(gemm_bs_fp4_pair_kernel<FMT, NHQ, AMX>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM);
     if (e != cudaSuccess) return e;
-    gemm_bs_fp4_pair_kernel<FMT, NHQ, AMX><<<2 * clusters, kGemmThreads, P_SMEM, s>>>(*tmapA, *tmapB, *tmapSFA,
-                                                                                     *tmapSFB, *tmapD, p);
-    return cudaSuccess;
+    return launch_pdl(gemm_bs_fp4_pair_kernel<FMT, NHQ, AMX>, dim3(2 * clusters), dim3(kGemmThreads), P_SMEM, s,
+                      *tmapA, *tmapB, *tmapSFA, *tmapSFB, *tmapD, p);
 }
 
 cudaError_t launch_gemm_pair(const GemmParams& p, int fmt, const CUtensorMap* tmapA, const CUtensorMap* tmapB,

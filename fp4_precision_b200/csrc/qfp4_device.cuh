@@ -4,9 +4,12 @@
 #pragma once
 
 #include <cstdint>
+#include <cstdlib>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
+
+#include <utility>
 
 namespace qfp4 {
 
@@ -452,6 +455,39 @@ __device__ __forceinline__ void tc_commit_pair(uint64_t* bar) {
 // own tensor memory at `taddr`.
 __device__ __forceinline__ void tc_cp_pair_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
     asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+
+// ---------------------------------------------------------------------------
+// Programmatic dependent launch. Every kernel of the library is launched with
+// programmatic stream serialization, so the next kernel on the stream can be
+// scheduled while this one drains; each kernel does its set-up that touches
+// no global memory (barrier init, tensor-memory allocation, descriptor
+// prefetch), then waits (griddepcontrol.wait: the previous grid has completed
+// and its writes are visible) before its first global read or write, and
+// lets its own dependents launch (they start as its CTAs exit and wait the
+// same way). QFP4_PDL=0 launches without the attribute (same results).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+inline bool pdl_enabled() {
+    const char* e = std::getenv("QFP4_PDL");
+    return !(e != nullptr && e[0] == '0');
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = pdl_enabled() ? 1 : 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
 }  // namespace qfp4

@@ -809,6 +809,8 @@ __global__ void __launch_bounds__(kThreads, 2)
         ring_init(ring);
     }
     __syncthreads();
+    pdl_wait();  // the previous kernel's writes are visible (and its reads done)
+    pdl_launch_dependents();
 
     if (warp == kComputeWarps) {
         // ---------------- producer ----------------
@@ -1004,6 +1006,8 @@ __global__ void __launch_bounds__(kThreads, 2)
         ring_init(ring);
     }
     __syncthreads();
+    pdl_wait();  // the previous kernel's writes are visible (and its reads done)
+    pdl_launch_dependents();
 
     if (warp == kComputeWarps) {
         if (lane == 0) {
@@ -1350,6 +1354,8 @@ __global__ void __launch_bounds__(kThreads, 2)
         ring_init(ring);
     }
     __syncthreads();
+    pdl_wait();  // the previous kernel's writes are visible (and its reads done)
+    pdl_launch_dependents();
 
     if (warp == kComputeWarps) {
         if (lane == 0) {
@@ -1541,6 +1547,8 @@ __global__ void __launch_bounds__(kThreads, 2)
         ring_init(ring);
     }
     __syncthreads();
+    pdl_wait();  // the previous kernel's writes are visible (and its reads done)
+    pdl_launch_dependents();
     if (warp == kComputeWarps) {
         if (lane == 0) {
             int i = 0;
@@ -1598,9 +1606,9 @@ cudaError_t launch_persistent(Kern kern, int grid, int smem, const CUtensorMap& 
                               cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    kern<<<grid, kThreads, smem, s>>>(tmap, p);
+    e = launch_pdl(kern, dim3(grid), dim3(kThreads), (size_t)smem, s, tmap, p);
     count_launch();
-    return cudaGetLastError();
+    return e;
 }
 
 // A cooperative launch (all CTAs co-resident, as the fused kernels' grid
@@ -1694,6 +1702,8 @@ cudaError_t dispatch_nh(const QuantParams& p, int nh, int axis, const CUtensorMa
 
 // Max of n partial maxima (one CTA).
 __global__ void __launch_bounds__(256) reduce_max_kernel(const float* in, int n, float* out) {
+    pdl_wait();
+    pdl_launch_dependents();
     __shared__ float red[8];
     float m = 0.0f;
     for (int i = threadIdx.x; i < n; i += blockDim.x) m = fmaxf(m, in[i]);
@@ -1717,9 +1727,9 @@ int64_t quant_tiles(int axis, int64_t rows, int64_t k, int G) {
 }
 
 cudaError_t launch_reduce_max(const float* in, int n, float* out, cudaStream_t s) {
-    reduce_max_kernel<<<1, 256, 0, s>>>(in, n, out);
+    const cudaError_t e = launch_pdl(reduce_max_kernel, dim3(1), dim3(256), 0, s, in, n, out);
     count_launch();
-    return cudaGetLastError();
+    return e;
 }
 
 int col_group(int block, int nh) { return nh > block ? nh : block; }
