@@ -44,7 +44,8 @@ def parse():
     ap.add_argument("--no-sustained", action="store_true",
                     help="leave out the two-second sustained run of the step (its own key, not the headline)")
     ap.add_argument("--profile", choices=["gemm_fprop", "gemm_dgrad", "gemm_wgrad", "quant_row", "quant_col",
-                                          "quant_sr_row", "quant_sr_col", "amax_row", "amax_col"],
+                                          "quant_sr_row", "quant_sr_col", "amax_row", "amax_col",
+                                          "amax_rowcol"],
                     help="run only one kernel 3 times on a bounded case (for ncu captures), print nothing else")
     return ap.parse_args()
 
@@ -987,7 +988,10 @@ def run_profile(kind: str):
     else:
         T = inputs.normal((16384, 8192), 1e-3, 5, "prof", device=dev)
         axis = Q.ROW if kind.endswith("row") else Q.COL
-        if kind.startswith("amax"):
+        if kind == "amax_rowcol":  # both orientations' rotated amax from one read
+            for _ in range(3):
+                Q.amax_rowcol(T, Q.HAD_RAND16, seed, Q.make_seed(3, 4, 1, 2))
+        elif kind.startswith("amax"):
             for _ in range(3):
                 Q.amax(T, Q.HAD_RAND16, axis, seed)
         else:

@@ -33,6 +33,13 @@
  *  - Errors are negative status codes; nothing aborts, traps or prints.
  *  - Matrices are row-major. "rows x k" is the quantized orientation: k is the
  *    axis the blocks run along, which is the reduction axis of the GEMM.
+ *  - Kernels are launched with programmatic dependent launch (each waits for
+ *    the previous grid on the stream before touching memory, so stream order
+ *    holds as usual). Environment switches, read on every call, select
+ *    equivalent paths with the same results: QFP4_PDL=0 (plain launches),
+ *    QFP4_FUSED_AMAX=0 (no one-launch amax + quantization), QFP4_COL_BANDS=0
+ *    (group-walking column quantizer), QFP4_GEMM_PAIR=0/1 (GEMM kernel).
+ *  - Each call that touches the device opens an NVTX range named after it.
  */
 #ifndef QFP4_H_
 #define QFP4_H_
