@@ -409,7 +409,8 @@ def check_quartet2_error_half_of_sr():
     stochastic rounding. On N(0,1) data with and without a random 16x16
     rotation the mean squared error of the NVFP4 reconstruction (rotated
     domain, 4 rounding seeds) is within 0.4-0.6 of SR's; the part added by the
-    scale rounding (over RTN) is at least 10x smaller than SR's."""
+    scale rounding (over RTN) is at least 20x smaller than SR's (measured about
+    30x; the page says about two orders of magnitude)."""
     ratio = golden("pages.json")["quartet2_error_vs_plain_sr"]
     x = inputs.normal((256, 1024), 1.0, 9, "mse")
     for had in (O.HAD_RAND16, O.HAD_NONE):
@@ -419,7 +420,7 @@ def check_quartet2_error_half_of_sr():
             mse[rnd] = np.mean([np.mean((O.dequantize(O.quantize(x, O.NVFP4, rnd, had, O.ROW, 5, 0, 100 + s, 0))
                                          - v) ** 2) for s in range(4)])
         assert abs(mse[O.QUARTET2] / mse[O.SR] - ratio) < 0.1, mse
-        assert (mse[O.SR] - mse[O.RTN]) > 10 * (mse[O.QUARTET2] - mse[O.RTN]) > 0, mse
+        assert (mse[O.SR] - mse[O.RTN]) > 20 * (mse[O.QUARTET2] - mse[O.RTN]) > 0, mse
 
 
 def check_quartet2_alpha_range():
