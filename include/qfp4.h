@@ -37,7 +37,8 @@
  *    the previous grid on the stream before touching memory, so stream order
  *    holds as usual). Environment switches, read on every call, select
  *    equivalent paths with the same results: QFP4_PDL=0 (plain launches),
- *    QFP4_FUSED_AMAX=0 (no one-launch amax + quantization), QFP4_COL_BANDS=0
+ *    QFP4_FUSED_AMAX=1 (one-launch amax + quantization of an NVFP4 tensor
+ *    that fits in L2, a cooperative launch; off by default), QFP4_COL_BANDS=0
  *    (group-walking column quantizer), QFP4_GEMM_PAIR=0/1 (GEMM kernel).
  *  - Each call that touches the device opens an NVTX range named after it.
  */

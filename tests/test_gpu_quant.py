@@ -305,19 +305,20 @@ def test_argument_errors():
 @pytest.mark.parametrize("had", [Q.HAD_NONE, Q.HAD_DET16, Q.HAD_RAND16], ids=["none", "det16", "rand16"])
 @pytest.mark.parametrize("rnd", [Q.RTN, Q.QUARTET2], ids=["rtn", "q2"])
 def test_fused_amax_matches_oracle(rnd, had, axis, monkeypatch):
-    """NVFP4 tensors that fit in L2 are quantized by one cooperative launch that
-    takes the rotated amax itself (a first pass, a grid barrier, then the
-    quantizing pass); QFP4_FUSED_AMAX=0 runs the separate amax pass instead.
+    """With QFP4_FUSED_AMAX=1, NVFP4 tensors that fit in L2 are quantized by one
+    cooperative launch that takes the rotated amax itself (a first pass, a grid
+    barrier, then the quantizing pass); by default the separate amax pass runs
+    instead (an amax launch, then the quantizer, which reduces the partials).
     Both give the oracle's codes, scales and tensor scale, on a shape with
     ragged tiles and on the full sweep tensor [8192 x 4096] (67 MB)."""
     for shape in ((384, 448), (8192, 4096)):
         x = sweep_like(*shape) if shape[0] < 8192 else inputs.workload("sweep")["T"]
         ref = oracle_quant(x, Q.NVFP4, rnd, had, axis)
         xd = x.cuda()
+        monkeypatch.setenv("QFP4_FUSED_AMAX", "1")
         Q.launch_count(reset=True)
         assert_same(gpu_quant(xd, Q.NVFP4, rnd, had, axis), ref, Q.NVFP4)
-        fused_launches = Q.launch_count(reset=True)
-        monkeypatch.setenv("QFP4_FUSED_AMAX", "0")
-        assert_same(gpu_quant(xd, Q.NVFP4, rnd, had, axis), ref, Q.NVFP4)
-        assert Q.launch_count(reset=True) == fused_launches + 1  # amax pass + quantizer (it reduces the partials)
+        assert Q.launch_count(reset=True) == 1  # one cooperative launch
         monkeypatch.delenv("QFP4_FUSED_AMAX")
+        assert_same(gpu_quant(xd, Q.NVFP4, rnd, had, axis), ref, Q.NVFP4)
+        assert Q.launch_count(reset=True) == 2  # amax pass + quantizer
