@@ -778,6 +778,19 @@ __device__ int fused_amax_pass(const QuantParams& p, Ring<STAGES>& ring, int til
     return total > (int64_t)blockIdx.x ? (int)((total - blockIdx.x + gridDim.x - 1) / gridDim.x) : 0;
 }
 
+// Occupancy of the persistent quantizers: two CTAs per SM with a 3-stage ring
+// (the memory-bound modes need the deeper ring), or three CTAs per SM with a
+// 2-stage ring (at most 75 registers) for NVFP4 with per-element SR or Quartet
+// II, which are bound by instruction issue and gain from the extra warps
+// (measured on the 940 MB dY: Quartet II rows 1-3 %, SR rows 4 % faster; RTN
+// rows 6 % slower with the shallower ring).
+template <int STAGES>
+constexpr int kCtasPerSm = STAGES == 2 ? 3 : 2;
+template <int FMT, int RND>
+constexpr bool issue_bound_mode() {
+    return FMT == kNvfp4 && (RND == kSr || RND == kQuartet2);
+}
+
 // ===========================================================================
 // Row mode
 // ===========================================================================
@@ -785,7 +798,7 @@ __device__ int fused_amax_pass(const QuantParams& p, Ring<STAGES>& ring, int til
 // pass over the tiles takes the rotated amax, a grid barrier, then the
 // quantizing pass re-reads the tiles (from L2).
 template <int FMT, int RND, int NH, bool AMAX_ONLY, int STAGES, bool FUSED = false>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, kCtasPerSm<STAGES>)
     quant_row_kernel(const __grid_constant__ CUtensorMap tmap, const QuantParams p) {
     using Grp = Group<FMT, RND, NH>;
     constexpr int NB = Grp::NB;
@@ -1324,7 +1337,7 @@ __device__ __forceinline__ void dual_row_work(const QuantParams& p, float s_enc_
 // sign vector, the row tensor amax and random streams), as the row kernel
 // would: one read of x gives both orientations.
 template <int FMT, int RND, int NH, int STAGES, int NH_ROW = -1, bool FUSED = false>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, kCtasPerSm<STAGES>)
     quant_col64_kernel(const __grid_constant__ CUtensorMap tmap, const QuantParams p) {
     constexpr bool kDual = NH_ROW >= 0;
     using Grp = Group<FMT, RND, NH>;
@@ -1644,9 +1657,10 @@ cudaError_t launch_t(const QuantParams& p, int axis, const CUtensorMap* tmap, in
     if (axis == 0) {
         const int64_t tiles =
             ((p.rows + kRowTileRows - 1) / kRowTileRows) * ((p.k + kRowTileCols - 1) / kRowTileCols);
-        if (grid <= 0) grid = persistent_grid(tiles, 2);
-        const int smem = kRowStages * kRowTileRows * kRowTileCols * 2 + 1024;
-        return launch_persistent(quant_row_kernel<FMT, RND, NH, AMAX_ONLY, kRowStages>, grid, smem, *tmap, p, s);
+        constexpr int S = (!AMAX_ONLY && issue_bound_mode<FMT, RND>()) ? 2 : kRowStages;
+        if (grid <= 0) grid = persistent_grid(tiles, kCtasPerSm<S>);
+        const int smem = S * kRowTileRows * kRowTileCols * 2 + 1024;
+        return launch_persistent(quant_row_kernel<FMT, RND, NH, AMAX_ONLY, S>, grid, smem, *tmap, p, s);
     } else {
         constexpr int NB = (FMT == kNvfp4) ? 16 : 32;
         constexpr int G = AMAX_ONLY ? ((NH > 16) ? NH : 16) : ((NH > NB) ? NH : NB);
@@ -1661,10 +1675,11 @@ cudaError_t launch_t(const QuantParams& p, int axis, const CUtensorMap* tmap, in
 // Column mode over 64-row bands (axis code 2; the quantized axis a multiple of 64).
 template <int FMT, int RND, int NH>
 cudaError_t launch_col64(const QuantParams& p, const CUtensorMap* tmap, cudaStream_t s) {
-    constexpr int S = 3;
+    constexpr int S = issue_bound_mode<FMT, RND>() ? 2 : 3;
     const int64_t tiles = ((p.rows + 127) / 128 * 2) * ((p.k + 255) / 256);
     const int smem = S * 256 * 64 * 2 + 1024;
-    return launch_persistent(quant_col64_kernel<FMT, RND, NH, S>, persistent_grid(tiles, 2), smem, *tmap, p, s);
+    return launch_persistent(quant_col64_kernel<FMT, RND, NH, S>, persistent_grid(tiles, kCtasPerSm<S>), smem,
+                             *tmap, p, s);
 }
 
 // The fused (one-launch) NVFP4 quantization: packed unit, RTN or Quartet II,
