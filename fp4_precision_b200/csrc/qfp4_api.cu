@@ -8,6 +8,7 @@
 #include <cuda_runtime.h>
 #include <nvtx3/nvToolsExt.h>
 
+#include <algorithm>
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
@@ -1104,6 +1105,46 @@ int qfp4_selftest_wait_timeout(int64_t limit_ns, void* stream) {
     if (rc) return rc;
     if (limit_ns <= 0 || limit_ns > (int64_t)kWaitLimitNs) return QFP4_ERR_INVALID_ARG;
     qfp4::wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>((uint64_t)limit_ns);
+    count_launch();
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? QFP4_OK : cuda_fail(e);
+}
+
+// ---- rounding self-test ---------------------------------------------------------
+namespace qfp4 {
+namespace {
+// The quantizers' element and scale rounding steps, one value per thread.
+__global__ void rounding_selftest_kernel(int32_t op, const float* x, const uint32_t* w, uint8_t* codes, int64_t n) {
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
+        const float v = x[i];
+        uint32_t code;
+        if (op == QFP4_ROUND_E2M1_SR || op == QFP4_ROUND_E2M1_RN) {
+            float r[8] = {op == QFP4_ROUND_E2M1_SR ? e2m1_sr_value(v, w[i] << 16) : v, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            code = e2m1x8_rn(r) & 0xFu;
+        } else if (op == QFP4_ROUND_E4M3_SR) {
+            code = e4m3_sr(v, w[i]);
+        } else if (op == QFP4_ROUND_E4M3_RN) {
+            code = e4m3_rn(v);
+        } else {
+            code = e8m0_sr(v, uniform24(w[i]));
+        }
+        codes[i] = (uint8_t)code;
+    }
+}
+}  // namespace
+}  // namespace qfp4
+
+int qfp4_selftest_rounding(int32_t op, const float* x, const uint32_t* w, uint8_t* codes, int64_t n, void* stream) {
+    const ApiRange range("qfp4_selftest_rounding");
+    const int rc = bind_context(static_cast<cudaStream_t>(stream));
+    if (rc) return rc;
+    if (op < QFP4_ROUND_E2M1_SR || op > QFP4_ROUND_E8M0_SR || n < 0) return QFP4_ERR_INVALID_ARG;
+    const bool needs_w = op != QFP4_ROUND_E2M1_RN && op != QFP4_ROUND_E4M3_RN;
+    if (n == 0) return QFP4_OK;
+    if (!x || !codes || (needs_w && !w)) return QFP4_ERR_INVALID_ARG;
+    const int64_t blocks = std::min<int64_t>((n + 255) / 256, 148 * 8);
+    qfp4::rounding_selftest_kernel<<<(unsigned)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(op, x, w, codes, n);
     count_launch();
     const cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? QFP4_OK : cuda_fail(e);

@@ -82,8 +82,6 @@ __device__ __forceinline__ uint4 philox_quad(uint64_t seed, uint32_t tag_stream,
 
 // Uniform in [0, 1) on the 2^-24 grid.
 __device__ __forceinline__ float uniform24(uint32_t w) { return __uint2float_rn(w >> 8) * 0x1p-24f; }
-// Uniform in [0, 1) on the 2^-16 grid from a 16-bit value (element SR).
-__device__ __forceinline__ float uniform16(uint32_t h) { return __uint2float_rn(h) * 0x1p-16f; }
 
 // ---------------------------------------------------------------------------
 // bf16 pairs -> fp32 (exact)
@@ -111,26 +109,27 @@ __device__ __forceinline__ uint32_t e2m1x8_rn(const float* v) {
     return mag | (out & nonzero);
 }
 
-// E2M1 magnitude grid step for |u| < 6: 0.5 below 2, 1 below 4, 2 above.
-__device__ __forceinline__ float e2m1_step(float a) { return a < 2.0f ? 0.5f : (a < 4.0f ? 1.0f : 2.0f); }
-
-// Stochastic rounding of u onto the E2M1 grid with uniform rho: the lower grid
-// neighbour lo, gap `step`, round up iff rho < (|u| - lo) / step; |u| >= 6 -> 6.
-// Returns the exactly representable rounded value (sign kept).
-__device__ __forceinline__ float e2m1_sr_value(float u, float rho) {
-    const float a = fabsf(u);
-    float m;
-    if (a >= 6.0f) {
-        m = 6.0f;
-    } else {
-        const float inv_step = a < 2.0f ? 2.0f : (a < 4.0f ? 1.0f : 0.5f);
-        const float step = e2m1_step(a);
-        const float t = a * inv_step;      // = a / step exactly (power-of-two step)
-        const float fl = floorf(t);
-        const float p = t - fl;            // exact: fraction of an exactly scaled value
-        m = (fl + (rho < p ? 1.0f : 0.0f)) * step;
-    }
-    return copysignf(m, u);
+// Stochastic rounding of u onto the E2M1 grid with a 16-bit draw h, given as
+// hs = h << 16: the lower grid neighbour lo, gap `step`, round up iff
+// h * 2^-16 < (|u| - lo) / step; the result is the chosen grid value with the
+// sign of u (magnitudes above 6 come out as 6 or 8 and saturate to 6 in the
+// E2M1 conversion). Exact, in integer steps: with C the power of two just
+// above |u| (at least 2), y = |u| + C rounded upward lies in [C, 2C] and the
+// E2M1 gap of |u|'s binade, C/4, is y's top two mantissa bits, so lo + C is y
+// with the lower 21 bits cleared and y's lower 21 bits are ceil((|u| - lo) /
+// ulp(y)); h * 2^-16 < (|u| - lo) / step <=> 32 h < (|u| - lo) / ulp(y) <=>
+// 32 h < ceil(...) for integer h, i.e. h << 16 < y << 11 unsigned. When the
+// upward rounding carries into the gap bits (|u| within an ulp below a grid
+// point) the fraction left is 0 and the result is that grid point, which is
+// also the exact outcome there (the true fraction exceeds 1 - 2^-16).
+__device__ __forceinline__ float e2m1_sr_value(float u, uint32_t hs) {
+    const uint32_t b = __float_as_uint(u);
+    const uint32_t cb = max((b & 0x7F800000u) + 0x00800000u, 0x40000000u);
+    const float c = __uint_as_float(cb);
+    const uint32_t yb = __float_as_uint(__fadd_ru(fabsf(u), c));
+    const uint32_t mb = (yb & 0xFFE00000u) + (hs < (yb << 11) ? 0x00200000u : 0u);
+    const float m = __fsub_rn(__uint_as_float(mb), c);  // exact: mb in [c, 2c]
+    return __uint_as_float(__float_as_uint(m) | (b & 0x80000000u));
 }
 
 // E2M1 code value (signed) of a 4-bit code.

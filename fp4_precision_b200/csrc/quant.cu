@@ -112,25 +112,28 @@ __device__ __forceinline__ void fwht(float* v) {
     if constexpr (N == 32) fwht_stage<N, 16>(v);
 }
 
-// One stride of the halving tree: s[j] += s[j + ST] for j < ST. Scalar
-// __fadd_rn, like the products that feed the tree (__fmul_rn): those are never
-// merged into a fused multiply-add, whereas a packed f32x2 product feeding a
-// packed sum was (by the assembler, even as explicit mul.rn.f32x2 /
-// add.rn.f32x2), which moved alpha by an ulp in about 15 % of blocks.
+// One stride of the halving tree: s[j] += s[j + ST] for j < ST.
 template <int ST>
 __device__ __forceinline__ void tree_stage(float* s) {
 #pragma unroll
     for (int j = 0; j < ST; ++j) s[j] = __fadd_rn(s[j], s[j + ST]);
 }
 
-// Halving-stride tree sum of n fp32 terms (s[j] += s[j + stride], stride n/2 .. 1).
+// Halving-stride tree sum of N = 8 or 16 fp32 terms (s[j] += s[j + stride],
+// stride N/2 .. 1).
 template <int N>
 __device__ __forceinline__ float tree_sum(float* s) {
-    if constexpr (N == 32) tree_stage<16>(s);
-    tree_stage<8>(s);
+    if constexpr (N == 16) tree_stage<8>(s);
     tree_stage<4>(s);
     tree_stage<2>(s);
     return __fadd_rn(s[0], s[1]);
+}
+
+// First stride of <a, b> over a block of NB terms in the halving-stride
+// order: a[j] b[j] fused onto the rounded a[j + NB/2] b[j + NB/2] (one
+// multiply-add); tree_sum<NB/2> of these gives the dot product.
+__device__ __forceinline__ float dot_first(float a0, float b0, float a1, float b1) {
+    return __fmaf_rn(a0, b0, __fmul_rn(a1, b1));
 }
 
 // E2M1 pair (one byte) -> two fp32 values (exact through f16).
@@ -324,26 +327,29 @@ struct Group {
                     const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
                     for (int h = 0; h < 4; ++h) {
-                        vb[e8 + 2 * h] = e2m1_sr_value(vb[e8 + 2 * h], uniform16(ws[h] & 0xFFFFu));
-                        vb[e8 + 2 * h + 1] = e2m1_sr_value(vb[e8 + 2 * h + 1], uniform16(ws[h] >> 16));
+                        vb[e8 + 2 * h] = e2m1_sr_value(vb[e8 + 2 * h], ws[h] << 16);
+                        vb[e8 + 2 * h + 1] = e2m1_sr_value(vb[e8 + 2 * h + 1], ws[h] & 0xFFFF0000u);
                     }
                 }
             }
 #pragma unroll
             for (int e8 = 0; e8 < NB; e8 += 8) cb[e8 / 8] = e2m1x8_rn(vb + e8);
             if constexpr (RND == kQuartet2) {
-                // alpha = T(u*u) / T(u*q), T the halving-stride tree sum
-                float sa[NB], sb[NB];
+                // alpha = <u, u> / <u, q>, each sum's first stride by
+                // dot_first on element pairs (j, j + NB/2), then the tree
+                constexpr int H = NB / 2;
+                float sa[H], sb[H];
 #pragma unroll
-                for (int e = 0; e < NB; e += 2) {
-                    const float2 q = e2m1x2_decode((cb[e / 8] >> (4 * (e & 7))) & 0xFFu);
-                    sa[e] = __fmul_rn(vb[e], vb[e]);
-                    sa[e + 1] = __fmul_rn(vb[e + 1], vb[e + 1]);
-                    sb[e] = __fmul_rn(vb[e], q.x);
-                    sb[e + 1] = __fmul_rn(vb[e + 1], q.y);
+                for (int j = 0; j < H; j += 2) {
+                    const float2 q0 = e2m1x2_decode((cb[j / 8] >> (4 * (j & 7))) & 0xFFu);
+                    const float2 q1 = e2m1x2_decode((cb[(j + H) / 8] >> (4 * ((j + H) & 7))) & 0xFFu);
+                    sa[j] = dot_first(vb[j], vb[j], vb[j + H], vb[j + H]);
+                    sa[j + 1] = dot_first(vb[j + 1], vb[j + 1], vb[j + H + 1], vb[j + H + 1]);
+                    sb[j] = dot_first(vb[j], q0.x, vb[j + H], q1.x);
+                    sb[j + 1] = dot_first(vb[j + 1], q0.y, vb[j + H + 1], q1.y);
                 }
-                const float num = tree_sum<NB>(sa);
-                const float den = tree_sum<NB>(sb);
+                const float num = tree_sum<H>(sa);
+                const float den = tree_sum<H>(sb);
                 const float alpha = (den == 0.0f) ? 1.0f : __fdiv_rn(num, den);
                 const float t = __fmul_rn(S, alpha);
                 const uint32_t rw = srng.word(p, block0 + b);
@@ -491,14 +497,17 @@ __device__ __forceinline__ void fwht_pair_stage(float2* P) {
         }
 }
 
-// Halving-stride tree sum of the 16 terms of each lane of a pair, in scalar
-// __fadd_rn (see tree_stage: the terms are products, and a packed sum of
-// packed products was fused into multiply-adds).
-__device__ __forceinline__ float2 tree_sum_pair(float2* s) {
+// dot_tree of the 16 terms of each lane of a pair (two blocks at once): the
+// first stride as packed multiply-adds onto packed products, the tree over
+// the 8 partial sums as packed sums.
+__device__ __forceinline__ float2 dot_tree_pair(const float2* a, const float2* b) {
+    float2 s[8];
 #pragma unroll
-    for (int st = 8; st >= 1; st >>= 1)
+    for (int j = 0; j < 8; ++j) s[j] = __ffma2_rn(a[j], b[j], __fmul2_rn(a[j + 8], b[j + 8]));
 #pragma unroll
-        for (int j = 0; j < st; ++j) s[j] = f2(__fadd_rn(s[j].x, s[j + st].x), __fadd_rn(s[j].y, s[j + st].y));
+    for (int st = 4; st >= 1; st >>= 1)
+#pragma unroll
+        for (int j = 0; j < st; ++j) s[j] = __fadd2_rn(s[j], s[j + st]);
     return s[0];
 }
 
@@ -593,24 +602,21 @@ __device__ __forceinline__ uint32_t nv64_quantize(Load load, const SignFlips& sf
             cw[3] = e2m1x8_words(P[8].y, P[9].y, P[10].y, P[11].y, P[12].y, P[13].y, P[14].y, P[15].y);
             scw |= sc2 << (16 * bp);
         } else {
-            // RTN codes and their values q; alpha = T(u u) / T(u q) per lane
+            // RTN codes and their values q; alpha = <u, u> / <u, q> per lane
             uint32_t h[4][4];
             cw[0] = e2m1x8_words_dec(P[0].x, P[1].x, P[2].x, P[3].x, P[4].x, P[5].x, P[6].x, P[7].x, h[0]);
             cw[1] = e2m1x8_words_dec(P[8].x, P[9].x, P[10].x, P[11].x, P[12].x, P[13].x, P[14].x, P[15].x, h[1]);
             cw[2] = e2m1x8_words_dec(P[0].y, P[1].y, P[2].y, P[3].y, P[4].y, P[5].y, P[6].y, P[7].y, h[2]);
             cw[3] = e2m1x8_words_dec(P[8].y, P[9].y, P[10].y, P[11].y, P[12].y, P[13].y, P[14].y, P[15].y, h[3]);
-            float2 uu[16], uq[16];
+            float2 Q[16];
 #pragma unroll
             for (int j = 0; j < 16; j += 2) {
                 const float2 qx = __half22float2(*reinterpret_cast<const __half2*>(&h[j / 8][(j % 8) / 2]));
                 const float2 qy = __half22float2(*reinterpret_cast<const __half2*>(&h[2 + j / 8][(j % 8) / 2]));
-                // scalar products (never fused with the tree's sums)
-                uu[j] = f2(__fmul_rn(P[j].x, P[j].x), __fmul_rn(P[j].y, P[j].y));
-                uu[j + 1] = f2(__fmul_rn(P[j + 1].x, P[j + 1].x), __fmul_rn(P[j + 1].y, P[j + 1].y));
-                uq[j] = f2(__fmul_rn(P[j].x, qx.x), __fmul_rn(P[j].y, qy.x));
-                uq[j + 1] = f2(__fmul_rn(P[j + 1].x, qx.y), __fmul_rn(P[j + 1].y, qy.y));
+                Q[j] = f2(qx.x, qy.x);
+                Q[j + 1] = f2(qx.y, qy.y);
             }
-            const float2 num = tree_sum_pair(uu), den = tree_sum_pair(uq);
+            const float2 num = dot_tree_pair(P, P), den = dot_tree_pair(P, Q);
             const float a0 = (den.x == 0.0f) ? 1.0f : __fdiv_rn(num.x, den.x);
             const float a1 = (den.y == 0.0f) ? 1.0f : __fdiv_rn(num.y, den.y);
             const float2 ts = __fmul2_rn(f2(e0.y, e1.y), f2(a0, a1));

@@ -30,6 +30,7 @@ OK, ERR_INVALID_ARG, ERR_MISALIGNED, ERR_UNSUPPORTED_ARCH, ERR_WORKSPACE, ERR_CU
 ERR_TOO_LARGE = -7
 ERR_BOUNDS = -8
 NOALLOC_SCRATCH_BYTES = 32 << 20
+ROUND_E2M1_SR, ROUND_E2M1_RN, ROUND_E4M3_SR, ROUND_E4M3_RN, ROUND_E8M0_SR = 0, 1, 2, 3, 4
 
 
 class Seed(ctypes.Structure):
@@ -99,6 +100,7 @@ _SIGNATURES = {
                                                ctypes.POINTER(Seed), _VOID]),
     "qfp4_status": (ctypes.c_int, [_VOID]),
     "qfp4_selftest_wait_timeout": (ctypes.c_int, [_I64, _VOID]),
+    "qfp4_selftest_rounding": (ctypes.c_int, [_I32, _VOID, _VOID, _VOID, _I64, _VOID]),
     "qfp4_launch_count": (_I64, [_I32]),
 }
 
@@ -372,6 +374,17 @@ def linear_bwd(dY, X, W, rec: Recipe, seed: Seed, dX=None, dW=None, workspace=No
 def status(stream=None):
     """Synchronize and raise if a kernel reported a device-side error."""
     _check(lib().qfp4_status(_stream(stream)), "qfp4_status")
+
+
+def selftest_rounding(op: int, x: torch.Tensor, w: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """The quantizers' rounding step `op` (ROUND_*) applied to each fp32 of x
+    with the uint32 random words w (int32 storage): one code byte per value."""
+    assert x.dtype == torch.float32 and x.is_contiguous()
+    assert w is None or (w.dtype == torch.int32 and w.is_contiguous() and w.numel() == x.numel())
+    codes = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    _check(lib().qfp4_selftest_rounding(op, _ptr(x), _ptr(w), _ptr(codes), x.numel(), _stream(stream)),
+           "qfp4_selftest_rounding")
+    return codes
 
 
 class Fp4Linear(torch.autograd.Function):

@@ -390,6 +390,39 @@ int64_t qfp4_launch_count(int32_t reset);
  * Returns QFP4_OK (launched), QFP4_ERR_INVALID_ARG or QFP4_ERR_CUDA. */
 int qfp4_selftest_wait_timeout(int64_t limit_ns, void* stream);
 
+/* Self-test of the quantizers' element and scale rounding steps: applies one
+ * of them, as the quantizer kernels inline it, to each of n fp32 values and
+ * writes one code byte per value. Lets a test compare the exact decision of
+ * the device code with the definition at chosen points (grid points, the
+ * stochastic-rounding thresholds themselves and their neighbouring floats),
+ * which the quantizers' own inputs reach only by chance.
+ *   op QFP4_ROUND_E2M1_SR: stochastic rounding onto E2M1 with the 16-bit
+ *     draw r = w[i] & 0xFFFF (round up iff r * 2^-16 < the fraction between
+ *     the two grid neighbours, |x| >= 6 gives 6; [NVIDIA NVFP4] "Kak eto
+ *     rabotaet", [Quartet II] on NVIDIA's recipe); |x| < 2^127.
+ *   op QFP4_ROUND_E2M1_RN: round-to-nearest-even onto E2M1, saturating at 6
+ *     ([AMD MXFP4] "Chto takoe MXFP4").
+ *   op QFP4_ROUND_E4M3_SR: stochastic rounding of x >= 0 onto E4M3 with the
+ *     uniform (w[i] >> 8) * 2^-24, saturating at 448 (the Quartet II scale
+ *     step, [Quartet II]).
+ *   op QFP4_ROUND_E4M3_RN: round-to-nearest-even of x >= 0 onto E4M3,
+ *     saturating at 448 (the NVFP4 block scale).
+ *   op QFP4_ROUND_E8M0_SR: stochastic rounding of x > 0 onto powers of two
+ *     with the uniform (w[i] >> 8) * 2^-24, as the E8M0 code (the Quartet II
+ *     scale step on an MXFP4 scale).
+ * x: n fp32 (device), w: n uint32 (device; may be NULL for the two RN ops),
+ * codes: n bytes (device, written; an E2M1 code is sign << 3 | magnitude
+ * index, magnitude 0 always code 0). Values outside an op's stated domain
+ * give unspecified codes. Stream-ordered. Returns QFP4_OK (launched),
+ * QFP4_ERR_INVALID_ARG (unknown op, n < 0, a NULL pointer that the op reads
+ * or writes) or QFP4_ERR_CUDA. */
+#define QFP4_ROUND_E2M1_SR 0
+#define QFP4_ROUND_E2M1_RN 1
+#define QFP4_ROUND_E4M3_SR 2
+#define QFP4_ROUND_E4M3_RN 3
+#define QFP4_ROUND_E8M0_SR 4
+int qfp4_selftest_rounding(int32_t op, const float* x, const uint32_t* w, uint8_t* codes, int64_t n, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -9,7 +9,8 @@
  * code) is taken on fp32 values computed in the same fp32 operation order the
  * method is stated in, so that its result is exactly defined. Distances to grid
  * points are compared in fp64, where they are exact. Build with
- * -ffp-contract=off (no fused multiply-add) and without fast-math.
+ * -ffp-contract=off (no fused multiply-add but the one written out, fmaf in
+ * dot_tree) and without fast-math.
  *
  * Sources (web pages on FP4 training; no code is printed on any of them):
  *  [Quartet II]  "Quartet II - obuchenie v NVFP4 s tochnymi nesmeshchyonnymi
@@ -290,6 +291,20 @@ static float tree_sum(float* s, int n) {
     return s[0];
 }
 
+/* <a, b> of n <= 32 fp32 terms in the same halving-stride order, the first
+ * stride taking the products: s[j] = a[j] b[j] + a[j + n/2] b[j + n/2] as one
+ * fused multiply-add of a[j] b[j] onto the rounded product a[j + n/2] b[j +
+ * n/2] (fmaf: exact product and sum, one rounding), then tree_sum of the n/2
+ * partial sums. Reading: the pages fix neither the precision nor the order of
+ * the Quartet II sums; this one is exactly defined, and the multiply-add
+ * leaves one rounding fewer per pair than a product followed by a sum. */
+static float dot_tree(const float* a, const float* b, int n) {
+    float s[16];
+    const int h = n / 2;
+    for (int j = 0; j < h; ++j) s[j] = fmaf(a[j], b[j], a[j + h] * b[j + h]);
+    return tree_sum(s, h);
+}
+
 /* Load quantized-axis segment `row` (length k) of x into seg as fp32. */
 static void load_segment(const uint16_t* x, int64_t ld, int axis, int64_t row, int64_t k, float* seg) {
     if (axis == AXIS_ROW)
@@ -373,7 +388,7 @@ int oracle_quantize_rows(const uint16_t* x, int64_t R, int64_t C, int64_t ld, in
 #pragma omp parallel
     {
         float* seg = (float*)malloc(sizeof(float) * (size_t)(k > 0 ? k : 1));
-        float u[32], prod[32];
+        float u[32], qval[32];
         uint8_t q[32];
 #pragma omp for schedule(static)
         for (int64_t ro = 0; ro < n_out; ++ro) {
@@ -440,10 +455,9 @@ int oracle_quantize_rows(const uint16_t* x, int64_t R, int64_t C, int64_t ld, in
                      * projection of u on q) makes it unbiased; alpha (about 0.94-1.06) is
                      * too fine for an FP8 scale, so S * alpha is stochastically rounded
                      * into the scale. The element codes stay round-to-nearest. */
-                    for (int j = 0; j < nb; ++j) prod[j] = u[j] * u[j];
-                    float num = tree_sum(prod, nb);
-                    for (int j = 0; j < nb; ++j) prod[j] = u[j] * (float)oracle_e2m1_value(q[j]);
-                    float den = tree_sum(prod, nb);
+                    for (int j = 0; j < nb; ++j) qval[j] = (float)oracle_e2m1_value(q[j]);
+                    float num = dot_tree(u, u, nb);
+                    float den = dot_tree(u, qval, nb);
                     alpha = (den == 0.0f) ? 1.0f : num / den;
                     float t = s_val * alpha;
                     float rho = uniform24(random_word(sr_seed, TAG_SCALE, sr_stream, (uint64_t)blk_index));

@@ -441,6 +441,33 @@ def check_quartet2_alpha_range():
     assert np.all(s_q2 <= t * (1 + 2.0**-3) + 1e-30) and np.all(s_q2 >= t * (1 - 2.0**-3))
 
 
+def check_quartet2_alpha_is_the_projection():
+    """[Quartet II]: the renormalisation of a block is the projection
+    <u, u> / <u, q> of its scaled values u on their RTN values q. Recomputed
+    here in fp64 from the oracle's own RTN output (u = rotated block / (S g),
+    q = the E2M1 values of its codes), the oracle's fp32 alpha agrees to within
+    the rounding of its fp32 sums (all terms u_j q_j share a sign, so nothing
+    cancels): 2^-18 relative. A term, index or operand wrong anywhere in the
+    two sums moves alpha by far more. Also: Quartet II keeps the RTN codes."""
+    x = inputs.normal((32, 256), 1.0, 21, "alpha_exact")
+    for fmt, had in ((O.NVFP4, O.HAD_RAND16), (O.NVFP4, O.HAD_NONE), (O.MXFP4, O.HAD_RAND32), (O.MXFP4, O.HAD_DET32)):
+        nb = O.BLOCK[fmt]
+        q_rtn = O.quantize(x, fmt, O.RTN, had, O.ROW, 9, 0)
+        q2 = O.quantize(x, fmt, O.QUARTET2, had, O.ROW, 9, 0, 13, 0)
+        assert np.array_equal(q2.codes, q_rtn.codes)
+        v = O.rotate(x, had, O.ROW, 9, 0).astype(np.float64)
+        step = O.scale_values(q_rtn) * (np.float64(q_rtn.g) if fmt == O.NVFP4 else 1.0)
+        u = v.reshape(32, -1, nb) / step[:, :, None]
+        e2m1 = np.array([O.e2m1_value(c) for c in range(16)])
+        q = e2m1[O.unpack_codes(q_rtn.codes)].reshape(32, -1, nb)
+        num, den = np.sum(u * u, axis=2), np.sum(u * q, axis=2)
+        ok = den > 0
+        assert ok.mean() > 0.99
+        alpha = num[ok] / den[ok]
+        rel = np.abs(q2.alpha[ok] / alpha - 1.0)
+        assert rel.max() < 2.0**-18, (fmt, had, rel.max())
+
+
 # ---------------------------------------------------------------------------
 # scales and reconstruction
 
@@ -623,7 +650,7 @@ ALL_CHECKS = [
     check_sr_threshold_exact_16bit, check_e4m3_sr_threshold_exact,
     check_e8m0_sr_threshold_exact,
     check_sr_unbiased_rtn_biased, check_quartet2_projection_unbiased, check_quartet2_error_half_of_sr,
-    check_quartet2_alpha_range,
+    check_quartet2_alpha_range, check_quartet2_alpha_is_the_projection,
     check_nvfp4_scales, check_mxfp4_scales, check_mxfp4_round_up, check_zero_and_degenerate, check_col_is_row_of_transpose,
     check_seed_determinism, check_gemm_brute_force, check_hadamard_cancels_in_gemm,
 ]

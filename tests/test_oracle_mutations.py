@@ -30,6 +30,9 @@ MUTATIONS = [
     ("philox_key_bump", "k1 += 0xBB67AE85u;", "k1 += 0xBB67AE86u;"),
     ("quartet2_alpha_inverted", "alpha = (den == 0.0f) ? 1.0f : num / den;", "alpha = (den == 0.0f) ? 1.0f : den / num;"),
     ("tree_sum_wrong_term", "s[j] = s[j] + s[j + stride];", "s[j] = s[j] + s[j + stride / 2];"),
+    ("dot_tree_first_stride_term", "s[j] = fmaf(a[j], b[j], a[j + h] * b[j + h]);",
+     "s[j] = fmaf(a[j], b[j], a[j + h] * b[j]);"),
+    ("dot_tree_half_dropped", "return tree_sum(s, h);", "return tree_sum(s, h / 2);"),
     ("nibble_order", "out[j / 2] = (uint8_t)(q[j] | (q[j + 1] << 4));", "out[j / 2] = (uint8_t)(q[j + 1] | (q[j] << 4));"),
     ("col_orientation", "for (int64_t j = 0; j < k; ++j) seg[j] = bf16_to_f32(x[j * ld + row]);",
      "for (int64_t j = 0; j < k; ++j) seg[j] = bf16_to_f32(x[(j ^ 1) * ld + row]);"),
