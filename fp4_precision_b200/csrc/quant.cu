@@ -23,9 +23,10 @@
 //     conflict-free; thread (column c, q) takes rows [Gq, Gq + G) of c.
 //
 // Every fp32 operation is the one the method states, in its order, with no
-// fused multiply-add (the library is built with --fmad=false; packed f32x2
-// adds and multiplies round each lane like the scalar instruction), so codes
-// and scales are exactly those of the definition.
+// fused multiply-add but the one the Quartet II sums define (their first
+// stride, written out as __fmaf_rn / __ffma2_rn; the library is built with
+// --fmad=false, and packed f32x2 operations round each lane like the scalar
+// instruction), so codes and scales are exactly those of the definition.
 #include "qfp4_device.cuh"
 #include "qfp4_internal.h"
 
