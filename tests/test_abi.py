@@ -99,3 +99,20 @@ def test_linear_workspace_covers_operands(lib):
 def test_launch_counter(lib):
     Q.launch_count(reset=True)
     assert Q.launch_count() == 0
+
+
+def test_binding_has_no_fallback(lib, monkeypatch):
+    """Without the built library the binding raises instead of computing
+    anything itself, and on a host without a GPU a quantization raises too
+    (no CPU path exists to fall back to)."""
+    import torch
+    monkeypatch.setattr(Q, "_lib", None)
+    monkeypatch.setattr(Q, "LIB_PATH", os.path.join(ROOT, "fp4_precision_b200", "no_such_libqfp4.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        Q.lib()
+    monkeypatch.undo()
+    if not torch.cuda.is_available():
+        x = torch.zeros((128, 128), dtype=torch.bfloat16)
+        with pytest.raises(Exception):
+            Q.quantize(x, Q.NVFP4, Q.RTN, Q.HAD_NONE, Q.ROW)
+
