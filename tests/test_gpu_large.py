@@ -66,3 +66,51 @@ def test_quantize_past_32_bit_indices():
             ref = O.quantize(x_cpu, Q.NVFP4, rnd, Q.HAD_NONE, axis, ROT, 1, SR, 5 + axis, amax=amax, rows_sel=rows)
             assert_rows_same(q, ref, rows)
             del q
+
+
+def test_gemm_past_31_bit_output_offsets():
+    """GEMM outputs past 2^31 bytes: D [40960 x 28672] in bf16 (2.35 GB) and in
+    fp32 (4.70 GB) from NVFP4 operands with K = 256, and the fp32 output again
+    accumulated into (D += A B^T). Sampled outputs around the row where the
+    byte offset crosses 2^31, and at the ends, are within 2^-18 * sum |a b| of
+    fp64 dot products of the oracle's quantization of the sampled rows (bf16
+    outputs add 2^-8 |D|)."""
+    M, N, K = 40960, 28672, 256
+    free, _ = torch.cuda.mem_get_info()
+    if free < 24 * 2**30:
+        pytest.skip("needs about 24 GB of free device memory")
+    dev = torch.device("cuda", 0)
+    A = inputs.normal((M, K), 1.0, 41, "A", device=dev)
+    B = inputs.normal((N, K), 1.0, 41, "B", device=dev)
+    seed_a, seed_b = Q.make_seed(ROT, SR, 0, 0), Q.make_seed(ROT, SR, 0, 1)
+    qa = Q.quantize(A, Q.NVFP4, Q.RTN, Q.HAD_RAND16, Q.ROW, seed_a)
+    qb = Q.quantize(B, Q.NVFP4, Q.RTN, Q.HAD_RAND16, Q.ROW, seed_b)
+    rng = np.random.default_rng(5)
+    ra = np.unique(np.concatenate([[0, 1, M - 1], [r + d for r in ((1 << 29) // N, (1 << 30) // N) for d in (-1, 0, 1)],
+                                   rng.choice(M, 8, replace=False)]))
+    rb = np.unique(np.concatenate([[0, 1, N // 2, N - 1], rng.choice(N, 12, replace=False)]))
+    Ad = O.dequantize(O.quantize(A.cpu(), Q.NVFP4, Q.RTN, Q.HAD_RAND16, Q.ROW, ROT, 0, SR, 0, rows_sel=ra))
+    Bd = O.dequantize(O.quantize(B.cpu(), Q.NVFP4, Q.RTN, Q.HAD_RAND16, Q.ROW, ROT, 0, SR, 1, rows_sel=rb))
+    ref = Ad @ Bd.T
+    bound = O.GEMM_REL_BOUND * (np.abs(Ad) @ np.abs(Bd).T)
+    ia, ib = torch.as_tensor(ra, device=dev), torch.as_tensor(rb, device=dev)
+
+    def check(D, tol, what):
+        got = D.index_select(0, ia).index_select(1, ib).double().cpu().numpy()
+        err = np.abs(got - ref)
+        assert np.all(err <= tol), f"{what}: {np.sum(err > tol)} of {err.size} sampled outputs out of bound"
+
+    D = Q.gemm(qa, qb, torch.bfloat16)
+    torch.cuda.synchronize()
+    Q.status()
+    check(D, bound + 2.0 ** -8 * np.abs(ref), "bf16")
+    del D
+    D = Q.gemm(qa, qb, torch.float32)
+    torch.cuda.synchronize()
+    Q.status()
+    check(D, bound, "fp32")
+    Q.gemm_accumulate(qa, qb, D)
+    torch.cuda.synchronize()
+    Q.status()
+    ref = 2.0 * ref
+    check(D, 2.0 * bound + np.abs(ref) * 2.0 ** -24, "fp32 accumulated")
