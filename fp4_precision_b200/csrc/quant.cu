@@ -113,6 +113,40 @@ __device__ __forceinline__ void fwht(float* v) {
     if constexpr (N == 32) fwht_stage<N, 16>(v);
 }
 
+// max(m, |H D x|) over G elements in groups of NH (no 1/sqrt(n_h)): the
+// butterflies but the last, whose two outputs only enter the maximum; of
+// RN(a + b) and RN(a - b) the larger magnitude is RN(|a| + |b|) (one exact
+// value has magnitude |a| + |b|, the other at most that, and rounding is
+// monotone and symmetric).
+template <int NH, int G>
+__device__ __forceinline__ float rot_abs_max(float m, float* v) {
+    if constexpr (NH == 0) {
+        return abs_max<G>(m, v);
+    } else {
+#pragma unroll
+        for (int hb = 0; hb < G / NH; ++hb) {
+            float* w = v + hb * NH;
+#pragma unroll
+            for (int j = 0; j < NH; j += 2) {
+                const float a = w[j], b = w[j + 1];
+                w[j] = __fadd_rn(a, b);
+                w[j + 1] = __fsub_rn(a, b);
+            }
+            fwht_stage<NH, 2>(w);
+            if constexpr (NH >= 16) fwht_stage<NH, 4>(w);
+            if constexpr (NH == 32) fwht_stage<NH, 8>(w);
+            float m1 = 0.0f;
+#pragma unroll
+            for (int j = 0; j < NH / 2; j += 2) {
+                m = fmaxf(m, __fadd_rn(fabsf(w[j]), fabsf(w[j + NH / 2])));
+                m1 = fmaxf(m1, __fadd_rn(fabsf(w[j + 1]), fabsf(w[j + 1 + NH / 2])));
+            }
+            m = fmaxf(m, m1);
+        }
+        return m;
+    }
+}
+
 // One stride of the halving tree: s[j] += s[j + ST] for j < ST.
 template <int ST>
 __device__ __forceinline__ void tree_stage(float* s) {
@@ -665,10 +699,24 @@ __device__ __forceinline__ float rot_amax64(Load load, const SignFlips& sf, floa
             fwht_pair_stage<1>(P);
             fwht_pair_stage<2>(P);
             fwht_pair_stage<4>(P);
-            fwht_pair_stage<8>(P);
+            // The last stage (half-width 8) only feeds the maximum: of RN(a + b)
+            // and RN(a - b) the larger magnitude is RN(|a| + |b|) (one of the two
+            // exact values has magnitude |a| + |b|, the other at most that, and
+            // rounding is monotone and symmetric), so one scalar sum per pair of
+            // outputs replaces the two packed ones, and half as many values
+            // enter the maximum.
+            float m1 = 0.0f;
+#pragma unroll
+            for (int j = 0; j < 8; j += 2) {
+                m = max3(m, __fadd_rn(fabsf(P[j].x), fabsf(P[j + 8].x)), __fadd_rn(fabsf(P[j].y), fabsf(P[j + 8].y)));
+                m1 = max3(m1, __fadd_rn(fabsf(P[j + 1].x), fabsf(P[j + 9].x)),
+                          __fadd_rn(fabsf(P[j + 1].y), fabsf(P[j + 9].y)));
+            }
+            m = fmaxf(m, m1);
+        } else {
+            const float2 am = abs_max_pair(P);
+            m = max3(m, am.x, am.y);
         }
-        const float2 am = abs_max_pair(P);
-        m = max3(m, am.x, am.y);
     }
     return m;
 }
@@ -937,8 +985,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<STAGES>)
                 v[8 * c8 + 6] = bf16lo(w3); v[8 * c8 + 7] = bf16hi(w3);
             }
             if constexpr (AMAX_ONLY) {
-                Group<kNvfp4, kRtn, NH>::template rotate<false>(v);
-                amax_acc = abs_max<G>(amax_acc, v);
+                amax_acc = rot_abs_max<NH, G>(amax_acc, v);
             } else {
                 Grp::rotate(v);
                 const int64_t j0 = col0 + g * G;
@@ -1141,8 +1188,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             const int64_t c = c0 + cc[ci];              // x column = output row
             const int64_t r_grp = r0 + (int64_t)G * q;  // first k index of this group
             if constexpr (AMAX_ONLY) {
-                Group<kNvfp4, kRtn, NH>::template rotate<false>(v);
-                amax_acc = abs_max<G>(amax_acc, v);
+                amax_acc = rot_abs_max<NH, G>(amax_acc, v);
                 if constexpr (DUAL) {
                     // Row orientation from the same tile: thread t takes shared-
                     // memory row t % 64 (some x-row of the tile; the max does not
@@ -1172,8 +1218,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                         vr[8 * c8 + 4] = bf16lo(w2); vr[8 * c8 + 5] = bf16hi(w2);
                         vr[8 * c8 + 6] = bf16lo(w3); vr[8 * c8 + 7] = bf16hi(w3);
                     }
-                    Group<kNvfp4, kRtn, NH>::template rotate<false>(vr);
-                    amax_row_acc = abs_max<16>(amax_row_acc, vr);
+                    amax_row_acc = rot_abs_max<NH, 16>(amax_row_acc, vr);
                 }
             } else {
                 uint32_t codes[G / 8];
