@@ -223,6 +223,9 @@ def run_ours(args, rank, world, local_rank):
     # with round-to-nearest one pass gives both quantizations
     fused_dy_amax, dual_dy = dy_plan(Q, c, M)
     dy_amax = torch.empty((2,), dtype=torch.float32, device=dev)
+    # X and W: the forward's amax read also gives the backward's tensor amaxes
+    xw = xw_plan(Q, c)
+    xw_amax = torch.empty((4,), dtype=torch.float32, device=dev)
 
     def step(ev=None, st=None):
         st = stream if st is None else st
@@ -236,7 +239,7 @@ def run_ours(args, rank, world, local_rank):
             if i in (2, 4):
                 quantize_dy(Q, dY, c, ops, qs, i, fused_dy_amax, dual_dy, dy_amax, ws, st)
             else:
-                Q.quantize(t, fmt, rnd, had, axis, sd, out=qs[i], workspace=ws, stream=st)
+                quantize_xw(Q, ops, qs, i, xw, xw_amax, ws, st)
             mark(i, 1)
             if i == 1:
                 mark(6, 0)
@@ -543,6 +546,37 @@ def quantize_dy(Q, dY, c, ops, qs, i, fused, dual, dy_amax, ws, stream):
     Q.quantize(t, fmt, rnd, had, axis, sd, amax_in=am if fused else None, out=qs[i], workspace=ws, stream=stream)
 
 
+def xw_plan(Q, c):
+    """Whether the forward takes the backward's NVFP4 tensor amaxes of X and W
+    in the read that gives its own (qfp4_amax_rowcol: the forward's Hadamard
+    along K, the backward GEMM's along the other axis), so that the backward
+    quantizes X and W without an amax pass of its own: (for X, for W). Both
+    GEMMs that use the operand must quantize it to NVFP4. (The linear layer's
+    entry points cannot do this: the forward and the backward are separate
+    calls.)"""
+    nv = lambda g: g.fmt == Q.NVFP4
+    return (nv(c[0]) and nv(c[2]), nv(c[0]) and nv(c[1]))
+
+
+def quantize_xw(Q, ops, qs, i, plan, xw_amax, ws, stream):
+    """Operand i (0: X along K, 1: W along K, 3: W along N, 5: X along the
+    tokens) of the step. With plan[X or W] the forward's call takes both
+    tensor amaxes of the operand in one read and the backward's call uses the
+    second (the same values the backward's own amax pass would give)."""
+    t, fmt, rnd, had, axis, sd = ops[i]
+    j = 0 if i in (0, 5) else 1
+    if not plan[j]:
+        Q.quantize(t, fmt, rnd, had, axis, sd, out=qs[i], workspace=ws, stream=stream)
+        return
+    am = xw_amax[2 * j:2 * j + 2]
+    if i in (0, 1):
+        b = 5 if i == 0 else 3
+        Q.amax_rowcol(t, had, sd, ops[b][5], out=am, workspace=ws, stream=stream, had_col=ops[b][3])
+        Q.quantize(t, fmt, rnd, had, axis, sd, amax_in=am[0:1], out=qs[i], workspace=ws, stream=stream)
+    else:
+        Q.quantize(t, fmt, rnd, had, axis, sd, amax_in=am[1:2], out=qs[i], workspace=ws, stream=stream)
+
+
 def layer_step(Q, X, W, dY, rec, seed, steps, stream, dev):
     """One linear layer's fwd+bwd through the six quantize and three GEMM calls
     (the same sequence as the headline step), timed with CUDA events on the
@@ -570,13 +604,15 @@ def layer_step(Q, X, W, dY, rec, seed, steps, stream, dev):
 
     fused_dy_amax, dual_dy = dy_plan(Q, c, M)
     dy_amax = torch.empty((2,), dtype=torch.float32, device=dev)
+    xw = xw_plan(Q, c)
+    xw_amax = torch.empty((4,), dtype=torch.float32, device=dev)
 
     def step(ev):
         for i, (t, fmt, rnd, had, axis, sd) in enumerate(ops):
             if i in (2, 4):
                 quantize_dy(Q, dY, c, ops, qs, i, fused_dy_amax, dual_dy, dy_amax, ws, stream)
             else:
-                Q.quantize(t, fmt, rnd, had, axis, sd, out=qs[i], workspace=ws, stream=stream)
+                quantize_xw(Q, ops, qs, i, xw, xw_amax, ws, stream)
             if i % 2 == 1:
                 a, b, D, odt = outs[i // 2]
                 if ev is not None:

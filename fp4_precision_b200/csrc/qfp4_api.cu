@@ -718,18 +718,19 @@ qfp4_seed op_seed(const qfp4_seed* s, uint32_t gemm, uint32_t operand) {
 
 // Both orientations' rotated amax. n_h <= 16: one read of x by the column
 // kernel (its tile serves 16-element groups of both axes); n_h = 32: two passes.
-int amax_rowcol_impl(const void* x, int64_t R, int64_t C, int64_t ld, int32_t had, const qfp4_seed* seed_row,
-                     const qfp4_seed* seed_col, float* amax_row, float* amax_col, void* workspace,
-                     size_t workspace_bytes, cudaStream_t s) {
+int amax_rowcol_impl(const void* x, int64_t R, int64_t C, int64_t ld, int32_t had_row, int32_t had_col,
+                     const qfp4_seed* seed_row, const qfp4_seed* seed_col, float* amax_row, float* amax_col,
+                     void* workspace, size_t workspace_bytes, cudaStream_t s) {
     int rc = bind_context(s);  // callers may run on threads without a current context
     if (rc) return rc;
     int sms = 0;
     if ((rc = check_device(&sms))) return rc;
     Geometry gr, gc;
-    if ((rc = validate_input(x, R, C, ld, had, QFP4_AXIS_ROW, &gr))) return rc;
-    if ((rc = validate_input(x, R, C, ld, had, QFP4_AXIS_COL, &gc))) return rc;
+    if ((rc = validate_input(x, R, C, ld, had_row, QFP4_AXIS_ROW, &gr))) return rc;
+    if ((rc = validate_input(x, R, C, ld, had_col, QFP4_AXIS_COL, &gc))) return rc;
     if (amax_row == nullptr || amax_col == nullptr) return QFP4_ERR_INVALID_ARG;
-    if (had_random(had) && (seed_row == nullptr || seed_col == nullptr)) return QFP4_ERR_INVALID_ARG;
+    if ((had_random(had_row) && seed_row == nullptr) || (had_random(had_col) && seed_col == nullptr))
+        return QFP4_ERR_INVALID_ARG;
     if (workspace == nullptr || workspace_bytes < qfp4_quantize_workspace_bytes()) return QFP4_ERR_WORKSPACE;
     if (!aligned16(workspace)) return QFP4_ERR_MISALIGNED;
     if (R == 0 || C == 0) {
@@ -737,12 +738,13 @@ int amax_rowcol_impl(const void* x, int64_t R, int64_t C, int64_t ld, int32_t ha
         if (e == cudaSuccess) e = cudaMemsetAsync(amax_col, 0, sizeof(float), s);
         return e == cudaSuccess ? QFP4_OK : cuda_fail(e);
     }
-    const uint32_t signs_row = had_random(had) ? host_sign_bits(seed_row->rot, seed_row->rot_stream) : 0u;
-    const uint32_t signs_col = had_random(had) ? host_sign_bits(seed_col->rot, seed_col->rot_stream) : 0u;
+    // a deterministic Hadamard is the random one with no sign flips
+    const uint32_t signs_row = had_random(had_row) ? host_sign_bits(seed_row->rot, seed_row->rot_stream) : 0u;
+    const uint32_t signs_col = had_random(had_col) ? host_sign_bits(seed_col->rot, seed_col->rot_stream) : 0u;
     float* partials = static_cast<float*>(workspace);
-    const int nh = had_n(had);
+    const int nh = had_n(had_col);
     cudaError_t e;
-    if (nh <= 16) {
+    if (nh <= 16 && had_n(had_row) == nh) {
         QuantParams p{};
         p.x = static_cast<const uint16_t*>(x);
         p.R = R; p.C = C; p.ld = ld;
@@ -768,11 +770,12 @@ int amax_rowcol_impl(const void* x, int64_t R, int64_t C, int64_t ld, int32_t ha
         if (e == cudaSuccess) e = launch_reduce_max(partials, n, amax_col, s);
         if (e == cudaSuccess) e = launch_reduce_max(partials + n, n, amax_row, s);
     } else {
+        // a 32-point Hadamard, or Hadamards of different sizes: one pass per orientation
         int n = 0;
-        if ((rc = run_amax(x, R, C, ld, had, QFP4_AXIS_ROW, signs_row, gr, partials, &n, sms, s))) return rc;
+        if ((rc = run_amax(x, R, C, ld, had_row, QFP4_AXIS_ROW, signs_row, gr, partials, &n, sms, s))) return rc;
         e = launch_reduce_max(partials, n, amax_row, s);
         if (e != cudaSuccess) return cuda_fail(e);
-        if ((rc = run_amax(x, R, C, ld, had, QFP4_AXIS_COL, signs_col, gc, partials, &n, sms, s))) return rc;
+        if ((rc = run_amax(x, R, C, ld, had_col, QFP4_AXIS_COL, signs_col, gc, partials, &n, sms, s))) return rc;
         e = launch_reduce_max(partials, n, amax_col, s);
     }
     return e == cudaSuccess ? QFP4_OK : cuda_fail(e);
@@ -855,12 +858,12 @@ int qfp4_amax(const void* x, int64_t R, int64_t C, int64_t ld, int32_t had, int3
     return e == cudaSuccess ? QFP4_OK : cuda_fail(e);
 }
 
-int qfp4_amax_rowcol(const void* x, int64_t R, int64_t C, int64_t ld, int32_t had, const qfp4_seed* seed_row,
-                     const qfp4_seed* seed_col, float* amax_row, float* amax_col, void* workspace,
-                     size_t workspace_bytes, void* stream) {
+int qfp4_amax_rowcol(const void* x, int64_t R, int64_t C, int64_t ld, int32_t had_row, int32_t had_col,
+                     const qfp4_seed* seed_row, const qfp4_seed* seed_col, float* amax_row, float* amax_col,
+                     void* workspace, size_t workspace_bytes, void* stream) {
     const ApiRange range("qfp4_amax_rowcol");
-    return amax_rowcol_impl(x, R, C, ld, had, seed_row, seed_col, amax_row, amax_col, workspace, workspace_bytes,
-                            static_cast<cudaStream_t>(stream));
+    return amax_rowcol_impl(x, R, C, ld, had_row, had_col, seed_row, seed_col, amax_row, amax_col, workspace,
+                            workspace_bytes, static_cast<cudaStream_t>(stream));
 }
 
 int qfp4_quantize(const void* x, int64_t R, int64_t C, int64_t ld, int32_t fmt, int32_t rounding, int32_t had,
@@ -1035,7 +1038,8 @@ int qfp4_linear_bwd(const void* dY, const void* X, const void* W, void* dX, void
     const float* am_row = nullptr;
     const float* am_col = nullptr;
     if (d.fmt == QFP4_NVFP4 && w.fmt == QFP4_NVFP4 && d.had == w.had && had_n(d.had) <= 16) {
-        if ((rc = amax_rowcol_impl(dY, M, N, N, d.had, &s0, &s2, dy_amax, dy_amax + 1, partials, pws, s))) return rc;
+        if ((rc = amax_rowcol_impl(dY, M, N, N, d.had, d.had, &s0, &s2, dy_amax, dy_amax + 1, partials, pws, s)))
+            return rc;
         am_row = dy_amax;
         am_col = dy_amax + 1;
     } else if (dual && d.fmt == QFP4_NVFP4) {

@@ -73,7 +73,7 @@ _SIGNATURES = {
     "qfp4_scale_offset": (_I64, [_I32, _I64, _I64, _I64, _I64]),
     "qfp4_quantize_workspace_bytes": (_SZ, []),
     "qfp4_amax": (ctypes.c_int, [_VOID, _I64, _I64, _I64, _I32, _I32, ctypes.POINTER(Seed), _VOID, _VOID, _SZ, _VOID]),
-    "qfp4_amax_rowcol": (ctypes.c_int, [_VOID, _I64, _I64, _I64, _I32, ctypes.POINTER(Seed), ctypes.POINTER(Seed),
+    "qfp4_amax_rowcol": (ctypes.c_int, [_VOID, _I64, _I64, _I64, _I32, _I32, ctypes.POINTER(Seed), ctypes.POINTER(Seed),
                                         _VOID, _VOID, _VOID, _SZ, _VOID]),
     "qfp4_quantize": (ctypes.c_int, [_VOID, _I64, _I64, _I64, _I32, _I32, _I32, _I32, ctypes.POINTER(Seed), _VOID,
                                      ctypes.POINTER(TensorDesc), _VOID, _SZ, _VOID]),
@@ -205,16 +205,18 @@ def amax(x: torch.Tensor, had: int = HAD_NONE, axis: int = ROW, seed: Seed | Non
 
 
 def amax_rowcol(x: torch.Tensor, had: int, seed_row: Seed | None = None, seed_col: Seed | None = None, out=None,
-                workspace=None, stream=None) -> torch.Tensor:
+                workspace=None, stream=None, had_col: int | None = None) -> torch.Tensor:
     """Both orientations' tensor amax in one call: out[0] as amax(x, had, ROW,
-    seed_row), out[1] as amax(x, had, COL, seed_col)."""
+    seed_row), out[1] as amax(x, had_col (default had), COL, seed_col)."""
     assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
     R, C = x.shape
     out = torch.empty((2,), dtype=torch.float32, device=x.device) if out is None else out
     ws = torch.empty((quantize_workspace_bytes(),), dtype=torch.uint8, device=x.device) if workspace is None else workspace
     seed_row = seed_row or make_seed()
     seed_col = seed_col or make_seed()
-    _check(lib().qfp4_amax_rowcol(_ptr(x), R, C, x.stride(0), had, ctypes.byref(seed_row), ctypes.byref(seed_col),
+    had_col = had if had_col is None else had_col
+    _check(lib().qfp4_amax_rowcol(_ptr(x), R, C, x.stride(0), had, had_col, ctypes.byref(seed_row),
+                                  ctypes.byref(seed_col),
                                   _ptr(out), ctypes.c_void_p(out.data_ptr() + 4), _ptr(ws), ws.numel(),
                                   _stream(stream)), "qfp4_amax_rowcol")
     return out

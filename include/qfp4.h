@@ -200,19 +200,23 @@ size_t qfp4_quantize_workspace_bytes(void);
 int qfp4_amax(const void* x, int64_t R, int64_t C, int64_t ld, int32_t had, int32_t axis, const qfp4_seed* seed,
               float* amax, void* workspace, size_t workspace_bytes, void* stream);
 /* qfp4_amax_rowcol: both orientations' tensor amax of x (bf16, R x C), as
- * qfp4_amax computes them: *amax_row with axis ROW and seed_row's sign
- * vector, *amax_col with axis COL and seed_col's (device fp32 each; the two
- * GEMMs that use x along both axes rotate with different sign vectors). A
- * Hadamard of size <= 16 (or none) takes one read of x; size 32 takes two.
- * Requirements: those of qfp4_amax for both axes (R and C multiples of n_h);
- * workspace >= qfp4_quantize_workspace_bytes(), 16-byte aligned.
+ * qfp4_amax computes them: *amax_row with axis ROW, had_row and seed_row's
+ * sign vector, *amax_col with axis COL, had_col and seed_col's (device fp32
+ * each; the two GEMMs that use x along both axes rotate with different sign
+ * vectors, and may use a deterministic Hadamard on one axis and a random one
+ * on the other). Hadamards of one size <= 16 (or none on both axes) take one
+ * read of x; size 32 or two different sizes take one read per axis.
+ * Requirements: those of qfp4_amax for both axes (R a multiple of had_col's
+ * size, C of had_row's); workspace >= qfp4_quantize_workspace_bytes(),
+ * 16-byte aligned.
  * This is the fused tensor-scale pass of the backward linear layer (dY is
  * quantized along N for Dgrad and along the tokens for Wgrad; pages: "New AMD
  * paper overturns conventional wisdom: FP4 training...", section
- * "Poiskovaya eksperimental'naya rabota", the three GEMMs of the layer). */
-int qfp4_amax_rowcol(const void* x, int64_t R, int64_t C, int64_t ld, int32_t had, const qfp4_seed* seed_row,
-                     const qfp4_seed* seed_col, float* amax_row, float* amax_col, void* workspace,
-                     size_t workspace_bytes, void* stream);
+ * "Poiskovaya eksperimental'naya rabota", the three GEMMs of the layer), and
+ * lets the forward take the backward's amaxes of X and W in its own read. */
+int qfp4_amax_rowcol(const void* x, int64_t R, int64_t C, int64_t ld, int32_t had_row, int32_t had_col,
+                     const qfp4_seed* seed_row, const qfp4_seed* seed_col, float* amax_row, float* amax_col,
+                     void* workspace, size_t workspace_bytes, void* stream);
 
 int qfp4_quantize(const void* x, int64_t R, int64_t C, int64_t ld, int32_t fmt, int32_t rounding, int32_t had,
                   int32_t axis, const qfp4_seed* seed, const float* amax_in, qfp4_tensor* out, void* workspace,

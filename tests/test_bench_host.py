@@ -42,6 +42,24 @@ def test_dy_plan_of_custom_recipes():
     assert bench.dy_plan(Q, c, 16384 + 32) == (True, False)  # tokens not a multiple of 64
 
 
+@pytest.mark.parametrize("name,plan", [
+    ("QUARTET2_NVFP4", (True, True)),   # NVFP4 in all three GEMMs: X and W amaxes from the forward's read
+    ("NVIDIA_NVFP4", (True, True)),
+    ("AMD_MXFP4_H", (False, False)),    # MXFP4 has no tensor amax
+])
+def test_xw_plan_of_the_presets(name, plan):
+    assert bench.xw_plan(Q, cfgs(name)) == plan
+
+
+def test_xw_plan_needs_nvfp4_on_both_gemms():
+    r = Q.recipe("QUARTET2_NVFP4")
+    c = [r.fprop, r.dgrad, r.wgrad]
+    c[2].fmt = Q.MXFP4
+    assert bench.xw_plan(Q, c) == (False, True)    # X's backward operand is MXFP4
+    c[2].fmt, c[1].fmt = Q.NVFP4, Q.MXFP4
+    assert bench.xw_plan(Q, c) == (True, False)
+
+
 def test_traffic_is_reported_only_for_the_profiled_sources(monkeypatch):
     root = helpers.scratch_dir("bench_root_")
     try:

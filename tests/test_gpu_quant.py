@@ -274,6 +274,28 @@ def test_amax_rowcol_matches_oracle(had, shape):
     assert np.float32(a[1]) == np.float32(np.abs(v_col).max())
 
 
+@pytest.mark.parametrize("hads", [(Q.HAD_DET16, Q.HAD_RAND16), (Q.HAD_RAND16, Q.HAD_DET16), (Q.HAD_NONE, Q.HAD_RAND16),
+                                  (Q.HAD_RAND32, Q.HAD_DET16)], ids=["det16-rand16", "rand16-det16", "none-rand16",
+                                                                     "rand32-det16"])
+@pytest.mark.parametrize("shape", [(352, 416), (384, 256), (8192, 4096)], ids=lambda s: "x".join(map(str, s)))
+def test_amax_rowcol_with_a_hadamard_per_axis(hads, shape):
+    """A Hadamard per orientation (the forward's deterministic one along K and
+    the backward's random one along the tokens, as the linear layer uses them):
+    one read of x when both have 16 points, one read per axis otherwise; each
+    amax equals the oracle's max |rotated x| with that axis's Hadamard."""
+    had_row, had_col = hads
+    R, C = shape
+    x = sweep_like(R, C)
+    s_row = Q.make_seed(SEED["rot"], SEED["sr"], 0, 0)
+    s_col = Q.make_seed(SEED["rot"], SEED["sr"], 2, 5)
+    a = Q.amax_rowcol(x.cuda(), had_row, s_row, s_col, had_col=had_col).cpu().numpy()
+    Q.status()
+    v_row = O.rotate(x, had_row, O.ROW, SEED["rot"], 0)
+    v_col = O.rotate(x, had_col, O.COL, SEED["rot"], 2)
+    assert np.float32(a[0]) == np.float32(np.abs(v_row).max())
+    assert np.float32(a[1]) == np.float32(np.abs(v_col).max())
+
+
 def test_determinism_and_seed_sensitivity():
     x = sweep_like(256, 256).cuda()
     a = gpu_quant(x, Q.NVFP4, Q.SR, Q.HAD_RAND16, Q.COL)
